@@ -1,0 +1,434 @@
+"""Benchmark of one decode step of joint-QKV latent attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1]
+                    [--impl ours|reference] [--splits G] [--kernel auto|simt|tcgen05]
+
+One step = the whole hot path for one batch: append the current token of
+every sequence (c = x W^d, written as row len-1), then decode attention over
+the latent cache (query projection and absorption, split-KV flash decoding,
+cross-split merge and value up-projection).  Inputs are synthetic and seeded
+(``synthetic``); the latent cache is far larger than L2, so no flush is
+needed between steps.  Prints one JSON line (rank 0).
+
+Multi-GPU (torchrun): every rank holds its own batch of sequences (weak
+scaling, no collective on the data path); the step time is the max over
+ranks.  ``--impl reference`` times the CPU oracle on this host's cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "decode-attn KV-tokens/s over C_qkv latent cache; achieved HBM GB/s vs peak"
+UNIT = "KV-tokens/s"
+TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+ROW_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "i8": 1, "i4": 0.5}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+
+def bench_inputs(cfg: int, device: str, rank: int = 0):
+    """Device-resident synthetic inputs of configuration ``cfg`` (the same
+    recipe on every rank, seeded by rank)."""
+    w = synthetic.CONFIGS[cfg]
+    lens = synthetic.lengths(w)
+    max_len = int(lens.max())
+    cs, _ = synthetic.direct_channel_scales(w)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed * 7919 + rank)
+    B, r = w.B, w.r
+    cs_t = torch.tensor(cs, dtype=torch.float32, device=device)
+    scales = None
+    if w.cache in ("f32", "f16", "bf16"):
+        cache = torch.empty((B, max_len, r), dtype=TORCH_DT[w.cache], device=device)
+        for b in range(B):   # per sequence keeps the fp32 temporary small
+            rows = torch.randn((max_len, r), generator=gen, device=device) * cs_t
+            cache[b].copy_(rows)
+    else:
+        # random codes on the symmetric grid and positive fp16 group scales
+        g = w.group
+        if w.cache == "i8":
+            cache = torch.randint(-127, 128, (B, max_len, r), generator=gen, device=device,
+                                  dtype=torch.int8)
+        else:
+            lo = torch.randint(-7, 8, (B, max_len, r // 2), generator=gen, device=device)
+            hi = torch.randint(-7, 8, (B, max_len, r // 2), generator=gen, device=device)
+            cache = ((lo & 0xF) | ((hi & 0xF) << 4)).to(torch.uint8)
+        grp = cs_t.view(r // g, g).amax(dim=1) * 3.0 / (7 if w.cache == "i4" else 127)
+        scales = (grp[None, None, :] * (0.5 + torch.rand((B, max_len, r // g), generator=gen,
+                                                          device=device))).to(torch.float16)
+    wuq, wuk, wuv = (torch.from_numpy(a).to(device=device, dtype=TORCH_DT[w.weight])
+                     for a in synthetic.direct_up_weights_np(w))
+    wd = torch.from_numpy(synthetic.direct_down_weight_np(w)).to(device=device,
+                                                               dtype=TORCH_DT[w.weight])
+    x = torch.from_numpy(synthetic.direct_new_tokens_np(w)).to(dtype=TORCH_DT[w.weight])
+    return dict(w=w, lens=lens, max_len=max_len, cache=cache, scales=scales, wuq=wuq, wuk=wuk,
+                wuv=wuv, wd=wd, x_host=x)
+
+
+def latent_bytes(w, lens) -> float:
+    """Latent-cache bytes one step reads: rows x row bytes (+ group scales)."""
+    rows = float(np.sum(lens))
+    b = rows * w.r * ROW_BYTES[w.cache]
+    if w.cache in ("i8", "i4"):
+        b += rows * (w.r // w.group) * 2
+    return b
+
+
+def weight_bytes(w) -> float:
+    """W^d and the three W^u read once per step (4 r E elements)."""
+    return 4.0 * w.r * w.E * (4 if w.weight == "f32" else 2)
+
+
+# ---------------------------------------------------------------------------
+# clocks, peaks, profiles
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "rank_joint_qkv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_name: str, workload: str, src_files):
+    """DRAM bytes per launch of the split kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_name, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_hash(src_files):
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import rank_joint_qkv_b200 as q
+
+    device = f"cuda:{local_rank}"
+    torch.cuda.set_device(device)
+    inp = bench_inputs(args.config, device, rank)
+    w, lens, max_len = inp["w"], inp["lens"], inp["max_len"]
+    kern = {"auto": q.QSVD_KERNEL_AUTO, "simt": q.QSVD_KERNEL_SIMT,
+            "tcgen05": q.QSVD_KERNEL_TCGEN05}[args.kernel]
+    dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
+                       out="f32", group=w.group, rope=w.rope, rope_base=w.rope_base,
+                       kernel=kern)
+    packed = q.qsvd_prepare_weights(dims, inp["wd"], inp["wuq"], inp["wuk"], inp["wuv"])
+    stream = torch.cuda.current_stream()
+    lens_dev = torch.from_numpy(lens).to(device)
+    pos_dev = (lens_dev - 1).to(torch.int32)
+    x_dev = inp["x_host"].to(device)
+    cnew = torch.empty((w.B, w.r), dtype=torch.float32, device=device)
+    out = torch.empty((w.B, w.E), dtype=torch.float32, device=device)
+    app_ws = torch.empty(q.append_workspace_bytes(dims), dtype=torch.uint8, device=device)
+    dec_ws = torch.empty(q.decode_workspace_bytes(dims, args.splits), dtype=torch.uint8,
+                         device=device)
+    cache, scales = inp["cache"], inp["scales"]
+
+    def step(ev_split=None):
+        q.qsvd_append_latent(dims, packed, x_dev, pos_dev, cache, scales, cnew, None, app_ws,
+                             stream=stream)
+        q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
+                           num_splits=args.splits, workspace=dec_ws,
+                           phases=q.QSVD_PHASE_PROLOGUE, stream=stream)
+        if ev_split is not None:
+            ev_split[0].record(stream)
+        q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
+                           num_splits=args.splits, workspace=dec_ws,
+                           phases=q.QSVD_PHASE_SPLIT, stream=stream)
+        if ev_split is not None:
+            ev_split[1].record(stream)
+        q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
+                           num_splits=args.splits, workspace=dec_ws,
+                           phases=q.QSVD_PHASE_COMBINE, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = q.kernel_launches()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    launches = q.kernel_launches() - launches0
+    ms = t0.elapsed_time(t1)
+    split_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_per_step = float(np.sum(lens))
+    value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+
+    # end to end through the public API with host buffers
+    x_pin = inp["x_host"].pin_memory()
+    lens_pin = torch.from_numpy(lens).pin_memory()
+    out_pin = torch.empty((w.B, w.E), dtype=torch.float32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ke = max(3, args.steps)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(ke):
+        x_dev.copy_(x_pin, non_blocking=True)
+        lens_dev.copy_(lens_pin, non_blocking=True)
+        torch.sub(lens_dev, 1, out=pos_dev)
+        step()
+        out_pin.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = tokens_per_step * ke * world / (float(e2e_t.item()) / 1e3)
+    h2d = x_pin.numel() * x_pin.element_size() + lens_pin.numel() * 4
+    d2h = out_pin.numel() * 4
+
+    if rank != 0:
+        return None
+    hbm_peak, _, peak_kind = measured_peaks()
+    split_mean = statistics.mean(split_ms)
+    lat_b = latent_bytes(w, lens)
+    achieved = lat_b / (split_mean / 1e3) / 1e9
+    kname = "split_tcgen05" if args.kernel == "tcgen05" else "split_simt"
+    workload = w.name
+    traffic = profiled_traffic(kname, workload, ["split_simt.cu", "internal.cuh"])
+    step_gbs = (lat_b + weight_bytes(w)) / (ms_max / args.steps / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.cache, "data": "synthetic",
+        "config": {"workload": workload, "E": w.E, "H": w.H, "d_h": w.d_h, "r": w.r,
+                   "batch_per_gpu": w.B, "kv_len": int(max_len),
+                   "tokens_per_step_per_gpu": int(tokens_per_step), "cache": w.cache,
+                   "weights": w.weight, "mode": "rope" if w.rope else "absorbed",
+                   "splits": args.splits, "kernel": args.kernel,
+                   "l2": "inputs larger than L2: %.0f MB latent read per step per GPU"
+                         % (lat_b / 1e6),
+                   "parallelism": f"dp{world}"},
+        "steps_per_s": args.steps * 1e3 / ms_max,
+        "step_hbm_gbs": step_gbs,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "kernel": kname, "peak_kind": peak_kind,
+                     "bytes_per_launch": lat_b, "launch_ms": split_mean},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+    }
+    line["clocks"] = clk.summary()
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, lens, budget_s=args.cpu_seconds)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, n_tokens: int, b: int):
+    """One sequence of the workload on the host: latent rows, new latent, W^u."""
+    from oracle import qsvd_ref as ref   # noqa: F401  (checked import for the timed leg)
+    c = synthetic.direct_latent_rows_np(w, b, n_tokens).astype(np.float64)
+    cnew = synthetic.direct_new_latent_np(w)[b:b + 1].astype(np.float64)
+    wuq, wuk, wuv = (a.astype(np.float64) for a in synthetic.direct_up_weights_np(w))
+    return c, cnew, wuq, wuk, wuv
+
+
+def time_oracle(w, n_tokens, budget_s, max_seqs=None):
+    from oracle import qsvd_ref as ref
+    rb = w.rope_base if w.rope else None
+    done_tokens, spent, seqs = 0, 0.0, 0
+    wts = None
+    while spent < budget_s and (max_seqs is None or seqs < max_seqs):
+        c, cnew, wuq, wuk, wuv = oracle_sample(w, n_tokens, seqs % w.B)
+        t = time.perf_counter()
+        ref.decode_materialized([c], [n_tokens], cnew, wuq, wuk, wuv, w.H, rope_base=rb)
+        spent += time.perf_counter() - t
+        done_tokens += n_tokens
+        seqs += 1
+    return done_tokens, spent, seqs
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, lens, budget_s=15.0):
+    n = int(min(int(np.max(lens)), 8192))
+    tokens, spent, seqs = time_oracle(w, n, budget_s)
+    return {"value": tokens / spent, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{seqs} sequence(s) of {n} tokens through the fp64 oracle "
+                      f"(keys/values materialised), {spent:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = synthetic.CONFIGS[args.config]
+    lens = synthetic.lengths(w)
+    n = int(min(int(np.max(lens)), 8192))
+    for _ in range(args.warmup):
+        time_oracle(w, min(n, 512), 0.0, max_seqs=1)
+    tokens, spent, seqs = 0, 0.0, 0
+    for _ in range(args.steps):
+        t, s, k = time_oracle(w, n, 0.0, max_seqs=1)
+        tokens += t
+        spent += s
+        seqs += k
+    value = tokens / spent
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": spent / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "E": w.E, "H": w.H, "d_h": w.d_h, "r": w.r,
+                   "mode": "rope" if w.rope else "absorbed",
+                   "sample_per_step": f"one sequence of {n} tokens"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"{seqs} sequence(s) of {n} tokens, one per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group(
+                "nccl", timeout=datetime.timedelta(seconds=300),
+                device_id=torch.device(f"cuda:{local_rank}"))
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,224 @@
+/*
+ * qsvd.h -- C ABI of the joint-QKV latent decode library (NVIDIA B200, sm_100a).
+ *
+ * The operation.  QSVD compresses the query, key and value projections of an
+ * attention layer jointly: [W_Q W_K W_V] (E x 3E) ~= W^d [W^u_q W^u_k W^u_v],
+ * with one shared down-projection W^d (E x r) and three up-projections W^u_*
+ * (r x E each).  Only the latent C = X W^d (L x r per sequence) is cached;
+ * keys and values are rebuilt from it on the fly as C W^u_k and C W^u_v.
+ *   - QSVD paper notes (Paper-Notes, NeurIPS 2025), section 关键设计,
+ *     "QKV联合SVD分解" (joint SVD, shared latent of size r x L, 4rE weights).
+ *   - QSVD paper digest, section Method, Step 1 (C_qkv buffered, K and V
+ *     recomputed on the fly) and Step 3 (H1/H2 rotations, beta split,
+ *     latent quantisation).
+ *   - WSVD paper digest, sections Problem and Method 3.4: a decoder that
+ *     re-reads the shared latent once per head moves more bytes than an
+ *     uncompressed cache; a fused flash-decoding kernel reconstructs keys
+ *     on-chip and applies rotary embedding.
+ * This library implements one decode step of that attention: every head
+ * reads the latent tile once from HBM (split-KV flash decoding), with the
+ * query absorbed into latent space (no rotary embedding) or with per-tile key
+ * reconstruction on the tensor cores followed by rotary embedding.
+ *
+ * Conventions shared by all calls:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, unless
+ *     the argument says "host".  The library never allocates device memory
+ *     and keeps no per-model state; scratch lives in a caller-provided
+ *     workspace whose size the library reports.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t passed
+ *     as void*; NULL is the legacy default stream).  No call synchronises.
+ *   - Row-major layouts; "B x E" means B rows of E contiguous elements.
+ *   - Heads: head h owns columns [h*d_h, (h+1)*d_h) of every E-wide matrix.
+ *   - Errors detectable on the host return a status and enqueue nothing.
+ *     Violations only visible on the device (a length or position out of
+ *     range) are clamped and recorded as bits in a device status word; no
+ *     kernel traps.
+ *   - Pointers must be 16-byte aligned.
+ */
+#ifndef QSVD_H
+#define QSVD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QSVD_ABI_VERSION 1
+
+typedef enum {
+  QSVD_OK = 0,
+  QSVD_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent or unsupported sizes */
+  QSVD_ERR_UNSUPPORTED = 2,  /* valid request that this build has no kernel for */
+  QSVD_ERR_WORKSPACE = 3,    /* workspace or packed buffer too small */
+  QSVD_ERR_CUDA = 4          /* a CUDA runtime call or kernel launch failed */
+} qsvd_status;
+
+typedef enum {
+  QSVD_F32 = 0,
+  QSVD_F16 = 1,
+  QSVD_BF16 = 2,
+  QSVD_I8 = 3,   /* latent cache only: int8 codes + fp16 group scales */
+  QSVD_I4 = 4    /* latent cache only: packed int4 codes + fp16 group scales */
+} qsvd_dtype;
+
+/* Split-KV granularity: sequences are cut into tiles of this many tokens. */
+#define QSVD_TILE_TOKENS 128
+
+/* Phases of qsvd_decode_attn (bit mask; 0 means all). */
+#define QSVD_PHASE_PROLOGUE 1u  /* query (c_new W^u_q), absorption or rotary */
+#define QSVD_PHASE_SPLIT 2u     /* split-KV attention over the latent tiles */
+#define QSVD_PHASE_COMBINE 4u   /* merge of the split partials, value up-projection */
+#define QSVD_PHASE_ALL 7u
+
+/* Device status bits (workspace word 0 for decode; `status` for append). */
+#define QSVD_STATUS_LEN_CLAMPED 1   /* some lengths[b] < 0 or > max_len (clamped) */
+#define QSVD_STATUS_POS_OOB 2       /* some pos[b] outside [0, max_len) (row not written) */
+#define QSVD_STATUS_SCALE_SAT 4     /* a group scale exceeded the fp16 range (saturated) */
+
+/* Split-kernel choice (qsvd_dims.kernel). */
+#define QSVD_KERNEL_AUTO 0
+#define QSVD_KERNEL_SIMT 1      /* CUDA-core split kernel: every dtype and mode */
+#define QSVD_KERNEL_TCGEN05 2   /* tensor-core split kernel (tcgen05, TMA) */
+
+typedef struct {
+  int E;               /* model width, E = H * d_h */
+  int H;               /* heads */
+  int d_h;             /* head dim (even; multiple of 8) */
+  int r;               /* retained rank (latent width; multiple of 32) */
+  int batch;           /* B sequences per call */
+  int max_len;         /* cache rows per sequence (capacity) */
+  int group;           /* channels per quantisation group (I8/I4 caches) */
+  int rope;            /* 0: no rotary embedding, query absorbed; 1: rotary */
+  float rope_base;     /* rotary base (e.g. 10000) */
+  float softmax_scale; /* score scale; <= 0 selects 1/sqrt(d_h) */
+  qsvd_dtype cache_dtype;   /* F32, F16, BF16, I8 or I4 */
+  qsvd_dtype weight_dtype;  /* F32, F16 or BF16: W^d, W^u_*, and append's x */
+  qsvd_dtype out_dtype;     /* F32, F16 or BF16 */
+  int h2;              /* 1: append applies H2 to the latent before quantising */
+  int h2_m;            /* order m of the small factor of H2 = H_{r/m} (x) Q_m */
+  int kernel;          /* QSVD_KERNEL_* */
+} qsvd_dims;
+
+/*
+ * qsvd_prepare_weights -- lay out the factors for the decode kernels.
+ * Source: QSVD paper notes, 关键设计 (shared W^d, separate W^u_q/k/v; the
+ * rotation identity Y = (X H1^T)(H1 W^d H2^T)(H2 W^u)); QSVD digest, Method,
+ * Step 3.
+ *   wd            device, E x r, weight_dtype: W^d.
+ *   wuq/wuk/wuv   device, r x E each, weight_dtype: W^u_q, W^u_k, W^u_v.
+ *   h2_q          HOST, h2_m x h2_m float32 row-major orthogonal matrix Q, or
+ *                 NULL.  When given, H2 = H_{r/h2_m} (x) Q (normalised
+ *                 Sylvester Hadamard; r/h2_m must be a power of two) is
+ *                 folded into the up-projections (W^u_* <- H2 W^u_*) and,
+ *                 unless dims->h2 == 1, into W^d (W^d <- W^d H2^T).  With
+ *                 dims->h2 == 1, W^d is kept and append rotates each latent.
+ *                 The fold runs in float32 and rounds once to weight_dtype.
+ *   packed        device buffer receiving the laid-out weights (owned by the
+ *                 caller, 256-byte aligned), or NULL to query the size.
+ *   packed_bytes  in: capacity of `packed`; out: bytes required.
+ * Rotary mode also stores a float32 cos/sin table for positions < max_len,
+ * built from float64 angles.  The packed buffer is read-only afterwards and
+ * may be shared by concurrent calls with the same dims.
+ * Errors: INVALID_ARG (dims, null inputs), WORKSPACE (capacity too small),
+ * CUDA (launch failure).
+ */
+qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd,
+                                 const void* wuq, const void* wuk,
+                                 const void* wuv, const float* h2_q,
+                                 void* packed, size_t* packed_bytes,
+                                 void* stream);
+
+/*
+ * qsvd_append_latent -- project one new token per sequence into the latent
+ * and write it into the cache.
+ * Source: QSVD digest, Method, Step 1 (C = X W^d is the buffered
+ * intermediate) and Step 3 (H2 rotation, latent quantisation); QSVD paper
+ * notes, 实验关键数据 (A8/A4 latent precisions).
+ *   x       device, B x E, weight_dtype: the new tokens' activations.
+ *   pos     device, B int32: row written for sequence b (0 <= pos < max_len).
+ *   cache   device, B x max_len rows; row layout by cache_dtype:
+ *             F32/F16/BF16: r elements;  I8: r int8 codes;
+ *             I4: r/2 bytes, element 2j in the low nibble, 2j+1 in the high
+ *             nibble (two's complement).
+ *   scales  device, B x max_len x (r/group) float16 (I8/I4 only; else NULL).
+ *   c_out   device, B x r float32, or NULL: receives c = x W^d (after H2
+ *           when dims->h2 == 1), i.e. the exact input of the quantiser.
+ *   status  device int32 word or NULL; bits QSVD_STATUS_* are OR-ed in.
+ *   workspace        device scratch (split-K partials of x W^d), or NULL to
+ *                    query the size into *workspace_bytes (in: capacity).
+ * Quantiser (I8/I4): per token and group of `group` channels,
+ *   scale = fp16_rn(amax / qmax) (IEEE float32 division; saturates at 65504
+ *   and sets QSVD_STATUS_SCALE_SAT), code = 0 if scale == 0 else
+ *   clamp(rint_half_even(c / scale), -qmax, qmax), qmax = 127 or 7.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed,
+                               const void* x, const int32_t* pos, void* cache,
+                               void* scales, float* c_out, int32_t* status,
+                               void* workspace, size_t* workspace_bytes,
+                               void* stream);
+
+/*
+ * qsvd_decode_attn -- one decode step of multi-head attention over the
+ * latent cache, output B x E.
+ * Source: QSVD digest, Method, Step 1 (keys/values rebuilt from C_qkv);
+ * WSVD digest, Method 3.4 (flash decoding over latent tiles, rotary keys).
+ *   qin            device, float32: B x r latent of the current token when
+ *                  qin_is_latent != 0 (q = qin W^u_q), else the B x E query.
+ *   cache, scales  as in qsvd_append_latent.
+ *   lengths        device, B int32: tokens attended by sequence b (rows
+ *                  0..len-1; the query sits at position len-1 for rotary).
+ *                  len == 0 gives a zero output row.  Values outside
+ *                  [0, max_len] are clamped and flagged.
+ *   num_splits     number of split CTAs G of the split phase (0: one wave on
+ *                  this device).  Tiles of 128 tokens are dealt to the G
+ *                  splits in equal contiguous runs over all sequences.
+ *   workspace      device scratch, or NULL to query the size into
+ *                  *workspace_bytes (in: capacity).  Layout (256-byte aligned
+ *                  sections): header (int32 status, G, tile, kernel), query
+ *                  buffers, then per split-partial slot s = split + b:
+ *                  m[s][H], l[s][H] (float32, log2 domain), z[s][H][r].
+ *   out            device, B x E, out_dtype.
+ *   phases         QSVD_PHASE_* mask (0 = all).  Running the phases as
+ *                  separate calls in order gives the same result.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed,
+                             const float* qin, int qin_is_latent,
+                             const void* cache, const void* scales,
+                             const int32_t* lengths, int num_splits,
+                             void* workspace, size_t* workspace_bytes,
+                             void* out, unsigned phases, void* stream);
+
+/*
+ * qsvd_combine_splits -- merge the split partials held in `workspace`
+ * (written by the split phase of qsvd_decode_attn with the same dims,
+ * lengths and num_splits) and apply the value up-projection: with M = max_s m_s,
+ * w_s = 2^(m_s - M):  z = sum_s w_s z_s / sum_s w_s l_s,  o_h = z_h W^u_{v,h}.
+ * Source: WSVD digest, Method 3.4 (flash decoding); QSVD digest, Step 1.
+ * Equivalent to qsvd_decode_attn with phases = QSVD_PHASE_COMBINE.
+ * Errors: INVALID_ARG, CUDA.
+ */
+qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
+                                void* workspace, int num_splits,
+                                const int32_t* lengths, void* out, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* qsvd_status_string(qsvd_status s);
+
+/* Message describing the last failing call on this host thread. */
+const char* qsvd_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t qsvd_kernel_launches(void);
+
+/* QSVD_ABI_VERSION of the loaded library. */
+int qsvd_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSVD_H */

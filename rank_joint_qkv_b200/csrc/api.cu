@@ -1,0 +1,280 @@
+// C-ABI layer: argument validation, layouts, phase dispatch.
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.cuh"
+
+namespace qsvd {
+
+static std::atomic<uint64_t> g_launches{0};
+static thread_local char g_err[512] = "";
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+cudaError_t check_launch() { return cudaGetLastError(); }
+
+static qsvd_status fail(qsvd_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+static qsvd_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(QSVD_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host-checkable constraints shared by all calls.
+static qsvd_status validate(const qsvd_dims* d) {
+  if (!d) return fail(QSVD_ERR_INVALID_ARG, "dims is NULL");
+  if (d->H <= 0 || d->d_h <= 0 || d->E != d->H * d->d_h)
+    return fail(QSVD_ERR_INVALID_ARG, "E (%d) must equal H (%d) * d_h (%d)", d->E, d->H, d->d_h);
+  if (d->E % 64) return fail(QSVD_ERR_INVALID_ARG, "E (%d) must be a multiple of 64", d->E);
+  if (d->d_h % 8 || d->d_h > 256)
+    return fail(QSVD_ERR_INVALID_ARG, "d_h (%d) must be a multiple of 8, at most 256", d->d_h);
+  if (d->r < 32 || d->r % 32 || d->r > 8192)
+    return fail(QSVD_ERR_INVALID_ARG, "r (%d) must be a multiple of 32 in [32, 8192]", d->r);
+  if (d->batch < 1) return fail(QSVD_ERR_INVALID_ARG, "batch must be >= 1");
+  if (d->max_len < 1) return fail(QSVD_ERR_INVALID_ARG, "max_len must be >= 1");
+  if (d->cache_dtype < QSVD_F32 || d->cache_dtype > QSVD_I4)
+    return fail(QSVD_ERR_INVALID_ARG, "unknown cache dtype %d", int(d->cache_dtype));
+  if (d->weight_dtype < QSVD_F32 || d->weight_dtype > QSVD_BF16)
+    return fail(QSVD_ERR_INVALID_ARG, "weight dtype must be F32, F16 or BF16");
+  if (d->out_dtype < QSVD_F32 || d->out_dtype > QSVD_BF16)
+    return fail(QSVD_ERR_INVALID_ARG, "out dtype must be F32, F16 or BF16");
+  if (cache_is_int(*d)) {
+    if (d->group < 32 || d->group % 32 || d->r % d->group)
+      return fail(QSVD_ERR_INVALID_ARG, "group (%d) must be a multiple of 32 dividing r (%d)",
+                  d->group, d->r);
+  }
+  if (d->rope) {
+    if (!(d->rope_base > 0.f)) return fail(QSVD_ERR_INVALID_ARG, "rope_base must be > 0");
+    if (d->d_h % 64) return fail(QSVD_ERR_UNSUPPORTED, "rotary mode needs d_h %% 64 == 0");
+  }
+  if (d->h2) {
+    if (d->h2_m < 1 || d->h2_m > 16 || d->r % d->h2_m || !is_pow2(d->r / d->h2_m))
+      return fail(QSVD_ERR_INVALID_ARG, "H2 needs r/h2_m a power of two, 1 <= h2_m <= 16");
+  }
+  if (d->kernel < QSVD_KERNEL_AUTO || d->kernel > QSVD_KERNEL_TCGEN05)
+    return fail(QSVD_ERR_INVALID_ARG, "unknown kernel choice %d", d->kernel);
+  return QSVD_OK;
+}
+
+static int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+// Split kernel actually used for these dims.
+static int pick_kernel(const qsvd_dims& d) {
+  if (d.kernel == QSVD_KERNEL_SIMT) return QSVD_KERNEL_SIMT;
+  if (d.kernel == QSVD_KERNEL_TCGEN05) return QSVD_KERNEL_TCGEN05;
+  return QSVD_KERNEL_SIMT;
+}
+
+static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel, int* G) {
+  const long long max_tiles = (long long)d.batch * ((d.max_len + kTile - 1) / kTile);
+  long long g = num_splits;
+  if (num_splits < 0) return fail(QSVD_ERR_INVALID_ARG, "num_splits must be >= 0");
+  if (g == 0) {
+    const int sms = device_sms();
+    if (sms <= 0) return fail(QSVD_ERR_CUDA, "no CUDA device to size the split grid");
+    if (kernel == QSVD_KERNEL_TCGEN05) {
+      g = sms;
+    } else {
+      const int hb = split_simt_grid_heads(d);
+      g = hb > 0 ? (2LL * sms + hb - 1) / hb : sms;
+    }
+  }
+  if (g > max_tiles) g = max_tiles;
+  if (g < 1) g = 1;
+  if (g > (1 << 20)) return fail(QSVD_ERR_INVALID_ARG, "num_splits too large");
+  *G = int(g);
+  return QSVD_OK;
+}
+
+static float score_scale_log2(const qsvd_dims& d) {
+  const double tau = d.softmax_scale > 0.f ? double(d.softmax_scale) : 1.0 / std::sqrt(double(d.d_h));
+  return float(tau * 1.4426950408889634);
+}
+
+}  // namespace qsvd
+
+using namespace qsvd;
+
+extern "C" {
+
+const char* qsvd_status_string(qsvd_status s) {
+  switch (s) {
+    case QSVD_OK: return "QSVD_OK";
+    case QSVD_ERR_INVALID_ARG: return "QSVD_ERR_INVALID_ARG";
+    case QSVD_ERR_UNSUPPORTED: return "QSVD_ERR_UNSUPPORTED";
+    case QSVD_ERR_WORKSPACE: return "QSVD_ERR_WORKSPACE";
+    case QSVD_ERR_CUDA: return "QSVD_ERR_CUDA";
+  }
+  return "QSVD_UNKNOWN_STATUS";
+}
+
+const char* qsvd_last_error(void) { return g_err; }
+
+uint64_t qsvd_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int qsvd_abi_version(void) { return QSVD_ABI_VERSION; }
+
+qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd, const void* wuq,
+                                 const void* wuk, const void* wuv, const float* h2_q,
+                                 void* packed, size_t* packed_bytes, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  if (!packed_bytes) return fail(QSVD_ERR_INVALID_ARG, "packed_bytes is NULL");
+  const qsvd_dims& d = *dims;
+  if (h2_q && (d.h2_m < 1 || d.h2_m > 16 || d.r % d.h2_m || !is_pow2(d.r / d.h2_m)))
+    return fail(QSVD_ERR_INVALID_ARG, "H2 needs r/h2_m a power of two, 1 <= h2_m <= 16");
+  const PackedLayout L = packed_layout(d);
+  if (!packed) { *packed_bytes = L.total; return QSVD_OK; }
+  if (d.h2 && !h2_q) return fail(QSVD_ERR_INVALID_ARG, "dims->h2 = 1 needs h2_q");
+  if (*packed_bytes < L.total)
+    return fail(QSVD_ERR_WORKSPACE, "packed buffer holds %zu bytes, %zu needed", *packed_bytes, L.total);
+  if (!wd || !wuq || !wuk || !wuv) return fail(QSVD_ERR_INVALID_ARG, "a weight pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(packed) & 255u) != 0)
+    return fail(QSVD_ERR_INVALID_ARG, "packed must be 256-byte aligned");
+  *packed_bytes = L.total;
+  cudaError_t e = launch_prepare(d, wd, wuq, wuk, wuv, h2_q, packed, L,
+                                 static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prepare_weights");
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed, const void* x,
+                               const int32_t* pos, void* cache, void* scales, float* c_out,
+                               int32_t* status, void* workspace, size_t* workspace_bytes,
+                               void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  const int KS = append_ksplit(d);
+  const size_t need = align256(size_t(KS) * d.batch * d.r * 4);
+  if (!workspace) { *workspace_bytes = need; return QSVD_OK; }
+  if (*workspace_bytes < need)
+    return fail(QSVD_ERR_WORKSPACE, "append workspace holds %zu bytes, %zu needed", *workspace_bytes, need);
+  if (!packed || !x || !pos || !cache) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (cache_is_int(d) && !scales) return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
+  if (!aligned16(x) || !aligned16(cache) || !aligned16(workspace))
+    return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const PackedLayout L = packed_layout(d);
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  const float h2_scale = d.h2 ? float(1.0 / std::sqrt(double(d.r / d.h2_m))) : 1.f;
+  cudaError_t e = launch_append(d, x, P + L.wd, reinterpret_cast<const float*>(P + L.h2q), h2_scale,
+                                pos, cache, scales, c_out, static_cast<float*>(workspace), KS,
+                                status, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append_latent");
+  return QSVD_OK;
+}
+
+static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const float* qin,
+                               int qin_is_latent, const void* cache, const void* scales,
+                               const int32_t* lengths, int num_splits, void* workspace,
+                               size_t* workspace_bytes, void* out, unsigned phases,
+                               cudaStream_t s) {
+  if (phases == 0) phases = QSVD_PHASE_ALL;
+  if (phases & ~QSVD_PHASE_ALL) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
+  const int kernel = pick_kernel(d);
+  if (kernel == QSVD_KERNEL_TCGEN05)
+    return fail(QSVD_ERR_UNSUPPORTED, "tensor-core split kernel not available for these dims");
+  if (!d.rope && split_simt_grid_heads(d) == 0)
+    return fail(QSVD_ERR_UNSUPPORTED, "rank too large for the CUDA-core split kernel");
+  int G = 0;
+  qsvd_status st = resolve_splits(d, num_splits, kernel, &G);
+  if (st != QSVD_OK) return st;
+  const WsLayout W = ws_layout(d, G);
+  if (!workspace) { *workspace_bytes = W.total; return QSVD_OK; }
+  if (*workspace_bytes < W.total)
+    return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, W.total);
+  if (!packed || !lengths) return fail(QSVD_ERR_INVALID_ARG, "packed/lengths is NULL");
+  if ((phases & QSVD_PHASE_PROLOGUE) && !qin) return fail(QSVD_ERR_INVALID_ARG, "qin is NULL");
+  if ((phases & QSVD_PHASE_SPLIT) && !cache) return fail(QSVD_ERR_INVALID_ARG, "cache is NULL");
+  if ((phases & QSVD_PHASE_SPLIT) && cache_is_int(d) && !scales)
+    return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
+  if ((phases & QSVD_PHASE_COMBINE) && !out) return fail(QSVD_ERR_INVALID_ARG, "out is NULL");
+  if (!aligned16(workspace) || (cache && !aligned16(cache)) || (qin && !aligned16(qin)))
+    return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+
+  const PackedLayout L = packed_layout(d);
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  uint8_t* Wb = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(Wb + W.hdr);
+  int32_t* sched = reinterpret_cast<int32_t*>(Wb + W.sched);
+  float* q = reinterpret_cast<float*>(Wb + W.q);
+  float* qt32 = reinterpret_cast<float*>(Wb + W.qt32);
+  void* qt16 = Wb + W.qt16;
+  float* qpart = reinterpret_cast<float*>(Wb + W.qpart);
+  float* pm = reinterpret_cast<float*>(Wb + W.pm);
+  float* pl = reinterpret_cast<float*>(Wb + W.pl);
+  float* pz = reinterpret_cast<float*>(Wb + W.pz);
+  float* opart = reinterpret_cast<float*>(Wb + W.opart);
+  const float* rope_tab = reinterpret_cast<const float*>(P + L.rope);
+  const float sl2 = score_scale_log2(d);
+  cudaError_t e;
+
+  if (phases & QSVD_PHASE_PROLOGUE) {
+    if ((e = launch_schedule(d, lengths, G, sched, hdr, kernel, s)) != cudaSuccess)
+      return cuda_fail(e, "schedule");
+    const float* q_given = qin_is_latent ? nullptr : qin;
+    if (qin_is_latent) {
+      if ((e = launch_q_partial(d, qin, P + L.wuq, qpart, W.KS, s)) != cudaSuccess)
+        return cuda_fail(e, "query projection");
+    }
+    if (d.rope)
+      e = launch_rope_query(d, qpart, W.KS, q_given, sched, rope_tab, sl2, q, s);
+    else
+      e = launch_absorb(d, qpart, W.KS, q_given, P + L.wuk, sl2, qt32, qt16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "query prologue");
+  }
+  if (phases & QSVD_PHASE_SPLIT) {
+    if (d.rope)
+      e = launch_split_simt_rope(d, q, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
+    else
+      e = launch_split_simt_absorbed(d, qt32, cache, scales, sched, G, pm, pl, pz, s);
+    if (e != cudaSuccess) return cuda_fail(e, "split phase");
+  }
+  if (phases & QSVD_PHASE_COMBINE) {
+    if ((e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, out, s)) != cudaSuccess)
+      return cuda_fail(e, "combine phase");
+  }
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed, const float* qin,
+                             int qin_is_latent, const void* cache, const void* scales,
+                             const int32_t* lengths, int num_splits, void* workspace,
+                             size_t* workspace_bytes, void* out, unsigned phases, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  return decode_impl(*dims, packed, qin, qin_is_latent, cache, scales, lengths, num_splits,
+                     workspace, workspace_bytes, out, phases, static_cast<cudaStream_t>(stream));
+}
+
+qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed, void* workspace,
+                                int num_splits, const int32_t* lengths, void* out,
+                                void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  if (!packed || !workspace || !lengths || !out)
+    return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  size_t cap = ~size_t(0);
+  return decode_impl(*dims, packed, nullptr, 1, nullptr, nullptr, lengths, num_splits, workspace,
+                     &cap, out, QSVD_PHASE_COMBINE, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,274 @@
+// Internal declarations of the joint-QKV latent decode library (sm_100a).
+//
+// Shared by the C-ABI layer (api.cu) and the kernel files.  Nothing here is
+// part of the public interface (include/qsvd.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/qsvd.h"
+
+namespace qsvd {
+
+constexpr int kTile = QSVD_TILE_TOKENS;   // tokens per split-KV tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- layouts
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline size_t dtype_bytes(qsvd_dtype t) {
+  switch (t) {
+    case QSVD_F32: return 4;
+    case QSVD_F16: case QSVD_BF16: return 2;
+    default: return 1;
+  }
+}
+
+// Bytes of one cache row (without scales).
+inline size_t cache_row_bytes(const qsvd_dims& d) {
+  switch (d.cache_dtype) {
+    case QSVD_F32: return size_t(d.r) * 4;
+    case QSVD_F16: case QSVD_BF16: return size_t(d.r) * 2;
+    case QSVD_I8: return size_t(d.r);
+    case QSVD_I4: return size_t(d.r) / 2;
+  }
+  return 0;
+}
+
+inline bool cache_is_int(const qsvd_dims& d) {
+  return d.cache_dtype == QSVD_I8 || d.cache_dtype == QSVD_I4;
+}
+
+// Packed weights: one device buffer, 256-byte aligned sections.
+struct PackedLayout {
+  size_t wd, wuq, wuk, wuv;   // native layouts: W^d E x r, W^u_* r x E
+  size_t wukT;                // W^u_k transposed, E x r (rotary tensor-core path)
+  size_t h2q;                 // h2_m x h2_m float32 (online H2 in append)
+  size_t rope;                // max_len x (d_h/2) x {cos, sin} float32
+  size_t total;
+};
+
+inline PackedLayout packed_layout(const qsvd_dims& d) {
+  PackedLayout p{};
+  const size_t wb = dtype_bytes(d.weight_dtype);
+  const size_t mat = size_t(d.E) * d.r * wb;
+  size_t o = 256;  // reserved header
+  p.wd = o;  o = align256(o + mat);
+  p.wuq = o; o = align256(o + mat);
+  p.wuk = o; o = align256(o + mat);
+  p.wuv = o; o = align256(o + mat);
+  p.wukT = o; if (d.rope) o = align256(o + mat);
+  p.h2q = o; o = align256(o + size_t(16) * 16 * 4);
+  p.rope = o; if (d.rope) o = align256(o + size_t(d.max_len) * (d.d_h / 2) * 2 * 4);
+  p.total = o;
+  return p;
+}
+
+// Workspace of qsvd_decode_attn.
+struct WsHeader {
+  int32_t status;
+  int32_t G;       // split CTAs of the split phase
+  int32_t tile;    // tokens per tile
+  int32_t kernel;  // split kernel used
+};
+
+struct WsLayout {
+  size_t hdr, sched, q, qt32, qt16, qpart, pm, pl, pz, opart, total;
+  int G, P, KS, JS;
+};
+
+// Split-K factor of the query projection and j-splits of the combine.
+inline int prologue_ksplit(const qsvd_dims& d) {
+  int ks = d.r / 128;
+  if (ks < 1) ks = 1;
+  if (ks > 4) ks = 4;
+  while (d.r % (ks * 32)) --ks;
+  return ks;
+}
+inline int combine_jsplit(const qsvd_dims& d) { return (d.r + 255) / 256; }
+
+inline WsLayout ws_layout(const qsvd_dims& d, int G) {
+  WsLayout w{};
+  w.G = G;
+  w.P = G + d.batch;
+  w.KS = prologue_ksplit(d);
+  w.JS = combine_jsplit(d);
+  const size_t B = d.batch, E = d.E, H = d.H, r = d.r;
+  size_t o = 0;
+  w.hdr = o;   o = align256(o + sizeof(WsHeader));
+  w.sched = o; o = align256(o + (2 * B + 1) * 4);
+  w.q = o;     o = align256(o + B * E * 4);
+  w.qt32 = o;  o = align256(o + B * H * r * 4);
+  w.qt16 = o;  o = align256(o + B * H * r * 2);
+  w.qpart = o; o = align256(o + size_t(w.KS) * B * E * 4);
+  w.pm = o;    o = align256(o + size_t(w.P) * H * 4);
+  w.pl = o;    o = align256(o + size_t(w.P) * H * 4);
+  w.pz = o;    o = align256(o + size_t(w.P) * H * r * 4);
+  w.opart = o; o = align256(o + size_t(w.JS) * B * E * 4);
+  w.total = o;
+  return w;
+}
+
+// -------------------------------------------------------- launch bookkeeping
+
+void note_launch();                 // counts kernels launched by this library
+cudaError_t check_launch();         // cudaGetLastError after a launch
+
+// ------------------------------------------------------------ kernel entry
+
+// Prologue (query side).
+cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
+                            WsHeader* hdr, int kernel, cudaStream_t s);
+cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
+                             float* qpart, int KS, cudaStream_t s);
+cudaError_t launch_absorb(const qsvd_dims& d, const float* qpart, int KS,
+                          const float* q_given, const void* wuk, float scale_log2,
+                          float* qt32, void* qt16, cudaStream_t s);
+cudaError_t launch_rope_query(const qsvd_dims& d, const float* qpart, int KS,
+                              const float* q_given, const int32_t* sched,
+                              const float* rope_tab, float scale_log2,
+                              float* qrot, cudaStream_t s);
+
+// Split phase.
+cudaError_t launch_split_simt_absorbed(const qsvd_dims& d, const float* qt32,
+                                       const void* cache, const void* scales,
+                                       const int32_t* sched, int G, float* pm,
+                                       float* pl, float* pz, cudaStream_t s);
+cudaError_t launch_split_simt_rope(const qsvd_dims& d, const float* qrot,
+                                   const void* wuk, const float* rope_tab,
+                                   const void* cache, const void* scales,
+                                   const int32_t* sched, int G, float* pm,
+                                   float* pl, float* pz, cudaStream_t s);
+int split_simt_grid_heads(const qsvd_dims& d);   // head blocks per split
+
+// Combine phase.
+cudaError_t launch_combine(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
+                           const float* pm, const float* pl, const float* pz,
+                           const void* wuv, float* opart, int JS, void* out,
+                           cudaStream_t s);
+
+// Append.
+int append_ksplit(const qsvd_dims& d);
+cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
+                          const float* h2q, float h2_scale, const int32_t* pos,
+                          void* cache, void* scales, float* c_out, float* cpart,
+                          int KS, int32_t* status, cudaStream_t s);
+
+// Prepare.
+cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
+                           const void* wuk, const void* wuv, const float* h2q_host,
+                           void* packed, const PackedLayout& L, cudaStream_t s);
+
+}  // namespace qsvd
+
+// ------------------------------------------------------------ device helpers
+
+namespace qsvd {
+namespace dev {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Number of tiles of a sequence of n tokens.
+__device__ __forceinline__ int tiles_of(int n) { return (n + kTile - 1) / kTile; }
+
+// Clamp a device length into [0, max_len]; flag out-of-range values.
+__device__ __forceinline__ int clamp_len(int n, int max_len, int32_t* status) {
+  if (n < 0 || n > max_len) {
+    if (status) atomicOr(status, QSVD_STATUS_LEN_CLAMPED);
+    n = n < 0 ? 0 : max_len;
+  }
+  return n;
+}
+
+// Split c of G covers global tiles [split_begin(c), split_begin(c + 1)).
+__device__ __forceinline__ long long split_begin(long long c, long long G, long long T) {
+  return (c * T) / G;
+}
+// The split whose range contains global tile t.
+__device__ __forceinline__ long long split_of_tile(long long t, long long G, long long T) {
+  return ((t + 1) * G - 1) / T;
+}
+
+// Sixteen bytes of a cache row converted to float.  Element index j0 is the
+// first of the vector; `scale` is the group scale for int caches.
+template <qsvd_dtype CT> struct CacheVec;
+
+template <> struct CacheVec<QSVD_F32> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const uint8_t* row, int j0, float s, float* o) {
+    float4 v = *reinterpret_cast<const float4*>(row + size_t(j0) * 4);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  }
+};
+template <> struct CacheVec<QSVD_F16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const uint8_t* row, int j0, float s, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + size_t(j0) * 2);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __half22float2(h[i]); o[2 * i] = f.x; o[2 * i + 1] = f.y; }
+  }
+};
+template <> struct CacheVec<QSVD_BF16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const uint8_t* row, int j0, float s, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + size_t(j0) * 2);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __bfloat1622float2(h[i]); o[2 * i] = f.x; o[2 * i + 1] = f.y; }
+  }
+};
+template <> struct CacheVec<QSVD_I8> {
+  static constexpr int N = 16;
+  __device__ __forceinline__ static void load(const uint8_t* row, int j0, float s, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + size_t(j0));
+    const int8_t* c = reinterpret_cast<const int8_t*>(&v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = float(c[i]) * s;
+  }
+};
+template <> struct CacheVec<QSVD_I4> {
+  static constexpr int N = 32;
+  __device__ __forceinline__ static void load(const uint8_t* row, int j0, float s, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + size_t(j0) / 2);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // nibble i of word k is element 8k + i (low nibble first)
+        int q = int((w[k] >> (4 * i)) & 0xFu);
+        q = (q ^ 8) - 8;  // sign-extend 4-bit two's complement
+        o[8 * k + i] = float(q) * s;
+      }
+    }
+  }
+};
+
+}  // namespace dev
+}  // namespace qsvd

@@ -1,0 +1,168 @@
+// Weight preparation (one-off per model layer).
+//
+// Copies the joint-SVD factors into one packed device buffer, optionally
+// folds the rotation H2 = H_n (x) Q_m into them (QSVD paper notes, 关键设计:
+// Y = (X H1^T)(H1 W^d H2^T)(H2 W^u)), stores W^u_k transposed for the rotary
+// tensor-core kernel and a float32 cos/sin table whose angles are formed in
+// float64 (positions up to 32k lose ~2^-9 rad if formed in float32).
+#include <cmath>
+
+#include "internal.cuh"
+
+namespace qsvd {
+namespace {
+
+// Apply H2 to NV vectors of length r stored with element stride es and
+// vector stride vs: v <- H2 v.  grid ceil(nvec/NV), block 256.
+template <typename WT>
+__global__ void __launch_bounds__(256)
+k_h2_fold(WT* __restrict__ base, int nvec, size_t es, size_t vs, int r, int m,
+          const float* __restrict__ q, float scale) {
+  constexpr int NV = 4;
+  extern __shared__ float v[];   // NV x r
+  __shared__ float qm[256];
+  const int v0 = blockIdx.x * NV;
+  const int nv = min(NV, nvec - v0);
+  for (int i = threadIdx.x; i < m * m; i += 256) qm[i] = q[i];
+  for (int i = threadIdx.x; i < NV * r; i += 256) {
+    const int k = i / r, j = i % r;
+    v[i] = k < nv ? dev::to_f(base[size_t(v0 + k) * vs + size_t(j) * es]) : 0.f;
+  }
+  __syncthreads();
+  const int n = r / m;
+  for (int len = 1; len < n; len <<= 1) {
+    for (int idx = threadIdx.x; idx < NV * (n / 2) * m; idx += 256) {
+      const int k = idx / ((n / 2) * m), rem = idx % ((n / 2) * m);
+      const int beta = rem % m, p = rem / m;
+      const int a0 = (p / len) * 2 * len + (p % len);
+      float* vk = v + k * r;
+      const int i0 = a0 * m + beta, i1 = (a0 + len) * m + beta;
+      const float u = vk[i0], w = vk[i1];
+      vk[i0] = u + w;
+      vk[i1] = u - w;
+    }
+    __syncthreads();
+  }
+  for (int idx = threadIdx.x; idx < NV * n; idx += 256) {
+    const int k = idx / n, a = idx % n;
+    float* vk = v + k * r;
+    float x[16], y[16];
+    for (int b = 0; b < m; ++b) x[b] = vk[a * m + b] * scale;
+    for (int b = 0; b < m; ++b) {
+      float s = 0.f;
+      for (int bb = 0; bb < m; ++bb) s = fmaf(qm[b * m + bb], x[bb], s);
+      y[b] = s;
+    }
+    for (int b = 0; b < m; ++b) vk[a * m + b] = y[b];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < NV * r; i += 256) {
+    const int k = i / r, j = i % r;
+    if (k < nv) base[size_t(v0 + k) * vs + size_t(j) * es] = dev::from_f<WT>(v[i]);
+  }
+}
+
+// dst[e][j] = src[j][e]  (src r x E)
+template <typename WT>
+__global__ void k_transpose(const WT* __restrict__ src, WT* __restrict__ dst, int r, int E) {
+  __shared__ WT t[32][33];
+  const int e0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int j = j0 + i, e = e0 + threadIdx.x;
+    if (j < r && e < E) t[i][threadIdx.x] = src[size_t(j) * E + e];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int e = e0 + i, j = j0 + threadIdx.x;
+    if (j < r && e < E) dst[size_t(e) * r + j] = t[threadIdx.x][i];
+  }
+}
+
+// tab[pos][i] = {cos, sin}(pos * base^(-2i/d_h)), angles in float64.
+__global__ void k_rope_table(float* __restrict__ tab, int max_len, int half, double log_base,
+                             int d_h) {
+  const size_t n = size_t(max_len) * half;
+  for (size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < n;
+       idx += size_t(gridDim.x) * blockDim.x) {
+    const int pos = int(idx / half), i = int(idx % half);
+    const double theta = exp(-(2.0 * i / d_h) * log_base);
+    double s, c;
+    sincos(double(pos) * theta, &s, &c);
+    tab[idx * 2 + 0] = float(c);
+    tab[idx * 2 + 1] = float(s);
+  }
+}
+
+template <typename WT>
+cudaError_t fold_t(WT* base, int nvec, size_t es, size_t vs, int r, int m, const float* q,
+                   float scale, cudaStream_t s) {
+  const size_t smem = size_t(4) * r * 4;
+  auto kern = k_h2_fold<WT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<(nvec + 3) / 4, 256, smem, s>>>(base, nvec, es, vs, r, m, q, scale);
+  note_launch();
+  return check_launch();
+}
+
+template <typename WT>
+cudaError_t prepare_t(const qsvd_dims& d, const float* h2q_host, uint8_t* P,
+                      const PackedLayout& L, cudaStream_t s) {
+  cudaError_t e;
+  WT* wd = reinterpret_cast<WT*>(P + L.wd);
+  WT* wu[3] = {reinterpret_cast<WT*>(P + L.wuq), reinterpret_cast<WT*>(P + L.wuk),
+               reinterpret_cast<WT*>(P + L.wuv)};
+  float* q = reinterpret_cast<float*>(P + L.h2q);
+  if (h2q_host) {
+    const int m = d.h2_m;
+    e = cudaMemcpyAsync(q, h2q_host, size_t(m) * m * 4, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    const double n = double(d.r / m);
+    const float scale = float(1.0 / std::sqrt(n));
+    for (int k = 0; k < 3; ++k) {   // W^u_* <- H2 W^u_*: columns are vectors
+      e = fold_t<WT>(wu[k], d.E, size_t(d.E), 1, d.r, m, q, scale, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (!d.h2) {                     // W^d <- W^d H2^T: rows are vectors
+      e = fold_t<WT>(wd, d.E, 1, size_t(d.r), d.r, m, q, scale, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  if (d.rope) {
+    dim3 grid((d.E + 31) / 32, (d.r + 31) / 32);
+    k_transpose<WT><<<grid, dim3(32, 8), 0, s>>>(wu[1], reinterpret_cast<WT*>(P + L.wukT), d.r, d.E);
+    note_launch();
+    if ((e = check_launch()) != cudaSuccess) return e;
+    const int half = d.d_h / 2;
+    const size_t n = size_t(d.max_len) * half;
+    const unsigned blocks = unsigned(std::min<size_t>((n + 255) / 256, 4096));
+    k_rope_table<<<blocks, 256, 0, s>>>(reinterpret_cast<float*>(P + L.rope), d.max_len, half,
+                                        std::log(double(d.rope_base)), d.d_h);
+    note_launch();
+    if ((e = check_launch()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
+                           const void* wuk, const void* wuv, const float* h2q_host,
+                           void* packed, const PackedLayout& L, cudaStream_t s) {
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  const size_t mat = size_t(d.E) * d.r * dtype_bytes(d.weight_dtype);
+  const void* src[4] = {wd, wuq, wuk, wuv};
+  const size_t off[4] = {L.wd, L.wuq, L.wuk, L.wuv};
+  for (int k = 0; k < 4; ++k) {
+    cudaError_t e = cudaMemcpyAsync(P + off[k], src[k], mat, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return e;
+  }
+  switch (d.weight_dtype) {
+    case QSVD_F32: return prepare_t<float>(d, h2q_host, P, L, s);
+    case QSVD_F16: return prepare_t<__half>(d, h2q_host, P, L, s);
+    case QSVD_BF16: return prepare_t<__nv_bfloat16>(d, h2q_host, P, L, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qsvd

@@ -1,0 +1,234 @@
+// Prologue of a decode step: the query side.
+//
+//   q   = c_new W^u_q                      (QSVD digest, Method, Step 1: Q is
+//                                            rebuilt from the shared latent)
+//   qt_h = (tau * log2 e) W^u_{k,h} q_h    (no rotary embedding: the query is
+//                                            absorbed into latent space so the
+//                                            scores are C qt_h)
+//   q_h <- (tau * log2 e) R(len-1) q_h     (rotary mode: WSVD digest, Method
+//                                            3.4, rotary keys; the query is
+//                                            rotated at its own position)
+//
+// These read W^u_q and W^u_k once per step (batched GEMVs, HBM-bound on the
+// weights) and are small next to the split phase.
+#include "internal.cuh"
+#include "gemv.cuh"
+
+namespace qsvd {
+namespace {
+
+using dev::to_f;
+
+// Query of sequence b, head h, dim d: sum of the split partials (or given).
+__device__ __forceinline__ float query_at(const float* qpart, int KS, const float* q_given,
+                                          int B, int E, int b, int e) {
+  if (q_given) return q_given[size_t(b) * E + e];
+  float s = 0.f;
+  for (int k = 0; k < KS; ++k) s += qpart[(size_t(k) * B + b) * E + e];
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// qt[b][h][j] = scale * sum_d W^u_k[j][h*d_h + d] * q[b][h*d_h + d]
+// grid (H, ceil(r/128)), block 128.  A thread computes 4 rows x 4 sequences.
+// ---------------------------------------------------------------------------
+template <typename WT, typename QT16>
+__global__ void __launch_bounds__(128)
+k_absorb(const float* __restrict__ qpart, int KS, const float* __restrict__ q_given,
+         const WT* __restrict__ W, float scale, float* __restrict__ qt32,
+         QT16* __restrict__ qt16, int B, int H, int d_h, int r, int E) {
+  extern __shared__ float sm[];
+  const int h = blockIdx.x;
+  const int j0 = blockIdx.y * 128;
+  const int jn = min(128, r - j0);
+  const int ld = d_h + 4;                  // padded row stride (floats)
+  float* ws = sm;                          // [128][ld]
+  float* qs = sm + 128 * ld;               // [32][ld]
+  // stage the W^u_k tile (rows j0.., columns of head h) as float
+  for (int i = threadIdx.x; i < 128 * d_h; i += 128) {
+    const int jr = i / d_h, d = i % d_h;
+    ws[jr * ld + d] = jr < jn ? to_f(W[size_t(j0 + jr) * E + h * d_h + d]) : 0.f;
+  }
+  const int tr = threadIdx.x / 4;    // rows tr + 32a, a < 4 (conflict-free float4 reads)
+  const int tb = threadIdx.x % 4;    // sequences b0 + tb + 4c, c < 4
+  for (int b0 = 0; b0 < B; b0 += 16) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 16 * d_h; i += 128) {
+      const int bb = i / d_h, d = i % d_h;
+      qs[bb * ld + d] = (b0 + bb < B) ? query_at(qpart, KS, q_given, B, E, b0 + bb, h * d_h + d) : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+    for (int d = 0; d < d_h; d += 4) {
+      float4 wv[4], qv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) wv[a] = *reinterpret_cast<const float4*>(&ws[(tr + 32 * a) * ld + d]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) qv[c] = *reinterpret_cast<const float4*>(&qs[(tb + 4 * c) * ld + d]);
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[a][c] = fmaf(wv[a].x, qv[c].x, acc[a][c]);
+          acc[a][c] = fmaf(wv[a].y, qv[c].y, acc[a][c]);
+          acc[a][c] = fmaf(wv[a].z, qv[c].z, acc[a][c]);
+          acc[a][c] = fmaf(wv[a].w, qv[c].w, acc[a][c]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = j0 + tr + 32 * a, b = b0 + tb + 4 * c;
+        if (j - j0 < jn && b < B) {
+          const float v = acc[a][c] * scale;
+          const size_t o = (size_t(b) * H + h) * r + j;
+          qt32[o] = v;
+          qt16[o] = dev::from_f<QT16>(v);
+        }
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Rotary query: q_h <- scale * R(len_b - 1) q_h, pairs (i, i + d_h/2).
+// grid (B), block 256.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_rope_query(const float* __restrict__ qpart, int KS, const float* __restrict__ q_given,
+             const int32_t* __restrict__ sched, const float* __restrict__ tab,
+             float scale, float* __restrict__ qrot, int B, int H, int d_h, int E) {
+  const int b = blockIdx.x;
+  const int n = sched[B + 1 + b];
+  const int pos = n > 0 ? n - 1 : 0;
+  const int half = d_h / 2;
+  for (int i = threadIdx.x; i < H * half; i += blockDim.x) {
+    const int h = i / half, k = i % half;
+    const int e0 = h * d_h + k, e1 = e0 + half;
+    const float a = query_at(qpart, KS, q_given, B, E, b, e0);
+    const float c = query_at(qpart, KS, q_given, B, E, b, e1);
+    const float cs = tab[(size_t(pos) * half + k) * 2 + 0];
+    const float sn = tab[(size_t(pos) * half + k) * 2 + 1];
+    qrot[size_t(b) * E + e0] = (a * cs - c * sn) * scale;
+    qrot[size_t(b) * E + e1] = (c * cs + a * sn) * scale;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV schedule: clamped lengths and the tile prefix over sequences.
+// sched[0..B] = tiles before sequence b (sched[B] = total), sched[B+1+b] = len.
+// grid 1, block 1024.  Also records G in the workspace header.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
+           int32_t* __restrict__ sched, WsHeader* hdr, int kernel) {
+  __shared__ int32_t part[1024];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    hdr->status = 0;   // reset before any thread flags a clamped length
+    hdr->G = G;
+    hdr->tile = kTile;
+    hdr->kernel = kernel;
+  }
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += 1024) {
+    const int b = b0 + threadIdx.x;
+    int nt = 0;
+    if (b < B) {
+      const int n = dev::clamp_len(lengths[b], max_len, &hdr->status);
+      sched[B + 1 + b] = n;
+      nt = dev::tiles_of(n);
+    }
+    part[threadIdx.x] = nt;
+    __syncthreads();
+    // inclusive Hillis-Steele scan
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int v = threadIdx.x >= o ? part[threadIdx.x - o] : 0;
+      __syncthreads();
+      part[threadIdx.x] += v;
+      __syncthreads();
+    }
+    if (b < B) sched[b + 1] = carry + part[threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += part[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) sched[0] = 0;
+}
+
+template <typename WT>
+cudaError_t q_partial_t(const qsvd_dims& d, const float* qin, const void* wuq, float* qpart,
+                        int KS, cudaStream_t s) {
+  dim3 grid((d.E + 63) / 64, KS, (d.batch + 31) / 32);
+  k_gemv_partial<float, WT><<<grid, 256, 0, s>>>(qin, static_cast<const WT*>(wuq), qpart,
+                                                 d.batch, d.r, d.E, KS);
+  note_launch();
+  return check_launch();
+}
+
+template <typename WT, typename QT16>
+cudaError_t absorb_t(const qsvd_dims& d, const float* qpart, int KS, const float* q_given,
+                     const void* wuk, float scale, float* qt32, void* qt16, cudaStream_t s) {
+  const size_t smem = size_t(128 + 16) * (d.d_h + 4) * 4;
+  auto kern = k_absorb<WT, QT16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(d.H, (d.r + 127) / 128);
+  kern<<<grid, 128, smem, s>>>(qpart, KS, q_given, static_cast<const WT*>(wuk), scale, qt32,
+                               static_cast<QT16*>(qt16), d.batch, d.H, d.d_h, d.r, d.E);
+  note_launch();
+  return check_launch();
+}
+
+}  // namespace
+
+cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
+                            WsHeader* hdr, int kernel, cudaStream_t s) {
+  k_schedule<<<1, 1024, 0, s>>>(lengths, d.batch, d.max_len, G, sched, hdr, kernel);
+  note_launch();
+  return check_launch();
+}
+
+cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
+                             float* qpart, int KS, cudaStream_t s) {
+  switch (d.weight_dtype) {
+    case QSVD_F32: return q_partial_t<float>(d, qin, wuq, qpart, KS, s);
+    case QSVD_F16: return q_partial_t<__half>(d, qin, wuq, qpart, KS, s);
+    case QSVD_BF16: return q_partial_t<__nv_bfloat16>(d, qin, wuq, qpart, KS, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_absorb(const qsvd_dims& d, const float* qpart, int KS, const float* q_given,
+                          const void* wuk, float scale, float* qt32, void* qt16, cudaStream_t s) {
+  const bool bf = d.cache_dtype == QSVD_BF16;
+  switch (d.weight_dtype) {
+    case QSVD_F32:
+      return bf ? absorb_t<float, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
+                : absorb_t<float, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+    case QSVD_F16:
+      return bf ? absorb_t<__half, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
+                : absorb_t<__half, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+    case QSVD_BF16:
+      return bf ? absorb_t<__nv_bfloat16, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
+                : absorb_t<__nv_bfloat16, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_rope_query(const qsvd_dims& d, const float* qpart, int KS,
+                              const float* q_given, const int32_t* sched,
+                              const float* rope_tab, float scale, float* qrot,
+                              cudaStream_t s) {
+  k_rope_query<<<d.batch, 256, 0, s>>>(qpart, KS, q_given, sched, rope_tab, scale, qrot,
+                                       d.batch, d.H, d.d_h, d.E);
+  note_launch();
+  return check_launch();
+}
+
+}  // namespace qsvd

@@ -1,0 +1,122 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+declared in include/qsvd.h, agrees with the header on the struct layout, and
+rejects invalid arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import rank_joint_qkv_b200 as q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qsvd.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsvd_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("qsvd_prepare_weights", "qsvd_append_latent", "qsvd_decode_attn",
+              "qsvd_combine_splits"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(q.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing
+    assert sorted(q.exported_symbols()) == declared_functions()
+
+
+def test_abi_version_matches_header():
+    m = re.search(r"#define QSVD_ABI_VERSION (\d+)", open(HEADER).read())
+    assert q.abi_version() == int(m.group(1))
+
+
+def test_struct_layout_matches_header():
+    """Compile a C probe against the header; compare sizeof/offsetof."""
+    fields = [f for f, _ in q.qsvd_dims._fields_]
+    body = "\n".join(f'printf("%zu ", offsetof(qsvd_dims, {f}));' for f in fields)
+    prog = f"""
+#include <stdio.h>
+#include <stddef.h>
+#include "qsvd.h"
+int main(void) {{ printf("%zu ", sizeof(qsvd_dims)); {body} return 0; }}
+"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "p.c")
+        open(c, "w").write(prog)
+        exe = os.path.join(d, "p")
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        got = list(map(int, subprocess.run([exe], capture_output=True, text=True,
+                                           check=True).stdout.split()))
+    want = [ctypes.sizeof(q.qsvd_dims)] + [getattr(q.qsvd_dims, f).offset for f in fields]
+    assert got == want
+
+
+def _dims(**kw):
+    base = dict(E=512, H=4, d_h=128, r=256, batch=2, max_len=300)
+    base.update(kw)
+    opts = {k: base.pop(k) for k in list(base) if k not in ("E", "H", "d_h", "r", "batch", "max_len")}
+    return q.make_dims(base["E"], base["H"], base["d_h"], base["r"], base["batch"],
+                       base["max_len"], **opts)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(E=500), dict(H=3), dict(r=100), dict(r=16), dict(batch=0), dict(max_len=0),
+    dict(cache="i4", group=100), dict(cache="i8", group=96), dict(d_h=130, E=520),
+    dict(h2=True, h2_m=3),                   # r/h2_m = 256/3 not an integer
+])
+def test_invalid_dims_rejected_on_host(bad):
+    d = _dims(**bad)
+    with pytest.raises(q.QsvdError) as e:
+        q.decode_workspace_bytes(d, num_splits=4)
+    assert e.value.status == q.QSVD_ERR_INVALID_ARG
+
+
+def test_rope_needs_d_h_multiple_of_64():
+    d = _dims(E=384, H=4, d_h=96, rope=True)
+    with pytest.raises(q.QsvdError) as e:
+        q.decode_workspace_bytes(d, num_splits=4)
+    assert e.value.status == q.QSVD_ERR_UNSUPPORTED
+
+
+def test_workspace_query_on_host():
+    d = _dims(max_len=3000)
+    n4 = q.decode_workspace_bytes(d, num_splits=4)
+    n8 = q.decode_workspace_bytes(d, num_splits=8)
+    # 4 more partial slots of H x r latent floats (m, l sections are padded)
+    assert n8 - n4 >= 4 * 4 * 256 * 4
+    assert n4 % 256 == 0
+    # splits beyond the number of 128-token tiles are not used
+    d2 = _dims(max_len=300)
+    assert q.decode_workspace_bytes(d2, num_splits=6) == q.decode_workspace_bytes(d2, num_splits=60)
+    assert q.append_workspace_bytes(d) > 0
+
+
+def test_too_small_workspace_and_null_pointers():
+    lib = ctypes.CDLL(q.LIB_PATH)
+    lib.qsvd_decode_attn.argtypes = q._sigs["qsvd_decode_attn"]
+    d = _dims()
+    n = ctypes.c_size_t(16)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check fails first
+    st = lib.qsvd_decode_attn(ctypes.byref(d), fake, fake, 1, fake, None, fake, 4, fake,
+                              ctypes.byref(n), fake, 0, None)
+    assert st == q.QSVD_ERR_WORKSPACE
+    n = ctypes.c_size_t(1 << 40)
+    st = lib.qsvd_decode_attn(ctypes.byref(d), None, fake, 1, fake, None, fake, 4, fake,
+                              ctypes.byref(n), fake, 0, None)
+    assert st == q.QSVD_ERR_INVALID_ARG
+    assert b"NULL" in q._lib.qsvd_last_error()
+
+
+def test_status_strings():
+    for s in range(5):
+        assert q._lib.qsvd_status_string(s).startswith(b"QSVD_")
