@@ -161,6 +161,30 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed,
                                void* stream);
 
 /*
+ * qsvd_append_latent_static -- qsvd_append_latent without a workspace.
+ * The paper has no counterpart: this is an interface variant for callers
+ * that cannot allocate device memory -- a serving engine or plugin host that
+ * owns every buffer and passes only the call's tensors, or a deployment with
+ * a fixed memory budget that forbids allocation after start-up.
+ * Same arguments, results and status bits as qsvd_append_latent, minus the
+ * workspace.  The split-K partials of x W^d go to a static device array of
+ * 1,048,576 floats (4 MiB) that every GPU loading the library holds until
+ * the process exits; requests needing more, i.e. ksplit * batch * r >
+ * 1,048,576 with ksplit = min(16, max(1, E / 512)) reduced to a divisor of
+ * E, return QSVD_ERR_WORKSPACE and enqueue nothing.  Nothing is allocated.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the array.  It needs no clearing (each call writes
+ *     every partial it reads), but calls that overlap on the GPU -- on
+ *     different streams, or from several host threads -- race on it and
+ *     must be serialised by the caller.
+ */
+qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const void* packed,
+                                      const void* x, const int32_t* pos, void* cache,
+                                      void* scales, float* c_out, int32_t* status,
+                                      void* stream);
+
+/*
  * qsvd_decode_attn -- one decode step of multi-head attention over the
  * latent cache, output B x E.
  * Source: QSVD digest, Method, Step 1 (keys/values rebuilt from C_qkv);

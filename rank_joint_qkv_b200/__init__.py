@@ -4,7 +4,7 @@ Argument marshalling only: every step of the decode path runs in the CUDA
 kernels of ``libqsvd.so``; PyTorch supplies device memory and streams.  The
 functions carry the C names of ``include/qsvd.h`` and raise ``QsvdError`` on a
 non-OK status.  Importing the package fails loudly when the library has not
-been built (``python -m rank_joint_qkv_b200.build``): there is no fallback.
+been built (``python rank_joint_qkv_b200/build.py``): there is no fallback.
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libqsvd.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m rank_joint_qkv_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python rank_joint_qkv_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -54,6 +54,7 @@ _sigs = {
     "qsvd_decode_attn": [_D, _P, _P, ctypes.c_int, _P, _P, _P, ctypes.c_int, _P, _SZ, _P,
                          ctypes.c_uint, _P],
     "qsvd_combine_splits": [_D, _P, _P, ctypes.c_int, _P, _P, _P],
+    "qsvd_append_latent_static": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -150,6 +151,16 @@ def qsvd_append_latent(dims: qsvd_dims, packed, x, pos, cache, scales=None, c_ou
                                    _ptr(workspace), ctypes.byref(n), _stream(stream)),
            "qsvd_append_latent")
     return workspace
+
+
+def qsvd_append_latent_static(dims: qsvd_dims, packed, x, pos, cache, scales=None,
+                              c_out=None, status=None, stream=None):
+    """qsvd_append_latent for callers that cannot allocate: no workspace, the
+    library's static device scratch instead (calls must not overlap)."""
+    _check(_lib.qsvd_append_latent_static(ctypes.byref(dims), _ptr(packed), _ptr(x), _ptr(pos),
+                                          _ptr(cache), _ptr(scales), _ptr(c_out), _ptr(status),
+                                          _stream(stream)),
+           "qsvd_append_latent_static")
 
 
 def decode_workspace_bytes(dims: qsvd_dims, num_splits: int = 0) -> int:

@@ -1,6 +1,8 @@
 """Build the CUDA library in-tree: rank_joint_qkv_b200/libqsvd.so (sm_100a).
 
-    python -m rank_joint_qkv_b200.build [--force] [-v]
+    python rank_joint_qkv_b200/build.py [--force] [-v]
+
+(run by path: importing the package loads the library this script builds)
 
 Every ``csrc/*.cu`` is compiled with nvcc for ``sm_100a`` (object files under
 ``_build/`` at the repository root, rebuilt when a source or header is newer)

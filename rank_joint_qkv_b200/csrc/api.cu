@@ -23,6 +23,8 @@ static qsvd_status fail(qsvd_status st, const char* fmt, ...) {
   return st;
 }
 
+qsvd_status set_error(qsvd_status st, const char* msg) { return fail(st, "%s", msg); }
+
 static qsvd_status cuda_fail(cudaError_t e, const char* where) {
   return fail(QSVD_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }

@@ -117,6 +117,7 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
 // -------------------------------------------------------- launch bookkeeping
 
 void note_launch();                 // counts kernels launched by this library
+qsvd_status set_error(qsvd_status st, const char* msg);   // records qsvd_last_error()
 cudaError_t check_launch();         // cudaGetLastError after a launch
 
 // ------------------------------------------------------------ kernel entry
