@@ -212,22 +212,29 @@ def run_ours(args, rank, world, local_rank):
                          device=device)
     cache, scales = inp["cache"], inp["scales"]
 
-    def step(ev_split=None):
+    def step(ev=None):
+        # ev: 5 events bracketing append | prologue | split | combine
+        if ev is not None:
+            ev[0].record(stream)
         q.qsvd_append_latent(dims, packed, x_dev, pos_dev, cache, scales, cnew, None, app_ws,
                              stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
                            phases=q.QSVD_PHASE_PROLOGUE, stream=stream)
-        if ev_split is not None:
-            ev_split[0].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
                            phases=q.QSVD_PHASE_SPLIT, stream=stream)
-        if ev_split is not None:
-            ev_split[1].record(stream)
+        if ev is not None:
+            ev[3].record(stream)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
                            phases=q.QSVD_PHASE_COMBINE, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -235,8 +242,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = q.kernel_launches()
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -252,7 +258,10 @@ def run_ours(args, rank, world, local_rank):
             torch.distributed.barrier()
     launches = q.kernel_launches() - launches0
     ms = t0.elapsed_time(t1)
-    split_ms = [a.elapsed_time(b) for a, b in ev]
+    phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
+                for k, name in enumerate(("append", "prologue", "split", "combine"))}
+    split_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    kernel_used = int(dec_ws[12:16].view(torch.int32).item())   # workspace header: kernel
     ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
@@ -290,9 +299,10 @@ def run_ours(args, rank, world, local_rank):
     split_mean = statistics.mean(split_ms)
     lat_b = latent_bytes(w, lens)
     achieved = lat_b / (split_mean / 1e3) / 1e9
-    kname = "split_tcgen05" if args.kernel == "tcgen05" else "split_simt"
+    kname = "k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05 else "k_split_abs"
+    src = ["split_tc.cu", "internal.cuh"] if kname == "k_split_tc" else ["split_simt.cu", "internal.cuh"]
     workload = w.name
-    traffic = profiled_traffic(kname, workload, ["split_simt.cu", "internal.cuh"])
+    traffic = profiled_traffic(kname, workload, src)
     step_gbs = (lat_b + weight_bytes(w)) / (ms_max / args.steps / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -307,6 +317,7 @@ def run_ours(args, rank, world, local_rank):
                          % (lat_b / 1e6),
                    "parallelism": f"dp{world}"},
         "steps_per_s": args.steps * 1e3 / ms_max,
+        "phase_ms": phase_ms,
         "step_hbm_gbs": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
@@ -397,7 +408,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")

@@ -76,6 +76,8 @@ typedef enum {
 #define QSVD_STATUS_LEN_CLAMPED 1   /* some lengths[b] < 0 or > max_len (clamped) */
 #define QSVD_STATUS_POS_OOB 2       /* some pos[b] outside [0, max_len) (row not written) */
 #define QSVD_STATUS_SCALE_SAT 4     /* a group scale exceeded the fp16 range (saturated) */
+#define QSVD_STATUS_TIMEOUT 8       /* a pipeline wait in the split kernel timed out (the
+                                       output of that call is invalid) */
 
 /* Split-kernel choice (qsvd_dims.kernel). */
 #define QSVD_KERNEL_AUTO 0
@@ -170,8 +172,9 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed,
  * workspace.  The split-K partials of x W^d go to a static device array of
  * 1,048,576 floats (4 MiB) that every GPU loading the library holds until
  * the process exits; requests needing more, i.e. ksplit * batch * r >
- * 1,048,576 with ksplit = min(16, max(1, E / 512)) reduced to a divisor of
- * E, return QSVD_ERR_WORKSPACE and enqueue nothing.  Nothing is allocated.
+ * 1,048,576, where ksplit <= 16 is the split of E the projection uses
+ * (chosen from E, r and batch), return QSVD_ERR_WORKSPACE and enqueue
+ * nothing; batch * r <= 65,536 always fits.  Nothing is allocated.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - Every call shares the array.  It needs no clearing (each call writes

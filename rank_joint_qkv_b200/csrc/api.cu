@@ -52,8 +52,9 @@ static qsvd_status validate(const qsvd_dims* d) {
   if (d->out_dtype < QSVD_F32 || d->out_dtype > QSVD_BF16)
     return fail(QSVD_ERR_INVALID_ARG, "out dtype must be F32, F16 or BF16");
   if (cache_is_int(*d)) {
-    if (d->group < 32 || d->group % 32 || d->r % d->group)
-      return fail(QSVD_ERR_INVALID_ARG, "group (%d) must be a multiple of 32 dividing r (%d)",
+    if (d->group < 32 || d->group > 1024 || d->group % 32 || d->r % d->group)
+      return fail(QSVD_ERR_INVALID_ARG,
+                  "group (%d) must be a multiple of 32 in [32, 1024] dividing r (%d)",
                   d->group, d->r);
   }
   if (d->rope) {
@@ -80,7 +81,7 @@ static int device_sms() {
 static int pick_kernel(const qsvd_dims& d) {
   if (d.kernel == QSVD_KERNEL_SIMT) return QSVD_KERNEL_SIMT;
   if (d.kernel == QSVD_KERNEL_TCGEN05) return QSVD_KERNEL_TCGEN05;
-  return QSVD_KERNEL_SIMT;
+  return split_tc_supported(d) ? QSVD_KERNEL_TCGEN05 : QSVD_KERNEL_SIMT;
 }
 
 static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel, int* G) {
@@ -191,9 +192,10 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
   if (phases == 0) phases = QSVD_PHASE_ALL;
   if (phases & ~QSVD_PHASE_ALL) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
   const int kernel = pick_kernel(d);
-  if (kernel == QSVD_KERNEL_TCGEN05)
-    return fail(QSVD_ERR_UNSUPPORTED, "tensor-core split kernel not available for these dims");
-  if (!d.rope && split_simt_grid_heads(d) == 0)
+  if (kernel == QSVD_KERNEL_TCGEN05 && !split_tc_supported(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "tensor-core split kernel needs a 16-bit cache, no rotary, r %% 128 == 0, H <= 32");
+  if (kernel == QSVD_KERNEL_SIMT && !d.rope && split_simt_grid_heads(d) == 0)
     return fail(QSVD_ERR_UNSUPPORTED, "rank too large for the CUDA-core split kernel");
   int G = 0;
   qsvd_status st = resolve_splits(d, num_splits, kernel, &G);
@@ -229,28 +231,34 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
   cudaError_t e;
 
   if (phases & QSVD_PHASE_PROLOGUE) {
-    if ((e = launch_schedule(d, lengths, G, sched, hdr, kernel, s)) != cudaSuccess)
+    int32_t* tickets = reinterpret_cast<int32_t*>(Wb + W.tickets);
+    if ((e = launch_schedule(d, lengths, G, sched, hdr, kernel, tickets, W.NT, s)) != cudaSuccess)
       return cuda_fail(e, "schedule");
-    const float* q_given = qin_is_latent ? nullptr : qin;
+    // q = c_new W^u_q (reduced into the workspace), or the query as given
+    const float* qsrc = qin;
     if (qin_is_latent) {
-      if ((e = launch_q_partial(d, qin, P + L.wuq, qpart, W.KS, s)) != cudaSuccess)
+      if ((e = launch_q_partial(d, qin, P + L.wuq, qpart, W.KS, q, tickets, s)) != cudaSuccess)
         return cuda_fail(e, "query projection");
+      qsrc = q;
     }
+    // rotary mode keeps the rotated query in the q section (qt32 is unused there)
     if (d.rope)
-      e = launch_rope_query(d, qpart, W.KS, q_given, sched, rope_tab, sl2, q, s);
+      e = launch_rope_query(d, qsrc, sched, rope_tab, sl2, qt32, s);
     else
-      e = launch_absorb(d, qpart, W.KS, q_given, P + L.wuk, sl2, qt32, qt16, s);
+      e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, qt16, s);
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (phases & QSVD_PHASE_SPLIT) {
     if (d.rope)
-      e = launch_split_simt_rope(d, q, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
+      e = launch_split_simt_rope(d, qt32, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
+    else if (kernel == QSVD_KERNEL_TCGEN05)
+      e = launch_split_tc(d, cache, qt16, sched, G, pm, pl, pz, &hdr->status, s);
     else
       e = launch_split_simt_absorbed(d, qt32, cache, scales, sched, G, pm, pl, pz, s);
     if (e != cudaSuccess) return cuda_fail(e, "split phase");
   }
   if (phases & QSVD_PHASE_COMBINE) {
-    if ((e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, out, s)) != cudaSuccess)
+    if ((e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, W.P, out, s)) != cudaSuccess)
       return cuda_fail(e, "combine phase");
   }
   return QSVD_OK;

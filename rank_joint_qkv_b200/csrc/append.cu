@@ -119,21 +119,94 @@ k_append_finish(const float* __restrict__ cpart, int KS, const float* __restrict
   }
 }
 
+// Without online H2 every group is independent: grid (B, r / chunk), one
+// thread per channel of the chunk (chunk = the quantisation group for int
+// caches).  Sums the split-K partials, writes c_out and the cache row.
+template <qsvd_dtype CT>
+__global__ void __launch_bounds__(1024)
+k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restrict__ pos,
+               uint8_t* __restrict__ cache, __half* __restrict__ scales,
+               float* __restrict__ c_out, int32_t* status, int B, int r, int max_len,
+               int chunk) {
+  __shared__ float wmax[32];
+  const int b = blockIdx.x;
+  const int j = blockIdx.y * chunk + threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float v = 0.f;
+  for (int k = 0; k < KS; ++k) v += cpart[(size_t(k) * B + b) * r + j];
+  if (c_out) c_out[size_t(b) * r + j] = v;
+  const int p = pos[b];
+  if (p < 0 || p >= max_len) {
+    if (threadIdx.x == 0 && blockIdx.y == 0 && status) atomicOr(status, QSVD_STATUS_POS_OOB);
+    return;
+  }
+  const size_t row = size_t(b) * max_len + p;
+  if (CT == QSVD_F32) { reinterpret_cast<float*>(cache)[row * r + j] = v; return; }
+  if (CT == QSVD_F16) { reinterpret_cast<__half*>(cache)[row * r + j] = __float2half_rn(v); return; }
+  if (CT == QSVD_BF16) {
+    reinterpret_cast<__nv_bfloat16*>(cache)[row * r + j] = __float2bfloat16_rn(v);
+    return;
+  }
+  // group amax over the chunk (== group)
+  float a = dev::warp_max(fabsf(v));
+  if (lane == 0) wmax[warp] = a;
+  __syncthreads();
+  if (warp == 0) {
+    a = lane < int(blockDim.x >> 5) ? wmax[lane] : 0.f;
+    a = dev::warp_max(a);
+    if (lane == 0) wmax[0] = a;
+  }
+  __syncthreads();
+  const int qmax = (CT == QSVD_I4) ? 7 : 127;
+  float s32 = __fdiv_rn(wmax[0], float(qmax));
+  if (s32 > 65504.f) {
+    s32 = 65504.f;
+    if (threadIdx.x == 0 && status) atomicOr(status, QSVD_STATUS_SCALE_SAT);
+  }
+  const __half s16 = __float2half_rn(s32);
+  const float sf = __half2float(s16);
+  if (threadIdx.x == 0) scales[row * (r / chunk) + blockIdx.y] = s16;
+  int q = 0;
+  if (sf != 0.f) q = max(-qmax, min(qmax, __float2int_rn(__fdiv_rn(v, sf))));
+  if (CT == QSVD_I8) {
+    reinterpret_cast<int8_t*>(cache)[row * r + j] = int8_t(q);
+  } else {
+    const int hi = __shfl_down_sync(0xffffffffu, q, 1);   // partner element j + 1
+    if ((j & 1) == 0) cache[row * (r / 2) + j / 2] = uint8_t((q & 0xF) | ((hi & 0xF) << 4));
+  }
+}
+
 template <typename WT>
 cudaError_t gemv_t(const qsvd_dims& d, const void* x, const void* wd, float* cpart, int KS,
                    cudaStream_t s) {
-  dim3 grid((d.r + 63) / 64, KS, (d.batch + 31) / 32);
+  dim3 grid((d.r + 255) / 256, KS, (d.batch + 15) / 16);
   k_gemv_partial<WT, WT><<<grid, 256, 0, s>>>(static_cast<const WT*>(x),
                                               static_cast<const WT*>(wd), cpart, d.batch,
-                                              d.E, d.r, KS);
+                                              d.E, d.r, KS, nullptr, nullptr);
   note_launch();
   return check_launch();
+}
+
+int append_chunk(const qsvd_dims& d) {
+  if (d.cache_dtype == QSVD_I8 || d.cache_dtype == QSVD_I4) return d.group;
+  for (int c : {256, 128, 64, 32})
+    if (d.r % c == 0) return c;
+  return 32;
 }
 
 template <qsvd_dtype CT>
 cudaError_t finish_t(const qsvd_dims& d, const float* cpart, int KS, const float* h2q,
                      float h2_scale, const int32_t* pos, void* cache, void* scales,
                      float* c_out, int32_t* status, cudaStream_t s) {
+  if (!d.h2) {
+    const int chunk = append_chunk(d);
+    dim3 grid(d.batch, d.r / chunk);
+    k_append_chunk<CT><<<grid, chunk, 0, s>>>(cpart, KS, pos, static_cast<uint8_t*>(cache),
+                                              static_cast<__half*>(scales), c_out, status,
+                                              d.batch, d.r, d.max_len, chunk);
+    note_launch();
+    return check_launch();
+  }
   const size_t smem = size_t(d.r) * 4;
   auto kern = k_append_finish<CT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -147,13 +220,7 @@ cudaError_t finish_t(const qsvd_dims& d, const float* cpart, int KS, const float
 
 }  // namespace
 
-int append_ksplit(const qsvd_dims& d) {
-  int ks = d.E / 512;
-  if (ks < 1) ks = 1;
-  if (ks > 16) ks = 16;
-  while (d.E % ks) --ks;
-  return ks;
-}
+int append_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.E, d.r, d.batch, 16); }
 
 cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
                           const float* h2q, float h2_scale, const int32_t* pos,

@@ -78,19 +78,15 @@ struct WsHeader {
 };
 
 struct WsLayout {
-  size_t hdr, sched, q, qt32, qt16, qpart, pm, pl, pz, opart, total;
-  int G, P, KS, JS;
+  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, total;
+  int G, P, KS, JS, NT;
 };
 
 // Split-K factor of the query projection and j-splits of the combine.
-inline int prologue_ksplit(const qsvd_dims& d) {
-  int ks = d.r / 128;
-  if (ks < 1) ks = 1;
-  if (ks > 4) ks = 4;
-  while (d.r % (ks * 32)) --ks;
-  return ks;
-}
-inline int combine_jsplit(const qsvd_dims& d) { return (d.r + 255) / 256; }
+int prologue_ksplit(const qsvd_dims& d);   // split of r in q = c_new W^u_q
+inline int combine_jsplit(const qsvd_dims& d) { return (d.r + 127) / 128; }
+
+int prologue_tickets(const qsvd_dims& d);  // ticket counters of that GEMV
 
 inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   WsLayout w{};
@@ -98,13 +94,15 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.P = G + d.batch;
   w.KS = prologue_ksplit(d);
   w.JS = combine_jsplit(d);
+  w.NT = prologue_tickets(d);
   const size_t B = d.batch, E = d.E, H = d.H, r = d.r;
   size_t o = 0;
   w.hdr = o;   o = align256(o + sizeof(WsHeader));
   w.sched = o; o = align256(o + (2 * B + 1) * 4);
+  w.tickets = o; o = align256(o + size_t(w.NT) * 4);
   w.q = o;     o = align256(o + B * E * 4);
-  w.qt32 = o;  o = align256(o + B * H * r * 4);
-  w.qt16 = o;  o = align256(o + B * H * r * 2);
+  w.qt32 = o;  o = align256(o + (H * r > E ? H * r : E) * B * 4);   // rotary mode: B x E query
+  w.qt16 = o;  o = align256(o + 2 * B * H * r * 2);   // [B][2][H][r] for bf16 hi/lo
   w.qpart = o; o = align256(o + size_t(w.KS) * B * E * 4);
   w.pm = o;    o = align256(o + size_t(w.P) * H * 4);
   w.pl = o;    o = align256(o + size_t(w.P) * H * 4);
@@ -124,16 +122,15 @@ cudaError_t check_launch();         // cudaGetLastError after a launch
 
 // Prologue (query side).
 cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
-                            WsHeader* hdr, int kernel, cudaStream_t s);
+                            WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,
+                            cudaStream_t s);
 cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
-                             float* qpart, int KS, cudaStream_t s);
-cudaError_t launch_absorb(const qsvd_dims& d, const float* qpart, int KS,
-                          const float* q_given, const void* wuk, float scale_log2,
+                             float* qpart, int KS, float* q, int32_t* tickets, cudaStream_t s);
+cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale_log2,
                           float* qt32, void* qt16, cudaStream_t s);
-cudaError_t launch_rope_query(const qsvd_dims& d, const float* qpart, int KS,
-                              const float* q_given, const int32_t* sched,
-                              const float* rope_tab, float scale_log2,
-                              float* qrot, cudaStream_t s);
+cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
+                              const float* rope_tab, float scale_log2, float* qrot,
+                              cudaStream_t s);
 
 // Split phase.
 cudaError_t launch_split_simt_absorbed(const qsvd_dims& d, const float* qt32,
@@ -146,11 +143,15 @@ cudaError_t launch_split_simt_rope(const qsvd_dims& d, const float* qrot,
                                    const int32_t* sched, int G, float* pm,
                                    float* pl, float* pz, cudaStream_t s);
 int split_simt_grid_heads(const qsvd_dims& d);   // head blocks per split
+bool split_tc_supported(const qsvd_dims& d);
+cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* qt16,
+                            const int32_t* sched, int G, float* pm, float* pl, float* pz,
+                            int32_t* status, cudaStream_t s);
 
 // Combine phase.
 cudaError_t launch_combine(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                            const float* pm, const float* pl, const float* pz,
-                           const void* wuv, float* opart, int JS, void* out,
+                           const void* wuv, float* opart, int JS, int P, void* out,
                            cudaStream_t s);
 
 // Append.

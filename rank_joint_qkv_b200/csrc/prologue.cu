@@ -19,24 +19,15 @@ namespace {
 
 using dev::to_f;
 
-// Query of sequence b, head h, dim d: sum of the split partials (or given).
-__device__ __forceinline__ float query_at(const float* qpart, int KS, const float* q_given,
-                                          int B, int E, int b, int e) {
-  if (q_given) return q_given[size_t(b) * E + e];
-  float s = 0.f;
-  for (int k = 0; k < KS; ++k) s += qpart[(size_t(k) * B + b) * E + e];
-  return s;
-}
-
 // ---------------------------------------------------------------------------
 // qt[b][h][j] = scale * sum_d W^u_k[j][h*d_h + d] * q[b][h*d_h + d]
 // grid (H, ceil(r/128)), block 128.  A thread computes 4 rows x 4 sequences.
 // ---------------------------------------------------------------------------
 template <typename WT, typename QT16>
 __global__ void __launch_bounds__(128)
-k_absorb(const float* __restrict__ qpart, int KS, const float* __restrict__ q_given,
-         const WT* __restrict__ W, float scale, float* __restrict__ qt32,
-         QT16* __restrict__ qt16, int B, int H, int d_h, int r, int E) {
+k_absorb(const float* __restrict__ q, const WT* __restrict__ W, float scale,
+         float* __restrict__ qt32, QT16* __restrict__ qt16, int B, int H, int d_h, int r,
+         int E) {
   extern __shared__ float sm[];
   const int h = blockIdx.x;
   const int j0 = blockIdx.y * 128;
@@ -44,18 +35,35 @@ k_absorb(const float* __restrict__ qpart, int KS, const float* __restrict__ q_gi
   const int ld = d_h + 4;                  // padded row stride (floats)
   float* ws = sm;                          // [128][ld]
   float* qs = sm + 128 * ld;               // [32][ld]
-  // stage the W^u_k tile (rows j0.., columns of head h) as float
-  for (int i = threadIdx.x; i < 128 * d_h; i += 128) {
-    const int jr = i / d_h, d = i % d_h;
-    ws[jr * ld + d] = jr < jn ? to_f(W[size_t(j0 + jr) * E + h * d_h + d]) : 0.f;
+  // stage the W^u_k tile (rows j0.., columns of head h) as float, 16-byte loads
+  {
+    constexpr int V = 16 / int(sizeof(WT));
+    const int vpr = d_h / V;
+    for (int i = threadIdx.x; i < 128 * vpr; i += 128) {
+      const int jr = i / vpr, v = i % vpr;
+      float f[V];
+      if (jr < jn) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(W + size_t(j0 + jr) * E + h * d_h + v * V);
+        const WT* e = reinterpret_cast<const WT*>(&raw);
+#pragma unroll
+        for (int k = 0; k < V; ++k) f[k] = to_f(e[k]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k) f[k] = 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < V; ++k) ws[jr * ld + v * V + k] = f[k];
+    }
   }
   const int tr = threadIdx.x / 4;    // rows tr + 32a, a < 4 (conflict-free float4 reads)
   const int tb = threadIdx.x % 4;    // sequences b0 + tb + 4c, c < 4
   for (int b0 = 0; b0 < B; b0 += 16) {
     __syncthreads();
-    for (int i = threadIdx.x; i < 16 * d_h; i += 128) {
-      const int bb = i / d_h, d = i % d_h;
-      qs[bb * ld + d] = (b0 + bb < B) ? query_at(qpart, KS, q_given, B, E, b0 + bb, h * d_h + d) : 0.f;
+    for (int i = threadIdx.x; i < 16 * (d_h / 4); i += 128) {
+      const int bb = i / (d_h / 4), d = 4 * (i % (d_h / 4));
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b0 + bb < B) v = *reinterpret_cast<const float4*>(q + size_t(b0 + bb) * E + h * d_h + d);
+      *reinterpret_cast<float4*>(&qs[bb * ld + d]) = v;
     }
     __syncthreads();
     float acc[4][4];
@@ -88,7 +96,13 @@ k_absorb(const float* __restrict__ qpart, int KS, const float* __restrict__ q_gi
           const float v = acc[a][c] * scale;
           const size_t o = (size_t(b) * H + h) * r + j;
           qt32[o] = v;
-          qt16[o] = dev::from_f<QT16>(v);
+          // 16-bit copy for the tensor cores, [B][2][H][r]: the rounded value
+          // and its rounding residual (hi + lo carries ~2x the mantissa bits;
+          // one 16-bit part alone perturbs peaked softmaxes by ~1e-2)
+          const QT16 hi = dev::from_f<QT16>(v);
+          const size_t o2 = ((size_t(b) * 2) * H + h) * r + j;
+          qt16[o2] = hi;
+          qt16[o2 + size_t(H) * r] = dev::from_f<QT16>(v - dev::to_f(hi));
         }
       }
   }
@@ -99,9 +113,9 @@ k_absorb(const float* __restrict__ qpart, int KS, const float* __restrict__ q_gi
 // grid (B), block 256.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-k_rope_query(const float* __restrict__ qpart, int KS, const float* __restrict__ q_given,
-             const int32_t* __restrict__ sched, const float* __restrict__ tab,
-             float scale, float* __restrict__ qrot, int B, int H, int d_h, int E) {
+k_rope_query(const float* __restrict__ q, const int32_t* __restrict__ sched,
+             const float* __restrict__ tab, float scale, float* __restrict__ qrot, int B,
+             int H, int d_h, int E) {
   const int b = blockIdx.x;
   const int n = sched[B + 1 + b];
   const int pos = n > 0 ? n - 1 : 0;
@@ -109,8 +123,8 @@ k_rope_query(const float* __restrict__ qpart, int KS, const float* __restrict__ 
   for (int i = threadIdx.x; i < H * half; i += blockDim.x) {
     const int h = i / half, k = i % half;
     const int e0 = h * d_h + k, e1 = e0 + half;
-    const float a = query_at(qpart, KS, q_given, B, E, b, e0);
-    const float c = query_at(qpart, KS, q_given, B, E, b, e1);
+    const float a = q[size_t(b) * E + e0];
+    const float c = q[size_t(b) * E + e1];
     const float cs = tab[(size_t(pos) * half + k) * 2 + 0];
     const float sn = tab[(size_t(pos) * half + k) * 2 + 1];
     qrot[size_t(b) * E + e0] = (a * cs - c * sn) * scale;
@@ -125,7 +139,9 @@ k_rope_query(const float* __restrict__ qpart, int KS, const float* __restrict__ 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
-           int32_t* __restrict__ sched, WsHeader* hdr, int kernel) {
+           int32_t* __restrict__ sched, WsHeader* hdr, int kernel,
+           int32_t* __restrict__ tickets, int n_tickets) {
+  for (int i = threadIdx.x; i < n_tickets; i += 1024) tickets[i] = 0;
   __shared__ int32_t part[1024];
   __shared__ int32_t carry;
   if (threadIdx.x == 0) {
@@ -163,23 +179,23 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
 
 template <typename WT>
 cudaError_t q_partial_t(const qsvd_dims& d, const float* qin, const void* wuq, float* qpart,
-                        int KS, cudaStream_t s) {
-  dim3 grid((d.E + 63) / 64, KS, (d.batch + 31) / 32);
+                        int KS, float* q, int32_t* tickets, cudaStream_t s) {
+  dim3 grid((d.E + 255) / 256, KS, (d.batch + 15) / 16);
   k_gemv_partial<float, WT><<<grid, 256, 0, s>>>(qin, static_cast<const WT*>(wuq), qpart,
-                                                 d.batch, d.r, d.E, KS);
+                                                 d.batch, d.r, d.E, KS, q, tickets);
   note_launch();
   return check_launch();
 }
 
 template <typename WT, typename QT16>
-cudaError_t absorb_t(const qsvd_dims& d, const float* qpart, int KS, const float* q_given,
-                     const void* wuk, float scale, float* qt32, void* qt16, cudaStream_t s) {
+cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float scale,
+                     float* qt32, void* qt16, cudaStream_t s) {
   const size_t smem = size_t(128 + 16) * (d.d_h + 4) * 4;
   auto kern = k_absorb<WT, QT16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(d.H, (d.r + 127) / 128);
-  kern<<<grid, 128, smem, s>>>(qpart, KS, q_given, static_cast<const WT*>(wuk), scale, qt32,
+  kern<<<grid, 128, smem, s>>>(q, static_cast<const WT*>(wuk), scale, qt32,
                                static_cast<QT16*>(qt16), d.batch, d.H, d.d_h, d.r, d.E);
   note_launch();
   return check_launch();
@@ -187,46 +203,50 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* qpart, int KS, const float
 
 }  // namespace
 
+int prologue_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.r, d.E, d.batch, 32); }
+int prologue_tickets(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch); }
+
 cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
-                            WsHeader* hdr, int kernel, cudaStream_t s) {
-  k_schedule<<<1, 1024, 0, s>>>(lengths, d.batch, d.max_len, G, sched, hdr, kernel);
+                            WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,
+                            cudaStream_t s) {
+  k_schedule<<<1, 1024, 0, s>>>(lengths, d.batch, d.max_len, G, sched, hdr, kernel, tickets,
+                                n_tickets);
   note_launch();
   return check_launch();
 }
 
 cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
-                             float* qpart, int KS, cudaStream_t s) {
+                             float* qpart, int KS, float* q, int32_t* tickets, cudaStream_t s) {
   switch (d.weight_dtype) {
-    case QSVD_F32: return q_partial_t<float>(d, qin, wuq, qpart, KS, s);
-    case QSVD_F16: return q_partial_t<__half>(d, qin, wuq, qpart, KS, s);
-    case QSVD_BF16: return q_partial_t<__nv_bfloat16>(d, qin, wuq, qpart, KS, s);
+    case QSVD_F32: return q_partial_t<float>(d, qin, wuq, qpart, KS, q, tickets, s);
+    case QSVD_F16: return q_partial_t<__half>(d, qin, wuq, qpart, KS, q, tickets, s);
+    case QSVD_BF16: return q_partial_t<__nv_bfloat16>(d, qin, wuq, qpart, KS, q, tickets, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_absorb(const qsvd_dims& d, const float* qpart, int KS, const float* q_given,
-                          const void* wuk, float scale, float* qt32, void* qt16, cudaStream_t s) {
+cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale,
+                          float* qt32, void* qt16, cudaStream_t s) {
   const bool bf = d.cache_dtype == QSVD_BF16;
   switch (d.weight_dtype) {
     case QSVD_F32:
-      return bf ? absorb_t<float, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
-                : absorb_t<float, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<float, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
+                : absorb_t<float, __half>(d, q, wuk, scale, qt32, qt16, s);
     case QSVD_F16:
-      return bf ? absorb_t<__half, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
-                : absorb_t<__half, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<__half, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
+                : absorb_t<__half, __half>(d, q, wuk, scale, qt32, qt16, s);
     case QSVD_BF16:
-      return bf ? absorb_t<__nv_bfloat16, __nv_bfloat16>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s)
-                : absorb_t<__nv_bfloat16, __half>(d, qpart, KS, q_given, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<__nv_bfloat16, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
+                : absorb_t<__nv_bfloat16, __half>(d, q, wuk, scale, qt32, qt16, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_rope_query(const qsvd_dims& d, const float* qpart, int KS,
-                              const float* q_given, const int32_t* sched,
+cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
                               const float* rope_tab, float scale, float* qrot,
                               cudaStream_t s) {
-  k_rope_query<<<d.batch, 256, 0, s>>>(qpart, KS, q_given, sched, rope_tab, scale, qrot,
-                                       d.batch, d.H, d.d_h, d.E);
+  k_rope_query<<<d.batch, 256, 0, s>>>(q, sched, rope_tab, scale, qrot, d.batch, d.H, d.d_h,
+                                       d.E);
   note_launch();
   return check_launch();
 }

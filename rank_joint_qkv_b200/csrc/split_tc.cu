@@ -1,0 +1,691 @@
+// Split phase on the 5th-generation tensor cores: absorbed query, 16-bit latent.
+//
+// Per 128-token latent tile of one sequence (QSVD digest, Method, Step 1: keys
+// and values are never rebuilt when no rotary embedding is applied; WSVD
+// digest, Problem: the shared latent must not be re-read once per head):
+//
+//   S   = C_tile Qt^T        (128 tokens x H heads, K = r)        tcgen05, TMEM
+//   P   = 2^(S - m)          (online softmax, log2 domain)        CUDA cores
+//   Z^T += C_tile^T P        (r x H in 128-channel chunks, K=128) tcgen05, TMEM
+//
+// Every head is served from the same staged tile, so HBM sees the latent
+// once per step.  The tile is streamed twice through shared memory in
+// 128-channel chunks -- once for S (from HBM, together with the matching
+// chunk of the absorbed query Qt) and once for Z (re-read from L2 a fraction
+// of a tile later) -- because a whole tile (128 x r x 2 bytes) does not fit in
+// shared memory.  The two streams are interleaved (S of tile i+1 with Z of
+// tile i) so the HBM stream never waits for the softmax.
+//
+// Roles (192 threads):
+//   warp 0     TMA producer (full tiles) / manual zero-filled loads (ragged
+//              last tile of a sequence: rows past its length never reach an
+//              MMA, so a NaN or Inf stored there cannot leak through P = 0)
+//   warp 1     TMEM allocation, single-thread tcgen05.mma issue and commits
+//   warps 2-5  softmax over the S accumulator (one TMEM lane = one token),
+//              conditional rescale of Z, P written to shared memory, and the
+//              per-segment epilogue (partials m, l, z to global memory)
+//
+// Precision: the absorbed query enters the MMA as hi + lo 16-bit parts and,
+// for bf16 latents, P does too (two accumulating MMAs); accumulation is fp32.
+//
+// Online softmax keeps a per-head reference m; P = 2^(s - m) is written with
+// m fixed until some score exceeds m + 8, and only then is m raised and the Z
+// accumulator rescaled (exactly: the same m is reported with z and l).
+//
+// Every wait is bounded (2 s of globaltimer); on expiry the kernel records
+// QSVD_STATUS_TIMEOUT in the workspace status word, drains its own work in
+// flight (bounded), frees its TMEM and returns.
+#include <cuda.h>
+
+#include "internal.cuh"
+
+namespace qsvd {
+namespace {
+
+constexpr int kThreadsTc = 192;
+constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
+constexpr int kMaxSlots = 8;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
+
+// ------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `parity` to complete; false after kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  while (!mbar_try(bar, parity)) {
+    if (gtimer() - t0 > kWaitNs) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// Named barrier over the 128 softmax threads, OR-reduction of a predicate.
+__device__ __forceinline__ int group_or(int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred)
+      : "memory");
+  return r;
+}
+__device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// kind::f16 instruction descriptor: fp32 accumulate, A/B f16 or bf16.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a_mn, bool b_mn) {
+  return (1u << 4) | (uint32_t(bf16) << 7) | (uint32_t(bf16) << 10) | (uint32_t(a_mn) << 15) |
+         (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// --------------------------------------------------------------- schedule
+
+struct TileIter {
+  const int32_t* ts;
+  const int32_t* ln;
+  long long g, te;
+  int b;
+  __device__ void init(const int32_t* sched, int B, long long tb, long long te_) {
+    ts = sched;
+    ln = sched + B + 1;
+    g = tb;
+    te = te_;
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ts[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    while (ts[b + 1] <= g) ++b;
+  }
+  __device__ void next() {
+    ++g;
+    if (g < te)
+      while (ts[b + 1] <= g) ++b;
+  }
+  __device__ int t0() const { return int(g - ts[b]) * kTile; }
+  __device__ int nvalid() const { return min(kTile, ln[b] - t0()); }
+  __device__ bool first(long long tb) const { return g == tb || g == ts[b]; }
+  __device__ bool last() const { return g == te - 1 || g + 1 == ts[b + 1]; }
+};
+
+struct Smem {
+  uint8_t* slots;
+  uint8_t* pbuf;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* z_done;
+  uint64_t* drain;
+  float* red;            // [4][NP]
+  uint32_t* tmem_holder;
+  volatile int* abort_flag;
+};
+
+// A slot holds a 128-channel chunk of the latent tile (two 64-channel boxes)
+// and, for S items, the matching chunk of the absorbed query: QS parts of NP
+// rows per box (QS = 2: the query as a rounded 16-bit part plus its 16-bit
+// rounding residual, summed by the MMA into adjacent accumulator columns).
+template <int NP, int QS>
+__host__ __device__ constexpr int slot_bytes() { return 2 * kBoxBytes + 2 * QS * NP * 128; }
+template <int NP>
+__host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T buffer
+constexpr int kMiscBytes = 2048;
+
+// P buffers: 2 (double buffer) x PS parts (bf16: hi + lo) x pbuf_bytes.
+template <int NP, int QS, int PS>
+__device__ Smem carve(uint8_t* base, int nslot) {
+  Smem s;
+  s.slots = base;
+  s.pbuf = base + size_t(nslot) * slot_bytes<NP, QS>();
+  uint8_t* m = s.pbuf + 2 * PS * pbuf_bytes<NP>();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(m);
+  s.full = bars;
+  s.empty = bars + kMaxSlots;
+  s.s_full = bars + 2 * kMaxSlots;
+  s.p_full = s.s_full + 2;
+  s.z_done = s.p_full + 2;
+  s.drain = s.z_done + 2;
+  s.red = reinterpret_cast<float*>(m + 256);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(m + 256 + 4 * NP * 4);
+  s.abort_flag = reinterpret_cast<volatile int*>(m + 256 + 4 * NP * 4 + 16);
+  return s;
+}
+
+__device__ __forceinline__ void set_abort(const Smem& s, int32_t* status) {
+  *s.abort_flag = 1;
+  atomicOr(status, QSVD_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int NP, bool BF16, int QS, int PS>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_q,
+           const uint8_t* __restrict__ cache, const int32_t* __restrict__ sched,
+           float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
+           int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int nslot) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const Smem s = carve<NP, QS, PS>(base, nslot);
+  constexpr int SW = QS * NP;                 // S accumulator columns per buffer
+  constexpr int ZC0 = 2 * SW;                 // first Z column
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NC = r / 128;
+  const long long T = sched[B];
+  const long long tb = dev::split_begin(blockIdx.x, G, T);
+  const long long te = dev::split_begin(blockIdx.x + 1, G, T);
+  if (tb >= te) return;   // uniform across the CTA, before any barrier or TMEM use
+  const int n = int(te - tb);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nslot; ++i) {
+      mbar_init(saddr(&s.full[i]), 1);
+      mbar_init(saddr(&s.empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(saddr(&s.s_full[i]), 1);
+      mbar_init(saddr(&s.p_full[i]), 1);
+      mbar_init(saddr(&s.z_done[i]), 1);
+    }
+    mbar_init(saddr(s.drain), 1);
+    *s.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     saddr(s.tmem_holder))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s.tmem_holder;
+  const uint32_t p_base = saddr(s.pbuf);
+  const uint32_t slot_base0 = saddr(s.slots);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    TileIter cur, prev;   // cur: tile of the S items (i), prev: tile of the Z items (i - 1)
+    cur.init(sched, B, tb, te);
+    prev.init(sched, B, tb, te);
+    const size_t row_bytes = size_t(r) * 2;
+    long long k = 0;
+    bool ok = true;
+    for (int i = 0; i <= n && ok; ++i) {
+      for (int j = 0; j < NC && ok; ++j) {
+        for (int kind = 0; kind < 2 && ok; ++kind) {   // 0: S of tile i, 1: Z of tile i-1
+          if ((kind == 0 && i >= n) || (kind == 1 && i == 0)) continue;
+          const TileIter& it = kind == 0 ? cur : prev;
+          const int slot = int(k % nslot);
+          const uint32_t ph = uint32_t(k / nslot) & 1u;
+          if (!mbar_wait(saddr(&s.empty[slot]), ph ^ 1u)) { ok = false; break; }
+          const uint32_t dst = slot_base0 + uint32_t(slot) * slot_bytes<NP, QS>();
+          const uint32_t full = saddr(&s.full[slot]);
+          const int nv = it.nvalid(), t0 = it.t0(), b = it.b;
+          if (nv == kTile) {
+            if (lane == 0) {
+              mbar_expect_tx(full, kind == 0 ? uint32_t(slot_bytes<NP, QS>()) : uint32_t(2 * kBoxBytes));
+              const int row = b * max_len + t0;
+              tma_load_2d(dst, &tm_c, 128 * j, row, full);
+              tma_load_2d(dst + kBoxBytes, &tm_c, 128 * j + 64, row, full);
+              if (kind == 0) {
+#pragma unroll
+                for (int box = 0; box < 2; ++box)
+#pragma unroll
+                  for (int part = 0; part < QS; ++part)
+                    tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
+                                128 * j + 64 * box, 0, QS * b + part, full);
+              }
+            }
+          } else {
+            // ragged tile: rows >= nv are written as zeros
+            uint8_t* d = s.slots + size_t(slot) * slot_bytes<NP, QS>();
+            const uint8_t* src = cache + (size_t(b) * max_len + t0) * row_bytes + size_t(256) * j;
+            for (int idx = lane; idx < 2 * 128 * 8; idx += 32) {
+              const int box = idx >> 10, t = (idx >> 3) & 127, c = idx & 7;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (t < nv) v = *reinterpret_cast<const uint4*>(src + size_t(t) * row_bytes + box * 128 + c * 16);
+              *reinterpret_cast<uint4*>(d + box * kBoxBytes + t * 128 + ((c ^ (t & 7)) << 4)) = v;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              if (kind == 0) {
+                mbar_expect_tx(full, uint32_t(2 * QS * NP * 128));
+#pragma unroll
+                for (int box = 0; box < 2; ++box)
+#pragma unroll
+                  for (int part = 0; part < QS; ++part)
+                    tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
+                                128 * j + 64 * box, 0, QS * b + part, full);
+              } else {
+                mbar_arrive(full);
+              }
+            }
+          }
+          __syncwarp();
+          ++k;
+          if (*s.abort_flag) ok = false;
+        }
+      }
+      if (i < n) cur.next();
+      if (i >= 1) prev.next();
+    }
+    if (!ok) {
+      if (lane == 0) set_abort(s, status);
+      // drain: every issued load lands (bounded) before the CTA exits
+      for (long long kk = (k > nslot ? k - nslot : 0); kk < k; ++kk)
+        mbar_wait(saddr(&s.full[kk % nslot]), uint32_t(kk / nslot) & 1u);
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
+      const uint32_t id_z = idesc_f16(128, NP, BF16, true, false);
+      TileIter prev;
+      prev.init(sched, B, tb, te);
+      long long k = 0;
+      bool ok = true;
+      for (int i = 0; i <= n && ok; ++i) {
+        const int pi = i - 1;
+        const bool prev_first = i >= 1 ? prev.first(tb) : false;
+        for (int j = 0; j < NC && ok; ++j) {
+          for (int kind = 0; kind < 2 && ok; ++kind) {
+            if ((kind == 0 && i >= n) || (kind == 1 && i == 0)) continue;
+            const int slot = int(k % nslot);
+            if (!mbar_wait(saddr(&s.full[slot]), uint32_t(k / nslot) & 1u)) { ok = false; break; }
+            if (kind == 1 && j == 0) {
+              if (!mbar_wait(saddr(&s.p_full[pi & 1]), uint32_t(pi >> 1) & 1u)) { ok = false; break; }
+            }
+            tc_fence_after();
+            const uint32_t sb = slot_base0 + uint32_t(slot) * slot_bytes<NP, QS>();
+            if (kind == 0) {
+              const uint32_t d = tmem + uint32_t((i & 1) * SW);
+#pragma unroll
+              for (int box = 0; box < 2; ++box)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t a = sdesc(sb + box * kBoxBytes + kk * 32, 16, 1024);
+                  const uint64_t bd = sdesc(sb + 2 * kBoxBytes + box * SW * 128 + kk * 32, 16, 1024);
+                  tc_mma(d, a, bd, id_s, (j | box | kk) != 0);
+                }
+              tc_commit(saddr(&s.empty[slot]));
+              if (j == NC - 1) tc_commit(saddr(&s.s_full[i & 1]));
+            } else {
+              const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
+              const uint32_t pb = p_base + uint32_t((pi & 1) * PS * pbuf_bytes<NP>());
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = sdesc(sb + ks * 16 * 128, kBoxBytes, 1024);
+#pragma unroll
+                for (int part = 0; part < PS; ++part) {   // P = P_hi (+ P_lo for bf16)
+                  const uint64_t bd = sdesc(pb + part * pbuf_bytes<NP>() + (ks >> 2) * NP * 128 +
+                                            (ks & 3) * 32, 16, 1024);
+                  tc_mma(d, a, bd, id_z, (prev_first && ks == 0 && part == 0) ? 0u : 1u);
+                }
+              }
+              tc_commit(saddr(&s.empty[slot]));
+              if (j == NC - 1) tc_commit(saddr(&s.z_done[pi & 1]));
+            }
+            ++k;
+            if (*s.abort_flag) ok = false;
+          }
+        }
+        if (i >= 1) prev.next();
+      }
+      if (!ok) set_abort(s, status);
+      tc_commit(saddr(s.drain));
+      mbar_wait(saddr(s.drain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ softmax and epilogue
+    const int q = warp & 3;
+    const int t = 32 * q + lane;              // token row in the tile == TMEM lane
+    const uint32_t lane_off = uint32_t(32 * q) << 16;
+    float m_run[NP], l_part[NP];
+    TileIter it;
+    it.init(sched, B, tb, te);
+    for (int i = 0; i < n; ++i) {
+      const int pb = i & 1;
+      const bool first = it.first(tb), last = it.last();
+      const int nv = it.nvalid();
+      if (first) {
+#pragma unroll
+        for (int h = 0; h < NP; ++h) { m_run[h] = -INFINITY; l_part[h] = 0.f; }
+      }
+      int fail = !mbar_wait(saddr(&s.s_full[pb]), uint32_t(i >> 1) & 1u);
+      if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+      tc_fence_after();
+      float sv[NP];
+#pragma unroll
+      for (int c = 0; c < NP / 16; ++c) tmem_ld16(tmem + lane_off + uint32_t(pb * SW + 16 * c), sv + 16 * c);
+      if (QS == 2) {   // S = C (q_hi + q_lo)
+        float lo[NP];
+#pragma unroll
+        for (int c = 0; c < NP / 16; ++c)
+          tmem_ld16(tmem + lane_off + uint32_t(pb * SW + NP + 16 * c), lo + 16 * c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < NP; ++h) sv[h] += lo[h];
+      }
+      tmem_wait_ld();
+      const bool valid = t < nv;
+      int need = 0;
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        if (!valid) sv[h] = -INFINITY;
+        need |= sv[h] > m_run[h] + kRescaleLog2;
+      }
+      if (group_or(need)) {
+        // exact tile max per head over the 128 rows
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+          const float v = dev::warp_max(sv[h]);
+          if (lane == 0) s.red[q * NP + h] = v;
+        }
+        group_sync();
+        float alpha[NP];
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+          const float mt = fmaxf(fmaxf(s.red[h], s.red[NP + h]), fmaxf(s.red[2 * NP + h], s.red[3 * NP + h]));
+          const float mn = fmaxf(m_run[h], mt);
+          alpha[h] = exp2f(m_run[h] - mn);
+          m_run[h] = mn;
+          l_part[h] *= alpha[h];
+        }
+        group_sync();
+        if (!first) {
+          // Z of the previous tile must be complete before it is rescaled
+          fail = !mbar_wait(saddr(&s.z_done[(i - 1) & 1]), uint32_t((i - 1) >> 1) & 1u);
+          if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+          tc_fence_after();
+          for (int c = 0; c < NC; ++c) {
+#pragma unroll
+            for (int h16 = 0; h16 < NP / 16; ++h16) {
+              float z[16];
+              const uint32_t ta = tmem + lane_off + uint32_t(ZC0 + c * NP + 16 * h16);
+              tmem_ld16(ta, z);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) z[e] *= alpha[16 * h16 + e];
+              tmem_st16(ta, z);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      // P = 2^(s - m) as the B operand of the Z MMA: P^T, K-major, 128B swizzle
+      if (i >= 2) {
+        fail = !mbar_wait(saddr(&s.z_done[pb]), uint32_t((i - 2) >> 1) & 1u);
+        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+      }
+      uint8_t* pbase = s.pbuf + pb * PS * pbuf_bytes<NP>() + (t >> 6) * NP * 128;
+      const int chunk = (t & 63) >> 3, within = (t & 7) * 2;
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        const float p = valid ? exp2f(sv[h] - m_run[h]) : 0.f;
+        l_part[h] += p;
+        uint8_t* dst = pbase + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
+        if (PS == 2) {
+          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+          *reinterpret_cast<__nv_bfloat16*>(dst) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(dst + pbuf_bytes<NP>()) =
+              __float2bfloat16_rn(p - __bfloat162float(hi));
+        } else {
+          *reinterpret_cast<__half*>(dst) = __float2half_rn(p);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      group_sync();
+      if (t == 0) mbar_arrive(saddr(&s.p_full[pb]));
+      if (last) {
+        fail = !mbar_wait(saddr(&s.z_done[pb]), uint32_t(i >> 1) & 1u);
+        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+        tc_fence_after();
+        const size_t slot = size_t(blockIdx.x) + it.b;
+        for (int c = 0; c < NC; ++c) {
+#pragma unroll
+          for (int h16 = 0; h16 < NP / 16; ++h16) {
+            float z[16];
+            tmem_ld16(tmem + lane_off + uint32_t(ZC0 + c * NP + 16 * h16), z);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int h = 16 * h16 + e;
+              if (h < H) pz[(slot * H + h) * r + 128 * c + t] = z[e];
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+          const float v = dev::warp_sum(l_part[h]);
+          if (lane == 0) s.red[q * NP + h] = v;
+        }
+        group_sync();
+        if (t < H && t < NP) {
+          pl[slot * H + t] = s.red[t] + s.red[NP + t] + s.red[2 * NP + t] + s.red[3 * NP + t];
+          pm[slot * H + t] = m_run[t];
+        }
+        group_sync();
+      }
+      it.next();
+      if (group_or(*s.abort_flag)) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+template <int NP, int QS, int PS>
+int nslots_for() {
+  int ns = (232448 - 1024 - 2 * PS * pbuf_bytes<NP>() - kMiscBytes) / slot_bytes<NP, QS>();
+  return ns > kMaxSlots ? kMaxSlots : ns;
+}
+
+template <int NP, bool BF16>
+cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
+                     const int32_t* sched, int G, float* pm, float* pl, float* pz,
+                     int32_t* status, cudaStream_t s) {
+  EncodeTiled enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tc, tq;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(d.r), cuuint64_t(d.batch) * d.max_len};
+    const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tc, dt, 2, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // query parts: qt16 holds [B][2][H][r] (hi, then the rounding residual)
+    constexpr int QS = 2;
+    const cuuint64_t dims[3] = {cuuint64_t(d.r), cuuint64_t(d.H), cuuint64_t(d.batch) * QS};
+    const cuuint64_t strides[2] = {cuuint64_t(d.r) * 2, cuuint64_t(d.H) * d.r * 2};
+    const cuuint32_t box[3] = {64, cuuint32_t(NP), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, dt, 3, const_cast<void*>(qt16), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
+  constexpr int PS = BF16 ? 2 : 1;   // P as hi + lo parts for bf16 (8-bit mantissa)
+  const int nslot = nslots_for<NP, QS, PS>();
+  const size_t smem = 1024 + size_t(nslot) * slot_bytes<NP, QS>() + 2 * PS * pbuf_bytes<NP>() + kMiscBytes;
+  auto kern = k_split_tc<NP, BF16, QS, PS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<G, kThreadsTc, smem, s>>>(tc, tq, static_cast<const uint8_t*>(cache), sched, pm, pl, pz,
+                                   status, d.batch, d.H, d.r, d.max_len, G, nslot);
+  note_launch();
+  return check_launch();
+}
+
+}  // namespace
+
+int split_tc_heads_padded(const qsvd_dims& d) { return d.H <= 16 ? 16 : (d.H <= 32 ? 32 : 0); }
+
+bool split_tc_supported(const qsvd_dims& d) {
+  if (d.rope) return false;
+  if (d.cache_dtype != QSVD_F16 && d.cache_dtype != QSVD_BF16) return false;
+  if (d.r % 128) return false;
+  const int np = split_tc_heads_padded(d);
+  if (np == 0) return false;
+  if ((2 * 2 + d.r / 128) * np > 512) return false;   // two S buffers of 2 np + Z
+  return true;
+}
+
+cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* qt16,
+                            const int32_t* sched, int G, float* pm, float* pl, float* pz,
+                            int32_t* status, cudaStream_t s) {
+  const bool bf = d.cache_dtype == QSVD_BF16;
+  const int np = split_tc_heads_padded(d);
+  if (np == 16) return bf ? launch_t<16, true>(d, cache, qt16, sched, G, pm, pl, pz, status, s)
+                          : launch_t<16, false>(d, cache, qt16, sched, G, pm, pl, pz, status, s);
+  return bf ? launch_t<32, true>(d, cache, qt16, sched, G, pm, pl, pz, status, s)
+            : launch_t<32, false>(d, cache, qt16, sched, G, pm, pl, pz, status, s);
+}
+
+}  // namespace qsvd

@@ -1,0 +1,115 @@
+"""Parity of the tensor-core split kernel (tcgen05 + TMA, absorbed query,
+fp16/bf16 latent) against the fp64 oracle and against the CUDA-core kernel.
+
+Bar: max |o_gpu - o_ref| / rms(o_ref) <= 2e-3 (P and the absorbed query are
+rounded to the latent's 16-bit type before the MMA; accumulation is fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import rank_joint_qkv_b200 as q
+import synthetic
+from oracle import inputs as oi
+from tests.gpu_util import GpuCase, rel_err
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+TC = q.QSVD_KERNEL_TCGEN05
+
+_CASES = {}
+
+
+def case(key):
+    if key not in _CASES:
+        base = synthetic.SHRUNK[1]   # E=512, H=4, r=256, B=3, L=300 (ragged tail)
+        w = {
+            "f16": base,
+            "bf16": synthetic.replace(base, cache="bf16", weight="bf16"),
+            "h32": synthetic.replace(base, E=4096, H=32, r=384, B=2, L=520),
+            "r768": synthetic.replace(base, E=1024, H=8, r=768, B=2, L=700),
+            "full": synthetic.replace(base, B=2, L=512),       # whole tiles only
+        }[key]
+        if w.E > 1024:
+            # direct seeded factors: skips the E x 3E SVD, which decode parity does not need
+            wuq, wuk, wuv = (a.astype(np.float64) for a in synthetic.direct_up_weights_np(w))
+            wd = synthetic.direct_down_weight_np(w).astype(np.float64)
+            _CASES[key] = oi.build_case(w, factors_override=(0.5, (wd, wuq, wuk, wuv), None))
+        else:
+            _CASES[key] = oi.build_case(w)
+    return _CASES[key]
+
+
+@pytest.mark.parametrize("key", ["full", "f16", "bf16", "h32", "r768"])
+def test_tc_matches_oracle(cuda_ok, key):
+    c = case(key)
+    g = GpuCase(c, kernel=TC)
+    got, ws = g.decode()
+    assert q.status_word(ws) == 0
+    err = rel_err(got, c.reference())
+    assert err <= TOL, f"{key}: {err:.3e}"
+
+
+@pytest.mark.parametrize("key", ["f16", "bf16"])
+def test_tc_agrees_with_simt(cuda_ok, key):
+    c = case(key)
+    a, _ = GpuCase(c, kernel=TC).decode()
+    b, _ = GpuCase(c, kernel=q.QSVD_KERNEL_SIMT).decode()
+    assert rel_err(a, b) <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 1000])
+def test_tc_split_invariance(cuda_ok, splits):
+    c = case("h32")
+    g = GpuCase(c, kernel=TC)
+    base, _ = g.decode(num_splits=1)
+    got, ws = g.decode(num_splits=splits)
+    assert q.status_word(ws) == 0
+    # each split rounds P = 2^(s - m_split) to fp16 against its own reference
+    # max, so split counts differ at the level of fp16 rounding (2^-11)
+    assert rel_err(got, base) <= 1e-3
+    assert rel_err(got, c.reference()) <= TOL
+
+
+@pytest.mark.parametrize("lens", [[1, 0, 2], [127, 128, 129], [255, 256, 257], [300, 1, 300]])
+def test_tc_edge_lengths(cuda_ok, lens):
+    w = synthetic.replace(synthetic.SHRUNK[1], B=len(lens), ragged=None, L=max(lens))
+    c = oi.build_case(w, lengths=np.array(lens, np.int32))
+    got, ws = GpuCase(c, kernel=TC).decode(num_splits=2)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(got[b] == 0.0)
+    assert rel_err(got, c.reference()) <= TOL
+    assert q.status_word(ws) == 0
+
+
+def test_tc_nan_padding_rows(cuda_ok):
+    """NaN in rows past each length (ragged tiles are zero-filled on load)."""
+    c = case("f16")
+    g = GpuCase(c, kernel=TC)
+    for b, n in enumerate(c.lengths):
+        g.cache[b, int(n):] = float("nan")
+    got, _ = g.decode(num_splits=4)
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, c.reference()) <= TOL
+
+
+def test_tc_large_score_range_rescales(cuda_ok):
+    """Scores spanning far more than 2^8 between tiles force the conditional
+    rescale of the latent accumulator."""
+    c = case("full")
+    g = GpuCase(c, kernel=TC)
+    # grow the latent along the sequence: later tiles dominate the softmax
+    caches, lens = [], c.lengths
+    w = c.w
+    for b in range(w.B):
+        n = int(lens[b])
+        ramp = np.linspace(0.2, 3.0, n)[:, None]
+        vals = c.caches[b] * ramp
+        dev = oi.to_device_dtype(vals, w.cache)
+        g.cache[b, :n] = oi.as_torch(dev, w.cache).to("cuda")
+        caches.append(oi.from_device_dtype(dev, w.cache))
+    c2 = oi.Case(**{**c.__dict__, "caches": caches})
+    got, ws = g.decode(num_splits=1)
+    assert q.status_word(ws) == 0
+    assert rel_err(got, c2.reference()) <= TOL

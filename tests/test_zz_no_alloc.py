@@ -77,8 +77,8 @@ def test_static_append_matches_workspace_append(cuda_ok, cache_dtype):
 
 
 def test_static_append_rejects_oversize_requests():
-    """ksplit(4096) = 8; 8 * 128 * 1536 floats > the 1,048,576-float scratch."""
-    dims = q.make_dims(4096, 32, 128, 1536, 128, 16, cache="f16", weight="f16")
+    """batch 512, r 4096: even ksplit = 1 needs 2,097,152 floats > 1,048,576."""
+    dims = q.make_dims(4096, 32, 128, 4096, 512, 16, cache="f16", weight="f16")
     lib = ctypes.CDLL(q.LIB_PATH)
     lib.qsvd_append_latent_static.argtypes = q._sigs["qsvd_append_latent_static"]
     lib.qsvd_append_latent_static.restype = ctypes.c_int
