@@ -237,7 +237,7 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     // q = c_new W^u_q (reduced into the workspace), or the query as given
     const float* qsrc = qin;
     if (qin_is_latent) {
-      if ((e = launch_q_partial(d, qin, P + L.wuq, qpart, W.KS, q, tickets, s)) != cudaSuccess)
+      if ((e = launch_q_partial(d, qin, P + L.wuq, qpart, W.KS, q, tickets, &hdr->status, s)) != cudaSuccess)
         return cuda_fail(e, "query projection");
       qsrc = q;
     }

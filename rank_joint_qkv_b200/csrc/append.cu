@@ -57,11 +57,8 @@ k_append_finish(const float* __restrict__ cpart, int KS, const float* __restrict
   __shared__ float qm[256];
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int j = threadIdx.x; j < r; j += 256) {
-    float s = 0.f;
-    for (int k = 0; k < KS; ++k) s += cpart[(size_t(k) * B + b) * r + j];
-    v[j] = s;
-  }
+  for (int j = threadIdx.x; j < r; j += 256)
+    v[j] = dev::sum_strided(cpart + size_t(b) * r + j, size_t(B) * r, KS);
   if (use_h2) {
     for (int i = threadIdx.x; i < h2_m * h2_m; i += 256) qm[i] = h2q[i];
   }
@@ -132,8 +129,7 @@ k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restric
   const int b = blockIdx.x;
   const int j = blockIdx.y * chunk + threadIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float v = 0.f;
-  for (int k = 0; k < KS; ++k) v += cpart[(size_t(k) * B + b) * r + j];
+  const float v = dev::sum_strided(cpart + size_t(b) * r + j, size_t(B) * r, KS);
   if (c_out) c_out[size_t(b) * r + j] = v;
   const int p = pos[b];
   if (p < 0 || p >= max_len) {
@@ -178,11 +174,14 @@ k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restric
 
 template <typename WT>
 cudaError_t gemv_t(const qsvd_dims& d, const void* x, const void* wd, float* cpart, int KS,
-                   cudaStream_t s) {
+                   int32_t* status, cudaStream_t s) {
+  auto kern = k_gemv_partial<WT, WT>;
+  const size_t smem = gemv_smem<WT>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
   dim3 grid((d.r + 255) / 256, KS, (d.batch + 15) / 16);
-  k_gemv_partial<WT, WT><<<grid, 256, 0, s>>>(static_cast<const WT*>(x),
-                                              static_cast<const WT*>(wd), cpart, d.batch,
-                                              d.E, d.r, KS, nullptr, nullptr);
+  kern<<<grid, 256, smem, s>>>(static_cast<const WT*>(x), static_cast<const WT*>(wd), cpart,
+                               d.batch, d.E, d.r, KS, nullptr, nullptr, status);
   note_launch();
   return check_launch();
 }
@@ -220,7 +219,7 @@ cudaError_t finish_t(const qsvd_dims& d, const float* cpart, int KS, const float
 
 }  // namespace
 
-int append_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.E, d.r, d.batch, 16); }
+int append_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.E, d.weight_dtype); }
 
 cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
                           const float* h2q, float h2_scale, const int32_t* pos,
@@ -228,9 +227,9 @@ cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
                           int KS, int32_t* status, cudaStream_t s) {
   cudaError_t e;
   switch (d.weight_dtype) {
-    case QSVD_F32: e = gemv_t<float>(d, x, wd, cpart, KS, s); break;
-    case QSVD_F16: e = gemv_t<__half>(d, x, wd, cpart, KS, s); break;
-    case QSVD_BF16: e = gemv_t<__nv_bfloat16>(d, x, wd, cpart, KS, s); break;
+    case QSVD_F32: e = gemv_t<float>(d, x, wd, cpart, KS, status, s); break;
+    case QSVD_F16: e = gemv_t<__half>(d, x, wd, cpart, KS, status, s); break;
+    case QSVD_BF16: e = gemv_t<__nv_bfloat16>(d, x, wd, cpart, KS, status, s); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

@@ -61,7 +61,7 @@ extern "C" qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const vo
   const size_t need = size_t(KS) * d.batch * d.r;
   if (need > kStaticScratchFloats)
     return set_error(QSVD_ERR_WORKSPACE,
-                     "qsvd_append_latent_static: ksplit(E) * batch * r exceeds the "
+                     "qsvd_append_latent_static: ceil(E / 128) * batch * r exceeds the "
                      "1048576-float static scratch; use qsvd_append_latent with a workspace");
   if (!packed || !x || !pos || !cache)
     return set_error(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");

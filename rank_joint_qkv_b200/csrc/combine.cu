@@ -126,9 +126,16 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
       float z = 0.f;
       if (bb < bn && jj < jn) {
         const int c0 = seg[2 * b], c1 = seg[2 * b + 1];
-        for (int c = c0; c <= c1; ++c) {
-          const float w = wt[c + b];
-          if (w != 0.f) z = fmaf(w, pz[((size_t(c) + b) * H + h) * r + j0 + jj], z);
+        // loads in batches of 8 so that they are in flight together
+        for (int cb = c0; cb <= c1; cb += 8) {
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            v[i] = (cb + i <= c1 && wt[cb + i + b] != 0.f)
+                       ? __ldcg(pz + ((size_t(cb + i) + b) * H + h) * r + j0 + jj) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (cb + i <= c1) z = fmaf(wt[cb + i + b], v[i], z);
         }
       }
       zs[bb * kJ + jj] = z;
@@ -173,9 +180,7 @@ __global__ void __launch_bounds__(256)
 k_combine_out(const float* __restrict__ opart, int JS, OT* __restrict__ out, size_t n) {
   const size_t i = size_t(blockIdx.x) * 256 + threadIdx.x;
   if (i >= n) return;
-  float s = 0.f;
-  for (int k = 0; k < JS; ++k) s += opart[size_t(k) * n + i];
-  out[i] = dev::from_f<OT>(s);
+  out[i] = dev::from_f<OT>(dev::sum_strided(opart + i, n, JS));
 }
 
 template <typename WT>

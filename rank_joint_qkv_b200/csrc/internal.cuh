@@ -125,7 +125,8 @@ cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, i
                             WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,
                             cudaStream_t s);
 cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
-                             float* qpart, int KS, float* q, int32_t* tickets, cudaStream_t s);
+                             float* qpart, int KS, float* q, int32_t* tickets, int32_t* status,
+                             cudaStream_t s);
 cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale_log2,
                           float* qt32, void* qt16, cudaStream_t s);
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
@@ -193,6 +194,22 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// sum_{k < n} p[k * stride] in order k = 0, 1, ..., with the loads issued in
+// batches of 8 so that they are in flight together (L2 path, no L1).
+__device__ __forceinline__ float sum_strided(const float* p, size_t stride, int n) {
+  float s = 0.f;
+  int k = 0;
+  for (; k + 8 <= n; k += 8) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __ldcg(p + size_t(k + i) * stride);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += v[i];
+  }
+  for (; k < n; ++k) s += __ldcg(p + size_t(k) * stride);
+  return s;
 }
 
 // Number of tiles of a sequence of n tokens.

@@ -179,10 +179,14 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
 
 template <typename WT>
 cudaError_t q_partial_t(const qsvd_dims& d, const float* qin, const void* wuq, float* qpart,
-                        int KS, float* q, int32_t* tickets, cudaStream_t s) {
+                        int KS, float* q, int32_t* tickets, int32_t* status, cudaStream_t s) {
+  auto kern = k_gemv_partial<float, WT>;
+  const size_t smem = gemv_smem<WT>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
   dim3 grid((d.E + 255) / 256, KS, (d.batch + 15) / 16);
-  k_gemv_partial<float, WT><<<grid, 256, 0, s>>>(qin, static_cast<const WT*>(wuq), qpart,
-                                                 d.batch, d.r, d.E, KS, q, tickets);
+  kern<<<grid, 256, smem, s>>>(qin, static_cast<const WT*>(wuq), qpart, d.batch, d.r, d.E, KS,
+                               q, tickets, status);
   note_launch();
   return check_launch();
 }
@@ -203,7 +207,7 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float 
 
 }  // namespace
 
-int prologue_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.r, d.E, d.batch, 32); }
+int prologue_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.r, d.weight_dtype); }
 int prologue_tickets(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch); }
 
 cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
@@ -216,11 +220,12 @@ cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, i
 }
 
 cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
-                             float* qpart, int KS, float* q, int32_t* tickets, cudaStream_t s) {
+                             float* qpart, int KS, float* q, int32_t* tickets, int32_t* status,
+                             cudaStream_t s) {
   switch (d.weight_dtype) {
-    case QSVD_F32: return q_partial_t<float>(d, qin, wuq, qpart, KS, q, tickets, s);
-    case QSVD_F16: return q_partial_t<__half>(d, qin, wuq, qpart, KS, q, tickets, s);
-    case QSVD_BF16: return q_partial_t<__nv_bfloat16>(d, qin, wuq, qpart, KS, q, tickets, s);
+    case QSVD_F32: return q_partial_t<float>(d, qin, wuq, qpart, KS, q, tickets, status, s);
+    case QSVD_F16: return q_partial_t<__half>(d, qin, wuq, qpart, KS, q, tickets, status, s);
+    case QSVD_BF16: return q_partial_t<__nv_bfloat16>(d, qin, wuq, qpart, KS, q, tickets, status, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -102,6 +102,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// Same, with an L2 eviction-priority policy (createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x,
+                                                 int y, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             int z, uint32_t bar) {
   asm volatile(
@@ -321,6 +340,10 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
     cur.init(sched, B, tb, te);
     prev.init(sched, B, tb, te);
     const size_t row_bytes = size_t(r) * 2;
+    // L2 policy: a chunk read for S is read once more for Z a tile later, so
+    // keep it (evict_last); after the Z read it is dead (evict_first).
+    const uint64_t pol_keep = policy_evict_last();
+    const uint64_t pol_drop = policy_evict_first();
     long long k = 0;
     bool ok = true;
     for (int i = 0; i <= n && ok; ++i) {
@@ -338,8 +361,9 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
             if (lane == 0) {
               mbar_expect_tx(full, kind == 0 ? uint32_t(slot_bytes<NP, QS>()) : uint32_t(2 * kBoxBytes));
               const int row = b * max_len + t0;
-              tma_load_2d(dst, &tm_c, 128 * j, row, full);
-              tma_load_2d(dst + kBoxBytes, &tm_c, 128 * j + 64, row, full);
+              const uint64_t pol = kind == 0 ? pol_keep : pol_drop;
+              tma_load_2d_hint(dst, &tm_c, 128 * j, row, full, pol);
+              tma_load_2d_hint(dst + kBoxBytes, &tm_c, 128 * j + 64, row, full, pol);
               if (kind == 0) {
 #pragma unroll
                 for (int box = 0; box < 2; ++box)
