@@ -184,6 +184,20 @@ def profiled_traffic(kernel_name: str, workload: str, src_files):
     return float(e["dram_bytes_per_launch"])
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """Max of a per-rank scalar over the process group (no-op for one rank)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_step_per_rank * steps * world / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
@@ -262,12 +276,9 @@ def run_ours(args, rank, world, local_rank):
                 for k, name in enumerate(("append", "prologue", "split", "combine"))}
     split_ms = [e[2].elapsed_time(e[3]) for e in ev]
     kernel_used = int(dec_ws[12:16].view(torch.int32).item())   # workspace header: kernel
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, device, world)
     tokens_per_step = float(np.sum(lens))
-    value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+    value = whole_job_rate(tokens_per_step, args.steps, world, ms_max)
 
     # end to end through the public API with host buffers
     x_pin = inp["x_host"].pin_memory()
@@ -285,11 +296,8 @@ def run_ours(args, rank, world, local_rank):
         out_pin.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = tokens_per_step * ke * world / (float(e2e_t.item()) / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
+    e2e_value = whole_job_rate(tokens_per_step, ke, world, e2e_ms)
     h2d = x_pin.numel() * x_pin.element_size() + lens_pin.numel() * 4
     d2h = out_pin.numel() * 4
 
