@@ -358,19 +358,23 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
           const uint32_t full = saddr(&s.full[slot]);
           const int nv = it.nvalid(), t0 = it.t0(), b = it.b;
           if (nv == kTile) {
-            if (lane == 0) {
+            // TMA operations issued by one thread are processed in order, so
+            // each operation of the item goes out from a different lane (the
+            // lanes rotate between items); lane 0 first posts the byte count.
+            if (lane == 0)
               mbar_expect_tx(full, kind == 0 ? uint32_t(slot_bytes<NP, QS>()) : uint32_t(2 * kBoxBytes));
+            __syncwarp();
+            const int op = (lane - int(8 * (k & 3))) & 31;      // this lane's operation index
+            const int nops = kind == 0 ? 2 + 2 * QS : 2;
+            if (op < nops) {
               const int row = b * max_len + t0;
-              const uint64_t pol = kind == 0 ? pol_keep : pol_drop;
-              tma_load_2d_hint(dst, &tm_c, 128 * j, row, full, pol);
-              tma_load_2d_hint(dst + kBoxBytes, &tm_c, 128 * j + 64, row, full, pol);
-              if (kind == 0) {
-#pragma unroll
-                for (int box = 0; box < 2; ++box)
-#pragma unroll
-                  for (int part = 0; part < QS; ++part)
-                    tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
-                                128 * j + 64 * box, 0, QS * b + part, full);
+              if (op < 2) {
+                tma_load_2d_hint(dst + op * kBoxBytes, &tm_c, 128 * j + 64 * op, row, full,
+                                 kind == 0 ? pol_keep : pol_drop);
+              } else {
+                const int box = (op - 2) / QS, part = (op - 2) % QS;
+                tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
+                            128 * j + 64 * box, 0, QS * b + part, full);
               }
             }
           } else {
@@ -386,17 +390,14 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
-              if (kind == 0) {
-                mbar_expect_tx(full, uint32_t(2 * QS * NP * 128));
-#pragma unroll
-                for (int box = 0; box < 2; ++box)
-#pragma unroll
-                  for (int part = 0; part < QS; ++part)
-                    tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
-                                128 * j + 64 * box, 0, QS * b + part, full);
-              } else {
-                mbar_arrive(full);
-              }
+              if (kind == 0) mbar_expect_tx(full, uint32_t(2 * QS * NP * 128));
+              else mbar_arrive(full);
+            }
+            __syncwarp();
+            if (kind == 0 && lane < 2 * QS) {
+              const int box = lane / QS, part = lane % QS;
+              tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
+                          128 * j + 64 * box, 0, QS * b + part, full);
             }
           }
           __syncwarp();
