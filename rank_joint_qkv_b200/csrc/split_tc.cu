@@ -13,15 +13,26 @@
 // 128-channel chunks -- once for S (from HBM, together with the matching
 // chunk of the absorbed query Qt) and once for Z (re-read from L2 a fraction
 // of a tile later) -- because a whole tile (128 x r x 2 bytes) does not fit in
-// shared memory.  The two streams are interleaved (S of tile i+1 with Z of
-// tile i) so the HBM stream never waits for the softmax.
+// shared memory.
 //
-// Roles (192 threads):
-//   warp 0     TMA producer (full tiles) / manual zero-filled loads (ragged
-//              last tile of a sequence: rows past its length never reach an
-//              MMA, so a NaN or Inf stored there cannot leak through P = 0)
-//   warp 1     TMEM allocation, single-thread tcgen05.mma issue and commits
-//   warps 2-5  softmax over the S accumulator (one TMEM lane = one token),
+// The two streams are independent pipelines, each with its own ring of
+// shared-memory slots, its own TMA producer warp and its own MMA-issuing
+// thread: a single thread issues one tcgen05.mma about every 100 cycles
+// whatever the shape, and the small-N MMAs of this kernel finish faster than
+// that, so two issuers keep the tensor core twice as busy as one.  Each
+// 128-channel chunk of the latent (two 64-channel swizzled boxes) arrives in
+// one 3D TMA operation, the matching query chunk (two boxes x hi/lo parts) in
+// one 4D operation.
+//
+// Roles (256 threads):
+//   warp 0     S producer: latent chunk + query chunk per slot (ragged last
+//              tile of a sequence: latent rows past its length are written as
+//              zeros by the warp, so a NaN or Inf stored there cannot leak
+//              through P = 0)
+//   warp 1     TMEM allocation; one thread issues the S MMAs
+//   warp 2     Z producer: latent chunk re-read per slot (same ragged rule)
+//   warp 3     one thread issues the Z MMAs
+//   warps 4-7  softmax over the S accumulator (one TMEM lane = one token),
 //              conditional rescale of Z, P written to shared memory, and the
 //              per-segment epilogue (partials m, l, z to global memory)
 //
@@ -42,9 +53,9 @@
 namespace qsvd {
 namespace {
 
-constexpr int kThreadsTc = 192;
+constexpr int kThreadsTc = 256;
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
-constexpr int kMaxSlots = 8;
+constexpr int kMaxSlots = 6;                   // per ring
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
@@ -94,23 +105,6 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// Same, with an L2 eviction-priority policy (createpolicy).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x,
-                                                 int y, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -121,12 +115,21 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            int z, uint32_t bar) {
+// 3D tiled load with an L2 eviction-priority policy (createpolicy).
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 int z, uint32_t bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -236,53 +239,152 @@ struct TileIter {
   __device__ bool last() const { return g == te - 1 || g + 1 == ts[b + 1]; }
 };
 
+// Shared-memory carve.  S ring slot: the latent chunk (two 64-channel boxes)
+// followed by the query chunk, QS parts of NP rows per box (QS = 2: the query
+// as a rounded 16-bit part plus its 16-bit rounding residual, summed by the
+// MMA into adjacent accumulator columns), laid out [box][part][row].  Z ring
+// slot: the latent chunk only.
+template <int NP, int QS>
+__host__ __device__ constexpr int s_slot_bytes() { return 2 * kBoxBytes + 2 * QS * NP * 128; }
+constexpr int kZSlotBytes = 2 * kBoxBytes;
+template <int NP>
+__host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T part
+constexpr int kMiscBytes = 2048;
+
 struct Smem {
-  uint8_t* slots;
+  uint8_t* sring;
+  uint8_t* zring;
   uint8_t* pbuf;
-  uint64_t* full;
-  uint64_t* empty;
-  uint64_t* s_full;
-  uint64_t* p_full;
-  uint64_t* z_done;
-  uint64_t* drain;
+  uint64_t* s_full;      // [kMaxSlots] S ring: data landed
+  uint64_t* s_empty;     // [kMaxSlots] S ring: MMAs done with the slot
+  uint64_t* z_full;      // [kMaxSlots]
+  uint64_t* z_empty;     // [kMaxSlots]
+  uint64_t* acc_full;    // [2] S accumulator of a tile complete
+  uint64_t* p_full;      // [2] P of a tile written (S accumulator read)
+  uint64_t* z_done;      // [2] Z MMAs of a tile complete
+  uint64_t* drain;       // [2] one per MMA issuer
   float* red;            // [4][NP]
   uint32_t* tmem_holder;
   volatile int* abort_flag;
 };
 
-// A slot holds a 128-channel chunk of the latent tile (two 64-channel boxes)
-// and, for S items, the matching chunk of the absorbed query: QS parts of NP
-// rows per box (QS = 2: the query as a rounded 16-bit part plus its 16-bit
-// rounding residual, summed by the MMA into adjacent accumulator columns).
-template <int NP, int QS>
-__host__ __device__ constexpr int slot_bytes() { return 2 * kBoxBytes + 2 * QS * NP * 128; }
-template <int NP>
-__host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T buffer
-constexpr int kMiscBytes = 2048;
-
 // P buffers: 2 (double buffer) x PS parts (bf16: hi + lo) x pbuf_bytes.
 template <int NP, int QS, int PS>
-__device__ Smem carve(uint8_t* base, int nslot) {
+__device__ Smem carve(uint8_t* base, int ns, int nz) {
   Smem s;
-  s.slots = base;
-  s.pbuf = base + size_t(nslot) * slot_bytes<NP, QS>();
+  s.sring = base;
+  s.zring = s.sring + size_t(ns) * s_slot_bytes<NP, QS>();
+  s.pbuf = s.zring + size_t(nz) * kZSlotBytes;
   uint8_t* m = s.pbuf + 2 * PS * pbuf_bytes<NP>();
   uint64_t* bars = reinterpret_cast<uint64_t*>(m);
-  s.full = bars;
-  s.empty = bars + kMaxSlots;
-  s.s_full = bars + 2 * kMaxSlots;
-  s.p_full = s.s_full + 2;
+  s.s_full = bars;
+  s.s_empty = bars + kMaxSlots;
+  s.z_full = bars + 2 * kMaxSlots;
+  s.z_empty = bars + 3 * kMaxSlots;
+  s.acc_full = bars + 4 * kMaxSlots;
+  s.p_full = s.acc_full + 2;
   s.z_done = s.p_full + 2;
   s.drain = s.z_done + 2;
-  s.red = reinterpret_cast<float*>(m + 256);
-  s.tmem_holder = reinterpret_cast<uint32_t*>(m + 256 + 4 * NP * 4);
-  s.abort_flag = reinterpret_cast<volatile int*>(m + 256 + 4 * NP * 4 + 16);
+  s.red = reinterpret_cast<float*>(m + 512);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(m + 512 + 4 * NP * 4);
+  s.abort_flag = reinterpret_cast<volatile int*>(m + 512 + 4 * NP * 4 + 16);
   return s;
 }
 
 __device__ __forceinline__ void set_abort(const Smem& s, int32_t* status) {
   *s.abort_flag = 1;
   atomicOr(status, QSVD_STATUS_TIMEOUT);
+}
+
+// Ring position: slot index and the parity of its current use.
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  int n;
+  __device__ explicit Ring(int n_) : n(n_) {}
+  __device__ void advance() {
+    if (++slot == n) { slot = 0; phase ^= 1u; }
+  }
+};
+
+// Zero-filled copy of a ragged latent chunk (rows >= nv) into a slot, by one
+// warp, in the 128-byte-swizzled layout TMA would have produced.
+__device__ __forceinline__ void ragged_chunk(uint8_t* d, const uint8_t* src, size_t row_bytes,
+                                             int nv, int lane) {
+  for (int idx = lane; idx < 2 * 128 * 8; idx += 32) {
+    const int box = idx >> 10, t = (idx >> 3) & 127, c = idx & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t < nv) v = *reinterpret_cast<const uint4*>(src + size_t(t) * row_bytes + box * 128 + c * 16);
+    *reinterpret_cast<uint4*>(d + box * kBoxBytes + t * 128 + ((c ^ (t & 7)) << 4)) = v;
+  }
+  fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
+  __syncwarp();
+}
+
+// Producer of one ring (warp-wide).  kind 0: S ring (latent from HBM, kept
+// in L2 for the Z re-read, plus the query chunk); kind 1: Z ring (latent
+// re-read, dropped from L2 after).  Returns false on a wait that expired.
+template <int NP, int QS>
+__device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_c, const CUtensorMap* tm_q,
+                        const uint8_t* cache, const int32_t* sched, int B, int r, int max_len,
+                        long long tb, long long te, int n, int nslots, int lane, long long* issued) {
+  const int NC = r / 128;
+  const size_t row_bytes = size_t(r) * 2;
+  uint8_t* ring = kind == 0 ? s.sring : s.zring;
+  const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
+  uint64_t* full = kind == 0 ? s.s_full : s.z_full;
+  uint64_t* empty = kind == 0 ? s.s_empty : s.z_empty;
+  const uint64_t policy = kind == 0 ? policy_evict_last() : policy_evict_first();
+  const uint32_t ring0 = saddr(ring);
+  TileIter it;
+  it.init(sched, B, tb, te);
+  Ring rg(nslots);
+  long long k = 0;
+  for (int i = 0; i < n; ++i) {
+    const int nv = it.nvalid(), b = it.b;
+    const int row = b * max_len + it.t0();
+    for (int j = 0; j < NC; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
+        *issued = k;
+        return false;
+      }
+      const uint32_t dst = ring0 + uint32_t(rg.slot) * slot_bytes;
+      const uint32_t fb = saddr(&full[rg.slot]);
+      if (nv == kTile) {
+        if (lane == 0) mbar_expect_tx(fb, slot_bytes);
+        __syncwarp();
+        // one operation per lane: TMA operations of one thread are processed in order
+        if (lane == 0) tma_load_3d_hint(dst, tm_c, 0, row, 2 * j, fb, policy);
+        if (kind == 0 && lane == 1) tma_load_4d(dst + 2 * kBoxBytes, tm_q, 0, 0, QS * b, 2 * j, fb);
+      } else {
+        ragged_chunk(ring + size_t(rg.slot) * slot_bytes,
+                     cache + (size_t(b) * max_len + it.t0()) * row_bytes + size_t(256) * j, row_bytes,
+                     nv, lane);
+        if (lane == 0) {
+          if (kind == 0) {
+            mbar_expect_tx(fb, uint32_t(2 * QS * NP * 128));
+            tma_load_4d(dst + 2 * kBoxBytes, tm_q, 0, 0, QS * b, 2 * j, fb);
+          } else {
+            mbar_arrive(fb);
+          }
+        }
+      }
+      __syncwarp();
+      rg.advance();
+      ++k;
+    }
+    it.next();
+    if (__any_sync(0xffffffffu, *s.abort_flag)) { *issued = k; return false; }
+  }
+  *issued = k;
+  return true;
+}
+
+// Wait (bounded) until the last `min(k, nslots)` loads of a ring have landed,
+// so that no copy is in flight when the CTA exits.
+__device__ void drain_ring(uint64_t* full, long long k, int nslots) {
+  for (long long kk = (k > nslots ? k - nslots : 0); kk < k; ++kk)
+    mbar_wait(saddr(&full[int(kk % nslots)]), uint32_t(kk / nslots) & 1u);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -292,11 +394,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_q,
            const uint8_t* __restrict__ cache, const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
-           int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int nslot) {
+           int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const Smem s = carve<NP, QS, PS>(base, nslot);
+  const Smem s = carve<NP, QS, PS>(base, ns, nz);
   constexpr int SW = QS * NP;                 // S accumulator columns per buffer
   constexpr int ZC0 = 2 * SW;                 // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -308,16 +410,20 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
   const int n = int(te - tb);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < nslot; ++i) {
-      mbar_init(saddr(&s.full[i]), 1);
-      mbar_init(saddr(&s.empty[i]), 1);
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(saddr(&s.s_full[i]), 1);
+      mbar_init(saddr(&s.s_empty[i]), 1);
+    }
+    for (int i = 0; i < nz; ++i) {
+      mbar_init(saddr(&s.z_full[i]), 1);
+      mbar_init(saddr(&s.z_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(saddr(&s.s_full[i]), 1);
+      mbar_init(saddr(&s.acc_full[i]), 1);
       mbar_init(saddr(&s.p_full[i]), 1);
       mbar_init(saddr(&s.z_done[i]), 1);
+      mbar_init(saddr(&s.drain[i]), 1);
     }
-    mbar_init(saddr(s.drain), 1);
     *s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -331,148 +437,96 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_holder;
-  const uint32_t p_base = saddr(s.pbuf);
-  const uint32_t slot_base0 = saddr(s.slots);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    TileIter cur, prev;   // cur: tile of the S items (i), prev: tile of the Z items (i - 1)
-    cur.init(sched, B, tb, te);
-    prev.init(sched, B, tb, te);
-    const size_t row_bytes = size_t(r) * 2;
-    // L2 policy: a chunk read for S is read once more for Z a tile later, so
-    // keep it (evict_last); after the Z read it is dead (evict_first).
-    const uint64_t pol_keep = policy_evict_last();
-    const uint64_t pol_drop = policy_evict_first();
-    long long k = 0;
-    bool ok = true;
-    for (int i = 0; i <= n && ok; ++i) {
-      for (int j = 0; j < NC && ok; ++j) {
-        for (int kind = 0; kind < 2 && ok; ++kind) {   // 0: S of tile i, 1: Z of tile i-1
-          if ((kind == 0 && i >= n) || (kind == 1 && i == 0)) continue;
-          const TileIter& it = kind == 0 ? cur : prev;
-          const int slot = int(k % nslot);
-          const uint32_t ph = uint32_t(k / nslot) & 1u;
-          if (!mbar_wait(saddr(&s.empty[slot]), ph ^ 1u)) { ok = false; break; }
-          const uint32_t dst = slot_base0 + uint32_t(slot) * slot_bytes<NP, QS>();
-          const uint32_t full = saddr(&s.full[slot]);
-          const int nv = it.nvalid(), t0 = it.t0(), b = it.b;
-          if (nv == kTile) {
-            // TMA operations issued by one thread are processed in order, so
-            // each operation of the item goes out from a different lane (the
-            // lanes rotate between items); lane 0 first posts the byte count.
-            if (lane == 0)
-              mbar_expect_tx(full, kind == 0 ? uint32_t(slot_bytes<NP, QS>()) : uint32_t(2 * kBoxBytes));
-            __syncwarp();
-            const int op = (lane - int(8 * (k & 3))) & 31;      // this lane's operation index
-            const int nops = kind == 0 ? 2 + 2 * QS : 2;
-            if (op < nops) {
-              const int row = b * max_len + t0;
-              if (op < 2) {
-                tma_load_2d_hint(dst + op * kBoxBytes, &tm_c, 128 * j + 64 * op, row, full,
-                                 kind == 0 ? pol_keep : pol_drop);
-              } else {
-                const int box = (op - 2) / QS, part = (op - 2) % QS;
-                tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
-                            128 * j + 64 * box, 0, QS * b + part, full);
-              }
-            }
-          } else {
-            // ragged tile: rows >= nv are written as zeros
-            uint8_t* d = s.slots + size_t(slot) * slot_bytes<NP, QS>();
-            const uint8_t* src = cache + (size_t(b) * max_len + t0) * row_bytes + size_t(256) * j;
-            for (int idx = lane; idx < 2 * 128 * 8; idx += 32) {
-              const int box = idx >> 10, t = (idx >> 3) & 127, c = idx & 7;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (t < nv) v = *reinterpret_cast<const uint4*>(src + size_t(t) * row_bytes + box * 128 + c * 16);
-              *reinterpret_cast<uint4*>(d + box * kBoxBytes + t * 128 + ((c ^ (t & 7)) << 4)) = v;
-            }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) {
-              if (kind == 0) mbar_expect_tx(full, uint32_t(2 * QS * NP * 128));
-              else mbar_arrive(full);
-            }
-            __syncwarp();
-            if (kind == 0 && lane < 2 * QS) {
-              const int box = lane / QS, part = lane % QS;
-              tma_load_3d(dst + 2 * kBoxBytes + (box * QS + part) * NP * 128, &tm_q,
-                          128 * j + 64 * box, 0, QS * b + part, full);
-            }
-          }
-          __syncwarp();
-          ++k;
-          if (*s.abort_flag) ok = false;
-        }
+  if (warp == 0 || warp == 2) {
+    // ----------------------------------------------------------- producers
+    const int kind = warp >> 1;
+    const int nslots = kind == 0 ? ns : nz;
+    long long issued = 0;
+    if (!produce<NP, QS>(kind, s, &tm_c, &tm_q, cache, sched, B, r, max_len, tb, te, n, nslots,
+                         lane, &issued)) {
+      if (lane == 0) {
+        set_abort(s, status);
+        drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
       }
-      if (i < n) cur.next();
-      if (i >= 1) prev.next();
     }
-    if (!ok) {
-      if (lane == 0) set_abort(s, status);
-      // drain: every issued load lands (bounded) before the CTA exits
-      for (long long kk = (k > nslot ? k - nslot : 0); kk < k; ++kk)
-        mbar_wait(saddr(&s.full[kk % nslot]), uint32_t(kk / nslot) & 1u);
-    }
+    __syncwarp();
   } else if (warp == 1) {
-    // --------------------------------------------------------------- MMA
+    // ----------------------------------------------------------- S MMAs
     if (lane == 0) {
-      const uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
-      const uint32_t id_z = idesc_f16(128, NP, BF16, true, false);
-      TileIter prev;
-      prev.init(sched, B, tb, te);
-      long long k = 0;
+      constexpr uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
+      const uint64_t da0 = sdesc(saddr(s.sring), 16, 1024);   // K-major, 128B swizzle
+      Ring rg(ns);
       bool ok = true;
-      for (int i = 0; i <= n && ok; ++i) {
-        const int pi = i - 1;
-        const bool prev_first = i >= 1 ? prev.first(tb) : false;
-        for (int j = 0; j < NC && ok; ++j) {
-          for (int kind = 0; kind < 2 && ok; ++kind) {
-            if ((kind == 0 && i >= n) || (kind == 1 && i == 0)) continue;
-            const int slot = int(k % nslot);
-            if (!mbar_wait(saddr(&s.full[slot]), uint32_t(k / nslot) & 1u)) { ok = false; break; }
-            if (kind == 1 && j == 0) {
-              if (!mbar_wait(saddr(&s.p_full[pi & 1]), uint32_t(pi >> 1) & 1u)) { ok = false; break; }
+      for (int i = 0; i < n && ok; ++i) {
+        // the accumulator buffer of tile i was last read by the softmax of tile i - 2
+        if (i >= 2 && !mbar_wait(saddr(&s.p_full[i & 1]), uint32_t((i - 2) >> 1) & 1u)) { ok = false; break; }
+        const uint32_t d = tmem + uint32_t((i & 1) * SW);
+        for (int j = 0; j < NC; ++j) {
+          if (!mbar_wait(saddr(&s.s_full[rg.slot]), rg.phase)) { ok = false; break; }
+          tc_fence_after();
+          // descriptor address field is in 16-byte units
+          const uint64_t sa = da0 + uint64_t((rg.slot * s_slot_bytes<NP, QS>()) >> 4);
+#pragma unroll
+          for (int box = 0; box < 2; ++box)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t a = sa + uint64_t((box * kBoxBytes + kk * 32) >> 4);
+              const uint64_t bd = sa + uint64_t((2 * kBoxBytes + box * SW * 128 + kk * 32) >> 4);
+              tc_mma(d, a, bd, id_s, (j | box | kk) != 0);
             }
-            tc_fence_after();
-            const uint32_t sb = slot_base0 + uint32_t(slot) * slot_bytes<NP, QS>();
-            if (kind == 0) {
-              const uint32_t d = tmem + uint32_t((i & 1) * SW);
-#pragma unroll
-              for (int box = 0; box < 2; ++box)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t a = sdesc(sb + box * kBoxBytes + kk * 32, 16, 1024);
-                  const uint64_t bd = sdesc(sb + 2 * kBoxBytes + box * SW * 128 + kk * 32, 16, 1024);
-                  tc_mma(d, a, bd, id_s, (j | box | kk) != 0);
-                }
-              tc_commit(saddr(&s.empty[slot]));
-              if (j == NC - 1) tc_commit(saddr(&s.s_full[i & 1]));
-            } else {
-              const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
-              const uint32_t pb = p_base + uint32_t((pi & 1) * PS * pbuf_bytes<NP>());
-#pragma unroll
-              for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a = sdesc(sb + ks * 16 * 128, kBoxBytes, 1024);
-#pragma unroll
-                for (int part = 0; part < PS; ++part) {   // P = P_hi (+ P_lo for bf16)
-                  const uint64_t bd = sdesc(pb + part * pbuf_bytes<NP>() + (ks >> 2) * NP * 128 +
-                                            (ks & 3) * 32, 16, 1024);
-                  tc_mma(d, a, bd, id_z, (prev_first && ks == 0 && part == 0) ? 0u : 1u);
-                }
-              }
-              tc_commit(saddr(&s.empty[slot]));
-              if (j == NC - 1) tc_commit(saddr(&s.z_done[pi & 1]));
-            }
-            ++k;
-            if (*s.abort_flag) ok = false;
-          }
+          tc_commit(saddr(&s.s_empty[rg.slot]));
+          rg.advance();
         }
-        if (i >= 1) prev.next();
+        if (!ok) break;
+        tc_commit(saddr(&s.acc_full[i & 1]));
+        if (*s.abort_flag) ok = false;
       }
       if (!ok) set_abort(s, status);
-      tc_commit(saddr(s.drain));
-      mbar_wait(saddr(s.drain), 0);
+      tc_commit(saddr(&s.drain[0]));
+      mbar_wait(saddr(&s.drain[0]), 0);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ----------------------------------------------------------- Z MMAs
+    if (lane == 0) {
+      constexpr uint32_t id_z = idesc_f16(128, NP, BF16, true, false);
+      const uint64_t za0 = sdesc(saddr(s.zring), kBoxBytes, 1024);   // MN-major C^T
+      const uint64_t pb0 = sdesc(saddr(s.pbuf), 16, 1024);            // P^T, K-major
+      TileIter it;
+      it.init(sched, B, tb, te);
+      Ring rg(nz);
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        const bool first = it.first(tb);
+        if (!mbar_wait(saddr(&s.p_full[i & 1]), uint32_t(i >> 1) & 1u)) { ok = false; break; }
+        const uint64_t pb = pb0 + uint64_t(((i & 1) * PS * pbuf_bytes<NP>()) >> 4);
+        for (int j = 0; j < NC; ++j) {
+          if (!mbar_wait(saddr(&s.z_full[rg.slot]), rg.phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
+          const uint64_t za = za0 + uint64_t((rg.slot * kZSlotBytes) >> 4);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t a = za + uint64_t((ks * 16 * 128) >> 4);
+#pragma unroll
+            for (int part = 0; part < PS; ++part) {   // P = P_hi (+ P_lo for bf16)
+              const uint64_t bd = pb + uint64_t((part * pbuf_bytes<NP>() + (ks >> 2) * NP * 128 +
+                                                 (ks & 3) * 32) >> 4);
+              tc_mma(d, a, bd, id_z, (first && ks == 0 && part == 0) ? 0u : 1u);
+            }
+          }
+          tc_commit(saddr(&s.z_empty[rg.slot]));
+          rg.advance();
+        }
+        if (!ok) break;
+        tc_commit(saddr(&s.z_done[i & 1]));
+        it.next();
+        if (*s.abort_flag) ok = false;
+      }
+      if (!ok) set_abort(s, status);
+      tc_commit(saddr(&s.drain[1]));
+      mbar_wait(saddr(&s.drain[1]), 0);
     }
     __syncwarp();
   } else {
@@ -491,7 +545,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
 #pragma unroll
         for (int h = 0; h < NP; ++h) { m_run[h] = -INFINITY; l_part[h] = 0.f; }
       }
-      int fail = !mbar_wait(saddr(&s.s_full[pb]), uint32_t(i >> 1) & 1u);
+      int fail = !mbar_wait(saddr(&s.acc_full[pb]), uint32_t(i >> 1) & 1u);
       if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
       tc_fence_after();
       float sv[NP];
@@ -639,10 +693,18 @@ EncodeTiled get_encode() {
   return fn;
 }
 
+constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
+
+// Slots per ring: as many S slots as fit while the Z ring keeps two.
 template <int NP, int QS, int PS>
-int nslots_for() {
-  int ns = (232448 - 1024 - 2 * PS * pbuf_bytes<NP>() - kMiscBytes) / slot_bytes<NP, QS>();
-  return ns > kMaxSlots ? kMaxSlots : ns;
+void ring_slots(int* ns, int* nz) {
+  const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
+  int s = (avail - 2 * kZSlotBytes) / s_slot_bytes<NP, QS>();
+  if (s > kMaxSlots) s = kMaxSlots;
+  int z = (avail - s * s_slot_bytes<NP, QS>()) / kZSlotBytes;
+  if (z > kMaxSlots) z = kMaxSlots;
+  *ns = s;
+  *nz = z;
 }
 
 template <int NP, bool BF16>
@@ -651,39 +713,46 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
                      int32_t* status, cudaStream_t s) {
   EncodeTiled enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
+  constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
+  constexpr int PS = BF16 ? 2 : 1;   // P as hi + lo parts for bf16 (8-bit mantissa)
   const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tc, tq;
   {
-    const cuuint64_t dims[2] = {cuuint64_t(d.r), cuuint64_t(d.batch) * d.max_len};
-    const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
-    const cuuint32_t box[2] = {64, 128};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tc, dt, 2, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    // latent rows [B * max_len][r] seen as {64 channels, row, 64-channel box}:
+    // one box {64, 128, 2} is a 128-token x 128-channel chunk, smem [box][row][64]
+    const cuuint64_t dims[3] = {64, cuuint64_t(d.batch) * d.max_len, cuuint64_t(d.r / 64)};
+    const cuuint64_t strides[2] = {cuuint64_t(d.r) * 2, 128};
+    const cuuint32_t box[3] = {64, 128, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tc, dt, 3, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
-    // query parts: qt16 holds [B][2][H][r] (hi, then the rounding residual)
-    constexpr int QS = 2;
-    const cuuint64_t dims[3] = {cuuint64_t(d.r), cuuint64_t(d.H), cuuint64_t(d.batch) * QS};
-    const cuuint64_t strides[2] = {cuuint64_t(d.r) * 2, cuuint64_t(d.H) * d.r * 2};
-    const cuuint32_t box[3] = {64, cuuint32_t(NP), 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    if (enc(&tq, dt, 3, const_cast<void*>(qt16), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    // query parts: qt16 holds [B][QS][H][r] (hi, then the rounding residual),
+    // seen as {64 channels, head, sequence * part, 64-channel box}; one box
+    // {64, NP, QS, 2} lands as smem [box][part][head][64].  Heads H..NP-1 are
+    // outside the map and arrive as zeros.
+    const cuuint64_t dims[4] = {64, cuuint64_t(d.H), cuuint64_t(d.batch) * QS, cuuint64_t(d.r / 64)};
+    const cuuint64_t strides[3] = {cuuint64_t(d.r) * 2, cuuint64_t(d.H) * d.r * 2, 128};
+    const cuuint32_t box[4] = {64, cuuint32_t(NP), QS, 2};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    if (enc(&tq, dt, 4, const_cast<void*>(qt16), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
-  constexpr int PS = BF16 ? 2 : 1;   // P as hi + lo parts for bf16 (8-bit mantissa)
-  const int nslot = nslots_for<NP, QS, PS>();
-  const size_t smem = 1024 + size_t(nslot) * slot_bytes<NP, QS>() + 2 * PS * pbuf_bytes<NP>() + kMiscBytes;
+  int ns = 0, nz = 0;
+  ring_slots<NP, QS, PS>(&ns, &nz);
+  if (ns < 2 || nz < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = 1024 + size_t(ns) * s_slot_bytes<NP, QS>() + size_t(nz) * kZSlotBytes +
+                      2 * PS * pbuf_bytes<NP>() + kMiscBytes;
   auto kern = k_split_tc<NP, BF16, QS, PS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   kern<<<G, kThreadsTc, smem, s>>>(tc, tq, static_cast<const uint8_t*>(cache), sched, pm, pl, pz,
-                                   status, d.batch, d.H, d.r, d.max_len, G, nslot);
+                                   status, d.batch, d.H, d.r, d.max_len, G, ns, nz);
   note_launch();
   return check_launch();
 }
