@@ -55,7 +55,7 @@ namespace {
 
 constexpr int kThreadsTc = 256;
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
-constexpr int kMaxSlots = 6;                   // per ring
+constexpr int kMaxSlots = 8;                   // per ring
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
@@ -114,6 +114,15 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+// 2D tiled load with an L2 eviction-priority policy (createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x,
+                                                 int y, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
 }
 // 3D tiled load with an L2 eviction-priority policy (createpolicy).
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -239,14 +248,20 @@ struct TileIter {
   __device__ bool last() const { return g == te - 1 || g + 1 == ts[b + 1]; }
 };
 
-// Shared-memory carve.  S ring slot: the latent chunk (two 64-channel boxes)
-// followed by the query chunk, QS parts of NP rows per box (QS = 2: the query
-// as a rounded 16-bit part plus its 16-bit rounding residual, summed by the
-// MMA into adjacent accumulator columns), laid out [box][part][row].  Z ring
-// slot: the latent chunk only.
+// Shared-memory carve.  Both rings carry items of 1/(r/64) of a tile.
+//   S slot: one 64-channel box of the latent tile (128 tokens x 128 bytes,
+//           swizzled) followed by the matching box of the absorbed query, QS
+//           parts of NP rows (QS = 2: the query as a rounded 16-bit part plus
+//           its 16-bit rounding residual, summed by the MMA into adjacent
+//           accumulator columns), laid out [part][row].
+//   Z slot: 64 tokens x 128 channels of the latent tile, two 64-channel
+//           boxes of 64 rows ([box][row][128 bytes]).
+// Small items keep both rings deep for the shared-memory budget, and the
+// split of that budget between the rings follows their share of the bytes.
 template <int NP, int QS>
-__host__ __device__ constexpr int s_slot_bytes() { return 2 * kBoxBytes + 2 * QS * NP * 128; }
-constexpr int kZSlotBytes = 2 * kBoxBytes;
+__host__ __device__ constexpr int s_slot_bytes() { return kBoxBytes + QS * NP * 128; }
+constexpr int kZBoxBytes = 64 * 128;             // 64 tokens x 64 channels x 2 bytes
+constexpr int kZSlotBytes = 2 * kZBoxBytes;
 template <int NP>
 __host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T part
 constexpr int kMiscBytes = 2048;
@@ -307,28 +322,35 @@ struct Ring {
   }
 };
 
-// Zero-filled copy of a ragged latent chunk (rows >= nv) into a slot, by one
-// warp, in the 128-byte-swizzled layout TMA would have produced.
-__device__ __forceinline__ void ragged_chunk(uint8_t* d, const uint8_t* src, size_t row_bytes,
-                                             int nv, int lane) {
-  for (int idx = lane; idx < 2 * 128 * 8; idx += 32) {
-    const int box = idx >> 10, t = (idx >> 3) & 127, c = idx & 7;
+// Zero-filled copy of latent rows into a slot by one warp, in the
+// 128-byte-swizzled layout TMA would have produced: `nbox` 64-channel boxes
+// of `rows` rows starting at tile row `row_lo`; tile rows >= nv become zeros.
+// `src` is the tile's first row at the first box's channel offset.
+__device__ __forceinline__ void ragged_rows(uint8_t* d, const uint8_t* src, size_t row_bytes,
+                                            int rows, int nbox, int row_lo, int nv, int lane) {
+  const int per_box = rows * 8;   // 16-byte vectors per box
+  for (int idx = lane; idx < nbox * per_box; idx += 32) {
+    const int box = idx / per_box, tt = (idx >> 3) % rows, c = idx & 7;
+    const int t = row_lo + tt;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (t < nv) v = *reinterpret_cast<const uint4*>(src + size_t(t) * row_bytes + box * 128 + c * 16);
-    *reinterpret_cast<uint4*>(d + box * kBoxBytes + t * 128 + ((c ^ (t & 7)) << 4)) = v;
+    *reinterpret_cast<uint4*>(d + box * rows * 128 + tt * 128 + ((c ^ (tt & 7)) << 4)) = v;
   }
   fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
   __syncwarp();
 }
 
-// Producer of one ring (warp-wide).  kind 0: S ring (latent from HBM, kept
-// in L2 for the Z re-read, plus the query chunk); kind 1: Z ring (latent
-// re-read, dropped from L2 after).  Returns false on a wait that expired.
+// Producer of one ring (warp-wide).  kind 0: S ring (latent box from HBM,
+// kept in L2 for the Z re-read, plus the query box); kind 1: Z ring (latent
+// re-read, dropped from L2 after).  Item u of a tile: S -> channel box u;
+// Z -> channels [128 (u / 2), +128) x tokens [64 (u % 2), +64).  Returns false
+// on a wait that expired or an abort.
 template <int NP, int QS>
-__device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_c, const CUtensorMap* tm_q,
-                        const uint8_t* cache, const int32_t* sched, int B, int r, int max_len,
-                        long long tb, long long te, int n, int nslots, int lane, long long* issued) {
-  const int NC = r / 128;
+__device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const CUtensorMap* tm_cz,
+                        const CUtensorMap* tm_q, const uint8_t* cache, const int32_t* sched, int B,
+                        int r, int max_len, long long tb, long long te, int n, int nslots, int lane,
+                        long long* issued) {
+  const int NI = r / 64;
   const size_t row_bytes = size_t(r) * 2;
   uint8_t* ring = kind == 0 ? s.sring : s.zring;
   const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
@@ -341,29 +363,40 @@ __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_c, const 
   Ring rg(nslots);
   long long k = 0;
   for (int i = 0; i < n; ++i) {
-    const int nv = it.nvalid(), b = it.b;
-    const int row = b * max_len + it.t0();
-    for (int j = 0; j < NC; ++j) {
+    const int nv = it.nvalid(), b = it.b, t0 = it.t0();
+    const int row = b * max_len + t0;
+    const uint8_t* tile = cache + size_t(row) * row_bytes;
+    for (int u = 0; u < NI; ++u) {
       if (!__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
         *issued = k;
         return false;
       }
       const uint32_t dst = ring0 + uint32_t(rg.slot) * slot_bytes;
       const uint32_t fb = saddr(&full[rg.slot]);
-      if (nv == kTile) {
+      const int lo = kind == 0 ? 0 : 64 * (u & 1);        // first tile row of the item
+      const int hi = kind == 0 ? kTile : lo + 64;
+      if (nv >= hi) {
         if (lane == 0) mbar_expect_tx(fb, slot_bytes);
         __syncwarp();
-        // one operation per lane: TMA operations of one thread are processed in order
-        if (lane == 0) tma_load_3d_hint(dst, tm_c, 0, row, 2 * j, fb, policy);
-        if (kind == 0 && lane == 1) tma_load_4d(dst + 2 * kBoxBytes, tm_q, 0, 0, QS * b, 2 * j, fb);
+        // TMA operations of one thread are processed one after another, so the
+        // issuing lanes rotate between items and the item's two operations
+        // go out from different lanes
+        const int ln = int(k & 15) * 2;
+        if (kind == 0) {
+          if (lane == ln) tma_load_2d_hint(dst, tm_cs, 64 * u, row, fb, policy);
+          if (lane == ln + 1) tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
+        } else if (lane == ln) {
+          tma_load_3d_hint(dst, tm_cz, 0, row + lo, 2 * (u >> 1), fb, policy);
+        }
       } else {
-        ragged_chunk(ring + size_t(rg.slot) * slot_bytes,
-                     cache + (size_t(b) * max_len + it.t0()) * row_bytes + size_t(256) * j, row_bytes,
-                     nv, lane);
+        // last tile of a sequence: rows past its length are written as zeros
+        uint8_t* d = ring + size_t(rg.slot) * slot_bytes;
+        if (kind == 0) ragged_rows(d, tile + 128 * u, row_bytes, kTile, 1, 0, nv, lane);
+        else ragged_rows(d, tile + 256 * (u >> 1), row_bytes, 64, 2, lo, nv, lane);
         if (lane == 0) {
           if (kind == 0) {
-            mbar_expect_tx(fb, uint32_t(2 * QS * NP * 128));
-            tma_load_4d(dst + 2 * kBoxBytes, tm_q, 0, 0, QS * b, 2 * j, fb);
+            mbar_expect_tx(fb, uint32_t(QS * NP * 128));
+            tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
           } else {
             mbar_arrive(fb);
           }
@@ -391,7 +424,8 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 
 template <int NP, bool BF16, int QS, int PS>
 __global__ void __launch_bounds__(kThreadsTc, 1)
-k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_q,
+k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
+           const __grid_constant__ CUtensorMap tm_q,
            const uint8_t* __restrict__ cache, const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
            int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz) {
@@ -402,7 +436,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
   constexpr int SW = QS * NP;                 // S accumulator columns per buffer
   constexpr int ZC0 = 2 * SW;                 // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NC = r / 128;
+  const int NI = r / 64;                      // ring items per tile
+  const int NC = r / 128;                     // 128-channel Z accumulator chunks
   const long long T = sched[B];
   const long long tb = dev::split_begin(blockIdx.x, G, T);
   const long long te = dev::split_begin(blockIdx.x + 1, G, T);
@@ -443,7 +478,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
     const int kind = warp >> 1;
     const int nslots = kind == 0 ? ns : nz;
     long long issued = 0;
-    if (!produce<NP, QS>(kind, s, &tm_c, &tm_q, cache, sched, B, r, max_len, tb, te, n, nslots,
+    if (!produce<NP, QS>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te, n, nslots,
                          lane, &issued)) {
       if (lane == 0) {
         set_abort(s, status);
@@ -462,19 +497,17 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
         // the accumulator buffer of tile i was last read by the softmax of tile i - 2
         if (i >= 2 && !mbar_wait(saddr(&s.p_full[i & 1]), uint32_t((i - 2) >> 1) & 1u)) { ok = false; break; }
         const uint32_t d = tmem + uint32_t((i & 1) * SW);
-        for (int j = 0; j < NC; ++j) {
+        for (int u = 0; u < NI; ++u) {
           if (!mbar_wait(saddr(&s.s_full[rg.slot]), rg.phase)) { ok = false; break; }
           tc_fence_after();
           // descriptor address field is in 16-byte units
           const uint64_t sa = da0 + uint64_t((rg.slot * s_slot_bytes<NP, QS>()) >> 4);
 #pragma unroll
-          for (int box = 0; box < 2; ++box)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t a = sa + uint64_t((box * kBoxBytes + kk * 32) >> 4);
-              const uint64_t bd = sa + uint64_t((2 * kBoxBytes + box * SW * 128 + kk * 32) >> 4);
-              tc_mma(d, a, bd, id_s, (j | box | kk) != 0);
-            }
+          for (int kk = 0; kk < 4; ++kk) {   // K = 16 channels per MMA
+            const uint64_t a = sa + uint64_t((kk * 32) >> 4);
+            const uint64_t bd = sa + uint64_t((kBoxBytes + kk * 32) >> 4);
+            tc_mma(d, a, bd, id_s, (u | kk) != 0);
+          }
           tc_commit(saddr(&s.s_empty[rg.slot]));
           rg.advance();
         }
@@ -491,7 +524,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
     // ----------------------------------------------------------- Z MMAs
     if (lane == 0) {
       constexpr uint32_t id_z = idesc_f16(128, NP, BF16, true, false);
-      const uint64_t za0 = sdesc(saddr(s.zring), kBoxBytes, 1024);   // MN-major C^T
+      const uint64_t za0 = sdesc(saddr(s.zring), kZBoxBytes, 1024);  // MN-major C^T
       const uint64_t pb0 = sdesc(saddr(s.pbuf), 16, 1024);            // P^T, K-major
       TileIter it;
       it.init(sched, B, tb, te);
@@ -501,19 +534,19 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUt
         const bool first = it.first(tb);
         if (!mbar_wait(saddr(&s.p_full[i & 1]), uint32_t(i >> 1) & 1u)) { ok = false; break; }
         const uint64_t pb = pb0 + uint64_t(((i & 1) * PS * pbuf_bytes<NP>()) >> 4);
-        for (int j = 0; j < NC; ++j) {
+        for (int u = 0; u < NI; ++u) {
+          const int j = u >> 1, h = u & 1;   // 128-channel chunk, 64-token half
           if (!mbar_wait(saddr(&s.z_full[rg.slot]), rg.phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
           const uint64_t za = za0 + uint64_t((rg.slot * kZSlotBytes) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t a = za + uint64_t((ks * 16 * 128) >> 4);
+          for (int kk = 0; kk < 4; ++kk) {   // K = 16 tokens per MMA
+            const uint64_t a = za + uint64_t((kk * 16 * 128) >> 4);
 #pragma unroll
             for (int part = 0; part < PS; ++part) {   // P = P_hi (+ P_lo for bf16)
-              const uint64_t bd = pb + uint64_t((part * pbuf_bytes<NP>() + (ks >> 2) * NP * 128 +
-                                                 (ks & 3) * 32) >> 4);
-              tc_mma(d, a, bd, id_z, (first && ks == 0 && part == 0) ? 0u : 1u);
+              const uint64_t bd = pb + uint64_t((part * pbuf_bytes<NP>() + h * NP * 128 + kk * 32) >> 4);
+              tc_mma(d, a, bd, id_z, (first && h == 0 && kk == 0 && part == 0) ? 0u : 1u);
             }
           }
           tc_commit(saddr(&s.z_empty[rg.slot]));
@@ -695,13 +728,16 @@ EncodeTiled get_encode() {
 
 constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
 
-// Slots per ring: as many S slots as fit while the Z ring keeps two.
+// Slots per ring.  Per tile the S ring carries r/64 x (latent box + query
+// box) and the Z ring r/64 x half a latent chunk; every load sees about the
+// same latency, so each ring's slots are its share of the bytes.
 template <int NP, int QS, int PS>
 void ring_slots(int* ns, int* nz) {
   const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
-  int s = (avail - 2 * kZSlotBytes) / s_slot_bytes<NP, QS>();
+  const int sb = s_slot_bytes<NP, QS>();
+  int s = int(double(avail) * sb / (sb + kZSlotBytes)) / sb;
   if (s > kMaxSlots) s = kMaxSlots;
-  int z = (avail - s * s_slot_bytes<NP, QS>()) / kZSlotBytes;
+  int z = (avail - s * sb) / kZSlotBytes;
   if (z > kMaxSlots) z = kMaxSlots;
   *ns = s;
   *nz = z;
@@ -716,15 +752,27 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
   constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
   constexpr int PS = BF16 ? 2 : 1;   // P as hi + lo parts for bf16 (8-bit mantissa)
   const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUtensorMap tc, tq;
+  const cuuint64_t rows = cuuint64_t(d.batch) * d.max_len;
+  CUtensorMap tcs, tcz, tq;
   {
-    // latent rows [B * max_len][r] seen as {64 channels, row, 64-channel box}:
-    // one box {64, 128, 2} is a 128-token x 128-channel chunk, smem [box][row][64]
-    const cuuint64_t dims[3] = {64, cuuint64_t(d.batch) * d.max_len, cuuint64_t(d.r / 64)};
+    // S items: latent rows [B * max_len][r], one box {64 channels, 128 rows}
+    const cuuint64_t dims[2] = {cuuint64_t(d.r), rows};
+    const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tcs, dt, 2, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // Z items: the same rows seen as {64 channels, row, 64-channel box}; one
+    // box {64, 64, 2} is 64 tokens x 128 channels, smem [box][row][64]
+    const cuuint64_t dims[3] = {64, rows, cuuint64_t(d.r / 64)};
     const cuuint64_t strides[2] = {cuuint64_t(d.r) * 2, 128};
-    const cuuint32_t box[3] = {64, 128, 2};
+    const cuuint32_t box[3] = {64, 64, 2};
     const cuuint32_t es[3] = {1, 1, 1};
-    if (enc(&tc, dt, 3, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    if (enc(&tcz, dt, 3, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -732,11 +780,11 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
   {
     // query parts: qt16 holds [B][QS][H][r] (hi, then the rounding residual),
     // seen as {64 channels, head, sequence * part, 64-channel box}; one box
-    // {64, NP, QS, 2} lands as smem [box][part][head][64].  Heads H..NP-1 are
+    // {64, NP, QS, 1} lands as smem [part][head][64].  Heads H..NP-1 are
     // outside the map and arrive as zeros.
     const cuuint64_t dims[4] = {64, cuuint64_t(d.H), cuuint64_t(d.batch) * QS, cuuint64_t(d.r / 64)};
     const cuuint64_t strides[3] = {cuuint64_t(d.r) * 2, cuuint64_t(d.H) * d.r * 2, 128};
-    const cuuint32_t box[4] = {64, cuuint32_t(NP), QS, 2};
+    const cuuint32_t box[4] = {64, cuuint32_t(NP), QS, 1};
     const cuuint32_t es[4] = {1, 1, 1, 1};
     if (enc(&tq, dt, 4, const_cast<void*>(qt16), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -751,8 +799,8 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
   auto kern = k_split_tc<NP, BF16, QS, PS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<G, kThreadsTc, smem, s>>>(tc, tq, static_cast<const uint8_t*>(cache), sched, pm, pl, pz,
-                                   status, d.batch, d.H, d.r, d.max_len, G, ns, nz);
+  kern<<<G, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache), sched, pm, pl,
+                                   pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz);
   note_launch();
   return check_launch();
 }
