@@ -206,6 +206,32 @@ __device__ __forceinline__ int group_or(int pred) {
 }
 __device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Reduce v[0..N) over the 32 lanes of a warp (N a power of two <= 32) with a
+// transposing butterfly: each round a lane keeps the half of its elements
+// whose index bit matches its own lane bit and adds the partner's copy of
+// that half, so lane L ends with the reduction of element L % N after
+// N - 1 + log2(32 / N) shuffles (32 separate reductions would take 5 N).
+// v is overwritten.
+struct OpAdd { __device__ float operator()(float a, float b) const { return a + b; } };
+struct OpMax { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+template <int N, typename Op>
+__device__ __forceinline__ float warp_reduce_transposed(float (&v)[N], int lane, Op op) {
+#pragma unroll
+  for (int k = N / 2; k >= 1; k >>= 1) {
+    const bool upper = (lane & k) != 0;
+#pragma unroll
+    for (int j = 0; j < k; ++j) {
+      const float send = upper ? v[j] : v[j + k];
+      const float keep = upper ? v[j + k] : v[j];
+      v[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, k));
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int k = N; k < 32; k <<= 1) x = op(x, __shfl_xor_sync(0xffffffffu, x, k));
+  return x;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
@@ -603,10 +629,12 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       }
       if (group_or(need)) {
         // exact tile max per head over the 128 rows
+        {
+          float tmp[NP];
 #pragma unroll
-        for (int h = 0; h < NP; ++h) {
-          const float v = dev::warp_max(sv[h]);
-          if (lane == 0) s.red[q * NP + h] = v;
+          for (int h = 0; h < NP; ++h) tmp[h] = sv[h];
+          const float v = warp_reduce_transposed<NP>(tmp, lane, OpMax());
+          if (lane < NP) s.red[q * NP + lane] = v;
         }
         group_sync();
         float alpha[NP];
@@ -669,23 +697,33 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
         tc_fence_after();
         const size_t slot = size_t(blockIdx.x) + it.b;
+        // z^T chunk c: TMEM lane = channel 128 c + t, column = head; the
+        // load of chunk c + 1 is in flight while chunk c is stored
+        float* zrow = pz + slot * size_t(H) * r + t;
+        float zc[NP], zn[NP];
+#pragma unroll
+        for (int h16 = 0; h16 < NP / 16; ++h16)
+          tmem_ld16(tmem + lane_off + uint32_t(ZC0 + 16 * h16), zc + 16 * h16);
+        tmem_wait_ld();
         for (int c = 0; c < NC; ++c) {
+          if (c + 1 < NC) {
 #pragma unroll
-          for (int h16 = 0; h16 < NP / 16; ++h16) {
-            float z[16];
-            tmem_ld16(tmem + lane_off + uint32_t(ZC0 + c * NP + 16 * h16), z);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int h = 16 * h16 + e;
-              if (h < H) pz[(slot * H + h) * r + 128 * c + t] = z[e];
-            }
+            for (int h16 = 0; h16 < NP / 16; ++h16)
+              tmem_ld16(tmem + lane_off + uint32_t(ZC0 + (c + 1) * NP + 16 * h16), zn + 16 * h16);
           }
-        }
+          float* zp = zrow + 128 * c;   // row pointer stepped by r: no per-store index arithmetic
 #pragma unroll
-        for (int h = 0; h < NP; ++h) {
-          const float v = dev::warp_sum(l_part[h]);
-          if (lane == 0) s.red[q * NP + h] = v;
+          for (int h = 0; h < NP; ++h) {
+            if (h < H) *zp = zc[h];
+            zp += r;
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < NP; ++h) zc[h] = zn[h];
+        }
+        {
+          const float v = warp_reduce_transposed<NP>(l_part, lane, OpAdd());   // l_part is dead after
+          if (lane < NP) s.red[q * NP + lane] = v;
         }
         group_sync();
         if (t < H && t < NP) {
@@ -728,16 +766,20 @@ EncodeTiled get_encode() {
 
 constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
 
-// Slots per ring.  Per tile the S ring carries r/64 x (latent box + query
-// box) and the Z ring r/64 x half a latent chunk; every load sees about the
-// same latency, so each ring's slots are its share of the bytes.
+// Slots per ring.  About 96 KB in flight per ring measured best on the
+// LLaVA-7B-shaped layer (fp16 latent, r = 1536, 32 heads): 4 S slots and 6 Z
+// slots took 115.7 us, 5 + 5 118.8 us, 4 + 7 118.8 us, 3 + 7 117.8 us --
+// beyond that, more bytes in flight only lengthen every load's latency.
+constexpr int kRingTargetBytes = 96 * 1024;
 template <int NP, int QS, int PS>
 void ring_slots(int* ns, int* nz) {
   const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
   const int sb = s_slot_bytes<NP, QS>();
-  int s = int(double(avail) * sb / (sb + kZSlotBytes)) / sb;
+  int s = kRingTargetBytes / sb;
   if (s > kMaxSlots) s = kMaxSlots;
-  int z = (avail - s * sb) / kZSlotBytes;
+  int zbytes = avail - s * sb;
+  if (zbytes > kRingTargetBytes) zbytes = kRingTargetBytes;
+  int z = zbytes / kZSlotBytes;
   if (z > kMaxSlots) z = kMaxSlots;
   *ns = s;
   *nz = z;
