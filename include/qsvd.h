@@ -172,7 +172,7 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed,
  * workspace.  The split-K partials of x W^d go to a static device array of
  * 1,048,576 floats (4 MiB) that every GPU loading the library holds until
  * the process exits; requests needing more, i.e. ksplit * batch * r >
- * 1,048,576 with ksplit = ceil(E / 128) for 16-bit weights (ceil(E / 64)
+ * 1,048,576 with ksplit = ceil(E / 512) for 16-bit weights (ceil(E / 64)
  * for float32), return QSVD_ERR_WORKSPACE and enqueue nothing.  Nothing is
  * allocated.
  *   - The first call on each device looks up the array's device address

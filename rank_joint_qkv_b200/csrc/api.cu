@@ -15,6 +15,18 @@ static thread_local char g_err[512] = "";
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 cudaError_t check_launch() { return cudaGetLastError(); }
 
+TensorMapEncode tensor_map_encoder() {
+  static TensorMapEncode fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<TensorMapEncode>(p);
+    return TensorMapEncode(nullptr);
+  }();
+  return fn;
+}
+
 static qsvd_status fail(qsvd_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);

@@ -175,15 +175,8 @@ k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restric
 template <typename WT>
 cudaError_t gemv_t(const qsvd_dims& d, const void* x, const void* wd, float* cpart, int KS,
                    int32_t* status, cudaStream_t s) {
-  auto kern = k_gemv_partial<WT, WT>;
-  const size_t smem = gemv_smem<WT>();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((d.r + 255) / 256, KS, (d.batch + 15) / 16);
-  kern<<<grid, 256, smem, s>>>(static_cast<const WT*>(x), static_cast<const WT*>(wd), cpart,
-                               d.batch, d.E, d.r, KS, nullptr, nullptr, status);
-  note_launch();
-  return check_launch();
+  return launch_gemv<WT, WT>(static_cast<const WT*>(x), static_cast<const WT*>(wd), cpart, d.batch,
+                             d.E, d.r, KS, nullptr, nullptr, status, s);
 }
 
 int append_chunk(const qsvd_dims& d) {

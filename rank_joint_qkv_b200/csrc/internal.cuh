@@ -4,6 +4,7 @@
 // part of the public interface (include/qsvd.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -118,6 +119,14 @@ void note_launch();                 // counts kernels launched by this library
 qsvd_status set_error(qsvd_status st, const char* msg);   // records qsvd_last_error()
 cudaError_t check_launch();         // cudaGetLastError after a launch
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point
+// (no link against the driver library); null if the driver lacks it.
+using TensorMapEncode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncode tensor_map_encoder();
+
 // ------------------------------------------------------------ kernel entry
 
 // Prologue (query side).
@@ -210,6 +219,32 @@ __device__ __forceinline__ float sum_strided(const float* p, size_t stride, int 
   }
   for (; k < n; ++k) s += __ldcg(p + size_t(k) * stride);
   return s;
+}
+
+// Reduce v[0..N) over the 32 lanes of a warp (N a power of two <= 32) with a
+// transposing butterfly: each round a lane keeps the half of its elements
+// whose index bit matches its own lane bit and adds the partner's copy of
+// that half, so lane L ends with the reduction of element L % N after
+// N - 1 + log2(32 / N) shuffles (32 separate reductions would take 5 N).
+// v is overwritten.
+struct OpAdd { __device__ float operator()(float a, float b) const { return a + b; } };
+struct OpMax { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+template <int N, typename Op>
+__device__ __forceinline__ float warp_reduce_transposed(float (&v)[N], int lane, Op op) {
+#pragma unroll
+  for (int k = N / 2; k >= 1; k >>= 1) {
+    const bool upper = (lane & k) != 0;
+#pragma unroll
+    for (int j = 0; j < k; ++j) {
+      const float send = upper ? v[j] : v[j + k];
+      const float keep = upper ? v[j + k] : v[j];
+      v[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, k));
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int k = N; k < 32; k <<= 1) x = op(x, __shfl_xor_sync(0xffffffffu, x, k));
+  return x;
 }
 
 // Number of tiles of a sequence of n tokens.

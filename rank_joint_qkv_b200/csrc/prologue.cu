@@ -180,15 +180,8 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
 template <typename WT>
 cudaError_t q_partial_t(const qsvd_dims& d, const float* qin, const void* wuq, float* qpart,
                         int KS, float* q, int32_t* tickets, int32_t* status, cudaStream_t s) {
-  auto kern = k_gemv_partial<float, WT>;
-  const size_t smem = gemv_smem<WT>();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((d.E + 255) / 256, KS, (d.batch + 15) / 16);
-  kern<<<grid, 256, smem, s>>>(qin, static_cast<const WT*>(wuq), qpart, d.batch, d.r, d.E, KS,
-                               q, tickets, status);
-  note_launch();
-  return check_launch();
+  return launch_gemv<float, WT>(qin, static_cast<const WT*>(wuq), qpart, d.batch, d.r, d.E, KS, q,
+                                tickets, status, s);
 }
 
 template <typename WT, typename QT16>
@@ -208,7 +201,7 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float 
 }  // namespace
 
 int prologue_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.r, d.weight_dtype); }
-int prologue_tickets(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch); }
+int prologue_tickets(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch, d.weight_dtype); }
 
 cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
                             WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,

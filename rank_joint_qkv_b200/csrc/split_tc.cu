@@ -206,31 +206,6 @@ __device__ __forceinline__ int group_or(int pred) {
 }
 __device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Reduce v[0..N) over the 32 lanes of a warp (N a power of two <= 32) with a
-// transposing butterfly: each round a lane keeps the half of its elements
-// whose index bit matches its own lane bit and adds the partner's copy of
-// that half, so lane L ends with the reduction of element L % N after
-// N - 1 + log2(32 / N) shuffles (32 separate reductions would take 5 N).
-// v is overwritten.
-struct OpAdd { __device__ float operator()(float a, float b) const { return a + b; } };
-struct OpMax { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
-template <int N, typename Op>
-__device__ __forceinline__ float warp_reduce_transposed(float (&v)[N], int lane, Op op) {
-#pragma unroll
-  for (int k = N / 2; k >= 1; k >>= 1) {
-    const bool upper = (lane & k) != 0;
-#pragma unroll
-    for (int j = 0; j < k; ++j) {
-      const float send = upper ? v[j] : v[j + k];
-      const float keep = upper ? v[j + k] : v[j];
-      v[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, k));
-    }
-  }
-  float x = v[0];
-#pragma unroll
-  for (int k = N; k < 32; k <<= 1) x = op(x, __shfl_xor_sync(0xffffffffu, x, k));
-  return x;
-}
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -633,7 +608,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           float tmp[NP];
 #pragma unroll
           for (int h = 0; h < NP; ++h) tmp[h] = sv[h];
-          const float v = warp_reduce_transposed<NP>(tmp, lane, OpMax());
+          const float v = dev::warp_reduce_transposed<NP>(tmp, lane, dev::OpMax());
           if (lane < NP) s.red[q * NP + lane] = v;
         }
         group_sync();
@@ -722,7 +697,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           for (int h = 0; h < NP; ++h) zc[h] = zn[h];
         }
         {
-          const float v = warp_reduce_transposed<NP>(l_part, lane, OpAdd());   // l_part is dead after
+          const float v = dev::warp_reduce_transposed<NP>(l_part, lane, dev::OpAdd());   // l_part is dead after
           if (lane < NP) s.red[q * NP + lane] = v;
         }
         group_sync();
@@ -745,24 +720,6 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 }
 
 // ------------------------------------------------------------------- host
-
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled get_encode() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
 
 constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
 
@@ -789,7 +746,7 @@ template <int NP, bool BF16>
 cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
                      const int32_t* sched, int G, float* pm, float* pl, float* pz,
                      int32_t* status, cudaStream_t s) {
-  EncodeTiled enc = get_encode();
+  TensorMapEncode enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
   constexpr int PS = BF16 ? 2 : 1;   // P as hi + lo parts for bf16 (8-bit mantissa)
