@@ -19,55 +19,57 @@ constexpr int kJ = 128;   // latent rows (of W^u_v) per CTA
 constexpr int kBC = 16;   // sequences per pass
 
 // grid (H, ceil(r / kJ)), block 256.
-// smem: ws[kJ][d_h] W^u_v tile (float), zs[kBC][kJ] merged latents,
-//       red[KSP][kBC][d_h] partial outputs, wt[P] per-slot merge weight
-//       2^(m_s - M) / L (indexed by slot), seg[B][2] slot ranges.
+// smem: ws[kJ][d_h] W^u_v tile (16-bit, as stored), zs[kBC][kJ] merged
+//       latents, red[KSP][kBC][d_h] partial outputs, wt[P] per-slot merge
+//       weight 2^(m_s - M) / L (indexed by slot), ts[B + 1] tile starts,
+//       seg[B][2] slot ranges.
+// Every stage issues all of a thread's loads before it uses one of them:
+// the W^u_v tile by cp.async (it lands while the weights and the merge run),
+// the partials of 8 splits per thread at a time; registers are capped for
+// three CTAs per SM, so that the whole grid is resident at once.
 template <typename WT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sched,
               const float* __restrict__ pm, const float* __restrict__ pl,
               const float* __restrict__ pz, const WT* __restrict__ wuv,
               float* __restrict__ opart, int B, int H, int d_h, int r, int E, int P) {
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) uint8_t csm[];
   const int DQ = d_h / 4;                 // output quads per sequence
   const int KSP = 256 / (4 * DQ);         // k-splits of the V-up tile
-  float* ws = sm;                         // kJ * d_h
-  float* zs = ws + kJ * d_h;              // kBC * kJ
+  WT* ws = reinterpret_cast<WT*>(csm);                                   // kJ * d_h
+  float* zs = reinterpret_cast<float*>(csm + size_t(kJ) * d_h * sizeof(WT));   // kBC * kJ
   float* red = zs + kBC * kJ;             // KSP * kBC * d_h
   float* wt = red + KSP * kBC * d_h;      // P
-  int* seg = reinterpret_cast<int*>(wt + P);   // B x {c0, c1}
+  int* ts = reinterpret_cast<int*>(wt + P);   // B + 1
+  int* seg = ts + B + 1;                  // B x {c0, c1}
   const int h = blockIdx.x;
   const int js = blockIdx.y;
   const int j0 = js * kJ;
-  const int jn = min(kJ, r - j0);
+  const int jn = min(kJ, r - j0);         // a multiple of 32
   const long long G = hdr->G;
-  const int32_t* tstart = sched;
-  const long long T = tstart[B];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // W^u_v tile, 16-byte loads
+  // W^u_v tile rows j0 .. j0 + jn - 1, head h's columns: 16-byte async copies
   {
-    constexpr int V = 16 / int(sizeof(WT));
-    const int vpr = d_h / V;
+    const int vpr = d_h * int(sizeof(WT)) / 16;   // d_h is a multiple of 8
+    const uint32_t ws_s = static_cast<uint32_t>(__cvta_generic_to_shared(ws));
     for (int i = threadIdx.x; i < kJ * vpr; i += 256) {
       const int jj = i / vpr, v = i % vpr;
-      float f[V];
       if (jj < jn) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(wuv + size_t(j0 + jj) * E + h * d_h + v * V);
-        const WT* e = reinterpret_cast<const WT*>(&raw);
-#pragma unroll
-        for (int k = 0; k < V; ++k) f[k] = dev::to_f(e[k]);
+        const WT* src = wuv + size_t(j0 + jj) * E + h * d_h + v * (16 / int(sizeof(WT)));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ws_s + 16u * i), "l"(src) : "memory");
       } else {
-#pragma unroll
-        for (int k = 0; k < V; ++k) f[k] = 0.f;
+        reinterpret_cast<uint4*>(ws)[i] = make_uint4(0, 0, 0, 0);
       }
-#pragma unroll
-      for (int k = 0; k < V; ++k) ws[jj * d_h + v * V + k] = f[k];
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
+  for (int i = threadIdx.x; i <= B; i += 256) ts[i] = sched[i];
+  __syncthreads();
+  const long long T = ts[B];
   // merge weights, one warp per sequence; lane i holds slots c0 + i + 32 k
   for (int b = warp; b < B; b += 8) {
-    const long long t0 = tstart[b], t1 = tstart[b + 1];
+    const long long t0 = ts[b], t1 = ts[b + 1];
     int c0 = 0, c1 = -1;
     if (t1 > t0) {
       c0 = int(dev::split_of_tile(t0, G, T));
@@ -80,24 +82,21 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
       const int c = c0 + lane + 32 * k;
-      mv[k] = -INFINITY;
-      lv[k] = 0.f;
-      if (c <= c1 && dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T)) {
-        mv[k] = pm[(size_t(c) + b) * H + h];
-        lv[k] = pl[(size_t(c) + b) * H + h];
-      }
+      const bool live = c <= c1 && dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T);
+      mv[k] = live ? __ldcg(pm + (size_t(c) + b) * H + h) : -INFINITY;
+      lv[k] = live ? __ldcg(pl + (size_t(c) + b) * H + h) : 0.f;
       M = fmaxf(M, mv[k]);
     }
     for (int c = c0 + lane + 32 * NR; c <= c1; c += 32)   // long runs of splits
       if (dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T))
-        M = fmaxf(M, pm[(size_t(c) + b) * H + h]);
+        M = fmaxf(M, __ldcg(pm + (size_t(c) + b) * H + h));
     M = dev::warp_max(M);
     float L = 0.f;
 #pragma unroll
     for (int k = 0; k < NR; ++k) L += exp2f(mv[k] - M) * lv[k];
     for (int c = c0 + lane + 32 * NR; c <= c1; c += 32)
       if (dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T))
-        L += exp2f(pm[(size_t(c) + b) * H + h] - M) * pl[(size_t(c) + b) * H + h];
+        L += exp2f(__ldcg(pm + (size_t(c) + b) * H + h) - M) * __ldcg(pl + (size_t(c) + b) * H + h);
     L = dev::warp_sum(L);
     const float invL = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
@@ -107,38 +106,49 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
     }
     for (int c = c0 + lane + 32 * NR; c <= c1; c += 32) {
       const bool live = dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T);
-      wt[c + b] = live ? exp2f(pm[(size_t(c) + b) * H + h] - M) * invL : 0.f;
+      wt[c + b] = live ? exp2f(__ldcg(pm + (size_t(c) + b) * H + h) - M) * invL : 0.f;
     }
   }
   __syncthreads();
-  const int jj = threadIdx.x & (kJ - 1);
-  const int bsub = threadIdx.x / kJ;          // 0 or 1
   // V-up tile: thread -> 4 sequences x 4 output dims over one k-split
   const int ksp = threadIdx.x / (4 * DQ);
   const int bq = (threadIdx.x % (4 * DQ)) / DQ;
   const int dq = threadIdx.x % DQ;
   const int kper = kJ / KSP;
+  // merge: thread -> channel quad qd of sequences mb and mb + 8
+  const int mb = threadIdx.x >> 5, qd = threadIdx.x & 31;
+  bool waited = false;
   for (int bc = 0; bc < B; bc += kBC) {
     const int bn = min(kBC, B - bc);
-    // merged latent z[b][j] = sum_s w_s z_s[j]; the loads are independent
-    for (int bb = bsub; bb < kBC; bb += 2) {
+#pragma unroll 1
+    for (int bb = mb; bb < kBC; bb += 8) {
       const int b = bc + bb;
-      float z = 0.f;
-      if (bb < bn && jj < jn) {
+      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (bb < bn && 4 * qd < jn) {
         const int c0 = seg[2 * b], c1 = seg[2 * b + 1];
-        // loads in batches of 8 so that they are in flight together
+        const float* base = pz + size_t(h) * r + j0 + 4 * qd;
         for (int cb = c0; cb <= c1; cb += 8) {
-          float v[8];
+          float4 v[8];
+          float w[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            v[i] = (cb + i <= c1 && wt[cb + i + b] != 0.f)
-                       ? __ldcg(pz + ((size_t(cb + i) + b) * H + h) * r + j0 + jj) : 0.f;
+          for (int i = 0; i < 8; ++i) {
+            w[i] = cb + i <= c1 ? wt[cb + i + b] : 0.f;
+            v[i] = w[i] != 0.f
+                       ? __ldcg(reinterpret_cast<const float4*>(base + (size_t(cb + i) + b) * H * r))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (cb + i <= c1) z = fmaf(wt[cb + i + b], v[i], z);
+          for (int i = 0; i < 8; ++i) {
+            z.x = fmaf(w[i], v[i].x, z.x); z.y = fmaf(w[i], v[i].y, z.y);
+            z.z = fmaf(w[i], v[i].z, z.z); z.w = fmaf(w[i], v[i].w, z.w);
+          }
         }
       }
-      zs[bb * kJ + jj] = z;
+      reinterpret_cast<float4*>(zs + bb * kJ)[qd] = z;
+    }
+    if (!waited) {   // the W^u_v tile has landed
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      waited = true;
     }
     __syncthreads();
     float acc[4][4];
@@ -148,14 +158,19 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
       for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
     const int kend = ksp < KSP ? (ksp + 1) * kper : 0;   // spare threads when 256 % d_h != 0
     for (int k = ksp * kper; k < kend; ++k) {
-      const float4 w4 = *reinterpret_cast<const float4*>(&ws[k * d_h + 4 * dq]);
+      float w4[4];
+      {
+        const WT* wp = ws + k * d_h + 4 * dq;
+        w4[0] = dev::to_f(wp[0]); w4[1] = dev::to_f(wp[1]);
+        w4[2] = dev::to_f(wp[2]); w4[3] = dev::to_f(wp[3]);
+      }
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         const float z = zs[(4 * bq + a) * kJ + k];
-        acc[a][0] = fmaf(z, w4.x, acc[a][0]);
-        acc[a][1] = fmaf(z, w4.y, acc[a][1]);
-        acc[a][2] = fmaf(z, w4.z, acc[a][2]);
-        acc[a][3] = fmaf(z, w4.w, acc[a][3]);
+        acc[a][0] = fmaf(z, w4[0], acc[a][0]);
+        acc[a][1] = fmaf(z, w4[1], acc[a][1]);
+        acc[a][2] = fmaf(z, w4[2], acc[a][2]);
+        acc[a][3] = fmaf(z, w4[3], acc[a][3]);
       }
     }
     if (ksp < KSP) {
@@ -188,11 +203,14 @@ cudaError_t vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                   const float* pm, const float* pl, const float* pz, const void* wuv,
                   float* opart, int JS, int P, cudaStream_t s) {
   const int ksp = 256 / d.d_h;   // k-splits of the V-up tile (4 x 4 outputs per thread)
-  const size_t smem = (size_t(kJ) * d.d_h + size_t(kBC) * kJ + size_t(ksp) * kBC * d.d_h + P) * 4 +
+  const size_t smem = size_t(kJ) * d.d_h * sizeof(WT) +
+                      (size_t(kBC) * kJ + size_t(ksp) * kBC * d.d_h + P) * 4 + size_t(d.batch + 1) * 4 +
                       size_t(d.batch) * 8;
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   auto kern = k_combine_vup<WT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e == cudaSuccess)   // room for three CTAs per SM
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(d.H, JS);
   kern<<<grid, 256, smem, s>>>(hdr, sched, pm, pl, pz, static_cast<const WT*>(wuv), opart,
