@@ -257,7 +257,7 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (d.rope)
       e = launch_rope_query(d, qsrc, sched, rope_tab, sl2, qt32, s);
     else
-      e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, qt16, s);
+      e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, qt16, &hdr->status, s);
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (phases & QSVD_PHASE_SPLIT) {

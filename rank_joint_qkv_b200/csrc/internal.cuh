@@ -137,7 +137,7 @@ cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* w
                              float* qpart, int KS, float* q, int32_t* tickets, int32_t* status,
                              cudaStream_t s);
 cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale_log2,
-                          float* qt32, void* qt16, cudaStream_t s);
+                          float* qt32, void* qt16, int32_t* status, cudaStream_t s);
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
                               const float* rope_tab, float scale_log2, float* qrot,
                               cudaStream_t s);

@@ -109,6 +109,167 @@ k_absorb(const float* __restrict__ q, const WT* __restrict__ W, float scale,
 }
 
 // ---------------------------------------------------------------------------
+// Absorbed query on the tensor cores, for 16-bit weights and d_h a multiple
+// of 64:  qt[b][h][j] = scale * sum_dd q[b][h d_h + dd] W^u_k[j][h d_h + dd].
+// Per head a 16-row product (M = 16 sequences, N = 128 rows j of W^u_k per
+// CTA, K = d_h), so it takes the GEMV's form: the W^u_k tile arrives by TMA
+// into 128-byte-swizzled rows whose d_h values are K-contiguous (ldmatrix
+// gives the B fragments directly), q enters as a 16-bit part plus its
+// rounding residual, with fp16 weights scaled per sequence by a power of two.
+// grid (H, ceil(r / 128)), block 128.
+// ---------------------------------------------------------------------------
+template <typename WT, typename QT16>
+__global__ void __launch_bounds__(128)
+k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ q, float scale,
+             float* __restrict__ qt32, QT16* __restrict__ qt16, int B, int H, int d_h, int r, int E,
+             int32_t* status) {
+  using namespace gemv_mma;
+  constexpr bool BF16 = std::is_same<WT, __nv_bfloat16>::value;
+  constexpr bool SCALE = !BF16;           // fp16 range needs the power-of-two scale
+  extern __shared__ uint8_t asm_raw[];
+  uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(asm_raw) + 1023) &
+                                             ~uintptr_t(1023));   // [d_h / 64][128 rows][128 B]
+  const int XP = d_h * 2 + 16;            // activation row pitch (bytes, padded)
+  uint8_t* xs = tile + d_h * 256;         // [2][16][XP]
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ float inv_scale[16];
+  __shared__ unsigned smax[16];
+  const int h = blockIdx.x, j0 = blockIdx.y * 128, jn = min(128, r - j0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t tile_s = static_cast<uint32_t>(__cvta_generic_to_shared(tile));
+  const uint32_t bar_s = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  const int NBOX = d_h / 64;
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_s) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_s),
+                 "r"(uint32_t(d_h * 256)) : "memory");
+    for (int c = 0; c < NBOX; ++c)
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+          " [%0], [%1, {%2, %3}], [%4];" ::"r"(tile_s + c * 16384),
+          "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"(h * d_h + 64 * c), "r"(j0), "r"(bar_s)
+          : "memory");
+  }
+  const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);   // ldmatrix: this lane's row of its 8x8 matrix
+  const int mcol = 8 * (lane >> 4);
+  const uint32_t xs_s = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+  bool waited = false;
+  for (int b0 = 0; b0 < B; b0 += 16) {
+    const int bn = min(16, B - b0);
+    // q slice of head h: thread tid holds dd = tid + 128 u of every sequence
+    float xv[16][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int dd = tid + 128 * u;
+      const int ddc = dd < d_h ? dd : 0;   // clamped: the loads stay unconditional
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        xv[j][u] = __ldg(q + size_t(b0 + (j < bn ? j : 0)) * E + h * d_h + ddc);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (!(j < bn && dd < d_h)) xv[j][u] = 0.f;
+    }
+    if (SCALE) {
+      if (tid < 16) smax[tid] = 0u;
+      float m[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) m[j] = fmaxf(fabsf(xv[j][0]), fabsf(xv[j][1]));
+      const float wm = dev::warp_reduce_transposed<16>(m, lane, dev::OpMax());   // lane L: sequence L % 16
+      __syncthreads();
+      if (lane < 16) atomicMax(&smax[lane], __float_as_uint(wm));   // non-negative floats order as integers
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float s = 1.f, inv = 1.f;
+      if (SCALE) {
+        const unsigned mb = smax[j];
+        if (mb != 0u) {
+          const int e = max(int((mb >> 23) & 0xFFu) - 127, -112);
+          s = __uint_as_float(unsigned(141 - e) << 23);
+          inv = __uint_as_float(unsigned(113 + e) << 23);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int dd = tid + 128 * u;
+        if (dd < d_h) {
+          const float v = xv[j][u] * s;
+          const WT hi = dev::from_f<WT>(v);
+          reinterpret_cast<WT*>(xs + j * XP)[dd] = hi;
+          reinterpret_cast<WT*>(xs + (16 + j) * XP)[dd] = dev::from_f<WT>(v - dev::to_f(hi));
+        }
+      }
+      if (tid == 0) inv_scale[j] = inv;
+    }
+    if (!waited) {   // the W^u_k tile (bounded wait: 2 s; on expiry flag it and stop)
+      bool ok = mbar_try(bar_s, 0);
+      if (!ok) {
+        const uint64_t t0 = gtimer();
+        while (!(ok = mbar_try(bar_s, 0)))
+          if (gtimer() - t0 > 2000000000ull) break;
+      }
+      if (!__syncthreads_and(ok)) {
+        if (tid == 0 && status) atomicOr(status, QSVD_STATUS_TIMEOUT);
+        return;
+      }
+      waited = true;
+    } else {
+      __syncthreads();
+    }
+    // warp w: rows j 32 w .. 32 w + 31 (4 n-tiles), k over d_h
+    float acc[4][4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    for (int kk = 0; kk < d_h / 16; ++kk) {
+      uint32_t a[2][4];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) ldsm_x4(xs_s + (p * 16 + mrow) * XP + (16 * kk + mcol) * 2, a[p]);
+      const int dd = 16 * kk + 8 * ((lane >> 3) & 1);
+      const int c = dd >> 6, chunk = (dd & 63) >> 3;
+#pragma unroll
+      for (int jp = 0; jp < 2; ++jp) {
+        const int j = 32 * warp + 8 * (2 * jp + (lane >> 4)) + (lane & 7);
+        uint32_t bfr[4];   // n-tile 2 jp: k lo, k hi; n-tile 2 jp + 1: k lo, k hi
+        ldsm_x4(tile_s + c * 16384 + j * 128 + ((chunk ^ (j & 7)) << 4), bfr);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          mma16816<BF16>(acc[2 * jp], a[p], bfr[0], bfr[1]);
+          mma16816<BF16>(acc[2 * jp + 1], a[p], bfr[2], bfr[3]);
+        }
+      }
+    }
+    // fragment: (row g = sequence, cols 2t, 2t+1 = rows j) and (row g + 8)
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int jl = 32 * warp + 8 * t + 2 * t4;
+      if (jl >= jn) continue;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int bb = g + 8 * half;
+        if (bb >= bn) continue;
+        const int b = b0 + bb;
+        const float sc = scale * inv_scale[bb];
+        const float v0 = acc[t][2 * half] * sc, v1 = acc[t][2 * half + 1] * sc;
+        const size_t o = (size_t(b) * H + h) * r + j0 + jl;
+        *reinterpret_cast<float2*>(qt32 + o) = make_float2(v0, v1);
+        // 16-bit copy for the tensor cores, [B][2][H][r]: the rounded value
+        // and its rounding residual
+        const QT16 h0 = dev::from_f<QT16>(v0), h1 = dev::from_f<QT16>(v1);
+        const QT16 l0 = dev::from_f<QT16>(v0 - dev::to_f(h0)), l1 = dev::from_f<QT16>(v1 - dev::to_f(h1));
+        const size_t o2 = ((size_t(b) * 2) * H + h) * r + j0 + jl;
+        QT16 hv[2] = {h0, h1}, lv[2] = {l0, l1};
+        *reinterpret_cast<uint32_t*>(qt16 + o2) = *reinterpret_cast<const uint32_t*>(hv);
+        *reinterpret_cast<uint32_t*>(qt16 + o2 + size_t(H) * r) = *reinterpret_cast<const uint32_t*>(lv);
+      }
+    }
+    __syncthreads();   // xs is restaged for the next 16 sequences
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Rotary query: q_h <- scale * R(len_b - 1) q_h, pairs (i, i + d_h/2).
 // grid (B), block 256.
 // ---------------------------------------------------------------------------
@@ -186,7 +347,33 @@ cudaError_t q_partial_t(const qsvd_dims& d, const float* qin, const void* wuq, f
 
 template <typename WT, typename QT16>
 cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float scale,
-                     float* qt32, void* qt16, cudaStream_t s) {
+                     float* qt32, void* qt16, int32_t* status, cudaStream_t s) {
+  if constexpr (sizeof(WT) == 2) {
+    if (d.d_h % 64 == 0 && d.d_h <= 256) {
+      TensorMapEncode enc = tensor_map_encoder();
+      if (!enc) return cudaErrorNotSupported;
+      CUtensorMap tm;
+      const cuuint64_t dims[2] = {cuuint64_t(d.E), cuuint64_t(d.r)};
+      const cuuint64_t strides[1] = {cuuint64_t(d.E) * 2};
+      const cuuint32_t box[2] = {64, 128};
+      const cuuint32_t es[2] = {1, 1};
+      const CUtensorMapDataType dt = std::is_same<WT, __nv_bfloat16>::value
+                                         ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      if (enc(&tm, dt, 2, const_cast<void*>(wuk), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+      const int smem = 1024 + d.d_h * 256 + 2 * 16 * (d.d_h * 2 + 16);
+      auto kern = k_absorb_mma<WT, QT16>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      dim3 grid(d.H, (d.r + 127) / 128);
+      kern<<<grid, 128, smem, s>>>(tm, q, scale, qt32, static_cast<QT16*>(qt16), d.batch, d.H, d.d_h,
+                                   d.r, d.E, status);
+      note_launch();
+      return check_launch();
+    }
+  }
   const size_t smem = size_t(128 + 16) * (d.d_h + 4) * 4;
   auto kern = k_absorb<WT, QT16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -224,18 +411,18 @@ cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* w
 }
 
 cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale,
-                          float* qt32, void* qt16, cudaStream_t s) {
+                          float* qt32, void* qt16, int32_t* status, cudaStream_t s) {
   const bool bf = d.cache_dtype == QSVD_BF16;
   switch (d.weight_dtype) {
     case QSVD_F32:
-      return bf ? absorb_t<float, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
-                : absorb_t<float, __half>(d, q, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<float, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, status, s)
+                : absorb_t<float, __half>(d, q, wuk, scale, qt32, qt16, status, s);
     case QSVD_F16:
-      return bf ? absorb_t<__half, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
-                : absorb_t<__half, __half>(d, q, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<__half, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, status, s)
+                : absorb_t<__half, __half>(d, q, wuk, scale, qt32, qt16, status, s);
     case QSVD_BF16:
-      return bf ? absorb_t<__nv_bfloat16, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, s)
-                : absorb_t<__nv_bfloat16, __half>(d, q, wuk, scale, qt32, qt16, s);
+      return bf ? absorb_t<__nv_bfloat16, __nv_bfloat16>(d, q, wuk, scale, qt32, qt16, status, s)
+                : absorb_t<__nv_bfloat16, __half>(d, q, wuk, scale, qt32, qt16, status, s);
     default: return cudaErrorInvalidValue;
   }
 }
