@@ -226,29 +226,30 @@ def run_ours(args, rank, world, local_rank):
                          device=device)
     cache, scales = inp["cache"], inp["scales"]
 
-    def step(ev=None):
+    def step(ev=None, st=None):
         # ev: 5 events bracketing append | prologue | split | combine
+        st = stream if st is None else st
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         q.qsvd_append_latent(dims, packed, x_dev, pos_dev, cache, scales, cnew, None, app_ws,
-                             stream=stream)
+                             stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
-                           phases=q.QSVD_PHASE_PROLOGUE, stream=stream)
+                           phases=q.QSVD_PHASE_PROLOGUE, stream=st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
-                           phases=q.QSVD_PHASE_SPLIT, stream=stream)
+                           phases=q.QSVD_PHASE_SPLIT, stream=st)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
         q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
                            num_splits=args.splits, workspace=dec_ws,
-                           phases=q.QSVD_PHASE_COMBINE, stream=stream)
+                           phases=q.QSVD_PHASE_COMBINE, stream=st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -256,25 +257,50 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
 
+    # eager pass: the four API calls per step, with events between the phases
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = q.kernel_launches()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches_per_step = (q.kernel_launches() - launches0) // args.steps
+    ms_eager = max_over_ranks(t0.elapsed_time(t1), device, world)
+    phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
+                for k, name in enumerate(("append", "prologue", "split", "combine"))}
+    split_ms = [e[2].elapsed_time(e[3]) for e in ev]
+
+    # timed pass: one step captured as a CUDA graph (the same kernels with the
+    # same arguments, without the host work between launches), replayed
+    graph = None
+    if not args.eager:
+        gstream = torch.cuda.Stream(device)
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            step(st=gstream)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    run = (lambda: graph.replay()) if graph is not None else (lambda: step())
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
         t0.record(stream)
         for i in range(args.steps):
-            step(ev[i])
+            run()
         t1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
-    launches = q.kernel_launches() - launches0
+    launches = launches_per_step * args.steps
     ms = t0.elapsed_time(t1)
-    phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
-                for k, name in enumerate(("append", "prologue", "split", "combine"))}
-    split_ms = [e[2].elapsed_time(e[3]) for e in ev]
     kernel_used = int(dec_ws[12:16].view(torch.int32).item())   # workspace header: kernel
     ms_max = max_over_ranks(ms, device, world)
     tokens_per_step = float(np.sum(lens))
@@ -325,6 +351,9 @@ def run_ours(args, rank, world, local_rank):
                          % (lat_b / 1e6),
                    "parallelism": f"dp{world}"},
         "steps_per_s": args.steps * 1e3 / ms_max,
+        "timing": ("CUDA-graph replay of one captured step (the kernels of the four API calls)"
+                   if graph is not None else "eager API calls"),
+        "ms_per_step_eager": ms_eager / args.steps,
         "phase_ms": phase_ms,
         "step_hbm_gbs": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -424,6 +453,8 @@ def main():
     ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the API calls as issued instead of a CUDA-graph replay of one step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
