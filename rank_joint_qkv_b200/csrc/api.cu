@@ -264,7 +264,7 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (d.rope)
       e = launch_split_simt_rope(d, qt32, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
     else if (kernel == QSVD_KERNEL_TCGEN05)
-      e = launch_split_tc(d, cache, qt16, sched, G, pm, pl, pz, &hdr->status, s);
+      e = launch_split_tc(d, cache, scales, qt16, sched, G, pm, pl, pz, &hdr->status, s);
     else
       e = launch_split_simt_absorbed(d, qt32, cache, scales, sched, G, pm, pl, pz, s);
     if (e != cudaSuccess) return cuda_fail(e, "split phase");

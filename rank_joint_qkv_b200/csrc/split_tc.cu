@@ -48,6 +48,8 @@
 // flight (bounded), frees its TMEM and returns.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "internal.cuh"
 
 namespace qsvd {
@@ -56,6 +58,8 @@ namespace {
 constexpr int kThreadsTc = 256;
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
 constexpr int kMaxSlots = 8;                   // per ring
+constexpr int kMaxGroupBufs = 4;               // S accumulators per channel group (quantised latent)
+constexpr int kMaxRaw = 8;                     // raw-code slots per stream (quantised latent)
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
@@ -114,6 +118,14 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 // 2D tiled load with an L2 eviction-priority policy (createpolicy).
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x,
@@ -279,19 +291,34 @@ struct Smem {
   uint64_t* p_full;      // [2] P of a tile written (S accumulator read)
   uint64_t* z_done;      // [2] Z MMAs of a tile complete
   uint64_t* drain;       // [2] one per MMA issuer
+  uint64_t* sg_full;     // [kMaxGroupBufs] quantised latent: S of one channel group complete
+  uint64_t* sg_empty;    // [kMaxGroupBufs] ... read by the softmax
+  uint8_t* sraw;         // quantised latent: raw-code rings (S, Z) and two tiles of Z scales
+  uint8_t* zraw;
+  uint8_t* zscale;
+  uint64_t* sraw_full;   // [kMaxRaw]
+  uint64_t* zraw_full;   // [kMaxRaw]
   float* red;            // [4][NP]
   uint32_t* tmem_holder;
   volatile int* abort_flag;
 };
 
 // P buffers: 2 (double buffer) x PS parts (bf16: hi + lo) x pbuf_bytes.
+// Quantised latent: raw codes of one item (S: 128 rows x 64 channels; Z: 64
+// rows x 128 channels) are QB x 1024 bytes; Z scales of one tile 128 x r/128.
+__host__ __device__ constexpr int raw_bytes(int qb) { return qb * 1024; }
+__host__ __device__ inline int zscale_bytes(int r) { return 256 * (r / 128); }
+
 template <int NP, int QS, int PS>
-__device__ Smem carve(uint8_t* base, int ns, int nz) {
+__device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   Smem s;
   s.sring = base;
   s.zring = s.sring + size_t(ns) * s_slot_bytes<NP, QS>();
   s.pbuf = s.zring + size_t(nz) * kZSlotBytes;
-  uint8_t* m = s.pbuf + 2 * PS * pbuf_bytes<NP>();
+  s.sraw = s.pbuf + 2 * PS * pbuf_bytes<NP>();
+  s.zraw = s.sraw + size_t(nraw) * raw_bytes(qb);
+  s.zscale = s.zraw + size_t(nraw) * raw_bytes(qb);
+  uint8_t* m = s.zscale + (qb ? 2 * zscale_bytes(r) : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(m);
   s.s_full = bars;
   s.s_empty = bars + kMaxSlots;
@@ -301,9 +328,13 @@ __device__ Smem carve(uint8_t* base, int ns, int nz) {
   s.p_full = s.acc_full + 2;
   s.z_done = s.p_full + 2;
   s.drain = s.z_done + 2;
-  s.red = reinterpret_cast<float*>(m + 512);
-  s.tmem_holder = reinterpret_cast<uint32_t*>(m + 512 + 4 * NP * 4);
-  s.abort_flag = reinterpret_cast<volatile int*>(m + 512 + 4 * NP * 4 + 16);
+  s.sg_full = s.drain + 2;
+  s.sg_empty = s.sg_full + kMaxGroupBufs;
+  s.sraw_full = s.sg_empty + kMaxGroupBufs;
+  s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + 2 kMaxRaw = 64 barriers
+  s.red = reinterpret_cast<float*>(m + 640);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(m + 640 + 4 * NP * 4);
+  s.abort_flag = reinterpret_cast<volatile int*>(m + 640 + 4 * NP * 4 + 16);
   return s;
 }
 
@@ -339,6 +370,229 @@ __device__ __forceinline__ void ragged_rows(uint8_t* d, const uint8_t* src, size
   }
   fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
   __syncwarp();
+}
+
+// ------------------------------------------------- quantised latent rows
+// Symmetric int4 (two's complement nibbles, channel 2j in the low nibble of
+// byte j) and int8 codes, turned into exact fp16 integers by offset binary:
+// (code + 2^(b-1)) in the mantissa of 1024.0, minus (1024 + 2^(b-1)).
+
+// Eight int4 codes (one 32-bit word) -> four half2 as 32-bit words, channels
+// in order (o0 = c0 c1, o1 = c2 c3, o2 = c4 c5, o3 = c6 c7).  Nibbles 0 and 4,
+// 1 and 5 (then 2 and 6, 3 and 7 after a byte shift) land in the mantissas of
+// a half2 of 1024.0 each (the odd ones 16x too high, scaled back by an exact
+// fma); byte permutes restore channel order.
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ void int4x8_to_half(uint32_t w, __half2 s2, bool scaled, uint32_t& o0,
+                                               uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+  const uint32_t x = w ^ 0x88888888u;   // offset binary: code + 8 in 0..15
+  const __half2 b1032 = u2h(0x64086408u), s16 = u2h(0x2C002C00u), b72 = u2h(0xD480D480u);   // 1032, 1/16, -72
+  __half2 ha = __hsub2(u2h((x & 0x000F000Fu) | 0x64006400u), b1032);          // c0, c4
+  __half2 hb = __hfma2(u2h((x & 0x00F000F0u) | 0x64006400u), s16, b72);       // c1, c5
+  __half2 hc = __hsub2(u2h(((x >> 8) & 0x000F000Fu) | 0x64006400u), b1032);   // c2, c6
+  __half2 hd = __hfma2(u2h(((x >> 8) & 0x00F000F0u) | 0x64006400u), s16, b72); // c3, c7
+  if (scaled) { ha = __hmul2(ha, s2); hb = __hmul2(hb, s2); hc = __hmul2(hc, s2); hd = __hmul2(hd, s2); }
+  const uint32_t ua = h2u(ha), ub = h2u(hb), uc = h2u(hc), ud = h2u(hd);
+  o0 = __byte_perm(ua, ub, 0x5410);
+  o1 = __byte_perm(uc, ud, 0x5410);
+  o2 = __byte_perm(ua, ub, 0x7632);
+  o3 = __byte_perm(uc, ud, 0x7632);
+}
+// Four int8 codes (one 32-bit word) -> two half2 words: each byte (offset
+// binary) placed under an 0x64 high byte, minus 1024 + 128.
+__device__ __forceinline__ void int8x4_to_half(uint32_t w, __half2 s2, bool scaled, uint32_t& o0,
+                                               uint32_t& o1) {
+  const uint32_t x = w ^ 0x80808080u;
+  const __half2 bias = u2h(0x64806480u);   // 1152
+  __half2 lo = __hsub2(u2h(__byte_perm(x, 0x64646464u, 0x5140)), bias);
+  __half2 hi = __hsub2(u2h(__byte_perm(x, 0x64646464u, 0x5342)), bias);
+  if (scaled) { lo = __hmul2(lo, s2); hi = __hmul2(hi, s2); }
+  o0 = h2u(lo);
+  o1 = h2u(hi);
+}
+// One 16-byte vector of codes -> QB == 4: 32 channels (four 16-byte fp16
+// chunks), QB == 8: 16 channels (two chunks); optionally times a scale
+// (one fp16 rounding of the exact product).
+template <int QB>
+__device__ __forceinline__ void codes_to_half(const uint4& v, bool scaled, __half2 s2, uint4 (&out)[QB == 4 ? 4 : 2]) {
+  if (QB == 4) {
+    int4x8_to_half(v.x, s2, scaled, out[0].x, out[0].y, out[0].z, out[0].w);
+    int4x8_to_half(v.y, s2, scaled, out[1].x, out[1].y, out[1].z, out[1].w);
+    int4x8_to_half(v.z, s2, scaled, out[2].x, out[2].y, out[2].z, out[2].w);
+    int4x8_to_half(v.w, s2, scaled, out[3].x, out[3].y, out[3].z, out[3].w);
+  } else {
+    int8x4_to_half(v.x, s2, scaled, out[0].x, out[0].y);
+    int8x4_to_half(v.y, s2, scaled, out[0].z, out[0].w);
+    int8x4_to_half(v.z, s2, scaled, out[1].x, out[1].y);
+    int8x4_to_half(v.w, s2, scaled, out[1].z, out[1].w);
+  }
+}
+
+// Explicit shared-space 16-byte accesses (a generic pointer into shared
+// memory would be split into narrower generic stores).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// S item of a quantised tile from its raw codes in shared memory
+// ([128 rows][QB x 8 bytes]): channel box u as fp16 integers, unscaled (the
+// group scales are applied to S per token), in the 128-byte-swizzled K-major
+// layout; rows >= nv are zeros.  Warp-wide.
+template <int QB>
+__device__ __forceinline__ void convert_s_box(uint32_t d, uint32_t raw, int nv, int lane) {
+  constexpr int RPB = QB * 8;             // raw bytes per row: 32 (int4), 64 (int8)
+  constexpr int VPR = RPB / 16;           // 16-byte vectors per row
+  constexpr int CPV = QB == 4 ? 4 : 2;    // 16-byte fp16 chunks per vector
+  constexpr int NV = 128 * VPR / 32;      // vectors per lane: 8 (int4), 16 (int8)
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int v = lane + 32 * i, t = v / VPR, q = v % VPR;
+    const uint4 rv = t < nv ? lds128(raw + t * RPB + q * 16) : make_uint4(0, 0, 0, 0);
+    uint4 out[CPV];
+    codes_to_half<QB>(rv, false, __half2(), out);   // zero codes give zeros
+#pragma unroll
+    for (int c = 0; c < CPV; ++c) sts128(d + t * 128 + (((q * CPV + c) ^ (t & 7)) << 4), out[c]);
+  }
+  fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
+  __syncwarp();
+}
+
+// Z item of a quantised tile from its raw codes in shared memory ([64 rows]
+// [QB x 16 bytes]): channels 128 j .. 128 j + 127 of rows 64 h .. 64 h + 63,
+// dequantised (code x group scale, one fp16 rounding of the exact product),
+// two 64-channel boxes of 64 rows, 128-byte swizzled; rows >= nv are zeros.
+// tsc: the tile's scales [128][ngroups] (shared or global memory).
+template <int QB>
+__device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const __half* tsc,
+                                               int ngroups, int j, int h, int nv, int lane) {
+  constexpr int RPB = QB * 16;            // raw bytes per row: 64 (int4), 128 (int8)
+  constexpr int VPR = RPB / 16;
+  constexpr int CPV = QB == 4 ? 4 : 2;
+  constexpr int NV = 64 * VPR / 32;       // vectors per lane: 8 (int4), 16 (int8)
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR, t = 64 * h + tt;
+    const bool in = t < nv;
+    const uint4 rv = in ? lds128(raw + tt * RPB + q * 16) : make_uint4(0, 0, 0, 0);
+    const __half sc = in ? tsc[t * ngroups + j] : __float2half(0.f);
+    uint4 out[CPV];
+    codes_to_half<QB>(rv, true, __halves2half2(sc, sc), out);
+    const int ch = q * (CPV * 8);         // first channel of the vector within the 128
+    const int box = ch >> 6, c0 = (ch & 63) >> 3;
+#pragma unroll
+    for (int c = 0; c < CPV; ++c) sts128(d + box * kZBoxBytes + tt * 128 + (((c0 + c) ^ (tt & 7)) << 4), out[c]);
+  }
+  fence_proxy_async();
+  __syncwarp();
+}
+
+// Bulk (untiled) copy global -> shared, completion on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Producer of one ring for a quantised latent (warp-wide).  The raw codes of
+// each item arrive by TMA into a ring of nraw slots, issued nraw items ahead
+// (nraw <= items per tile); the warp converts them into the fp16 slot the
+// MMAs read (S: exact integers, plus the query box by TMA; Z: dequantised,
+// with the tile's scales, which ride with the tile's first Z item when their
+// block is 16-byte aligned and the tile is full).
+template <int NP, int QS, int QB>
+__device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, const CUtensorMap* tm_q,
+                          const __half* scales, const int32_t* sched, int B, int r, int max_len,
+                          long long tb, long long te, int n, int nslots, int nraw, int lane,
+                          long long* issued, long long* raw_issued) {
+  const int NI = r / 64, NG = r / 128;
+  uint8_t* ring = kind == 0 ? s.sring : s.zring;
+  const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
+  uint64_t* full = kind == 0 ? s.s_full : s.z_full;
+  uint64_t* empty = kind == 0 ? s.s_empty : s.z_empty;
+  uint8_t* raw = kind == 0 ? s.sraw : s.zraw;
+  uint64_t* rfull = kind == 0 ? s.sraw_full : s.zraw_full;
+  const uint32_t ring0 = saddr(ring), raw0 = saddr(raw), zsc0 = saddr(s.zscale);
+  constexpr uint32_t RB = uint32_t(raw_bytes(QB));
+  const uint32_t ZSB = uint32_t(zscale_bytes(r));
+  const long long total = (long long)n * NI;
+  // issue side: nraw items ahead of the conversion
+  TileIter ia;
+  ia.init(sched, B, tb, te);
+  int ia_i = 0, ua = 0;
+  long long ki = 0;
+  auto issue_one = [&]() {
+    const int slot = int(ki % nraw);
+    const uint32_t fb = saddr(&rfull[slot]);
+    const int row = ia.b * max_len + ia.t0();
+    const size_t sc_off = size_t(row) * NG * 2;
+    const bool sc_bulk = kind == 1 && ua == 0 && ia.nvalid() == kTile && sc_off % 16 == 0;
+    if (lane == int(ki & 31)) {   // rotating issuing lane
+      mbar_expect_tx(fb, RB + (sc_bulk ? ZSB : 0u));
+      if (kind == 0) tma_load_2d(raw0 + slot * RB, tm_raw, ua * (QB * 8), row, fb);
+      else tma_load_2d(raw0 + slot * RB, tm_raw, (ua >> 1) * (QB * 16), row + 64 * (ua & 1), fb);
+      if (sc_bulk)
+        bulk_load(zsc0 + (ia_i & 1) * ZSB, reinterpret_cast<const uint8_t*>(scales) + sc_off, ZSB, fb);
+    }
+    ++ki;
+    if (++ua == NI) {
+      ua = 0;
+      if (++ia_i < n) ia.next();
+    }
+  };
+  for (long long x = 0; x < total && x < nraw; ++x) issue_one();
+  TileIter it;
+  it.init(sched, B, tb, te);
+  Ring rg(nslots);
+  long long k = 0;
+  for (int i = 0; i < n; ++i) {
+    const int nv = it.nvalid(), b = it.b;
+    const int row = b * max_len + it.t0();
+    const size_t sc_off = size_t(row) * NG * 2;
+    const bool sc_smem = kind == 1 && nv == kTile && sc_off % 16 == 0;
+    const __half* tsc = sc_smem ? reinterpret_cast<const __half*>(s.zscale + (i & 1) * ZSB)
+                                : scales + size_t(row) * NG;
+    for (int u = 0; u < NI; ++u) {
+      const int rs = int(k % nraw);
+      if (!__all_sync(0xffffffffu, mbar_wait(saddr(&rfull[rs]), uint32_t(k / nraw) & 1u)) ||
+          !__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
+        *issued = k;
+        *raw_issued = ki;
+        return false;
+      }
+      const uint32_t dst = ring0 + uint32_t(rg.slot) * slot_bytes;
+      const uint32_t fb = saddr(&full[rg.slot]);
+      if (kind == 0) {
+        if (lane == 0) {   // the query box; the slot completes on this and the codes' arrival
+          mbar_expect_tx(fb, uint32_t(QS * NP * 128));
+          tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
+        }
+        convert_s_box<QB>(dst, raw0 + uint32_t(rs) * RB, nv, lane);
+      } else {
+        convert_z_item<QB>(dst, raw0 + uint32_t(rs) * RB, tsc, NG, u >> 1, u & 1, nv, lane);
+      }
+      if (lane == 0) mbar_arrive(fb);
+      // the raw slot has been read: refill it nraw items ahead
+      if (ki < total) issue_one();
+      __syncwarp();
+      rg.advance();
+      ++k;
+    }
+    it.next();
+    if (__any_sync(0xffffffffu, *s.abort_flag)) {
+      *issued = k;
+      *raw_issued = ki;
+      return false;
+    }
+  }
+  *issued = k;
+  *raw_issued = ki;
+  return true;
 }
 
 // Producer of one ring (warp-wide).  kind 0: S ring (latent box from HBM,
@@ -423,19 +677,24 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int NP, bool BF16, int QS, int PS>
+// QB = 0: 16-bit latent; QB = 4 / 8: int4 / int8 codes with fp16 scales per
+// group of 128 channels (S per group into a ring of nsg TMEM buffers, the
+// scales applied per token by the softmax; Z from the dequantised latent).
+template <int NP, bool BF16, int QS, int PS, int QB>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
            const __grid_constant__ CUtensorMap tm_q,
-           const uint8_t* __restrict__ cache, const int32_t* __restrict__ sched,
+           const uint8_t* __restrict__ cache, const __half* __restrict__ scales,
+           const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
-           int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz) {
+           int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz,
+           int nsg, int nraw) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const Smem s = carve<NP, QS, PS>(base, ns, nz);
+  const Smem s = carve<NP, QS, PS>(base, ns, nz, nraw, QB, r);
   constexpr int SW = QS * NP;                 // S accumulator columns per buffer
-  constexpr int ZC0 = 2 * SW;                 // first Z column
+  const int ZC0 = (QB ? nsg : 2) * SW;        // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = r / 64;                      // ring items per tile
   const int NC = r / 128;                     // 128-channel Z accumulator chunks
@@ -447,8 +706,16 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
-      mbar_init(saddr(&s.s_full[i]), 1);
+      mbar_init(saddr(&s.s_full[i]), QB ? 2 : 1);   // quantised: query TMA + converted codes
       mbar_init(saddr(&s.s_empty[i]), 1);
+    }
+    for (int i = 0; i < kMaxGroupBufs; ++i) {
+      mbar_init(saddr(&s.sg_full[i]), 1);
+      mbar_init(saddr(&s.sg_empty[i]), 1);
+    }
+    for (int i = 0; i < kMaxRaw; ++i) {
+      mbar_init(saddr(&s.sraw_full[i]), 1);
+      mbar_init(saddr(&s.zraw_full[i]), 1);
     }
     for (int i = 0; i < nz; ++i) {
       mbar_init(saddr(&s.z_full[i]), 1);
@@ -478,13 +745,18 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     // ----------------------------------------------------------- producers
     const int kind = warp >> 1;
     const int nslots = kind == 0 ? ns : nz;
-    long long issued = 0;
-    if (!produce<NP, QS>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te, n, nslots,
-                         lane, &issued)) {
-      if (lane == 0) {
-        set_abort(s, status);
-        drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
-      }
+    long long issued = 0, raw_issued = 0;
+    bool ok;
+    if constexpr (QB != 0)   // quantised latent: tm_cs / tm_cz map the raw codes
+      ok = produce_q<NP, QS, QB>(kind, s, kind == 0 ? &tm_cs : &tm_cz, &tm_q, scales, sched, B, r,
+                                 max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
+    else
+      ok = produce<NP, QS>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te, n,
+                           nslots, lane, &issued);
+    if (!ok && lane == 0) {
+      set_abort(s, status);
+      drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
+      if (QB) drain_ring(kind == 0 ? s.sraw_full : s.zraw_full, raw_issued, nraw);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -493,27 +765,38 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       constexpr uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
       const uint64_t da0 = sdesc(saddr(s.sring), 16, 1024);   // K-major, 128B swizzle
       Ring rg(ns);
+      Ring gr(QB ? nsg : 1);   // quantised latent: per-group S buffers
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
         // the accumulator buffer of tile i was last read by the softmax of tile i - 2
-        if (i >= 2 && !mbar_wait(saddr(&s.p_full[i & 1]), uint32_t((i - 2) >> 1) & 1u)) { ok = false; break; }
-        const uint32_t d = tmem + uint32_t((i & 1) * SW);
+        if (!QB && i >= 2 && !mbar_wait(saddr(&s.p_full[i & 1]), uint32_t((i - 2) >> 1) & 1u)) { ok = false; break; }
+        uint32_t d = tmem + uint32_t((i & 1) * SW);
         for (int u = 0; u < NI; ++u) {
+          if (QB && (u & 1) == 0) {
+            // a group (128 channels, two boxes) starts: its buffer must be free
+            if (!mbar_wait(saddr(&s.sg_empty[gr.slot]), gr.phase ^ 1u)) { ok = false; break; }
+            d = tmem + uint32_t(gr.slot * SW);
+          }
           if (!mbar_wait(saddr(&s.s_full[rg.slot]), rg.phase)) { ok = false; break; }
           tc_fence_after();
           // descriptor address field is in 16-byte units
           const uint64_t sa = da0 + uint64_t((rg.slot * s_slot_bytes<NP, QS>()) >> 4);
+          const int first = QB ? (u & 1) : u;   // accumulate from the group's (or tile's) first box on
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {   // K = 16 channels per MMA
             const uint64_t a = sa + uint64_t((kk * 32) >> 4);
             const uint64_t bd = sa + uint64_t((kBoxBytes + kk * 32) >> 4);
-            tc_mma(d, a, bd, id_s, (u | kk) != 0);
+            tc_mma(d, a, bd, id_s, (first | kk) != 0);
           }
           tc_commit(saddr(&s.s_empty[rg.slot]));
           rg.advance();
+          if (QB && (u & 1) == 1) {
+            tc_commit(saddr(&s.sg_full[gr.slot]));
+            gr.advance();
+          }
         }
         if (!ok) break;
-        tc_commit(saddr(&s.acc_full[i & 1]));
+        if (!QB) tc_commit(saddr(&s.acc_full[i & 1]));
         if (*s.abort_flag) ok = false;
       }
       if (!ok) set_abort(s, status);
@@ -571,6 +854,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     float m_run[NP], l_part[NP];
     TileIter it;
     it.init(sched, B, tb, te);
+    Ring sgr(QB ? nsg : 1);   // quantised latent: the per-group S buffers
     for (int i = 0; i < n; ++i) {
       const int pb = i & 1;
       const bool first = it.first(tb), last = it.last();
@@ -579,22 +863,51 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 #pragma unroll
         for (int h = 0; h < NP; ++h) { m_run[h] = -INFINITY; l_part[h] = 0.f; }
       }
-      int fail = !mbar_wait(saddr(&s.acc_full[pb]), uint32_t(i >> 1) & 1u);
-      if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
-      tc_fence_after();
+      int fail = 0;
       float sv[NP];
+      if (QB) {
+        // s_t = sum_g scale_{t,g} (codes_{t,g} . qt_g), one TMEM buffer per group
 #pragma unroll
-      for (int c = 0; c < NP / 16; ++c) tmem_ld16(tmem + lane_off + uint32_t(pb * SW + 16 * c), sv + 16 * c);
-      if (QS == 2) {   // S = C (q_hi + q_lo)
-        float lo[NP];
+        for (int h = 0; h < NP; ++h) sv[h] = 0.f;
+        const __half* tsc = scales + (size_t(it.b) * max_len + it.t0() + t) * NC;
+        for (int g = 0; g < NC; ++g) {
+          const float sg = t < nv ? __half2float(tsc[g]) : 0.f;
+          fail = group_or(!mbar_wait(saddr(&s.sg_full[sgr.slot]), sgr.phase));   // uniform
+          if (fail) break;
+          tc_fence_after();
+          const uint32_t tg = tmem + lane_off + uint32_t(sgr.slot * SW);
 #pragma unroll
-        for (int c = 0; c < NP / 16; ++c)
-          tmem_ld16(tmem + lane_off + uint32_t(pb * SW + NP + 16 * c), lo + 16 * c);
+          for (int c = 0; c < NP / 16; ++c) {
+            float hi[16], lo[16];
+            tmem_ld16(tg + uint32_t(16 * c), hi);
+            tmem_ld16(tg + uint32_t(NP + 16 * c), lo);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) sv[16 * c + e] = fmaf(sg, hi[e] + lo[e], sv[16 * c + e]);
+          }
+          tc_fence_before();
+          group_sync();
+          if (t == 0) mbar_arrive(saddr(&s.sg_empty[sgr.slot]));
+          sgr.advance();
+        }
+        if (fail) { if (t == 0) set_abort(s, status); break; }
+      } else {
+        fail = !mbar_wait(saddr(&s.acc_full[pb]), uint32_t(i >> 1) & 1u);
+        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < NP / 16; ++c) tmem_ld16(tmem + lane_off + uint32_t(pb * SW + 16 * c), sv + 16 * c);
+        if (QS == 2) {   // S = C (q_hi + q_lo)
+          float lo[NP];
+#pragma unroll
+          for (int c = 0; c < NP / 16; ++c)
+            tmem_ld16(tmem + lane_off + uint32_t(pb * SW + NP + 16 * c), lo + 16 * c);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < NP; ++h) sv[h] += lo[h];
+        }
         tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < NP; ++h) sv[h] += lo[h];
       }
-      tmem_wait_ld();
       const bool valid = t < nv;
       int need = 0;
 #pragma unroll
@@ -742,8 +1055,8 @@ void ring_slots(int* ns, int* nz) {
   *nz = z;
 }
 
-template <int NP, bool BF16>
-cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
+template <int NP, bool BF16, int QB>
+cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                      const int32_t* sched, int G, float* pm, float* pl, float* pz,
                      int32_t* status, cudaStream_t s) {
   TensorMapEncode enc = tensor_map_encoder();
@@ -753,7 +1066,26 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
   const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t rows = cuuint64_t(d.batch) * d.max_len;
   CUtensorMap tcs, tcz, tq;
-  {
+  memset(&tcs, 0, sizeof(tcs));
+  memset(&tcz, 0, sizeof(tcz));
+  if (QB) {
+    // quantised latent: raw code rows [B * max_len][r QB / 8] bytes; S item
+    // box {QB x 8 bytes, 128 rows} (64 channels), Z item box {QB x 16 bytes,
+    // 64 rows} (128 channels); no swizzle (the warps convert them)
+    const cuuint64_t rb = cuuint64_t(d.r) * QB / 8;
+    const cuuint64_t dims[2] = {rb, rows};
+    const cuuint64_t strides[1] = {rb};
+    const cuuint32_t es[2] = {1, 1};
+    const cuuint32_t bs[2] = {cuuint32_t(QB * 8), 128}, bz[2] = {cuuint32_t(QB * 16), 64};
+    if (enc(&tcs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides, bs, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        enc(&tcz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides, bz, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  if (!QB) {
     // S items: latent rows [B * max_len][r], one box {64 channels, 128 rows}
     const cuuint64_t dims[2] = {cuuint64_t(d.r), rows};
     const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
@@ -764,7 +1096,7 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
+  if (!QB) {
     // Z items: the same rows seen as {64 channels, row, 64-channel box}; one
     // box {64, 64, 2} is 64 tokens x 128 channels, smem [box][row][64]
     const cuuint64_t dims[3] = {64, rows, cuuint64_t(d.r / 64)};
@@ -790,16 +1122,34 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* qt16,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  int ns = 0, nz = 0;
+  int ns = 0, nz = 0, nraw = 0;
   ring_slots<NP, QS, PS>(&ns, &nz);
+  if constexpr (QB != 0) {
+    // quantised latent: the fp16 slots are filled by conversion (short
+    // latency), so three of each; the raw-code rings take the rest, at most
+    // one tile of items ahead (the Z scales are double-buffered per tile)
+    ns = nz = 3;
+    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>() - 2 * zscale_bytes(d.r) -
+                      ns * s_slot_bytes<NP, QS>() - nz * kZSlotBytes;
+    nraw = avail / (2 * raw_bytes(QB));
+    if (nraw > kMaxRaw) nraw = kMaxRaw;
+    if (nraw > d.r / 64) nraw = d.r / 64;
+    if (nraw < 2) return cudaErrorInvalidConfiguration;
+  }
   if (ns < 2 || nz < 2) return cudaErrorInvalidConfiguration;
+  // quantised latent: per-group S buffers in the TMEM left beside Z
+  int nsg = (512 - (d.r / 128) * NP) / (QS * NP);
+  if (nsg > kMaxGroupBufs) nsg = kMaxGroupBufs;
+  if (QB && nsg < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + size_t(ns) * s_slot_bytes<NP, QS>() + size_t(nz) * kZSlotBytes +
-                      2 * PS * pbuf_bytes<NP>() + kMiscBytes;
-  auto kern = k_split_tc<NP, BF16, QS, PS>;
+                      2 * PS * pbuf_bytes<NP>() +
+                      (QB ? 2 * size_t(nraw) * raw_bytes(QB) + 2 * zscale_bytes(d.r) : 0) + kMiscBytes;
+  auto kern = k_split_tc<NP, BF16, QS, PS, QB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<G, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache), sched, pm, pl,
-                                   pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz);
+  kern<<<G, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache),
+                                   static_cast<const __half*>(scales), sched, pm, pl, pz, status,
+                                   d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw);
   note_launch();
   return check_launch();
 }
@@ -810,23 +1160,34 @@ int split_tc_heads_padded(const qsvd_dims& d) { return d.H <= 16 ? 16 : (d.H <= 
 
 bool split_tc_supported(const qsvd_dims& d) {
   if (d.rope) return false;
-  if (d.cache_dtype != QSVD_F16 && d.cache_dtype != QSVD_BF16) return false;
+  const bool q = d.cache_dtype == QSVD_I4 || d.cache_dtype == QSVD_I8;
+  if (d.cache_dtype != QSVD_F16 && d.cache_dtype != QSVD_BF16 && !q) return false;
+  if (q && d.group != 128) return false;   // one scale group = one 128-channel Z chunk
   if (d.r % 128) return false;
   const int np = split_tc_heads_padded(d);
   if (np == 0) return false;
-  if ((2 * 2 + d.r / 128) * np > 512) return false;   // two S buffers of 2 np + Z
+  if ((2 * 2 + d.r / 128) * np > 512) return false;   // two S buffers (or group buffers) of 2 np + Z
   return true;
 }
 
-cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* qt16,
+cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s) {
-  const bool bf = d.cache_dtype == QSVD_BF16;
   const int np = split_tc_heads_padded(d);
-  if (np == 16) return bf ? launch_t<16, true>(d, cache, qt16, sched, G, pm, pl, pz, status, s)
-                          : launch_t<16, false>(d, cache, qt16, sched, G, pm, pl, pz, status, s);
-  return bf ? launch_t<32, true>(d, cache, qt16, sched, G, pm, pl, pz, status, s)
-            : launch_t<32, false>(d, cache, qt16, sched, G, pm, pl, pz, status, s);
+  switch (d.cache_dtype) {
+    case QSVD_BF16:
+      return np == 16 ? launch_t<16, true, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, true, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+    case QSVD_I4:
+      return np == 16 ? launch_t<16, false, 4>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 4>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+    case QSVD_I8:
+      return np == 16 ? launch_t<16, false, 8>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 8>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+    default:
+      return np == 16 ? launch_t<16, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+  }
 }
 
 }  // namespace qsvd

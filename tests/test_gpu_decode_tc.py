@@ -1,5 +1,6 @@
 """Parity of the tensor-core split kernel (tcgen05 + TMA, absorbed query,
-fp16/bf16 latent) against the fp64 oracle and against the CUDA-core kernel.
+fp16/bf16 latent, int4/int8 latent with group scales) against the fp64
+oracle and against the CUDA-core kernel.
 
 Bar: max |o_gpu - o_ref| / rms(o_ref) <= 2e-3 (P and the absorbed query are
 rounded to the latent's 16-bit type before the MMA; accumulation is fp32).
@@ -29,6 +30,11 @@ def case(key):
             "h32": synthetic.replace(base, E=4096, H=32, r=384, B=2, L=520),
             "r768": synthetic.replace(base, E=1024, H=8, r=768, B=2, L=700),
             "full": synthetic.replace(base, B=2, L=512),       # whole tiles only
+            # quantised latents: per-group S buffers, dequantised Z
+            "i4": synthetic.SHRUNK[3],                           # r 384, H2, ragged tail
+            "i8": synthetic.replace(synthetic.SHRUNK[3], cache="i8", name="shrunk-int8-h2"),
+            "i4h32": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=768, B=2, L=600,
+                                       h2_n=256),
         }[key]
         if w.E > 1024:
             # direct seeded factors: skips the E x 3E SVD, which decode parity does not need
@@ -40,7 +46,7 @@ def case(key):
     return _CASES[key]
 
 
-@pytest.mark.parametrize("key", ["full", "f16", "bf16", "h32", "r768"])
+@pytest.mark.parametrize("key", ["full", "f16", "bf16", "h32", "r768", "i4", "i8", "i4h32"])
 def test_tc_matches_oracle(cuda_ok, key):
     c = case(key)
     g = GpuCase(c, kernel=TC)
@@ -50,7 +56,7 @@ def test_tc_matches_oracle(cuda_ok, key):
     assert err <= TOL, f"{key}: {err:.3e}"
 
 
-@pytest.mark.parametrize("key", ["f16", "bf16"])
+@pytest.mark.parametrize("key", ["f16", "bf16", "i4", "i8"])
 def test_tc_agrees_with_simt(cuda_ok, key):
     c = case(key)
     a, _ = GpuCase(c, kernel=TC).decode()
