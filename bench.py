@@ -333,7 +333,8 @@ def run_ours(args, rank, world, local_rank):
     split_mean = statistics.mean(split_ms)
     lat_b = latent_bytes(w, lens)
     achieved = lat_b / (split_mean / 1e3) / 1e9
-    kname = ("k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05
+    kname = ("k_rope_scores" if (w.rope and kernel_used == q.QSVD_KERNEL_TCGEN05)
+             else "k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05
              else "k_split_rope" if w.rope else "k_split_abs")
     src = ["split_tc.cu", "internal.cuh"] if kname == "k_split_tc" else ["split_simt.cu", "internal.cuh"]
     workload = w.name

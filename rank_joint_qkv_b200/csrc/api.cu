@@ -93,6 +93,7 @@ static int device_sms() {
 static int pick_kernel(const qsvd_dims& d) {
   if (d.kernel == QSVD_KERNEL_SIMT) return QSVD_KERNEL_SIMT;
   if (d.kernel == QSVD_KERNEL_TCGEN05) return QSVD_KERNEL_TCGEN05;
+  if (d.rope) return rope_tc_supported(d) ? QSVD_KERNEL_TCGEN05 : QSVD_KERNEL_SIMT;
   return split_tc_supported(d) ? QSVD_KERNEL_TCGEN05 : QSVD_KERNEL_SIMT;
 }
 
@@ -103,7 +104,7 @@ static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel
   if (g == 0) {
     const int sms = device_sms();
     if (sms <= 0) return fail(QSVD_ERR_CUDA, "no CUDA device to size the split grid");
-    if (kernel == QSVD_KERNEL_TCGEN05) {
+    if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope) {   // rotary: the softmax runs on CUDA cores
       g = sms;
     } else {
       const int hb = split_simt_grid_heads(d);
@@ -204,9 +205,12 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
   if (phases == 0) phases = QSVD_PHASE_ALL;
   if (phases & ~QSVD_PHASE_ALL) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
   const int kernel = pick_kernel(d);
-  if (kernel == QSVD_KERNEL_TCGEN05 && !split_tc_supported(d))
+  if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope && !split_tc_supported(d))
     return fail(QSVD_ERR_UNSUPPORTED,
-                "tensor-core split kernel needs a 16-bit cache, no rotary, r %% 128 == 0, H <= 32");
+                "tensor-core split kernel needs a 16-bit or int4/int8 (group 128) cache, r %% 128 == 0, H <= 32");
+  if (kernel == QSVD_KERNEL_TCGEN05 && d.rope && !rope_tc_supported(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "tensor-core rotary path needs d_h == 128, r %% 64 == 0, cache and weights both fp16 or both bf16");
   if (kernel == QSVD_KERNEL_SIMT && !d.rope && split_simt_grid_heads(d) == 0)
     return fail(QSVD_ERR_UNSUPPORTED, "rank too large for the CUDA-core split kernel");
   int G = 0;
@@ -261,8 +265,16 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (phases & QSVD_PHASE_SPLIT) {
-    if (d.rope)
+    if (d.rope && kernel == QSVD_KERNEL_TCGEN05) {
+      float* scores = reinterpret_cast<float*>(Wb + W.scores);
+      const int sms = device_sms();
+      e = launch_rope_scores(d, cache, P + L.wukT, qt32, rope_tab, sched, sms > 0 ? sms : 1, scores,
+                             &hdr->status, s);
+      if (e == cudaSuccess)
+        e = launch_split_simt_scores(d, scores, cache, scales, sched, G, pm, pl, pz, s);
+    } else if (d.rope) {
       e = launch_split_simt_rope(d, qt32, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
+    }
     else if (kernel == QSVD_KERNEL_TCGEN05)
       e = launch_split_tc(d, cache, scales, qt16, sched, G, pm, pl, pz, &hdr->status, s);
     else

@@ -79,7 +79,7 @@ struct WsHeader {
 };
 
 struct WsLayout {
-  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, total;
+  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, scores, total;
   int G, P, KS, JS, NT;
 };
 
@@ -109,6 +109,7 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.pl = o;    o = align256(o + size_t(w.P) * H * 4);
   w.pz = o;    o = align256(o + size_t(w.P) * H * r * 4);
   w.opart = o; o = align256(o + size_t(w.JS) * B * E * 4);
+  w.scores = o; if (d.rope) o = align256(o + B * H * size_t(d.max_len) * 4);   // rotary: [B][H][max_len]
   w.total = o;
   return w;
 }
@@ -147,6 +148,16 @@ cudaError_t launch_split_simt_absorbed(const qsvd_dims& d, const float* qt32,
                                        const void* cache, const void* scales,
                                        const int32_t* sched, int G, float* pm,
                                        float* pl, float* pz, cudaStream_t s);
+// Rotary mode on the tensor cores: keys rebuilt from the latent, rotated,
+// scored against the rotary query into `scores` ([B][H][max_len]); then the
+// CUDA-core split kernel runs the softmax and the latent accumulation on them.
+bool rope_tc_supported(const qsvd_dims& d);
+cudaError_t launch_rope_scores(const qsvd_dims& d, const void* cache, const void* wukT,
+                               const float* qrot, const float* rope_tab, const int32_t* sched,
+                               int G, float* scores, int32_t* status, cudaStream_t s);
+cudaError_t launch_split_simt_scores(const qsvd_dims& d, const float* scores, const void* cache,
+                                     const void* scales, const int32_t* sched, int G, float* pm,
+                                     float* pl, float* pz, cudaStream_t s);
 cudaError_t launch_split_simt_rope(const qsvd_dims& d, const float* qrot,
                                    const void* wuk, const float* rope_tab,
                                    const void* cache, const void* scales,

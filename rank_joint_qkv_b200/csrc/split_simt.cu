@@ -88,12 +88,14 @@ __device__ __forceinline__ void stage_rows(float* dst, int ld, int TS, const uin
 // Absorbed split kernel.  grid (G, H/HB), block 256.
 // smem: qs[HB][r], cs[TS][r], zs[HB][r] (float), sc[TS*HB], red[8][64].
 // ---------------------------------------------------------------------------
-template <qsvd_dtype CT, int HB>
+// SG: the scores come precomputed (rotary mode: [B][H][max_len], log2 domain,
+// scaled) instead of from the absorbed query.
+template <qsvd_dtype CT, int HB, bool SG = false>
 __global__ void __launch_bounds__(kThreads)
 k_split_abs(const float* __restrict__ qt32, const uint8_t* __restrict__ cache,
             const __half* __restrict__ scales, const int32_t* __restrict__ sched,
             float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
-            int B, int H, int r, int max_len, int group, int G) {
+            int B, int H, int r, int max_len, int group, int G, const float* __restrict__ sgiven = nullptr) {
   constexpr int TS = 8;             // tokens per sub-tile
   constexpr int NV = TS * HB;       // scores per sub-tile
   extern __shared__ float sm[];
@@ -133,7 +135,7 @@ k_split_abs(const float* __restrict__ qt32, const uint8_t* __restrict__ cache,
     __syncthreads();
     for (int i = threadIdx.x; i < HB * r; i += kThreads) {
       const int hh = i / r, j = i % r;
-      qs[i] = qt32[(size_t(b) * H + h0 + hh) * r + j];
+      if (!SG) qs[i] = qt32[(size_t(b) * H + h0 + hh) * r + j];
       zs[i] = 0.f;
     }
     if (threadIdx.x < HB) { m_s[threadIdx.x] = -INFINITY; l_s[threadIdx.x] = 0.f; }
@@ -143,6 +145,12 @@ k_split_abs(const float* __restrict__ qt32, const uint8_t* __restrict__ cache,
       __syncthreads();
       stage_rows<CT>(cs, r, TS, seq_base, seq_scales, row_bytes, r, group, s0, nv);
       __syncthreads();
+      if (SG) {   // scores given: sc[tt][hh]
+        if (threadIdx.x < NV) {
+          const int tt = threadIdx.x / HB, hh = threadIdx.x % HB;
+          sc[threadIdx.x] = tt < nv ? sgiven[(size_t(b) * H + h0 + hh) * max_len + s0 + tt] : 0.f;
+        }
+      } else {
       // scores: each thread a strided slice of the channels
       float acc[NV];
 #pragma unroll
@@ -172,6 +180,7 @@ k_split_abs(const float* __restrict__ qt32, const uint8_t* __restrict__ cache,
 #pragma unroll
         for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
         sc[threadIdx.x] = s;
+      }
       }
       __syncthreads();
       // online softmax per head (log2 domain)
@@ -376,19 +385,32 @@ int head_block(const qsvd_dims& d) {
   return 0;
 }
 
-template <qsvd_dtype CT, int HB>
+template <qsvd_dtype CT, int HB, bool SG = false>
 cudaError_t abs_t(const qsvd_dims& d, const float* qt32, const void* cache, const void* scales,
-                  const int32_t* sched, int G, float* pm, float* pl, float* pz, cudaStream_t s) {
+                  const int32_t* sched, int G, float* pm, float* pl, float* pz, cudaStream_t s,
+                  const float* sgiven = nullptr) {
   const size_t smem = size_t(2 * HB + 8) * d.r * 4;
-  auto kern = k_split_abs<CT, HB>;
+  auto kern = k_split_abs<CT, HB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(G, d.H / HB);
   kern<<<grid, kThreads, smem, s>>>(qt32, static_cast<const uint8_t*>(cache),
                                     static_cast<const __half*>(scales), sched, pm, pl, pz,
-                                    d.batch, d.H, d.r, d.max_len, d.group, G);
+                                    d.batch, d.H, d.r, d.max_len, d.group, G, sgiven);
   note_launch();
   return check_launch();
+}
+
+template <qsvd_dtype CT>
+cudaError_t scores_ct(const qsvd_dims& d, const float* sgiven, const void* cache, const void* scales,
+                      const int32_t* sched, int G, float* pm, float* pl, float* pz, cudaStream_t s) {
+  switch (head_block(d)) {
+    case 8: return abs_t<CT, 8, true>(d, nullptr, cache, scales, sched, G, pm, pl, pz, s, sgiven);
+    case 4: return abs_t<CT, 4, true>(d, nullptr, cache, scales, sched, G, pm, pl, pz, s, sgiven);
+    case 2: return abs_t<CT, 2, true>(d, nullptr, cache, scales, sched, G, pm, pl, pz, s, sgiven);
+    case 1: return abs_t<CT, 1, true>(d, nullptr, cache, scales, sched, G, pm, pl, pz, s, sgiven);
+    default: return cudaErrorInvalidConfiguration;
+  }
 }
 
 template <qsvd_dtype CT>
@@ -451,6 +473,16 @@ cudaError_t launch_split_simt_absorbed(const qsvd_dims& d, const float* qt32, co
     case QSVD_I4: return abs_ct<QSVD_I4>(d, qt32, cache, scales, sched, G, pm, pl, pz, s);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_split_simt_scores(const qsvd_dims& d, const float* scores, const void* cache,
+                                     const void* scales, const int32_t* sched, int G, float* pm,
+                                     float* pl, float* pz, cudaStream_t s) {
+  switch (d.cache_dtype) {
+    case QSVD_F16: return scores_ct<QSVD_F16>(d, scores, cache, scales, sched, G, pm, pl, pz, s);
+    case QSVD_BF16: return scores_ct<QSVD_BF16>(d, scores, cache, scales, sched, G, pm, pl, pz, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_split_simt_rope(const qsvd_dims& d, const float* qrot, const void* wuk,

@@ -1032,6 +1032,220 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
   }
 }
 
+// ---------------------------------------------------------------------------
+// Rotary scores on the tensor cores (rotary mode, d_h = 128).
+//
+//   K_h = C_tile W^u_{k,h}      (128 tokens x 128, K = r)   tcgen05, two heads
+//                                                            per MMA (N = 256)
+//   s_{t,h} = (R(t) K_{h,t}) . q'_h                          CUDA cores
+//
+// where q'_h is the query already rotated to its position and scaled by
+// tau log2(e) (the prologue's rotary query).  Keys are rebuilt from the
+// shared latent as the QSVD digest's rotary reading requires (Method, Step
+// 1); the scores go to the workspace, [B][H][max_len] fp32, and the split
+// kernel that follows takes them instead of computing C . q~.
+//
+// Per CTA: the flattened tile range of the split schedule.  Per tile and head
+// pair the producer streams (latent box, W^u_k^T box) pairs through a ring,
+// one thread issues the MMAs into one of two TMEM buffers (256 columns each),
+// and four epilogue warps (one TMEM lane per token) apply the rotation with
+// the token's cos/sin row, staged once per tile in shared memory, and take the
+// dot products.  Every wait is bounded as in k_split_tc.
+// ---------------------------------------------------------------------------
+constexpr int kRopeSlotBytes = kBoxBytes + 256 * 128;   // latent box + 256 rows of W^u_k^T
+constexpr int kRopeTabPitch = 65;                        // floats per token row (bank-conflict free)
+
+template <bool BF16>
+__global__ void __launch_bounds__(192, 1)
+k_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_w,
+              const float* __restrict__ qrot, const float* __restrict__ rope_tab,
+              const int32_t* __restrict__ sched, float* __restrict__ scores, int32_t* __restrict__ status,
+              int B, int H, int E, int r, int max_len, int G, int ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = base;
+  float* tab_c = reinterpret_cast<float*>(ring + size_t(ns) * kRopeSlotBytes);   // [128][65] cos
+  float* tab_s = tab_c + 128 * kRopeTabPitch;                                       // [128][65] sin
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tab_s + 128 * kRopeTabPitch);
+  uint64_t* full = bars;                  // [kMaxSlots]
+  uint64_t* empty = bars + kMaxSlots;     // [kMaxSlots]
+  uint64_t* kfull = bars + 2 * kMaxSlots; // [2]
+  uint64_t* kempty = kfull + 2;           // [2]
+  uint64_t* drain = kempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NI = r / 64, NPAIR = (H + 1) / 2;
+  const long long T = sched[B];
+  const long long tb = dev::split_begin(blockIdx.x, G, T);
+  const long long te = dev::split_begin(blockIdx.x + 1, G, T);
+  if (tb >= te) return;   // uniform across the CTA, before any barrier or TMEM use
+  const int n = int(te - tb);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(saddr(&full[i]), 1);
+      mbar_init(saddr(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(saddr(&kfull[i]), 1);
+      mbar_init(saddr(&kempty[i]), 1);
+    }
+    mbar_init(saddr(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     saddr(tmem_holder))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t ring0 = saddr(ring);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    TileIter it;
+    it.init(sched, B, tb, te);
+    Ring rg(ns);
+    long long k = 0;
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int row = it.b * max_len + it.t0();   // rows past the length give keys nobody reads
+      for (int p = 0; p < NPAIR && ok; ++p)
+        for (int u = 0; u < NI; ++u) {
+          if (!__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) { ok = false; break; }
+          const uint32_t dst = ring0 + uint32_t(rg.slot) * kRopeSlotBytes;
+          const uint32_t fb = saddr(&full[rg.slot]);
+          if (lane == 0) mbar_expect_tx(fb, uint32_t(kRopeSlotBytes));
+          __syncwarp();
+          const int ln = int(k & 15) * 2;   // rotating issuing lanes
+          if (lane == ln) tma_load_2d(dst, &tm_c, 64 * u, row, fb);
+          if (lane == ln + 1) tma_load_2d(dst + kBoxBytes, &tm_w, 64 * u, 256 * p, fb);   // rows >= E are zeros
+          __syncwarp();
+          rg.advance();
+          ++k;
+        }
+      it.next();
+      if (__any_sync(0xffffffffu, *abort_flag)) ok = false;
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(status, QSVD_STATUS_TIMEOUT);
+      drain_ring(full, k, ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t id = idesc_f16(128, 256, BF16, false, false);
+      const uint64_t da0 = sdesc(ring0, 16, 1024);   // K-major, 128B swizzle
+      Ring rg(ns);
+      long long pc = 0;   // head pairs issued
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i)
+        for (int p = 0; p < NPAIR && ok; ++p, ++pc) {
+          const int kb = int(pc & 1);
+          if (pc >= 2 && !mbar_wait(saddr(&kempty[kb]), uint32_t((pc - 2) >> 1) & 1u)) { ok = false; break; }
+          const uint32_t d = tmem + uint32_t(kb * 256);
+          for (int u = 0; u < NI; ++u) {
+            if (!mbar_wait(saddr(&full[rg.slot]), rg.phase)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t sa = da0 + uint64_t((rg.slot * kRopeSlotBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)   // K = 16 channels per MMA
+              tc_mma(d, sa + uint64_t((kk * 32) >> 4), sa + uint64_t((kBoxBytes + kk * 32) >> 4), id,
+                     (u | kk) != 0);
+            tc_commit(saddr(&empty[rg.slot]));
+            rg.advance();
+          }
+          if (!ok) break;
+          tc_commit(saddr(&kfull[kb]));
+          if (*abort_flag) ok = false;
+        }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(status, QSVD_STATUS_TIMEOUT);
+      }
+      tc_commit(saddr(drain));
+      mbar_wait(saddr(drain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ rotation and scores
+    const int q = warp & 3;
+    const int t = 32 * q + lane;              // token row in the tile == TMEM lane
+    const uint32_t lane_off = uint32_t(32 * q) << 16;
+    float* tc = tab_c + t * kRopeTabPitch;    // this token's cos / sin row (private)
+    float* ts = tab_s + t * kRopeTabPitch;
+    TileIter it;
+    it.init(sched, B, tb, te);
+    long long pc = 0;
+    for (int i = 0; i < n; ++i) {
+      const int nv = it.nvalid(), b = it.b, t0 = it.t0();
+      if (t < nv) {   // the row of position t0 + t: 64 (cos, sin) pairs
+        const float4* src = reinterpret_cast<const float4*>(rope_tab + size_t(t0 + t) * 128);
+#pragma unroll 8
+        for (int v = 0; v < 32; ++v) {
+          const float4 x = __ldg(src + v);
+          tc[2 * v] = x.x; ts[2 * v] = x.y; tc[2 * v + 1] = x.z; ts[2 * v + 1] = x.w;
+        }
+      }
+      const float* qb = qrot + size_t(b) * E;
+      int fail = 0;
+      for (int p = 0; p < NPAIR; ++p, ++pc) {
+        const int kb = int(pc & 1);
+        fail = group_or(!mbar_wait(saddr(&kfull[kb]), uint32_t(pc >> 1) & 1u));   // uniform
+        if (fail) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = 2 * p + hh;
+          if (h >= H) break;
+          const float* qh = qb + h * 128;
+          const uint32_t ta = tmem + lane_off + uint32_t(kb * 256 + hh * 128);
+          float s = 0.f;
+#pragma unroll 1
+          for (int i0 = 0; i0 < 64; i0 += 16) {
+            float klo[16], khi[16];
+            tmem_ld16(ta + uint32_t(i0), klo);
+            tmem_ld16(ta + uint32_t(64 + i0), khi);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int j = i0 + e;
+              const float c = tc[j], sn = ts[j];
+              s = fmaf(__ldg(qh + j), fmaf(klo[e], c, -khi[e] * sn), s);
+              s = fmaf(__ldg(qh + 64 + j), fmaf(khi[e], c, klo[e] * sn), s);
+            }
+          }
+          if (t < nv) scores[(size_t(b) * H + h) * max_len + t0 + t] = s;
+        }
+        tc_fence_before();
+        group_sync();
+        if (t == 0) mbar_arrive(saddr(&kempty[kb]));
+      }
+      if (fail) {
+        if (t == 0) { *abort_flag = 1; atomicOr(status, QSVD_STATUS_TIMEOUT); }
+        break;
+      }
+      it.next();
+      if (group_or(*abort_flag)) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
 // ------------------------------------------------------------------- host
 
 constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
@@ -1154,6 +1368,47 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   return check_launch();
 }
 
+template <bool BF16>
+cudaError_t rope_scores_t(const qsvd_dims& d, const void* cache, const void* wukT, const float* qrot,
+                          const float* rope_tab, const int32_t* sched, int G, float* scores,
+                          int32_t* status, cudaStream_t s) {
+  TensorMapEncode enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tc, tw;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(d.r), cuuint64_t(d.batch) * d.max_len};
+    const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tc, dt, 2, const_cast<void*>(cache), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // W^u_k^T [E][r]: one box is 256 rows (two heads' d_h) x 64 channels
+    const cuuint64_t dims[2] = {cuuint64_t(d.r), cuuint64_t(d.E)};
+    const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
+    const cuuint32_t box[2] = {64, 256};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tw, dt, 2, const_cast<void*>(wukT), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  constexpr int ns = 3;
+  const size_t smem = 1024 + size_t(ns) * kRopeSlotBytes + 2 * 128 * kRopeTabPitch * 4 +
+                      (2 * kMaxSlots + 5) * 8 + 16;
+  auto kern = k_rope_scores<BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<G, 192, smem, s>>>(tc, tw, qrot, rope_tab, sched, scores, status, d.batch, d.H, d.E, d.r,
+                            d.max_len, G, ns);
+  note_launch();
+  return check_launch();
+}
+
 }  // namespace
 
 int split_tc_heads_padded(const qsvd_dims& d) { return d.H <= 16 ? 16 : (d.H <= 32 ? 32 : 0); }
@@ -1188,6 +1443,19 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
       return np == 16 ? launch_t<16, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
                       : launch_t<32, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
   }
+}
+
+bool rope_tc_supported(const qsvd_dims& d) {
+  return d.rope && d.d_h == 128 && d.r % 64 == 0 && d.cache_dtype == d.weight_dtype &&
+         (d.cache_dtype == QSVD_F16 || d.cache_dtype == QSVD_BF16);
+}
+
+cudaError_t launch_rope_scores(const qsvd_dims& d, const void* cache, const void* wukT,
+                               const float* qrot, const float* rope_tab, const int32_t* sched,
+                               int G, float* scores, int32_t* status, cudaStream_t s) {
+  return d.cache_dtype == QSVD_BF16
+             ? rope_scores_t<true>(d, cache, wukT, qrot, rope_tab, sched, G, scores, status, s)
+             : rope_scores_t<false>(d, cache, wukT, qrot, rope_tab, sched, G, scores, status, s);
 }
 
 }  // namespace qsvd

@@ -119,3 +119,35 @@ def test_tc_large_score_range_rescales(cuda_ok):
     got, ws = g.decode(num_splits=1)
     assert q.status_word(ws) == 0
     assert rel_err(got, c2.reference()) <= TOL
+
+
+# Rotary mode: keys rebuilt on the tensor cores (K_h = C W^u_{k,h}, two heads
+# per MMA), rotated and scored by CUDA cores, then the CUDA-core softmax and
+# latent accumulation on the given scores.
+_ROPE = {}
+
+
+def rope_case(key):
+    if key not in _ROPE:
+        w = {"s2": synthetic.SHRUNK[2],                      # bf16, r 256, even H
+             "s4": synthetic.SHRUNK[4],                      # bf16, r 384, H 5 (odd), ragged
+             "s2f16": synthetic.replace(synthetic.SHRUNK[2], cache="f16", weight="f16")}[key]
+        _ROPE[key] = oi.build_case(w)
+    return _ROPE[key]
+
+
+@pytest.mark.parametrize("key", ["s2", "s4", "s2f16"])
+def test_tc_rope_matches_oracle(cuda_ok, key):
+    c = rope_case(key)
+    got, ws = GpuCase(c, kernel=TC).decode()
+    assert q.status_word(ws) == 0
+    err = rel_err(got, c.reference())
+    assert err <= TOL, f"{key}: {err:.3e}"
+
+
+@pytest.mark.parametrize("key", ["s2", "s4"])
+def test_tc_rope_agrees_with_simt(cuda_ok, key):
+    c = rope_case(key)
+    a, _ = GpuCase(c, kernel=TC).decode()
+    b, _ = GpuCase(c, kernel=q.QSVD_KERNEL_SIMT).decode()
+    assert rel_err(a, b) <= TOL
