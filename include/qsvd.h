@@ -71,6 +71,12 @@ typedef enum {
 #define QSVD_PHASE_SPLIT 2u     /* split-KV attention over the latent tiles */
 #define QSVD_PHASE_COMBINE 4u   /* merge of the split partials, value up-projection */
 #define QSVD_PHASE_ALL 7u
+/* The two passes of the split phase in rotary mode on the tensor cores
+ * (QSVD_PHASE_SPLIT runs both): keys rebuilt from the latent, rotated and
+ * scored into the workspace; then the softmax and the latent accumulation
+ * over those scores.  Any other path rejects them with INVALID_ARG. */
+#define QSVD_PHASE_SPLIT_SCORES 8u
+#define QSVD_PHASE_SPLIT_ACCUM 16u
 
 /* Device status bits (workspace word 0 for decode; `status` for append). */
 #define QSVD_STATUS_LEN_CLAMPED 1   /* some lengths[b] < 0 or > max_len (clamped) */
@@ -209,7 +215,9 @@ qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const void* packed,
  *                  m[s][H], l[s][H] (float32, log2 domain), z[s][H][r].
  *   out            device, B x E, out_dtype.
  *   phases         QSVD_PHASE_* mask (0 = all).  Running the phases as
- *                  separate calls in order gives the same result.
+ *                  separate calls in order gives the same result; so does
+ *                  running the split as its two rotary passes
+ *                  (QSVD_PHASE_SPLIT_SCORES, then QSVD_PHASE_SPLIT_ACCUM).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed,

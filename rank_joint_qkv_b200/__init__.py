@@ -28,6 +28,7 @@ QSVD_OK, QSVD_ERR_INVALID_ARG, QSVD_ERR_UNSUPPORTED, QSVD_ERR_WORKSPACE, QSVD_ER
 QSVD_F32, QSVD_F16, QSVD_BF16, QSVD_I8, QSVD_I4 = range(5)
 QSVD_TILE_TOKENS = 128
 QSVD_PHASE_PROLOGUE, QSVD_PHASE_SPLIT, QSVD_PHASE_COMBINE, QSVD_PHASE_ALL = 1, 2, 4, 7
+QSVD_PHASE_SPLIT_SCORES, QSVD_PHASE_SPLIT_ACCUM = 8, 16
 QSVD_STATUS_LEN_CLAMPED, QSVD_STATUS_POS_OOB, QSVD_STATUS_SCALE_SAT, QSVD_STATUS_TIMEOUT = 1, 2, 4, 8
 QSVD_KERNEL_AUTO, QSVD_KERNEL_SIMT, QSVD_KERNEL_TCGEN05 = 0, 1, 2
 

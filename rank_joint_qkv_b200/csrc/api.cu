@@ -104,8 +104,8 @@ static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel
   if (g == 0) {
     const int sms = device_sms();
     if (sms <= 0) return fail(QSVD_ERR_CUDA, "no CUDA device to size the split grid");
-    if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope) {   // rotary: the softmax runs on CUDA cores
-      g = sms;
+    if (kernel == QSVD_KERNEL_TCGEN05 && (!d.rope || split_tc_scores_supported(d))) {
+      g = sms;   // one CTA per SM (persistent over its tile range)
     } else {
       const int hb = split_simt_grid_heads(d);
       g = hb > 0 ? (2LL * sms + hb - 1) / hb : sms;
@@ -203,8 +203,13 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
                                size_t* workspace_bytes, void* out, unsigned phases,
                                cudaStream_t s) {
   if (phases == 0) phases = QSVD_PHASE_ALL;
-  if (phases & ~QSVD_PHASE_ALL) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
+  constexpr unsigned kSub = QSVD_PHASE_SPLIT_SCORES | QSVD_PHASE_SPLIT_ACCUM;
+  if (phases & ~(QSVD_PHASE_ALL | kSub)) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
   const int kernel = pick_kernel(d);
+  if ((phases & kSub) && !(d.rope && kernel == QSVD_KERNEL_TCGEN05))
+    return fail(QSVD_ERR_INVALID_ARG, "split sub-phases exist in rotary mode on the tensor cores only");
+  if (phases & QSVD_PHASE_SPLIT) phases |= kSub;
+  const bool split_any = (phases & kSub) != 0;
   if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope && !split_tc_supported(d))
     return fail(QSVD_ERR_UNSUPPORTED,
                 "tensor-core split kernel needs a 16-bit or int4/int8 (group 128) cache, r %% 128 == 0, H <= 32");
@@ -222,8 +227,8 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, W.total);
   if (!packed || !lengths) return fail(QSVD_ERR_INVALID_ARG, "packed/lengths is NULL");
   if ((phases & QSVD_PHASE_PROLOGUE) && !qin) return fail(QSVD_ERR_INVALID_ARG, "qin is NULL");
-  if ((phases & QSVD_PHASE_SPLIT) && !cache) return fail(QSVD_ERR_INVALID_ARG, "cache is NULL");
-  if ((phases & QSVD_PHASE_SPLIT) && cache_is_int(d) && !scales)
+  if (split_any && !cache) return fail(QSVD_ERR_INVALID_ARG, "cache is NULL");
+  if (split_any && cache_is_int(d) && !scales)
     return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
   if ((phases & QSVD_PHASE_COMBINE) && !out) return fail(QSVD_ERR_INVALID_ARG, "out is NULL");
   if (!aligned16(workspace) || (cache && !aligned16(cache)) || (qin && !aligned16(qin)))
@@ -264,14 +269,18 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
       e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, qt16, &hdr->status, s);
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
-  if (phases & QSVD_PHASE_SPLIT) {
+  if (split_any) {
     if (d.rope && kernel == QSVD_KERNEL_TCGEN05) {
       float* scores = reinterpret_cast<float*>(Wb + W.scores);
       const int sms = device_sms();
-      e = launch_rope_scores(d, cache, P + L.wukT, qt32, rope_tab, sched, sms > 0 ? sms : 1, scores,
-                             &hdr->status, s);
-      if (e == cudaSuccess)
-        e = launch_split_simt_scores(d, scores, cache, scales, sched, G, pm, pl, pz, s);
+      e = cudaSuccess;
+      if (phases & QSVD_PHASE_SPLIT_SCORES)
+        e = launch_rope_scores(d, cache, P + L.wukT, qt32, rope_tab, sched, sms > 0 ? sms : 1,
+                               scores, &hdr->status, s);
+      if (e == cudaSuccess && (phases & QSVD_PHASE_SPLIT_ACCUM))
+        e = split_tc_scores_supported(d)
+                ? launch_split_tc_scores(d, scores, cache, sched, G, pm, pl, pz, &hdr->status, s)
+                : launch_split_simt_scores(d, scores, cache, scales, sched, G, pm, pl, pz, s);
     } else if (d.rope) {
       e = launch_split_simt_rope(d, qt32, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
     }

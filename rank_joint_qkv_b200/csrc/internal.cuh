@@ -149,12 +149,17 @@ cudaError_t launch_split_simt_absorbed(const qsvd_dims& d, const float* qt32,
                                        const int32_t* sched, int G, float* pm,
                                        float* pl, float* pz, cudaStream_t s);
 // Rotary mode on the tensor cores: keys rebuilt from the latent, rotated,
-// scored against the rotary query into `scores` ([B][H][max_len]); then the
-// CUDA-core split kernel runs the softmax and the latent accumulation on them.
+// scored against the rotary query into `scores` ([B][H][max_len]); then a
+// split kernel runs the softmax and the latent accumulation on them (the
+// tensor-core one when split_tc_scores_supported, else the CUDA-core one).
 bool rope_tc_supported(const qsvd_dims& d);
 cudaError_t launch_rope_scores(const qsvd_dims& d, const void* cache, const void* wukT,
                                const float* qrot, const float* rope_tab, const int32_t* sched,
                                int G, float* scores, int32_t* status, cudaStream_t s);
+bool split_tc_scores_supported(const qsvd_dims& d);
+cudaError_t launch_split_tc_scores(const qsvd_dims& d, const float* scores, const void* cache,
+                                   const int32_t* sched, int G, float* pm, float* pl, float* pz,
+                                   int32_t* status, cudaStream_t s);
 cudaError_t launch_split_simt_scores(const qsvd_dims& d, const float* scores, const void* cache,
                                      const void* scales, const int32_t* sched, int G, float* pm,
                                      float* pl, float* pz, cudaStream_t s);

@@ -275,6 +275,9 @@ template <int NP, int QS>
 __host__ __device__ constexpr int s_slot_bytes() { return kBoxBytes + QS * NP * 128; }
 constexpr int kZBoxBytes = 64 * 128;             // 64 tokens x 64 channels x 2 bytes
 constexpr int kZSlotBytes = 2 * kZBoxBytes;
+// Scores given (SG): no S pass; ring A carries Z items too.
+template <int NP, int QS, bool SG>
+__host__ __device__ constexpr int a_slot_bytes() { return SG ? kZSlotBytes : s_slot_bytes<NP, QS>(); }
 template <int NP>
 __host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T part
 constexpr int kMiscBytes = 2048;
@@ -309,11 +312,11 @@ struct Smem {
 __host__ __device__ constexpr int raw_bytes(int qb) { return qb * 1024; }
 __host__ __device__ inline int zscale_bytes(int r) { return 256 * (r / 128); }
 
-template <int NP, int QS, int PS>
+template <int NP, int QS, int PS, bool SG>
 __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   Smem s;
   s.sring = base;
-  s.zring = s.sring + size_t(ns) * s_slot_bytes<NP, QS>();
+  s.zring = s.sring + size_t(ns) * a_slot_bytes<NP, QS, SG>();
   s.pbuf = s.zring + size_t(nz) * kZSlotBytes;
   s.sraw = s.pbuf + 2 * PS * pbuf_bytes<NP>();
   s.zraw = s.sraw + size_t(nraw) * raw_bytes(qb);
@@ -598,20 +601,23 @@ __device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, co
 // Producer of one ring (warp-wide).  kind 0: S ring (latent box from HBM,
 // kept in L2 for the Z re-read, plus the query box); kind 1: Z ring (latent
 // re-read, dropped from L2 after).  Item u of a tile: S -> channel box u;
-// Z -> channels [128 (u / 2), +128) x tokens [64 (u % 2), +64).  Returns false
-// on a wait that expired or an abort.
-template <int NP, int QS>
+// Z -> channels [128 (u / 2), +128) x tokens [64 (u % 2), +64).  SG (scores
+// given): both rings carry Z items, ring `kind` the chunks u / 2 of its
+// parity, read once (dropped from L2 after).  Returns false on a wait that
+// expired or an abort.
+template <int NP, int QS, bool SG>
 __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const CUtensorMap* tm_cz,
                         const CUtensorMap* tm_q, const uint8_t* cache, const int32_t* sched, int B,
                         int r, int max_len, long long tb, long long te, int n, int nslots, int lane,
                         long long* issued) {
   const int NI = r / 64;
   const size_t row_bytes = size_t(r) * 2;
+  const bool zk = SG || kind == 1;   // this ring carries Z items
   uint8_t* ring = kind == 0 ? s.sring : s.zring;
-  const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
+  const uint32_t slot_bytes = zk ? uint32_t(kZSlotBytes) : uint32_t(s_slot_bytes<NP, QS>());
   uint64_t* full = kind == 0 ? s.s_full : s.z_full;
   uint64_t* empty = kind == 0 ? s.s_empty : s.z_empty;
-  const uint64_t policy = kind == 0 ? policy_evict_last() : policy_evict_first();
+  const uint64_t policy = zk ? policy_evict_first() : policy_evict_last();
   const uint32_t ring0 = saddr(ring);
   TileIter it;
   it.init(sched, B, tb, te);
@@ -622,14 +628,15 @@ __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const
     const int row = b * max_len + t0;
     const uint8_t* tile = cache + size_t(row) * row_bytes;
     for (int u = 0; u < NI; ++u) {
+      if (SG && ((u >> 1) & 1) != kind) continue;   // the other ring's chunk
       if (!__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
         *issued = k;
         return false;
       }
       const uint32_t dst = ring0 + uint32_t(rg.slot) * slot_bytes;
       const uint32_t fb = saddr(&full[rg.slot]);
-      const int lo = kind == 0 ? 0 : 64 * (u & 1);        // first tile row of the item
-      const int hi = kind == 0 ? kTile : lo + 64;
+      const int lo = zk ? 64 * (u & 1) : 0;               // first tile row of the item
+      const int hi = zk ? lo + 64 : kTile;
       if (nv >= hi) {
         if (lane == 0) mbar_expect_tx(fb, slot_bytes);
         __syncwarp();
@@ -637,7 +644,7 @@ __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const
         // issuing lanes rotate between items and the item's two operations
         // go out from different lanes
         const int ln = int(k & 15) * 2;
-        if (kind == 0) {
+        if (!zk) {
           if (lane == ln) tma_load_2d_hint(dst, tm_cs, 64 * u, row, fb, policy);
           if (lane == ln + 1) tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
         } else if (lane == ln) {
@@ -646,10 +653,10 @@ __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const
       } else {
         // last tile of a sequence: rows past its length are written as zeros
         uint8_t* d = ring + size_t(rg.slot) * slot_bytes;
-        if (kind == 0) ragged_rows(d, tile + 128 * u, row_bytes, kTile, 1, 0, nv, lane);
+        if (!zk) ragged_rows(d, tile + 128 * u, row_bytes, kTile, 1, 0, nv, lane);
         else ragged_rows(d, tile + 256 * (u >> 1), row_bytes, 64, 2, lo, nv, lane);
         if (lane == 0) {
-          if (kind == 0) {
+          if (!zk) {
             mbar_expect_tx(fb, uint32_t(QS * NP * 128));
             tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
           } else {
@@ -680,21 +687,25 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 // QB = 0: 16-bit latent; QB = 4 / 8: int4 / int8 codes with fp16 scales per
 // group of 128 channels (S per group into a ring of nsg TMEM buffers, the
 // scales applied per token by the softmax; Z from the dequantised latent).
-template <int NP, bool BF16, int QS, int PS, int QB>
+// SG: scores given ([B][H][max_len] fp32, log2 domain: the rotary mode's
+// scores kernel), no S pass; warps 1 and 3 both issue Z MMAs, each for the
+// 128-channel chunks of one parity, fed by its own ring.
+template <int NP, bool BF16, int QS, int PS, int QB, bool SG>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
            const __grid_constant__ CUtensorMap tm_q,
            const uint8_t* __restrict__ cache, const __half* __restrict__ scales,
-           const int32_t* __restrict__ sched,
+           const float* __restrict__ scores, const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
            int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz,
            int nsg, int nraw) {
+  static_assert(!(SG && QB), "scores given: 16-bit latent only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const Smem s = carve<NP, QS, PS>(base, ns, nz, nraw, QB, r);
+  const Smem s = carve<NP, QS, PS, SG>(base, ns, nz, nraw, QB, r);
   constexpr int SW = QS * NP;                 // S accumulator columns per buffer
-  const int ZC0 = (QB ? nsg : 2) * SW;        // first Z column
+  const int ZC0 = SG ? 0 : (QB ? nsg : 2) * SW;   // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = r / 64;                      // ring items per tile
   const int NC = r / 128;                     // 128-channel Z accumulator chunks
@@ -724,7 +735,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     for (int i = 0; i < 2; ++i) {
       mbar_init(saddr(&s.acc_full[i]), 1);
       mbar_init(saddr(&s.p_full[i]), 1);
-      mbar_init(saddr(&s.z_done[i]), 1);
+      mbar_init(saddr(&s.z_done[i]), SG ? 2 : 1);   // SG: one commit per Z issuer
       mbar_init(saddr(&s.drain[i]), 1);
     }
     *s.abort_flag = 0;
@@ -751,15 +762,15 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       ok = produce_q<NP, QS, QB>(kind, s, kind == 0 ? &tm_cs : &tm_cz, &tm_q, scales, sched, B, r,
                                  max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
     else
-      ok = produce<NP, QS>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te, n,
-                           nslots, lane, &issued);
+      ok = produce<NP, QS, SG>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te,
+                               n, nslots, lane, &issued);
     if (!ok && lane == 0) {
       set_abort(s, status);
       drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
       if (QB) drain_ring(kind == 0 ? s.sraw_full : s.zraw_full, raw_issued, nraw);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 && !SG) {
     // ----------------------------------------------------------- S MMAs
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
@@ -804,15 +815,19 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       mbar_wait(saddr(&s.drain[0]), 0);
     }
     __syncwarp();
-  } else if (warp == 3) {
+  } else if (warp == 3 || (SG && warp == 1)) {
     // ----------------------------------------------------------- Z MMAs
     if (lane == 0) {
+      const int kind = warp >> 1;   // SG: ring and chunk parity of this issuer
+      const bool ra = SG && kind == 0;
+      uint64_t* zfull = ra ? s.s_full : s.z_full;
+      uint64_t* zempty = ra ? s.s_empty : s.z_empty;
       constexpr uint32_t id_z = idesc_f16(128, NP, BF16, true, false);
-      const uint64_t za0 = sdesc(saddr(s.zring), kZBoxBytes, 1024);  // MN-major C^T
-      const uint64_t pb0 = sdesc(saddr(s.pbuf), 16, 1024);            // P^T, K-major
+      const uint64_t za0 = sdesc(saddr(ra ? s.sring : s.zring), kZBoxBytes, 1024);  // MN-major C^T
+      const uint64_t pb0 = sdesc(saddr(s.pbuf), 16, 1024);                          // P^T, K-major
       TileIter it;
       it.init(sched, B, tb, te);
-      Ring rg(nz);
+      Ring rg(ra ? ns : nz);
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
         const bool first = it.first(tb);
@@ -820,7 +835,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         const uint64_t pb = pb0 + uint64_t(((i & 1) * PS * pbuf_bytes<NP>()) >> 4);
         for (int u = 0; u < NI; ++u) {
           const int j = u >> 1, h = u & 1;   // 128-channel chunk, 64-token half
-          if (!mbar_wait(saddr(&s.z_full[rg.slot]), rg.phase)) { ok = false; break; }
+          if (SG && (j & 1) != kind) continue;
+          if (!mbar_wait(saddr(&zfull[rg.slot]), rg.phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
           const uint64_t za = za0 + uint64_t((rg.slot * kZSlotBytes) >> 4);
@@ -833,7 +849,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
               tc_mma(d, a, bd, id_z, (first && h == 0 && kk == 0 && part == 0) ? 0u : 1u);
             }
           }
-          tc_commit(saddr(&s.z_empty[rg.slot]));
+          tc_commit(saddr(&zempty[rg.slot]));
           rg.advance();
         }
         if (!ok) break;
@@ -842,8 +858,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         if (*s.abort_flag) ok = false;
       }
       if (!ok) set_abort(s, status);
-      tc_commit(saddr(&s.drain[1]));
-      mbar_wait(saddr(&s.drain[1]), 0);
+      tc_commit(saddr(&s.drain[kind]));
+      mbar_wait(saddr(&s.drain[kind]), 0);
     }
     __syncwarp();
   } else {
@@ -891,6 +907,12 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           sgr.advance();
         }
         if (fail) { if (t == 0) set_abort(s, status); break; }
+      } else if (SG) {
+        // head h's scores of this tile: 128 consecutive floats per warp-row
+        const float* sc = scores + size_t(it.b) * H * max_len + it.t0() + t;
+        const bool ok = t < nv;
+#pragma unroll
+        for (int h = 0; h < NP; ++h) sv[h] = (ok && h < H) ? __ldg(sc + size_t(h) * max_len) : -INFINITY;
       } else {
         fail = !mbar_wait(saddr(&s.acc_full[pb]), uint32_t(i >> 1) & 1u);
         if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
@@ -1269,10 +1291,10 @@ void ring_slots(int* ns, int* nz) {
   *nz = z;
 }
 
-template <int NP, bool BF16, int QB>
+template <int NP, bool BF16, int QB, bool SG = false>
 cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
-                     const int32_t* sched, int G, float* pm, float* pl, float* pz,
-                     int32_t* status, cudaStream_t s) {
+                     const float* scores, const int32_t* sched, int G, float* pm, float* pl,
+                     float* pz, int32_t* status, cudaStream_t s) {
   TensorMapEncode enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
@@ -1282,6 +1304,7 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   CUtensorMap tcs, tcz, tq;
   memset(&tcs, 0, sizeof(tcs));
   memset(&tcz, 0, sizeof(tcz));
+  memset(&tq, 0, sizeof(tq));
   if (QB) {
     // quantised latent: raw code rows [B * max_len][r QB / 8] bytes; S item
     // box {QB x 8 bytes, 128 rows} (64 channels), Z item box {QB x 16 bytes,
@@ -1299,7 +1322,7 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  if (!QB) {
+  if (!QB && !SG) {
     // S items: latent rows [B * max_len][r], one box {64 channels, 128 rows}
     const cuuint64_t dims[2] = {cuuint64_t(d.r), rows};
     const cuuint64_t strides[1] = {cuuint64_t(d.r) * 2};
@@ -1322,7 +1345,7 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
+  if (!SG) {
     // query parts: qt16 holds [B][QS][H][r] (hi, then the rounding residual),
     // seen as {64 channels, head, sequence * part, 64-channel box}; one box
     // {64, NP, QS, 1} lands as smem [part][head][64].  Heads H..NP-1 are
@@ -1350,19 +1373,25 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
     if (nraw > d.r / 64) nraw = d.r / 64;
     if (nraw < 2) return cudaErrorInvalidConfiguration;
   }
+  if constexpr (SG) {
+    // no S items: both rings carry Z items and share the budget
+    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
+    ns = nz = avail / kZSlotBytes / 2;
+    if (ns > kMaxSlots) ns = nz = kMaxSlots;
+  }
   if (ns < 2 || nz < 2) return cudaErrorInvalidConfiguration;
   // quantised latent: per-group S buffers in the TMEM left beside Z
   int nsg = (512 - (d.r / 128) * NP) / (QS * NP);
   if (nsg > kMaxGroupBufs) nsg = kMaxGroupBufs;
   if (QB && nsg < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = 1024 + size_t(ns) * s_slot_bytes<NP, QS>() + size_t(nz) * kZSlotBytes +
+  const size_t smem = 1024 + size_t(ns) * a_slot_bytes<NP, QS, SG>() + size_t(nz) * kZSlotBytes +
                       2 * PS * pbuf_bytes<NP>() +
                       (QB ? 2 * size_t(nraw) * raw_bytes(QB) + 2 * zscale_bytes(d.r) : 0) + kMiscBytes;
-  auto kern = k_split_tc<NP, BF16, QS, PS, QB>;
+  auto kern = k_split_tc<NP, BF16, QS, PS, QB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   kern<<<G, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache),
-                                   static_cast<const __half*>(scales), sched, pm, pl, pz, status,
+                                   static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status,
                                    d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw);
   note_launch();
   return check_launch();
@@ -1429,20 +1458,39 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s) {
   const int np = split_tc_heads_padded(d);
+  const float* ns = nullptr;
   switch (d.cache_dtype) {
     case QSVD_BF16:
-      return np == 16 ? launch_t<16, true, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, true, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, true, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, true, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
     case QSVD_I4:
-      return np == 16 ? launch_t<16, false, 4>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, false, 4>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
     case QSVD_I8:
-      return np == 16 ? launch_t<16, false, 8>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, false, 8>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
     default:
-      return np == 16 ? launch_t<16, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, false, 0>(d, cache, scales, qt16, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, false, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
+                      : launch_t<32, false, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
   }
+}
+
+bool split_tc_scores_supported(const qsvd_dims& d) {
+  if (d.cache_dtype != QSVD_F16 && d.cache_dtype != QSVD_BF16) return false;
+  if (d.r % 128) return false;
+  const int np = split_tc_heads_padded(d);
+  return np != 0 && (d.r / 128) * np <= 512;   // Z accumulators only
+}
+
+cudaError_t launch_split_tc_scores(const qsvd_dims& d, const float* scores, const void* cache,
+                                   const int32_t* sched, int G, float* pm, float* pl, float* pz,
+                                   int32_t* status, cudaStream_t s) {
+  const int np = split_tc_heads_padded(d);
+  if (d.cache_dtype == QSVD_BF16)
+    return np == 16 ? launch_t<16, true, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s)
+                    : launch_t<32, true, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s);
+  return np == 16 ? launch_t<16, false, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s)
+                  : launch_t<32, false, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s);
 }
 
 bool rope_tc_supported(const qsvd_dims& d) {

@@ -49,7 +49,7 @@ class GpuCase:
         self.out_dtype = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[out]
 
     def decode(self, *, num_splits=0, lengths=None, phases_separately=False, qin=None,
-               qin_is_latent=True):
+               qin_is_latent=True, split_phases=None):
         w = self.case.w
         out = torch.full((w.B, w.E), float("nan"), dtype=self.out_dtype, device=DEV)
         lens = self.lengths if lengths is None else lengths
@@ -59,7 +59,7 @@ class GpuCase:
                                     self.scales, lens, out, num_splits=num_splits)
         else:
             ws = None
-            for ph in (q.QSVD_PHASE_PROLOGUE, q.QSVD_PHASE_SPLIT):
+            for ph in (q.QSVD_PHASE_PROLOGUE,) + tuple(split_phases or (q.QSVD_PHASE_SPLIT,)):
                 ws = q.qsvd_decode_attn(self.dims, self.packed, qi, qin_is_latent, self.cache,
                                         self.scales, lens, out, num_splits=num_splits,
                                         workspace=ws, phases=ph)

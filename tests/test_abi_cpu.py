@@ -120,3 +120,33 @@ def test_too_small_workspace_and_null_pointers():
 def test_status_strings():
     for s in range(5):
         assert q._lib.qsvd_status_string(s).startswith(b"QSVD_")
+
+
+def test_header_constants_match_binding():
+    """Every QSVD_PHASE_ / QSVD_STATUS_ / QSVD_KERNEL_ value of the header
+    has the same value in the Python binding."""
+    src = open(HEADER).read()
+    consts = dict(re.findall(r"#define (QSVD_(?:PHASE|STATUS|KERNEL)_[A-Z0-9_]+) (\d+)u?", src))
+    assert any(k.startswith("QSVD_PHASE_SPLIT_") for k in consts)
+    assert "QSVD_KERNEL_TCGEN05" in consts
+    for name, val in consts.items():
+        assert getattr(q, name) == int(val), name
+
+
+def test_split_sub_phases_rejected_outside_rotary_tensor_path():
+    """The sub-phase bits are refused on the host for the absorbed path and
+    for the rotary CUDA-core path (before the device is touched)."""
+    lib = ctypes.CDLL(q.LIB_PATH)
+    lib.qsvd_decode_attn.argtypes = q._sigs["qsvd_decode_attn"]
+    fake = ctypes.c_void_p(1 << 20)
+    for d in (_dims(), _dims(rope=True, kernel=q.QSVD_KERNEL_SIMT)):
+        for ph in (q.QSVD_PHASE_SPLIT_SCORES, q.QSVD_PHASE_SPLIT_ACCUM):
+            n = ctypes.c_size_t(1 << 40)
+            st = lib.qsvd_decode_attn(ctypes.byref(d), fake, fake, 1, fake, None, fake, 4, fake,
+                                      ctypes.byref(n), fake, ph, None)
+            assert st == q.QSVD_ERR_INVALID_ARG
+            assert b"sub-phases" in q._lib.qsvd_last_error()
+    n = ctypes.c_size_t(1 << 40)
+    st = lib.qsvd_decode_attn(ctypes.byref(_dims()), fake, fake, 1, fake, None, fake, 4, fake,
+                              ctypes.byref(n), fake, 32, None)
+    assert st == q.QSVD_ERR_INVALID_ARG

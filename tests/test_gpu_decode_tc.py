@@ -122,21 +122,26 @@ def test_tc_large_score_range_rescales(cuda_ok):
 
 
 # Rotary mode: keys rebuilt on the tensor cores (K_h = C W^u_{k,h}, two heads
-# per MMA), rotated and scored by CUDA cores, then the CUDA-core softmax and
-# latent accumulation on the given scores.
+# per MMA), rotated and scored by CUDA cores; then the softmax and latent
+# accumulation on the given scores -- on the tensor cores when r % 128 == 0
+# and H <= 32 (Z only, two MMA issuers on alternating 128-channel chunks),
+# else on CUDA cores (r = 320 below).
 _ROPE = {}
 
 
 def rope_case(key):
     if key not in _ROPE:
-        w = {"s2": synthetic.SHRUNK[2],                      # bf16, r 256, even H
-             "s4": synthetic.SHRUNK[4],                      # bf16, r 384, H 5 (odd), ragged
-             "s2f16": synthetic.replace(synthetic.SHRUNK[2], cache="f16", weight="f16")}[key]
+        base = synthetic.SHRUNK[2]
+        w = {"s2": base,                                     # bf16, r 256, even H
+             "s4": synthetic.SHRUNK[4],                      # bf16, r 384 (odd chunk count), H 5, ragged
+             "s2f16": synthetic.replace(base, cache="f16", weight="f16"),
+             "h32": synthetic.replace(base, E=4096, H=32, r=384, B=2, L=520),
+             "r320": synthetic.replace(base, r=320)}[key]    # CUDA-core softmax on given scores
         _ROPE[key] = oi.build_case(w)
     return _ROPE[key]
 
 
-@pytest.mark.parametrize("key", ["s2", "s4", "s2f16"])
+@pytest.mark.parametrize("key", ["s2", "s4", "s2f16", "h32", "r320"])
 def test_tc_rope_matches_oracle(cuda_ok, key):
     c = rope_case(key)
     got, ws = GpuCase(c, kernel=TC).decode()
@@ -145,9 +150,54 @@ def test_tc_rope_matches_oracle(cuda_ok, key):
     assert err <= TOL, f"{key}: {err:.3e}"
 
 
-@pytest.mark.parametrize("key", ["s2", "s4"])
+@pytest.mark.parametrize("key", ["s2", "s4", "h32"])
 def test_tc_rope_agrees_with_simt(cuda_ok, key):
     c = rope_case(key)
     a, _ = GpuCase(c, kernel=TC).decode()
     b, _ = GpuCase(c, kernel=q.QSVD_KERNEL_SIMT).decode()
     assert rel_err(a, b) <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 3, 1000])
+def test_tc_rope_split_invariance(cuda_ok, splits):
+    c = rope_case("h32")
+    got, ws = GpuCase(c, kernel=TC).decode(num_splits=splits)
+    assert q.status_word(ws) == 0
+    assert rel_err(got, c.reference()) <= TOL
+
+
+@pytest.mark.parametrize("lens", [[1, 0, 2], [127, 128, 129], [300, 1, 257]])
+def test_tc_rope_edge_lengths(cuda_ok, lens):
+    w = synthetic.replace(synthetic.SHRUNK[2], B=len(lens), ragged=None, L=max(lens))
+    c = oi.build_case(w, lengths=np.array(lens, np.int32))
+    got, ws = GpuCase(c, kernel=TC).decode(num_splits=2)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(got[b] == 0.0)
+    assert rel_err(got, c.reference()) <= TOL
+    assert q.status_word(ws) == 0
+
+
+def test_tc_rope_nan_padding_rows(cuda_ok):
+    """NaN in rows past each length: neither the keys nor the latent
+    accumulation of the given-scores pass may pick them up."""
+    c = rope_case("s4")
+    g = GpuCase(c, kernel=TC)
+    for b, n in enumerate(c.lengths):
+        g.cache[b, int(n):] = float("nan")
+    got, _ = g.decode(num_splits=4)
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, c.reference()) <= TOL
+
+
+@pytest.mark.parametrize("key", ["s4", "r320"])
+def test_tc_rope_split_passes_as_separate_calls(cuda_ok, key):
+    """The rotary split run as its two passes (scores, then the softmax and
+    latent accumulation), each its own call, gives the one-call result."""
+    c = rope_case(key)
+    g = GpuCase(c, kernel=TC)
+    whole, _ = g.decode(num_splits=5)
+    parts, ws = g.decode(num_splits=5, phases_separately=True,
+                         split_phases=(q.QSVD_PHASE_SPLIT_SCORES, q.QSVD_PHASE_SPLIT_ACCUM))
+    assert q.status_word(ws) == 0
+    assert np.array_equal(whole, parts)
