@@ -104,8 +104,11 @@ static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel
   if (g == 0) {
     const int sms = device_sms();
     if (sms <= 0) return fail(QSVD_ERR_CUDA, "no CUDA device to size the split grid");
-    if (kernel == QSVD_KERNEL_TCGEN05 && (!d.rope || split_tc_scores_supported(d))) {
+    if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope) {
       g = sms;   // one CTA per SM (persistent over its tile range)
+    } else if (kernel == QSVD_KERNEL_TCGEN05 && split_tc_scores_supported(d)) {
+      g = sms / split_tc_scores_parts(d);   // ch CTAs per split, one per SM
+      if (g < 1) g = 1;
     } else {
       const int hb = split_simt_grid_heads(d);
       g = hb > 0 ? (2LL * sms + hb - 1) / hb : sms;

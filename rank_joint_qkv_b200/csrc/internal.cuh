@@ -157,6 +157,7 @@ cudaError_t launch_rope_scores(const qsvd_dims& d, const void* cache, const void
                                const float* qrot, const float* rope_tab, const int32_t* sched,
                                int G, float* scores, int32_t* status, cudaStream_t s);
 bool split_tc_scores_supported(const qsvd_dims& d);
+int split_tc_scores_parts(const qsvd_dims& d);   // CTAs sharing one split's channels
 cudaError_t launch_split_tc_scores(const qsvd_dims& d, const float* scores, const void* cache,
                                    const int32_t* sched, int G, float* pm, float* pl, float* pz,
                                    int32_t* status, cudaStream_t s);

@@ -301,7 +301,10 @@ struct Smem {
   uint8_t* zscale;
   uint64_t* sraw_full;   // [kMaxRaw]
   uint64_t* zraw_full;   // [kMaxRaw]
-  float* red;            // [4][NP]
+  float* red;            // [4][NP] per-warp partial max / sum
+  float* m_run;          // [NP] running reference max per head (log2 domain)
+  float* l_run;          // [NP] running sum of P per head
+  float* alpha;          // [NP] rescale factor of the current tile
   uint32_t* tmem_holder;
   volatile int* abort_flag;
 };
@@ -335,10 +338,41 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   s.sg_empty = s.sg_full + kMaxGroupBufs;
   s.sraw_full = s.sg_empty + kMaxGroupBufs;
   s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + 2 kMaxRaw = 64 barriers
+  static_assert(640 + 4 * NP * 4 + 32 + 3 * NP * 4 <= kMiscBytes, "misc region");
   s.red = reinterpret_cast<float*>(m + 640);
   s.tmem_holder = reinterpret_cast<uint32_t*>(m + 640 + 4 * NP * 4);
   s.abort_flag = reinterpret_cast<volatile int*>(m + 640 + 4 * NP * 4 + 16);
+  s.m_run = reinterpret_cast<float*>(m + 640 + 4 * NP * 4 + 32);
+  s.l_run = s.m_run + NP;
+  s.alpha = s.l_run + NP;
   return s;
+}
+
+// Per-head reduction over the 32 lanes of a warp into red[0..NP): lane L
+// writes head L (and 32 + L for NP = 48, reduced as 32 + 16).  v is consumed.
+template <int NP, typename Op>
+__device__ __forceinline__ void reduce_heads(float (&v)[NP], float* red, int lane, Op op) {
+  if constexpr (NP <= 32) {
+    const float x = dev::warp_reduce_transposed<NP>(v, lane, op);
+    if (lane < NP) red[lane] = x;
+  } else {
+    static_assert(NP == 48, "heads padded to 16, 32 or 48");
+    float a[32], b[16];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) a[h] = v[h];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) b[h] = v[32 + h];
+    const float xa = dev::warp_reduce_transposed<32>(a, lane, op);
+    red[lane] = xa;
+    const float xb = dev::warp_reduce_transposed<16>(b, lane, op);
+    if (lane < 16) red[32 + lane] = xb;
+  }
+}
+
+// SG with a channel split over `ch` CTAs: 128-channel chunk j belongs to CTA
+// part j % ch, and there to the issuer (and ring) (j / ch) % 2.
+__device__ __forceinline__ bool sg_owns(int j, int ch, int cpart, int kind) {
+  return j % ch == cpart && ((j / ch) & 1) == kind;
 }
 
 __device__ __forceinline__ void set_abort(const Smem& s, int32_t* status) {
@@ -602,14 +636,14 @@ __device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, co
 // kept in L2 for the Z re-read, plus the query box); kind 1: Z ring (latent
 // re-read, dropped from L2 after).  Item u of a tile: S -> channel box u;
 // Z -> channels [128 (u / 2), +128) x tokens [64 (u % 2), +64).  SG (scores
-// given): both rings carry Z items, ring `kind` the chunks u / 2 of its
-// parity, read once (dropped from L2 after).  Returns false on a wait that
-// expired or an abort.
+// given): both rings carry Z items, ring `kind` the chunks sg_owns gives it,
+// read once (dropped from L2 after).  Returns false on a wait that expired
+// or an abort.
 template <int NP, int QS, bool SG>
 __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const CUtensorMap* tm_cz,
                         const CUtensorMap* tm_q, const uint8_t* cache, const int32_t* sched, int B,
                         int r, int max_len, long long tb, long long te, int n, int nslots, int lane,
-                        long long* issued) {
+                        long long* issued, int ch, int cpart) {
   const int NI = r / 64;
   const size_t row_bytes = size_t(r) * 2;
   const bool zk = SG || kind == 1;   // this ring carries Z items
@@ -628,7 +662,7 @@ __device__ bool produce(int kind, const Smem& s, const CUtensorMap* tm_cs, const
     const int row = b * max_len + t0;
     const uint8_t* tile = cache + size_t(row) * row_bytes;
     for (int u = 0; u < NI; ++u) {
-      if (SG && ((u >> 1) & 1) != kind) continue;   // the other ring's chunk
+      if (SG && !sg_owns(u >> 1, ch, cpart, kind)) continue;   // another ring's (or CTA's) chunk
       if (!__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
         *issued = k;
         return false;
@@ -688,8 +722,11 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 // group of 128 channels (S per group into a ring of nsg TMEM buffers, the
 // scales applied per token by the softmax; Z from the dequantised latent).
 // SG: scores given ([B][H][max_len] fp32, log2 domain: the rotary mode's
-// scores kernel), no S pass; warps 1 and 3 both issue Z MMAs, each for the
-// 128-channel chunks of one parity, fed by its own ring.
+// scores kernel), no S pass; warps 1 and 3 both issue Z MMAs, each for
+// alternate 128-channel chunks, fed by its own ring.  When the Z accumulator
+// of all chunks does not fit TMEM, `ch` CTAs share one tile range (split g =
+// blockIdx.x / ch), each owning every ch-th chunk; all of them run the same
+// softmax on the same scores and part 0 writes m and l.
 template <int NP, bool BF16, int QS, int PS, int QB, bool SG>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
@@ -698,7 +735,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
            const float* __restrict__ scores, const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
            int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz,
-           int nsg, int nraw) {
+           int nsg, int nraw, int ch) {
   static_assert(!(SG && QB), "scores given: 16-bit latent only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -709,9 +746,12 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = r / 64;                      // ring items per tile
   const int NC = r / 128;                     // 128-channel Z accumulator chunks
+  const int g = SG ? int(blockIdx.x) / ch : int(blockIdx.x);       // split
+  const int cpart = SG ? int(blockIdx.x) % ch : 0;                 // channel part
+  const int NCL = SG ? (NC - cpart + ch - 1) / ch : NC;            // chunks held in TMEM
   const long long T = sched[B];
-  const long long tb = dev::split_begin(blockIdx.x, G, T);
-  const long long te = dev::split_begin(blockIdx.x + 1, G, T);
+  const long long tb = dev::split_begin(g, G, T);
+  const long long te = dev::split_begin(g + 1, G, T);
   if (tb >= te) return;   // uniform across the CTA, before any barrier or TMEM use
   const int n = int(te - tb);
 
@@ -763,7 +803,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
                                  max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
     else
       ok = produce<NP, QS, SG>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te,
-                               n, nslots, lane, &issued);
+                               n, nslots, lane, &issued, ch, cpart);
     if (!ok && lane == 0) {
       set_abort(s, status);
       drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
@@ -835,10 +875,10 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         const uint64_t pb = pb0 + uint64_t(((i & 1) * PS * pbuf_bytes<NP>()) >> 4);
         for (int u = 0; u < NI; ++u) {
           const int j = u >> 1, h = u & 1;   // 128-channel chunk, 64-token half
-          if (SG && (j & 1) != kind) continue;
+          if (SG && !sg_owns(j, ch, cpart, kind)) continue;
           if (!mbar_wait(saddr(&zfull[rg.slot]), rg.phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d = tmem + uint32_t(ZC0 + j * NP);
+          const uint32_t d = tmem + uint32_t(ZC0 + (SG ? j / ch : j) * NP);
           const uint64_t za = za0 + uint64_t((rg.slot * kZSlotBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {   // K = 16 tokens per MMA
@@ -867,7 +907,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     const int q = warp & 3;
     const int t = 32 * q + lane;              // token row in the tile == TMEM lane
     const uint32_t lane_off = uint32_t(32 * q) << 16;
-    float m_run[NP], l_part[NP];
+    // m and l per head live in shared memory (identical for the four warps);
+    // thread t < NP owns head t's entries
     TileIter it;
     it.init(sched, B, tb, te);
     Ring sgr(QB ? nsg : 1);   // quantised latent: the per-group S buffers
@@ -875,10 +916,6 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       const int pb = i & 1;
       const bool first = it.first(tb), last = it.last();
       const int nv = it.nvalid();
-      if (first) {
-#pragma unroll
-        for (int h = 0; h < NP; ++h) { m_run[h] = -INFINITY; l_part[h] = 0.f; }
-      }
       int fail = 0;
       float sv[NP];
       if (QB) {
@@ -886,8 +923,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 #pragma unroll
         for (int h = 0; h < NP; ++h) sv[h] = 0.f;
         const __half* tsc = scales + (size_t(it.b) * max_len + it.t0() + t) * NC;
-        for (int g = 0; g < NC; ++g) {
-          const float sg = t < nv ? __half2float(tsc[g]) : 0.f;
+        for (int grp = 0; grp < NC; ++grp) {
+          const float sg = t < nv ? __half2float(tsc[grp]) : 0.f;
           fail = group_or(!mbar_wait(saddr(&s.sg_full[sgr.slot]), sgr.phase));   // uniform
           if (fail) break;
           tc_fence_after();
@@ -931,11 +968,11 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         tmem_wait_ld();
       }
       const bool valid = t < nv;
-      int need = 0;
+      int need = first;   // a segment starts: m and l are set below
 #pragma unroll
       for (int h = 0; h < NP; ++h) {
         if (!valid) sv[h] = -INFINITY;
-        need |= sv[h] > m_run[h] + kRescaleLog2;
+        need |= sv[h] > s.m_run[h] + kRescaleLog2;
       }
       if (group_or(need)) {
         // exact tile max per head over the 128 rows
@@ -943,18 +980,17 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           float tmp[NP];
 #pragma unroll
           for (int h = 0; h < NP; ++h) tmp[h] = sv[h];
-          const float v = dev::warp_reduce_transposed<NP>(tmp, lane, dev::OpMax());
-          if (lane < NP) s.red[q * NP + lane] = v;
+          reduce_heads<NP>(tmp, s.red + q * NP, lane, dev::OpMax());
         }
         group_sync();
-        float alpha[NP];
-#pragma unroll
-        for (int h = 0; h < NP; ++h) {
-          const float mt = fmaxf(fmaxf(s.red[h], s.red[NP + h]), fmaxf(s.red[2 * NP + h], s.red[3 * NP + h]));
-          const float mn = fmaxf(m_run[h], mt);
-          alpha[h] = exp2f(m_run[h] - mn);
-          m_run[h] = mn;
-          l_part[h] *= alpha[h];
+        if (t < NP) {
+          const float mt = fmaxf(fmaxf(s.red[t], s.red[NP + t]), fmaxf(s.red[2 * NP + t], s.red[3 * NP + t]));
+          const float mo = first ? -INFINITY : s.m_run[t];
+          const float mn = fmaxf(mo, mt);
+          const float a = exp2f(mo - mn);
+          s.alpha[t] = a;
+          s.m_run[t] = mn;
+          s.l_run[t] = first ? 0.f : s.l_run[t] * a;
         }
         group_sync();
         if (!first) {
@@ -962,7 +998,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           fail = !mbar_wait(saddr(&s.z_done[(i - 1) & 1]), uint32_t((i - 1) >> 1) & 1u);
           if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
           tc_fence_after();
-          for (int c = 0; c < NC; ++c) {
+          for (int c = 0; c < NCL; ++c) {
 #pragma unroll
             for (int h16 = 0; h16 < NP / 16; ++h16) {
               float z[16];
@@ -970,7 +1006,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
               tmem_ld16(ta, z);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 16; ++e) z[e] *= alpha[16 * h16 + e];
+              for (int e = 0; e < 16; ++e) z[e] *= s.alpha[16 * h16 + e];
               tmem_st16(ta, z);
             }
           }
@@ -986,8 +1022,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       const int chunk = (t & 63) >> 3, within = (t & 7) * 2;
 #pragma unroll
       for (int h = 0; h < NP; ++h) {
-        const float p = valid ? exp2f(sv[h] - m_run[h]) : 0.f;
-        l_part[h] += p;
+        const float p = valid ? exp2f(sv[h] - s.m_run[h]) : 0.f;
+        sv[h] = p;
         uint8_t* dst = pbase + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
         if (PS == 2) {
           const __nv_bfloat16 hi = __float2bfloat16_rn(p);
@@ -1002,45 +1038,49 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       tc_fence_before();
       group_sync();
       if (t == 0) mbar_arrive(saddr(&s.p_full[pb]));
+      // l += this tile's P summed over its 128 tokens (after the hand-off)
+      reduce_heads<NP>(sv, s.red + q * NP, lane, dev::OpAdd());
+      group_sync();
+      if (t < NP) s.l_run[t] += (s.red[t] + s.red[NP + t]) + (s.red[2 * NP + t] + s.red[3 * NP + t]);
       if (last) {
         fail = !mbar_wait(saddr(&s.z_done[pb]), uint32_t(i >> 1) & 1u);
         if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
         tc_fence_after();
-        const size_t slot = size_t(blockIdx.x) + it.b;
-        // z^T chunk c: TMEM lane = channel 128 c + t, column = head; the
-        // load of chunk c + 1 is in flight while chunk c is stored
+        const size_t slot = size_t(g) + it.b;
+        // z^T chunk c: TMEM lane = channel 128 c + t, column = head, taken
+        // EW head columns at a time (registers); the load of chunk c + 1 is
+        // in flight while chunk c is stored
+        constexpr int EW = NP % 32 == 0 ? 32 : 16;
         float* zrow = pz + slot * size_t(H) * r + t;
-        float zc[NP], zn[NP];
+#pragma unroll 1
+        for (int hg = 0; hg < NP / EW; ++hg) {
+          float zc[EW], zn[EW];
+          const uint32_t tcol = tmem + lane_off + uint32_t(ZC0 + hg * EW);
 #pragma unroll
-        for (int h16 = 0; h16 < NP / 16; ++h16)
-          tmem_ld16(tmem + lane_off + uint32_t(ZC0 + 16 * h16), zc + 16 * h16);
-        tmem_wait_ld();
-        for (int c = 0; c < NC; ++c) {
-          if (c + 1 < NC) {
-#pragma unroll
-            for (int h16 = 0; h16 < NP / 16; ++h16)
-              tmem_ld16(tmem + lane_off + uint32_t(ZC0 + (c + 1) * NP + 16 * h16), zn + 16 * h16);
-          }
-          float* zp = zrow + 128 * c;   // row pointer stepped by r: no per-store index arithmetic
-#pragma unroll
-          for (int h = 0; h < NP; ++h) {
-            if (h < H) *zp = zc[h];
-            zp += r;
-          }
+          for (int e16 = 0; e16 < EW / 16; ++e16) tmem_ld16(tcol + uint32_t(16 * e16), zc + 16 * e16);
           tmem_wait_ld();
+          for (int c = 0; c < NCL; ++c) {
+            if (c + 1 < NCL) {
 #pragma unroll
-          for (int h = 0; h < NP; ++h) zc[h] = zn[h];
+              for (int e16 = 0; e16 < EW / 16; ++e16)
+                tmem_ld16(tcol + uint32_t((c + 1) * NP + 16 * e16), zn + 16 * e16);
+            }
+            // row pointer stepped by r: no per-store index arithmetic
+            float* zp = zrow + size_t(hg * EW) * r + 128 * (SG ? c * ch + cpart : c);
+#pragma unroll
+            for (int e = 0; e < EW; ++e) {
+              if (hg * EW + e < H) *zp = zc[e];
+              zp += r;
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < EW; ++e) zc[e] = zn[e];
+          }
         }
-        {
-          const float v = dev::warp_reduce_transposed<NP>(l_part, lane, dev::OpAdd());   // l_part is dead after
-          if (lane < NP) s.red[q * NP + lane] = v;
+        if (cpart == 0 && t < H && t < NP) {   // the thread that owns head t's m and l
+          pl[slot * H + t] = s.l_run[t];
+          pm[slot * H + t] = s.m_run[t];
         }
-        group_sync();
-        if (t < H && t < NP) {
-          pl[slot * H + t] = s.red[t] + s.red[NP + t] + s.red[2 * NP + t] + s.red[3 * NP + t];
-          pm[slot * H + t] = m_run[t];
-        }
-        group_sync();
       }
       it.next();
       if (group_or(*s.abort_flag)) break;
@@ -1294,7 +1334,7 @@ void ring_slots(int* ns, int* nz) {
 template <int NP, bool BF16, int QB, bool SG = false>
 cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                      const float* scores, const int32_t* sched, int G, float* pm, float* pl,
-                     float* pz, int32_t* status, cudaStream_t s) {
+                     float* pz, int32_t* status, cudaStream_t s, int ch = 1) {
   TensorMapEncode enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
@@ -1390,9 +1430,9 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   auto kern = k_split_tc<NP, BF16, QS, PS, QB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<G, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache),
-                                   static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status,
-                                   d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw);
+  kern<<<G * ch, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache),
+                                        static_cast<const __half*>(scales), scores, sched, pm, pl, pz,
+                                        status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch);
   note_launch();
   return check_launch();
 }
@@ -1475,22 +1515,38 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
   }
 }
 
+// Scores given: heads padded to 16, 32 or 48 (softmax registers), and the
+// Z accumulator of the 128-channel chunks a CTA holds within TMEM's 512
+// columns -- shared over ch CTAs when all chunks do not fit.
+static int sg_heads_padded(const qsvd_dims& d) {
+  return d.H <= 16 ? 16 : (d.H <= 32 ? 32 : (d.H <= 48 ? 48 : 0));
+}
+
+int split_tc_scores_parts(const qsvd_dims& d) {
+  const int np = sg_heads_padded(d), nc = d.r / 128;
+  if (np == 0 || nc == 0) return 0;
+  int ch = 1;
+  while ((nc + ch - 1) / ch * np > 512) ++ch;
+  return ch <= 8 ? ch : 0;
+}
+
 bool split_tc_scores_supported(const qsvd_dims& d) {
   if (d.cache_dtype != QSVD_F16 && d.cache_dtype != QSVD_BF16) return false;
   if (d.r % 128) return false;
-  const int np = split_tc_heads_padded(d);
-  return np != 0 && (d.r / 128) * np <= 512;   // Z accumulators only
+  return split_tc_scores_parts(d) != 0;
 }
 
 cudaError_t launch_split_tc_scores(const qsvd_dims& d, const float* scores, const void* cache,
                                    const int32_t* sched, int G, float* pm, float* pl, float* pz,
                                    int32_t* status, cudaStream_t s) {
-  const int np = split_tc_heads_padded(d);
+  const int np = sg_heads_padded(d), ch = split_tc_scores_parts(d);
+  if (ch == 0) return cudaErrorInvalidConfiguration;
+#define QSVD_SG(NP, BF)                                                                         \
+  launch_t<NP, BF, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s, ch)
   if (d.cache_dtype == QSVD_BF16)
-    return np == 16 ? launch_t<16, true, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s)
-                    : launch_t<32, true, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s);
-  return np == 16 ? launch_t<16, false, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s)
-                  : launch_t<32, false, 0, true>(d, cache, nullptr, nullptr, scores, sched, G, pm, pl, pz, status, s);
+    return np == 16 ? QSVD_SG(16, true) : np == 32 ? QSVD_SG(32, true) : QSVD_SG(48, true);
+  return np == 16 ? QSVD_SG(16, false) : np == 32 ? QSVD_SG(32, false) : QSVD_SG(48, false);
+#undef QSVD_SG
 }
 
 bool rope_tc_supported(const qsvd_dims& d) {

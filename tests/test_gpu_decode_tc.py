@@ -36,14 +36,17 @@ def case(key):
             "i4h32": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=768, B=2, L=600,
                                        h2_n=256),
         }[key]
-        if w.E > 1024:
-            # direct seeded factors: skips the E x 3E SVD, which decode parity does not need
-            wuq, wuk, wuv = (a.astype(np.float64) for a in synthetic.direct_up_weights_np(w))
-            wd = synthetic.direct_down_weight_np(w).astype(np.float64)
-            _CASES[key] = oi.build_case(w, factors_override=(0.5, (wd, wuq, wuk, wuv), None))
-        else:
-            _CASES[key] = oi.build_case(w)
+        _CASES[key] = _build(w)
     return _CASES[key]
+
+
+def _build(w):
+    if w.E > 1024:
+        # direct seeded factors: skips the E x 3E SVD, which decode parity does not need
+        wuq, wuk, wuv = (a.astype(np.float64) for a in synthetic.direct_up_weights_np(w))
+        wd = synthetic.direct_down_weight_np(w).astype(np.float64)
+        return oi.build_case(w, factors_override=(0.5, (wd, wuq, wuk, wuv), None))
+    return oi.build_case(w)
 
 
 @pytest.mark.parametrize("key", ["full", "f16", "bf16", "h32", "r768", "i4", "i8", "i4h32"])
@@ -136,12 +139,20 @@ def rope_case(key):
              "s4": synthetic.SHRUNK[4],                      # bf16, r 384 (odd chunk count), H 5, ragged
              "s2f16": synthetic.replace(base, cache="f16", weight="f16"),
              "h32": synthetic.replace(base, E=4096, H=32, r=384, B=2, L=520),
+             # heads padded to 48; Z of all chunks beyond TMEM: two CTAs per
+             # split, 9 + 9 chunks (r 2304) and 6 + 5 chunks (r 1408)
+             "h40": synthetic.replace(synthetic.SHRUNK[4], E=5120, H=40, r=2304, B=2, L=300,
+                                      ragged=(150, 300)),
+             "h40r1408": synthetic.replace(base, E=5120, H=40, r=1408, B=2, L=280),
+             "h40r384": synthetic.replace(base, E=5120, H=40, r=384, B=2, L=260),
+             "h32r2304": synthetic.replace(base, E=4096, H=32, r=2304, B=2, L=270),
              "r320": synthetic.replace(base, r=320)}[key]    # CUDA-core softmax on given scores
-        _ROPE[key] = oi.build_case(w)
+        _ROPE[key] = _build(w)
     return _ROPE[key]
 
 
-@pytest.mark.parametrize("key", ["s2", "s4", "s2f16", "h32", "r320"])
+@pytest.mark.parametrize("key", ["s2", "s4", "s2f16", "h32", "h40", "h40r1408", "h40r384",
+                                 "h32r2304", "r320"])
 def test_tc_rope_matches_oracle(cuda_ok, key):
     c = rope_case(key)
     got, ws = GpuCase(c, kernel=TC).decode()
@@ -150,7 +161,7 @@ def test_tc_rope_matches_oracle(cuda_ok, key):
     assert err <= TOL, f"{key}: {err:.3e}"
 
 
-@pytest.mark.parametrize("key", ["s2", "s4", "h32"])
+@pytest.mark.parametrize("key", ["s2", "s4", "h32", "h40"])
 def test_tc_rope_agrees_with_simt(cuda_ok, key):
     c = rope_case(key)
     a, _ = GpuCase(c, kernel=TC).decode()
@@ -158,9 +169,10 @@ def test_tc_rope_agrees_with_simt(cuda_ok, key):
     assert rel_err(a, b) <= TOL
 
 
-@pytest.mark.parametrize("splits", [1, 3, 1000])
-def test_tc_rope_split_invariance(cuda_ok, splits):
-    c = rope_case("h32")
+@pytest.mark.parametrize("key,splits", [("h32", 1), ("h32", 3), ("h32", 1000), ("h40", 1),
+                                        ("h40", 7)])
+def test_tc_rope_split_invariance(cuda_ok, key, splits):
+    c = rope_case(key)
     got, ws = GpuCase(c, kernel=TC).decode(num_splits=splits)
     assert q.status_word(ws) == 0
     assert rel_err(got, c.reference()) <= TOL
