@@ -210,7 +210,8 @@ def run_ours(args, rank, world, local_rank):
     inp = bench_inputs(args.config, device, rank)
     w, lens, max_len = inp["w"], inp["lens"], inp["max_len"]
     kern = {"auto": q.QSVD_KERNEL_AUTO, "simt": q.QSVD_KERNEL_SIMT,
-            "tcgen05": q.QSVD_KERNEL_TCGEN05}[args.kernel]
+            "tcgen05": q.QSVD_KERNEL_TCGEN05, "cta": q.QSVD_KERNEL_TCGEN05_CTA,
+            "cluster": q.QSVD_KERNEL_TCGEN05_CLUSTER}[args.kernel]
     dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
                        out="f32", group=w.group, rope=w.rope, rope_base=w.rope_base,
                        kernel=kern)
@@ -236,7 +237,7 @@ def run_ours(args, rank, world, local_rank):
     decode(q.QSVD_PHASE_ALL, stream)
     torch.cuda.synchronize()
     kernel_used = int(dec_ws[12:16].view(torch.int32).item())   # workspace header: kernel
-    rope_tc = w.rope and kernel_used == q.QSVD_KERNEL_TCGEN05
+    rope_tc = w.rope and kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
     # the phases of one step, one API call each; rotary mode on the tensor
     # cores runs the split as its two passes so that the scores pass (the
     # dominant kernel there) is timed on its own
@@ -343,9 +344,11 @@ def run_ours(args, rank, world, local_rank):
     dom_mean = statistics.mean(dom_ms)
     lat_b = latent_bytes(w, lens)
     kname = ("k_rope_scores" if rope_tc
-             else "k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05
+             else "k_split_cl" if kernel_used == q.QSVD_KERNEL_TCGEN05_CLUSTER
+             else "k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
              else "k_split_rope" if w.rope else "k_split_abs")
-    src = (["split_tc.cu", "internal.cuh"] if kname in ("k_split_tc", "k_rope_scores")
+    src = (["split_cluster.cu", "tc_common.cuh", "internal.cuh"] if kname == "k_split_cl"
+           else ["split_tc.cu", "tc_common.cuh", "internal.cuh"] if kname in ("k_split_tc", "k_rope_scores")
            else ["split_simt.cu", "internal.cuh"])
     workload = w.name
     traffic = profiled_traffic(kname, workload, src)
@@ -473,7 +476,7 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--splits", type=int, default=0)
-    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05", "cta", "cluster"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",

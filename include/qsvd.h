@@ -88,7 +88,15 @@ typedef enum {
 /* Split-kernel choice (qsvd_dims.kernel). */
 #define QSVD_KERNEL_AUTO 0
 #define QSVD_KERNEL_SIMT 1      /* CUDA-core split kernel: every dtype and mode */
-#define QSVD_KERNEL_TCGEN05 2   /* tensor-core split kernel (tcgen05, TMA) */
+#define QSVD_KERNEL_TCGEN05 2   /* tensor cores (tcgen05, TMA): one CTA per split where
+                                   that kernel applies, else the cluster kernel */
+#define QSVD_KERNEL_TCGEN05_CTA 3      /* tensor cores, one CTA per split */
+#define QSVD_KERNEL_TCGEN05_CLUSTER 4  /* tensor cores, the latent channels of a tile
+                                          spread over a thread-block cluster (absorbed
+                                          mode, fp16/bf16 cache, r = 128 k or 256 k with
+                                          2 <= k <= 8, H <= 32) */
+/* The workspace header records the kernel that ran: SIMT, TCGEN05_CTA or
+ * TCGEN05_CLUSTER. */
 
 typedef struct {
   int E;               /* model width, E = H * d_h */

@@ -31,6 +31,7 @@ QSVD_PHASE_PROLOGUE, QSVD_PHASE_SPLIT, QSVD_PHASE_COMBINE, QSVD_PHASE_ALL = 1, 2
 QSVD_PHASE_SPLIT_SCORES, QSVD_PHASE_SPLIT_ACCUM = 8, 16
 QSVD_STATUS_LEN_CLAMPED, QSVD_STATUS_POS_OOB, QSVD_STATUS_SCALE_SAT, QSVD_STATUS_TIMEOUT = 1, 2, 4, 8
 QSVD_KERNEL_AUTO, QSVD_KERNEL_SIMT, QSVD_KERNEL_TCGEN05 = 0, 1, 2
+QSVD_KERNEL_TCGEN05_CTA, QSVD_KERNEL_TCGEN05_CLUSTER = 3, 4
 
 DTYPE_CODE = {"f32": QSVD_F32, "f16": QSVD_F16, "bf16": QSVD_BF16, "i8": QSVD_I8, "i4": QSVD_I4}
 

@@ -77,7 +77,7 @@ static qsvd_status validate(const qsvd_dims* d) {
     if (d->h2_m < 1 || d->h2_m > 16 || d->r % d->h2_m || !is_pow2(d->r / d->h2_m))
       return fail(QSVD_ERR_INVALID_ARG, "H2 needs r/h2_m a power of two, 1 <= h2_m <= 16");
   }
-  if (d->kernel < QSVD_KERNEL_AUTO || d->kernel > QSVD_KERNEL_TCGEN05)
+  if (d->kernel < QSVD_KERNEL_AUTO || d->kernel > QSVD_KERNEL_TCGEN05_CLUSTER)
     return fail(QSVD_ERR_INVALID_ARG, "unknown kernel choice %d", d->kernel);
   return QSVD_OK;
 }
@@ -89,12 +89,25 @@ static int device_sms() {
   return sms;
 }
 
-// Split kernel actually used for these dims.
+// Split kernel actually used for these dims: SIMT, TCGEN05_CTA or
+// TCGEN05_CLUSTER (the rotary tensor-core path counts as one CTA per split).
+// The tensor-core choice prefers one CTA per split: on the LLaVA-7B fp16
+// workload it measured 112 us against 515 us for the cluster kernel, whose
+// per-tile cross-CTA exchange of partial scores sits on the softmax's path.
 static int pick_kernel(const qsvd_dims& d) {
-  if (d.kernel == QSVD_KERNEL_SIMT) return QSVD_KERNEL_SIMT;
-  if (d.kernel == QSVD_KERNEL_TCGEN05) return QSVD_KERNEL_TCGEN05;
-  if (d.rope) return rope_tc_supported(d) ? QSVD_KERNEL_TCGEN05 : QSVD_KERNEL_SIMT;
-  return split_tc_supported(d) ? QSVD_KERNEL_TCGEN05 : QSVD_KERNEL_SIMT;
+  const bool cl = split_cl_supported(d);
+  switch (d.kernel) {
+    case QSVD_KERNEL_SIMT:
+    case QSVD_KERNEL_TCGEN05_CTA:
+    case QSVD_KERNEL_TCGEN05_CLUSTER:
+      return d.kernel;
+    case QSVD_KERNEL_TCGEN05:
+      if (d.rope || split_tc_supported(d)) return QSVD_KERNEL_TCGEN05_CTA;
+      return cl ? QSVD_KERNEL_TCGEN05_CLUSTER : QSVD_KERNEL_TCGEN05_CTA;
+    default:
+      if (d.rope) return rope_tc_supported(d) ? QSVD_KERNEL_TCGEN05_CTA : QSVD_KERNEL_SIMT;
+      return split_tc_supported(d) ? QSVD_KERNEL_TCGEN05_CTA : (cl ? QSVD_KERNEL_TCGEN05_CLUSTER : QSVD_KERNEL_SIMT);
+  }
 }
 
 static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel, int* G) {
@@ -104,9 +117,12 @@ static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel
   if (g == 0) {
     const int sms = device_sms();
     if (sms <= 0) return fail(QSVD_ERR_CUDA, "no CUDA device to size the split grid");
-    if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope) {
+    if (kernel == QSVD_KERNEL_TCGEN05_CLUSTER) {
+      g = split_cl_clusters(d);   // as many clusters as fit at once
+      if (g <= 0) return fail(QSVD_ERR_CUDA, "no cluster configuration fits this device");
+    } else if (kernel == QSVD_KERNEL_TCGEN05_CTA && !d.rope) {
       g = sms;   // one CTA per SM (persistent over its tile range)
-    } else if (kernel == QSVD_KERNEL_TCGEN05 && split_tc_scores_supported(d)) {
+    } else if (kernel == QSVD_KERNEL_TCGEN05_CTA && split_tc_scores_supported(d)) {
       g = sms / split_tc_scores_parts(d);   // ch CTAs per split, one per SM
       if (g < 1) g = 1;
     } else {
@@ -209,14 +225,17 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
   constexpr unsigned kSub = QSVD_PHASE_SPLIT_SCORES | QSVD_PHASE_SPLIT_ACCUM;
   if (phases & ~(QSVD_PHASE_ALL | kSub)) return fail(QSVD_ERR_INVALID_ARG, "unknown phase bits");
   const int kernel = pick_kernel(d);
-  if ((phases & kSub) && !(d.rope && kernel == QSVD_KERNEL_TCGEN05))
+  if ((phases & kSub) && !(d.rope && kernel == QSVD_KERNEL_TCGEN05_CTA))
     return fail(QSVD_ERR_INVALID_ARG, "split sub-phases exist in rotary mode on the tensor cores only");
   if (phases & QSVD_PHASE_SPLIT) phases |= kSub;
   const bool split_any = (phases & kSub) != 0;
-  if (kernel == QSVD_KERNEL_TCGEN05 && !d.rope && !split_tc_supported(d))
+  if (kernel == QSVD_KERNEL_TCGEN05_CLUSTER && !split_cl_supported(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "cluster split kernel needs absorbed mode, a 16-bit cache, r = 128 k or 256 k (2 <= k <= 8), H <= 32");
+  if (kernel == QSVD_KERNEL_TCGEN05_CTA && !d.rope && !split_tc_supported(d))
     return fail(QSVD_ERR_UNSUPPORTED,
                 "tensor-core split kernel needs a 16-bit or int4/int8 (group 128) cache, r %% 128 == 0, H <= 32");
-  if (kernel == QSVD_KERNEL_TCGEN05 && d.rope && !rope_tc_supported(d))
+  if (kernel == QSVD_KERNEL_TCGEN05_CTA && d.rope && !rope_tc_supported(d))
     return fail(QSVD_ERR_UNSUPPORTED,
                 "tensor-core rotary path needs d_h == 128, r %% 64 == 0, cache and weights both fp16 or both bf16");
   if (kernel == QSVD_KERNEL_SIMT && !d.rope && split_simt_grid_heads(d) == 0)
@@ -273,7 +292,7 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (split_any) {
-    if (d.rope && kernel == QSVD_KERNEL_TCGEN05) {
+    if (d.rope && kernel == QSVD_KERNEL_TCGEN05_CTA) {
       float* scores = reinterpret_cast<float*>(Wb + W.scores);
       const int sms = device_sms();
       e = cudaSuccess;
@@ -287,7 +306,9 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     } else if (d.rope) {
       e = launch_split_simt_rope(d, qt32, P + L.wuk, rope_tab, cache, scales, sched, G, pm, pl, pz, s);
     }
-    else if (kernel == QSVD_KERNEL_TCGEN05)
+    else if (kernel == QSVD_KERNEL_TCGEN05_CLUSTER)
+      e = launch_split_cl(d, cache, qt16, sched, G, pm, pl, pz, &hdr->status, s);
+    else if (kernel == QSVD_KERNEL_TCGEN05_CTA)
       e = launch_split_tc(d, cache, scales, qt16, sched, G, pm, pl, pz, &hdr->status, s);
     else
       e = launch_split_simt_absorbed(d, qt32, cache, scales, sched, G, pm, pl, pz, s);

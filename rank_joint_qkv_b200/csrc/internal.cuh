@@ -171,6 +171,12 @@ cudaError_t launch_split_simt_rope(const qsvd_dims& d, const float* qrot,
                                    float* pl, float* pz, cudaStream_t s);
 int split_simt_grid_heads(const qsvd_dims& d);   // head blocks per split
 bool split_tc_supported(const qsvd_dims& d);
+// Absorbed mode, the tile's channels spread over a thread-block cluster;
+// G = the number of clusters (split_cl_clusters: as many as fit at once).
+bool split_cl_supported(const qsvd_dims& d);
+int split_cl_clusters(const qsvd_dims& d);
+cudaError_t launch_split_cl(const qsvd_dims& d, const void* cache, const void* qt16, const int32_t* sched,
+                            int G, float* pm, float* pl, float* pz, int32_t* status, cudaStream_t s);
 cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s);

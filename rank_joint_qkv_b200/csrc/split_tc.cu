@@ -51,6 +51,7 @@
 #include <cstring>
 
 #include "internal.cuh"
+#include "tc_common.cuh"
 
 namespace qsvd {
 namespace {
@@ -60,206 +61,8 @@ constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 
 constexpr int kMaxSlots = 8;                   // per ring
 constexpr int kMaxGroupBufs = 4;               // S accumulators per channel group (quantised latent)
 constexpr int kMaxRaw = 8;                     // raw-code slots per stream (quantised latent)
-constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
-// ------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait for the phase of `parity` to complete; false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = gtimer();
-  while (!mbar_try(bar, parity)) {
-    if (gtimer() - t0 > kWaitNs) return false;
-  }
-  return true;
-}
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// 2D tiled load with an L2 eviction-priority policy (createpolicy).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x,
-                                                 int y, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
-// 3D tiled load with an L2 eviction-priority policy (createpolicy).
-__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                                 int z, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            int z, int w, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 16 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15]))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// Named barrier over the 128 softmax threads, OR-reduction of a predicate.
-__device__ __forceinline__ int group_or(int pred) {
-  int r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.s32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
-      "selp.s32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred)
-      : "memory");
-  return r;
-}
-__device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
-         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
-}
-// kind::f16 instruction descriptor: fp32 accumulate, A/B f16 or bf16.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a_mn, bool b_mn) {
-  return (1u << 4) | (uint32_t(bf16) << 7) | (uint32_t(bf16) << 10) | (uint32_t(a_mn) << 15) |
-         (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
-}
-
-// --------------------------------------------------------------- schedule
-
-struct TileIter {
-  const int32_t* ts;
-  const int32_t* ln;
-  long long g, te;
-  int b;
-  __device__ void init(const int32_t* sched, int B, long long tb, long long te_) {
-    ts = sched;
-    ln = sched + B + 1;
-    g = tb;
-    te = te_;
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (ts[mid] <= g) lo = mid; else hi = mid - 1;
-    }
-    b = lo;
-    while (ts[b + 1] <= g) ++b;
-  }
-  __device__ void next() {
-    ++g;
-    if (g < te)
-      while (ts[b + 1] <= g) ++b;
-  }
-  __device__ int t0() const { return int(g - ts[b]) * kTile; }
-  __device__ int nvalid() const { return min(kTile, ln[b] - t0()); }
-  __device__ bool first(long long tb) const { return g == tb || g == ts[b]; }
-  __device__ bool last() const { return g == te - 1 || g + 1 == ts[b + 1]; }
-};
 
 // Shared-memory carve.  Both rings carry items of 1/(r/64) of a tile.
 //   S slot: one 64-channel box of the latent tile (128 tokens x 128 bytes,
@@ -348,27 +151,6 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   return s;
 }
 
-// Per-head reduction over the 32 lanes of a warp into red[0..NP): lane L
-// writes head L (and 32 + L for NP = 48, reduced as 32 + 16).  v is consumed.
-template <int NP, typename Op>
-__device__ __forceinline__ void reduce_heads(float (&v)[NP], float* red, int lane, Op op) {
-  if constexpr (NP <= 32) {
-    const float x = dev::warp_reduce_transposed<NP>(v, lane, op);
-    if (lane < NP) red[lane] = x;
-  } else {
-    static_assert(NP == 48, "heads padded to 16, 32 or 48");
-    float a[32], b[16];
-#pragma unroll
-    for (int h = 0; h < 32; ++h) a[h] = v[h];
-#pragma unroll
-    for (int h = 0; h < 16; ++h) b[h] = v[32 + h];
-    const float xa = dev::warp_reduce_transposed<32>(a, lane, op);
-    red[lane] = xa;
-    const float xb = dev::warp_reduce_transposed<16>(b, lane, op);
-    if (lane < 16) red[32 + lane] = xb;
-  }
-}
-
 // SG with a channel split over `ch` CTAs: 128-channel chunk j belongs to CTA
 // part j % ch, and there to the issuer (and ring) (j / ch) % 2.
 __device__ __forceinline__ bool sg_owns(int j, int ch, int cpart, int kind) {
@@ -380,16 +162,6 @@ __device__ __forceinline__ void set_abort(const Smem& s, int32_t* status) {
   atomicOr(status, QSVD_STATUS_TIMEOUT);
 }
 
-// Ring position: slot index and the parity of its current use.
-struct Ring {
-  int slot = 0;
-  uint32_t phase = 0;
-  int n;
-  __device__ explicit Ring(int n_) : n(n_) {}
-  __device__ void advance() {
-    if (++slot == n) { slot = 0; phase ^= 1u; }
-  }
-};
 
 // Zero-filled copy of latent rows into a slot by one warp, in the
 // 128-byte-swizzled layout TMA would have produced: `nbox` 64-channel boxes
@@ -1020,9 +792,18 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       }
       uint8_t* pbase = s.pbuf + pb * PS * pbuf_bytes<NP>() + (t >> 6) * NP * 128;
       const int chunk = (t & 63) >> 3, within = (t & 7) * 2;
+      float mr[NP];   // m into registers first: the P stores below would order each reload
+#pragma unroll
+      for (int h4 = 0; h4 < NP / 4; ++h4) {
+        const float4 v = reinterpret_cast<const float4*>(s.m_run)[h4];
+        mr[4 * h4] = v.x;
+        mr[4 * h4 + 1] = v.y;
+        mr[4 * h4 + 2] = v.z;
+        mr[4 * h4 + 3] = v.w;
+      }
 #pragma unroll
       for (int h = 0; h < NP; ++h) {
-        const float p = valid ? exp2f(sv[h] - s.m_run[h]) : 0.f;
+        const float p = valid ? exp2f(sv[h] - mr[h]) : 0.f;
         sv[h] = p;
         uint8_t* dst = pbase + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
         if (PS == 2) {

@@ -150,3 +150,14 @@ def test_split_sub_phases_rejected_outside_rotary_tensor_path():
     st = lib.qsvd_decode_attn(ctypes.byref(_dims()), fake, fake, 1, fake, None, fake, 4, fake,
                               ctypes.byref(n), fake, 32, None)
     assert st == q.QSVD_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(cache="i4"), dict(rope=True), dict(H=40, E=5120),
+                                 dict(r=64 * 3, E=512), dict(r=128 * 9 * 2, E=2304, H=18)])
+def test_cluster_kernel_refused_where_it_does_not_apply(bad):
+    """Forcing the cluster kernel on dims it does not cover is UNSUPPORTED,
+    decided on the host."""
+    d = _dims(kernel=q.QSVD_KERNEL_TCGEN05_CLUSTER, **bad)
+    with pytest.raises(q.QsvdError) as e:
+        q.decode_workspace_bytes(d, num_splits=4)
+    assert e.value.status == q.QSVD_ERR_UNSUPPORTED

@@ -1,6 +1,9 @@
-"""Parity of the tensor-core split kernel (tcgen05 + TMA, absorbed query,
+"""Parity of the tensor-core split kernels (tcgen05 + TMA, absorbed query,
 fp16/bf16 latent, int4/int8 latent with group scales) against the fp64
-oracle and against the CUDA-core kernel.
+oracle and against the CUDA-core kernel.  The 16-bit cases run both
+tensor-core variants: one CTA per split (CTA) and the tile's channels spread
+over a thread-block cluster (CL; r = 256 -> 2 CTAs, 384 -> 3, 768 -> 3,
+1536 -> 6, 2048 -> 8).
 
 Bar: max |o_gpu - o_ref| / rms(o_ref) <= 2e-3 (P and the absorbed query are
 rounded to the latent's 16-bit type before the MMA; accumulation is fp32).
@@ -17,6 +20,13 @@ from tests.gpu_util import GpuCase, rel_err
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
 TC = q.QSVD_KERNEL_TCGEN05
+CTA, CL = q.QSVD_KERNEL_TCGEN05_CTA, q.QSVD_KERNEL_TCGEN05_CLUSTER
+BOTH = [CTA, CL]
+
+
+def kernel_ran(ws):
+    """Split kernel recorded in the workspace header."""
+    return int(ws[12:16].view(torch.int32).item())
 
 _CASES = {}
 
@@ -35,6 +45,11 @@ def case(key):
             "i8": synthetic.replace(synthetic.SHRUNK[3], cache="i8", name="shrunk-int8-h2"),
             "i4h32": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=768, B=2, L=600,
                                        h2_n=256),
+            # cluster shapes: 6 CTAs of 256 channels (the LLaVA-7B rank), 8 of 256
+            "c6": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=300),
+            "c6bf": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=290, cache="bf16",
+                                      weight="bf16"),
+            "c8": synthetic.replace(base, E=2048, H=16, r=2048, B=2, L=280),
         }[key]
         _CASES[key] = _build(w)
     return _CASES[key]
@@ -49,28 +64,47 @@ def _build(w):
     return oi.build_case(w)
 
 
-@pytest.mark.parametrize("key", ["full", "f16", "bf16", "h32", "r768", "i4", "i8", "i4h32"])
-def test_tc_matches_oracle(cuda_ok, key):
+_KEYS16 = ["full", "f16", "bf16", "h32", "r768", "c6", "c6bf", "c8"]
+
+
+@pytest.mark.parametrize("key,kern", [(k, v) for k in _KEYS16 for v in BOTH] +
+                         [(k, CTA) for k in ("i4", "i8", "i4h32")])
+def test_tc_matches_oracle(cuda_ok, key, kern):
     c = case(key)
-    g = GpuCase(c, kernel=TC)
+    g = GpuCase(c, kernel=kern)
     got, ws = g.decode()
     assert q.status_word(ws) == 0
+    assert kernel_ran(ws) == kern
     err = rel_err(got, c.reference())
     assert err <= TOL, f"{key}: {err:.3e}"
 
 
-@pytest.mark.parametrize("key", ["f16", "bf16", "i4", "i8"])
-def test_tc_agrees_with_simt(cuda_ok, key):
+@pytest.mark.parametrize("key,kern", [("f16", CTA), ("f16", CL), ("bf16", CTA), ("bf16", CL),
+                                      ("c6", CL), ("i4", CTA), ("i8", CTA)])
+def test_tc_agrees_with_simt(cuda_ok, key, kern):
     c = case(key)
-    a, _ = GpuCase(c, kernel=TC).decode()
+    a, _ = GpuCase(c, kernel=kern).decode()
     b, _ = GpuCase(c, kernel=q.QSVD_KERNEL_SIMT).decode()
     assert rel_err(a, b) <= TOL
 
 
+def test_tc_auto_picks_one_cta_per_split(cuda_ok):
+    """The default and the generic tensor-core request run one CTA per split
+    (faster than the cluster kernel on the 16-bit workloads measured); the
+    cluster kernel runs when asked for."""
+    for kern in (q.QSVD_KERNEL_AUTO, TC):
+        for key in ("f16", "i4"):
+            _, ws = GpuCase(case(key), kernel=kern).decode()
+            assert kernel_ran(ws) == CTA
+    _, ws = GpuCase(case("f16"), kernel=CL).decode()
+    assert kernel_ran(ws) == CL
+
+
+@pytest.mark.parametrize("kern", BOTH)
 @pytest.mark.parametrize("splits", [1, 2, 3, 7, 1000])
-def test_tc_split_invariance(cuda_ok, splits):
+def test_tc_split_invariance(cuda_ok, splits, kern):
     c = case("h32")
-    g = GpuCase(c, kernel=TC)
+    g = GpuCase(c, kernel=kern)
     base, _ = g.decode(num_splits=1)
     got, ws = g.decode(num_splits=splits)
     assert q.status_word(ws) == 0
@@ -80,11 +114,12 @@ def test_tc_split_invariance(cuda_ok, splits):
     assert rel_err(got, c.reference()) <= TOL
 
 
+@pytest.mark.parametrize("kern", BOTH)
 @pytest.mark.parametrize("lens", [[1, 0, 2], [127, 128, 129], [255, 256, 257], [300, 1, 300]])
-def test_tc_edge_lengths(cuda_ok, lens):
+def test_tc_edge_lengths(cuda_ok, lens, kern):
     w = synthetic.replace(synthetic.SHRUNK[1], B=len(lens), ragged=None, L=max(lens))
     c = oi.build_case(w, lengths=np.array(lens, np.int32))
-    got, ws = GpuCase(c, kernel=TC).decode(num_splits=2)
+    got, ws = GpuCase(c, kernel=kern).decode(num_splits=2)
     for b, n in enumerate(lens):
         if n == 0:
             assert np.all(got[b] == 0.0)
@@ -92,10 +127,11 @@ def test_tc_edge_lengths(cuda_ok, lens):
     assert q.status_word(ws) == 0
 
 
-def test_tc_nan_padding_rows(cuda_ok):
+@pytest.mark.parametrize("kern", BOTH)
+def test_tc_nan_padding_rows(cuda_ok, kern):
     """NaN in rows past each length (ragged tiles are zero-filled on load)."""
     c = case("f16")
-    g = GpuCase(c, kernel=TC)
+    g = GpuCase(c, kernel=kern)
     for b, n in enumerate(c.lengths):
         g.cache[b, int(n):] = float("nan")
     got, _ = g.decode(num_splits=4)
@@ -103,11 +139,12 @@ def test_tc_nan_padding_rows(cuda_ok):
     assert rel_err(got, c.reference()) <= TOL
 
 
-def test_tc_large_score_range_rescales(cuda_ok):
+@pytest.mark.parametrize("kern", BOTH)
+def test_tc_large_score_range_rescales(cuda_ok, kern):
     """Scores spanning far more than 2^8 between tiles force the conditional
     rescale of the latent accumulator."""
     c = case("full")
-    g = GpuCase(c, kernel=TC)
+    g = GpuCase(c, kernel=kern)
     # grow the latent along the sequence: later tiles dominate the softmax
     caches, lens = [], c.lengths
     w = c.w
