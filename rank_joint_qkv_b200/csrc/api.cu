@@ -315,7 +315,15 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (e != cudaSuccess) return cuda_fail(e, "split phase");
   }
   if (phases & QSVD_PHASE_COMBINE) {
-    if ((e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, W.P, out, s)) != cudaSuccess)
+    if (combine_uses_gemv(d)) {
+      float* zm = reinterpret_cast<float*>(Wb + W.zm);
+      int32_t* tickets = reinterpret_cast<int32_t*>(Wb + W.tickets) + W.NTQ;
+      e = launch_combine_gemv(d, hdr, sched, pm, pl, pz, P + L.wuv, zm, opart, tickets, &hdr->status,
+                              out, s);
+    } else {
+      e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, W.P, out, s);
+    }
+    if (e != cudaSuccess)
       return cuda_fail(e, "combine phase");
   }
   return QSVD_OK;

@@ -53,6 +53,8 @@ k_append_finish(const float* __restrict__ cpart, int KS, const float* __restrict
                 uint8_t* __restrict__ cache, __half* __restrict__ scales,
                 float* __restrict__ c_out, int32_t* status, int B, int r, int max_len,
                 int group) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   extern __shared__ float v[];   // r
   __shared__ float qm[256];
   const int b = blockIdx.x;
@@ -125,6 +127,8 @@ k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restric
                uint8_t* __restrict__ cache, __half* __restrict__ scales,
                float* __restrict__ c_out, int32_t* status, int B, int r, int max_len,
                int chunk) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   __shared__ float wmax[32];
   const int b = blockIdx.x;
   const int j = blockIdx.y * chunk + threadIdx.x;
@@ -176,7 +180,7 @@ template <typename WT>
 cudaError_t gemv_t(const qsvd_dims& d, const void* x, const void* wd, float* cpart, int KS,
                    int32_t* status, cudaStream_t s) {
   return launch_gemv<WT, WT>(static_cast<const WT*>(x), static_cast<const WT*>(wd), cpart, d.batch,
-                             d.E, d.r, KS, nullptr, nullptr, status, s);
+                             d.E, d.r, KS, static_cast<float*>(nullptr), nullptr, status, s);
 }
 
 int append_chunk(const qsvd_dims& d) {
@@ -193,9 +197,11 @@ cudaError_t finish_t(const qsvd_dims& d, const float* cpart, int KS, const float
   if (!d.h2) {
     const int chunk = append_chunk(d);
     dim3 grid(d.batch, d.r / chunk);
-    k_append_chunk<CT><<<grid, chunk, 0, s>>>(cpart, KS, pos, static_cast<uint8_t*>(cache),
-                                              static_cast<__half*>(scales), c_out, status,
-                                              d.batch, d.r, d.max_len, chunk);
+    {
+      const cudaError_t le = launch_pdl(k_append_chunk<CT>, dim3(grid), dim3(chunk), 0, s,
+                                       cpart, KS, pos, static_cast<uint8_t*>(cache), static_cast<__half*>(scales), c_out, status, d.batch, d.r, d.max_len, chunk);
+      if (le != cudaSuccess) return le;
+    }
     note_launch();
     return check_launch();
   }
@@ -203,9 +209,11 @@ cudaError_t finish_t(const qsvd_dims& d, const float* cpart, int KS, const float
   auto kern = k_append_finish<CT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<d.batch, 256, smem, s>>>(cpart, KS, h2q, h2_scale, d.h2_m, d.h2 ? 1 : 0, pos,
-                                  static_cast<uint8_t*>(cache), static_cast<__half*>(scales),
-                                  c_out, status, d.batch, d.r, d.max_len, d.group);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(d.batch), dim3(256), smem, s,
+                                     cpart, KS, h2q, h2_scale, d.h2_m, d.h2 ? 1 : 0, pos, static_cast<uint8_t*>(cache), static_cast<__half*>(scales), c_out, status, d.batch, d.r, d.max_len, d.group);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }

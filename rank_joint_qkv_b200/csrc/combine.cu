@@ -10,10 +10,85 @@
 // CTA (h, js) owns rows [128 js, 128 js + 128) of head h's columns and
 // handles every sequence.  The per-split weights are computed first (one warp
 // per sequence), so the partial loads that follow are independent.
+#include "gemv.cuh"
 #include "internal.cuh"
 
 namespace qsvd {
 namespace {
+
+// ----------------------------------------------- merge, then V-up GEMV
+//
+// For 16-bit weights with d_h a multiple of 64 the two steps run as two
+// kernels: the merge, wide (one CTA per 512 channels of one (sequence,
+// head), four channels per thread), writes the merged latent
+// zm[b][h][r] = sum_s w_s z_s (w_s = 2^(m_s - M) / L); the V-up is the
+// tensor-core GEMV with head h's output columns reading row zm[b][h].
+
+constexpr int kMergeCh = 512;   // channels per merge CTA (128 threads x 4)
+constexpr int kMergeMaxSplits = 2048;   // weights kept in shared memory per (b, h)
+
+// grid (ceil(r / 512), H, B), block 128.
+__global__ void __launch_bounds__(128)
+k_merge(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sched,
+        const float* __restrict__ pm, const float* __restrict__ pl, const float* __restrict__ pz,
+        float* __restrict__ zm, int B, int H, int r) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
+  __shared__ float wt[kMergeMaxSplits];
+  __shared__ int cr[2];
+  const int ch = blockIdx.x * kMergeCh + 4 * threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long G = hdr->G;
+  if (warp == 0) {
+    // the slots of sequence b: splits c0..c1 (slot c + b); dead splits weigh 0
+    const long long T = sched[B], t0 = sched[b], t1 = sched[b + 1];
+    int c0 = 0, c1 = -1;
+    if (t1 > t0) {
+      c0 = int(dev::split_of_tile(t0, G, T));
+      c1 = int(dev::split_of_tile(t1 - 1, G, T));
+    }
+    float M = -INFINITY;
+    for (int c = c0 + lane; c <= c1; c += 32)
+      if (dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T))
+        M = fmaxf(M, __ldcg(pm + (size_t(c) + b) * H + h));
+    M = dev::warp_max(M);
+    float L = 0.f;
+    for (int c = c0 + lane; c <= c1; c += 32) {
+      float w = 0.f;
+      if (dev::split_begin(c, G, T) != dev::split_begin(c + 1, G, T)) {
+        w = exp2f(__ldcg(pm + (size_t(c) + b) * H + h) - M);
+        L += w * __ldcg(pl + (size_t(c) + b) * H + h);
+      }
+      wt[c - c0] = w;
+    }
+    L = dev::warp_sum(L);
+    const float invL = L > 0.f ? 1.f / L : 0.f;
+    __syncwarp();
+    for (int c = c0 + lane; c <= c1; c += 32) wt[c - c0] *= invL;
+    if (lane == 0) { cr[0] = c0; cr[1] = c1; }
+  }
+  __syncthreads();
+  if (ch >= r) return;
+  const int c0 = cr[0], c1 = cr[1];
+  const float* base = pz + size_t(h) * r + ch;
+  float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int cb = c0; cb <= c1; cb += 8) {   // eight splits' loads in flight, added in split order
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = cb + i <= c1 && wt[cb + i - c0] != 0.f
+                 ? __ldcg(reinterpret_cast<const float4*>(base + (size_t(cb + i) + b) * H * r))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float w = cb + i <= c1 ? wt[cb + i - c0] : 0.f;
+      z.x = fmaf(w, v[i].x, z.x); z.y = fmaf(w, v[i].y, z.y);
+      z.z = fmaf(w, v[i].z, z.z); z.w = fmaf(w, v[i].w, z.w);
+    }
+  }
+  *reinterpret_cast<float4*>(zm + (size_t(b) * H + h) * r + ch) = z;
+}
 
 constexpr int kJ = 128;   // latent rows (of W^u_v) per CTA
 constexpr int kBC = 16;   // sequences per pass
@@ -33,6 +108,8 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
               const float* __restrict__ pm, const float* __restrict__ pl,
               const float* __restrict__ pz, const WT* __restrict__ wuv,
               float* __restrict__ opart, int B, int H, int d_h, int r, int E, int P) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   extern __shared__ __align__(16) uint8_t csm[];
   const int DQ = d_h / 4;                 // output quads per sequence
   const int KSP = 256 / (4 * DQ);         // k-splits of the V-up tile
@@ -193,6 +270,8 @@ k_combine_vup(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sche
 template <typename OT>
 __global__ void __launch_bounds__(256)
 k_combine_out(const float* __restrict__ opart, int JS, OT* __restrict__ out, size_t n) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   const size_t i = size_t(blockIdx.x) * 256 + threadIdx.x;
   if (i >= n) return;
   out[i] = dev::from_f<OT>(dev::sum_strided(opart + i, n, JS));
@@ -213,8 +292,11 @@ cudaError_t vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(d.H, JS);
-  kern<<<grid, 256, smem, s>>>(hdr, sched, pm, pl, pz, static_cast<const WT*>(wuv), opart,
-                               d.batch, d.H, d.d_h, d.r, d.E, P);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(256), smem, s,
+                                     hdr, sched, pm, pl, pz, static_cast<const WT*>(wuv), opart, d.batch, d.H, d.d_h, d.r, d.E, P);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
@@ -222,12 +304,66 @@ cudaError_t vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
 template <typename OT>
 cudaError_t out_t(const qsvd_dims& d, const float* opart, int JS, void* out, cudaStream_t s) {
   const size_t n = size_t(d.batch) * d.E;
-  k_combine_out<OT><<<unsigned((n + 255) / 256), 256, 0, s>>>(opart, JS, static_cast<OT*>(out), n);
+  {
+    const cudaError_t le = launch_pdl(k_combine_out<OT>, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s,
+                                     opart, JS, static_cast<OT*>(out), n);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
 
+template <typename WT, typename OT>
+cudaError_t merge_vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
+                        const float* pm, const float* pl, const float* pz, const void* wuv,
+                        float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
+                        cudaStream_t s) {
+  const dim3 grid((d.r + kMergeCh - 1) / kMergeCh, d.H, d.batch);
+  {
+    const cudaError_t le = launch_pdl(k_merge, dim3(grid), dim3(128), 0, s,
+                                     hdr, sched, pm, pl, pz, zm, d.batch, d.H, d.r);
+    if (le != cudaSuccess) return le;
+  }
+  note_launch();
+  cudaError_t e = check_launch();
+  if (e != cudaSuccess) return e;
+  // o[b][h d_h + n] = zm[b][h] . W^u_v[:, h d_h + n]: activation row of
+  // column group h (d_h columns) is zm + b H r + h r
+  const XGroups xg{(long long)d.H * d.r, d.d_h, d.r};
+  return launch_gemv<float, WT, OT>(zm, static_cast<const WT*>(wuv), vpart, d.batch, d.r, d.E,
+                                    gemv_ksplit(d.r, d.weight_dtype), static_cast<OT*>(out), tickets,
+                                    status, s, xg);
+}
+
 }  // namespace
+
+bool combine_uses_gemv(const qsvd_dims& d) {
+  // a sequence of max_len tokens meets at most tiles + 1 splits: all their
+  // merge weights must fit the merge kernel's shared memory
+  const long long tiles = (d.max_len + kTile - 1) / kTile;
+  return (d.weight_dtype == QSVD_F16 || d.weight_dtype == QSVD_BF16) && d.d_h % 64 == 0 &&
+         d.r % 32 == 0 && tiles + 1 <= kMergeMaxSplits;
+}
+
+cudaError_t launch_combine_gemv(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
+                                const float* pm, const float* pl, const float* pz, const void* wuv,
+                                float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
+                                cudaStream_t s) {
+#define QSVD_MV(WT)                                                                                    \
+  switch (d.out_dtype) {                                                                               \
+    case QSVD_F32: return merge_vup_t<WT, float>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart, tickets,   \
+                                                 status, out, s);                                      \
+    case QSVD_F16: return merge_vup_t<WT, __half>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart, tickets,  \
+                                                  status, out, s);                                     \
+    case QSVD_BF16: return merge_vup_t<WT, __nv_bfloat16>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart,   \
+                                                          tickets, status, out, s);                    \
+    default: return cudaErrorInvalidValue;                                                             \
+  }
+  if (d.weight_dtype == QSVD_BF16) { QSVD_MV(__nv_bfloat16) }
+  if (d.weight_dtype == QSVD_F16) { QSVD_MV(__half) }
+#undef QSVD_MV
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_combine(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                            const float* pm, const float* pl, const float* pz,

@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(kGemvThreads)
 k_gemv_partial(const XT* __restrict__ x, const WT* __restrict__ W, float* __restrict__ part,
                int B, int K, int N, int KS, float* __restrict__ out,
                int32_t* __restrict__ ticket, int32_t* status) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   (void)status;                          // no waits left to time out
   constexpr int BC = 16;                 // sequences per CTA
   constexpr int RT = gemv_rows<WT>();    // rows per CTA
@@ -238,11 +240,19 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 
 // grid (ceil(N/64), KS = ceil(K/512), ceil(B/16)), block 128.  Writes partials
 // part[ks][b][n]; with `ticket` non-null the last CTA of each (column block,
-// sequence block) adds the KS partials in split order into `out`.
-template <typename XT, typename WT>
+// sequence block) adds the KS partials in split order into `out` (converted
+// to OT).  Activation row of sequence b for output column n:
+// x + b * xg.row + (n / xg.cols) * xg.step (xg.cols a multiple of 64); the
+// plain GEMV has row = K, step = 0.
+struct XGroups {
+  long long row;    // elements between sequences
+  int cols;         // output columns sharing one activation row
+  long long step;   // elements between consecutive column groups' rows
+};
+template <typename XT, typename WT, typename OT = float>
 __global__ void __launch_bounds__(128)
-k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x,
-           float* __restrict__ part, int B, int K, int N, int KS, float* __restrict__ out,
+k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x, XGroups xg,
+           float* __restrict__ part, int B, int K, int N, int KS, OT* __restrict__ out,
            int32_t* __restrict__ ticket, int32_t* status) {
   using namespace gemv_mma;
   constexpr bool BF16 = std::is_same<WT, __nv_bfloat16>::value;
@@ -280,6 +290,10 @@ k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x,
           : "memory");
   }
 
+  // the weight tile is in flight; everything below reads what earlier kernels wrote
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
+
   // activation slice, row k of sequence j at xs[j][k]; thread tid covers
   // k = 4 tid .. 4 tid + 3 of every sequence with one vector load each, all
   // 16 issued before any is used (rows is a multiple of 32)
@@ -288,11 +302,11 @@ k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x,
   // so that nothing stands between them.
   using Raw = typename std::conditional<sizeof(XT) == 4, float4, uint2>::type;
   const bool kin = 4 * tid < rows;
-  const XT* xrow = x + size_t(b0) * K + row0 + (kin ? 4 * tid : 0);
+  const XT* xrow = x + size_t(b0) * xg.row + size_t(col0 / xg.cols) * xg.step + row0 + (kin ? 4 * tid : 0);
   Raw raw[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j)
-    raw[j] = __ldg(reinterpret_cast<const Raw*>(xrow + size_t(j < bn ? j : 0) * K));
+    raw[j] = __ldg(reinterpret_cast<const Raw*>(xrow + size_t(j < bn ? j : 0) * xg.row));
   float xv[16][4];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -427,17 +441,26 @@ k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x,
         sum[4] += v[u][1].x; sum[5] += v[u][1].y; sum[6] += v[u][1].z; sum[7] += v[u][1].w;
       }
     }
-    float* orow = out + size_t(b0 + ob) * N + col0 + oc;
-    reinterpret_cast<float4*>(orow)[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
-    reinterpret_cast<float4*>(orow)[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+    OT* orow = out + size_t(b0 + ob) * N + col0 + oc;
+    if constexpr (std::is_same<OT, float>::value) {
+      reinterpret_cast<float4*>(orow)[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+      reinterpret_cast<float4*>(orow)[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) orow[e] = dev::from_f<OT>(sum[e]);
+    }
   }
   if (tid == 0) *tk = 0;   // ready for the next call
 }
 
 // Launch the GEMV: tensor cores for 16-bit weights, CUDA cores for fp32.
-template <typename XT, typename WT>
+// Per-group activation rows (xg) and a non-float output need the tensor-core
+// variant (16-bit weights).
+template <typename XT, typename WT, typename OT = float>
 cudaError_t launch_gemv(const XT* x, const WT* W, float* part, int B, int K, int N, int KS,
-                        float* out, int32_t* ticket, int32_t* status, cudaStream_t s) {
+                        OT* out, int32_t* ticket, int32_t* status, cudaStream_t s,
+                        XGroups xg = XGroups{0, 0, 0}) {
+  if (xg.cols == 0) xg = XGroups{K, N, 0};
   cudaError_t e;
   if constexpr (sizeof(WT) == 2) {
     const dim3 grid((N + gemv_mma::CT - 1) / gemv_mma::CT, KS, (B + 15) / 16);
@@ -455,20 +478,30 @@ cudaError_t launch_gemv(const XT* x, const WT* W, float* part, int B, int K, int
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-    auto kern = k_gemv_mma<XT, WT>;
+    auto kern = k_gemv_mma<XT, WT, OT>;
     const int smem = gemv_mma::smem_bytes<NPART>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 128, smem, s>>>(tm, x, part, B, K, N, KS, out, ticket, status);
+    {
+      const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(128), smem, s,
+                                       tm, x, xg, part, B, K, N, KS, out, ticket, status);
+      if (le != cudaSuccess) return le;
+    }
   } else {
+    static_assert(std::is_same<OT, float>::value, "CUDA-core GEMV writes fp32");
+    if (xg.step != 0 || xg.row != K) return cudaErrorInvalidValue;
     const dim3 grid((N + 255) / 256, KS, (B + 15) / 16);
     auto kern = k_gemv_partial<XT, WT>;
     const size_t smem = gemv_smem<WT>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kGemvThreads, smem, s>>>(x, W, part, B, K, N, KS, out, ticket, status);
+    {
+      const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(kGemvThreads), smem, s,
+                                       x, W, part, B, K, N, KS, out, ticket, status);
+      if (le != cudaSuccess) return le;
+    }
   }
   note_launch();
   return check_launch();

@@ -5,6 +5,8 @@
 #pragma once
 
 #include <cuda.h>
+
+#include <cstring>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -79,8 +81,8 @@ struct WsHeader {
 };
 
 struct WsLayout {
-  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, scores, total;
-  int G, P, KS, JS, NT;
+  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, zm, scores, total;
+  int G, P, KS, JS, NT, NTQ;   // NT tickets in all, the first NTQ for the query GEMV
 };
 
 // Split-K factor of the query projection and j-splits of the combine.
@@ -88,6 +90,7 @@ int prologue_ksplit(const qsvd_dims& d);   // split of r in q = c_new W^u_q
 inline int combine_jsplit(const qsvd_dims& d) { return (d.r + 127) / 128; }
 
 int prologue_tickets(const qsvd_dims& d);  // ticket counters of that GEMV
+int gemv_tickets_vup(const qsvd_dims& d);  // ticket counters of the combine's V-up GEMV
 
 inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   WsLayout w{};
@@ -95,7 +98,8 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.P = G + d.batch;
   w.KS = prologue_ksplit(d);
   w.JS = combine_jsplit(d);
-  w.NT = prologue_tickets(d);
+  w.NTQ = prologue_tickets(d);
+  w.NT = w.NTQ + gemv_tickets_vup(d);   // then the V-up GEMV's (combine)
   const size_t B = d.batch, E = d.E, H = d.H, r = d.r;
   size_t o = 0;
   w.hdr = o;   o = align256(o + sizeof(WsHeader));
@@ -108,7 +112,8 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.pm = o;    o = align256(o + size_t(w.P) * H * 4);
   w.pl = o;    o = align256(o + size_t(w.P) * H * 4);
   w.pz = o;    o = align256(o + size_t(w.P) * H * r * 4);
-  w.opart = o; o = align256(o + size_t(w.JS) * B * E * 4);
+  w.opart = o; o = align256(o + size_t(w.JS) * B * E * 4);   // also the V-up GEMV's partials
+  w.zm = o;    o = align256(o + B * H * r * 4);                 // merged latents [B][H][r]
   w.scores = o; if (d.rope) o = align256(o + B * H * size_t(d.max_len) * 4);   // rotary: [B][H][max_len]
   w.total = o;
   return w;
@@ -119,6 +124,33 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
 void note_launch();                 // counts kernels launched by this library
 qsvd_status set_error(qsvd_status st, const char* msg);   // records qsvd_last_error()
 cudaError_t check_launch();         // cudaGetLastError after a launch
+
+// Programmatic dependent launch.  The decode-step kernels are launched with
+// programmatic stream serialisation, so each may start while the previous
+// kernel in the stream is still running.  Every such kernel executes
+// dev::pdl_wait() -- which returns once the previous grid has completed and
+// its memory is visible -- before it reads or writes any global memory that
+// an earlier kernel produces or consumes; before the wait it only reads the
+// packed weights (written by qsvd_prepare_weights) and sets up its own shared
+// memory.  It calls dev::pdl_trigger() after the wait, so a kernel starts
+// only once its predecessor's predecessor has completed, and a chain of such
+// kernels stays ordered transitively.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point
 // (no link against the driver library); null if the driver lacks it.
@@ -181,7 +213,14 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s);
 
-// Combine phase.
+// Combine phase.  16-bit weights with d_h % 64 == 0: a merge kernel writes
+// the merged latents zm, then the tensor-core GEMV applies W^u_v per head;
+// otherwise one kernel merges and applies W^u_v per (head, 128 rows of r).
+bool combine_uses_gemv(const qsvd_dims& d);
+cudaError_t launch_combine_gemv(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
+                                const float* pm, const float* pl, const float* pz, const void* wuv,
+                                float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
+                                cudaStream_t s);
 cudaError_t launch_combine(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                            const float* pm, const float* pl, const float* pz,
                            const void* wuv, float* opart, int JS, int P, void* out,
@@ -205,6 +244,12 @@ cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
 
 namespace qsvd {
 namespace dev {
+
+// See launch_pdl.  A no-op when the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }

@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(128)
 k_absorb(const float* __restrict__ q, const WT* __restrict__ W, float scale,
          float* __restrict__ qt32, QT16* __restrict__ qt16, int B, int H, int d_h, int r,
          int E) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   extern __shared__ float sm[];
   const int h = blockIdx.x;
   const int j0 = blockIdx.y * 128;
@@ -123,6 +125,8 @@ __global__ void __launch_bounds__(128)
 k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ q, float scale,
              float* __restrict__ qt32, QT16* __restrict__ qt16, int B, int H, int d_h, int r, int E,
              int32_t* status) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   using namespace gemv_mma;
   constexpr bool BF16 = std::is_same<WT, __nv_bfloat16>::value;
   constexpr bool SCALE = !BF16;           // fp16 range needs the power-of-two scale
@@ -277,6 +281,8 @@ __global__ void __launch_bounds__(256)
 k_rope_query(const float* __restrict__ q, const int32_t* __restrict__ sched,
              const float* __restrict__ tab, float scale, float* __restrict__ qrot, int B,
              int H, int d_h, int E) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   const int b = blockIdx.x;
   const int n = sched[B + 1 + b];
   const int pos = n > 0 ? n - 1 : 0;
@@ -302,6 +308,8 @@ __global__ void __launch_bounds__(1024)
 k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
            int32_t* __restrict__ sched, WsHeader* hdr, int kernel,
            int32_t* __restrict__ tickets, int n_tickets) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   for (int i = threadIdx.x; i < n_tickets; i += 1024) tickets[i] = 0;
   __shared__ int32_t part[1024];
   __shared__ int32_t carry;
@@ -368,8 +376,11 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float 
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       dim3 grid(d.H, (d.r + 127) / 128);
-      kern<<<grid, 128, smem, s>>>(tm, q, scale, qt32, static_cast<QT16*>(qt16), d.batch, d.H, d.d_h,
-                                   d.r, d.E, status);
+      {
+        const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(128), smem, s,
+                                         tm, q, scale, qt32, static_cast<QT16*>(qt16), d.batch, d.H, d.d_h, d.r, d.E, status);
+        if (le != cudaSuccess) return le;
+      }
       note_launch();
       return check_launch();
     }
@@ -379,8 +390,11 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(d.H, (d.r + 127) / 128);
-  kern<<<grid, 128, smem, s>>>(q, static_cast<const WT*>(wuk), scale, qt32,
-                               static_cast<QT16*>(qt16), d.batch, d.H, d.d_h, d.r, d.E);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(128), smem, s,
+                                     q, static_cast<const WT*>(wuk), scale, qt32, static_cast<QT16*>(qt16), d.batch, d.H, d.d_h, d.r, d.E);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
@@ -389,12 +403,16 @@ cudaError_t absorb_t(const qsvd_dims& d, const float* q, const void* wuk, float 
 
 int prologue_ksplit(const qsvd_dims& d) { return gemv_ksplit(d.r, d.weight_dtype); }
 int prologue_tickets(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch, d.weight_dtype); }
+int gemv_tickets_vup(const qsvd_dims& d) { return gemv_tickets(d.E, d.batch, d.weight_dtype); }
 
 cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, int32_t* sched,
                             WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,
                             cudaStream_t s) {
-  k_schedule<<<1, 1024, 0, s>>>(lengths, d.batch, d.max_len, G, sched, hdr, kernel, tickets,
-                                n_tickets);
+  {
+    const cudaError_t le = launch_pdl(k_schedule, dim3(1), dim3(1024), 0, s,
+                                     lengths, d.batch, d.max_len, G, sched, hdr, kernel, tickets, n_tickets);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
@@ -430,8 +448,11 @@ cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, f
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
                               const float* rope_tab, float scale, float* qrot,
                               cudaStream_t s) {
-  k_rope_query<<<d.batch, 256, 0, s>>>(q, sched, rope_tab, scale, qrot, d.batch, d.H, d.d_h,
-                                       d.E);
+  {
+    const cudaError_t le = launch_pdl(k_rope_query, dim3(d.batch), dim3(256), 0, s,
+                                     q, sched, rope_tab, scale, qrot, d.batch, d.H, d.d_h, d.E);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }

@@ -96,6 +96,8 @@ k_split_abs(const float* __restrict__ qt32, const uint8_t* __restrict__ cache,
             const __half* __restrict__ scales, const int32_t* __restrict__ sched,
             float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
             int B, int H, int r, int max_len, int group, int G, const float* __restrict__ sgiven = nullptr) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   constexpr int TS = 8;             // tokens per sub-tile
   constexpr int NV = TS * HB;       // scores per sub-tile
   extern __shared__ float sm[];
@@ -242,6 +244,8 @@ k_split_rope(const float* __restrict__ qrot, const WT* __restrict__ wuk,
              const __half* __restrict__ scales, const int32_t* __restrict__ sched,
              float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
              int B, int H, int d_h, int r, int E, int max_len, int group, int G) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   constexpr int TS = 16;
   constexpr int JC = 32;
   extern __shared__ float sm[];
@@ -394,9 +398,11 @@ cudaError_t abs_t(const qsvd_dims& d, const float* qt32, const void* cache, cons
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(G, d.H / HB);
-  kern<<<grid, kThreads, smem, s>>>(qt32, static_cast<const uint8_t*>(cache),
-                                    static_cast<const __half*>(scales), sched, pm, pl, pz,
-                                    d.batch, d.H, d.r, d.max_len, d.group, G, sgiven);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s,
+                                     qt32, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), sched, pm, pl, pz, d.batch, d.H, d.r, d.max_len, d.group, G, sgiven);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
@@ -434,10 +440,11 @@ cudaError_t rope_t(const qsvd_dims& d, const float* qrot, const void* wuk, const
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(G, d.H);
-  kern<<<grid, kThreads, smem, s>>>(qrot, static_cast<const WT*>(wuk), tab,
-                                    static_cast<const uint8_t*>(cache),
-                                    static_cast<const __half*>(scales), sched, pm, pl, pz,
-                                    d.batch, d.H, d.d_h, d.r, d.E, d.max_len, d.group, G);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s,
+                                     qrot, static_cast<const WT*>(wuk), tab, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), sched, pm, pl, pz, d.batch, d.H, d.d_h, d.r, d.E, d.max_len, d.group, G);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }

@@ -508,6 +508,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
            int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz,
            int nsg, int nraw, int ch) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   static_assert(!(SG && QB), "scores given: 16-bit latent only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -904,6 +906,8 @@ k_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ 
               const float* __restrict__ qrot, const float* __restrict__ rope_tab,
               const int32_t* __restrict__ sched, float* __restrict__ scores, int32_t* __restrict__ status,
               int B, int H, int E, int r, int max_len, int G, int ns) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -1211,9 +1215,11 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   auto kern = k_split_tc<NP, BF16, QS, PS, QB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<G * ch, kThreadsTc, smem, s>>>(tcs, tcz, tq, static_cast<const uint8_t*>(cache),
-                                        static_cast<const __half*>(scales), scores, sched, pm, pl, pz,
-                                        status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(kThreadsTc), smem, s,
+                                     tcs, tcz, tq, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }
@@ -1253,8 +1259,11 @@ cudaError_t rope_scores_t(const qsvd_dims& d, const void* cache, const void* wuk
   auto kern = k_rope_scores<BF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<G, 192, smem, s>>>(tc, tw, qrot, rope_tab, sched, scores, status, d.batch, d.H, d.E, d.r,
-                            d.max_len, G, ns);
+  {
+    const cudaError_t le = launch_pdl(kern, dim3(G), dim3(192), smem, s,
+                                     tc, tw, qrot, rope_tab, sched, scores, status, d.batch, d.H, d.E, d.r, d.max_len, G, ns);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return check_launch();
 }

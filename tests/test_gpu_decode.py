@@ -33,13 +33,15 @@ def case_for(key):
             w = synthetic.replace(synthetic.SHRUNK[1], weight="f32", cache="f32")
         elif key == "s1-bf16":
             w = synthetic.replace(synthetic.SHRUNK[1], weight="bf16", cache="bf16")
+        elif key == "s1-dh96":   # 16-bit weights, d_h not a multiple of 64: one-kernel combine
+            w = synthetic.replace(synthetic.SHRUNK[1], E=384, H=4, d_h=96)
         else:
             w = synthetic.SHRUNK[int(key[1])]
         _CASES[key] = oi.build_case(w)
     return _CASES[key]
 
 
-ALL = ["cfg0", "s1", "s1-bf16", "s1-f32w", "s2", "s3", "s3-i8", "s4"]
+ALL = ["cfg0", "s1", "s1-bf16", "s1-f32w", "s1-dh96", "s2", "s3", "s3-i8", "s4"]
 
 
 @pytest.mark.parametrize("key", ALL)
@@ -57,12 +59,16 @@ def test_decode_matches_oracle(cuda_ok, key):
 @pytest.mark.parametrize("key", ["s1", "s3", "s4"])
 @pytest.mark.parametrize("splits", [1, 2, 5, 1000])
 def test_split_count_invariance(cuda_ok, key, splits):
-    """Any split count gives the same attention (log-sum-exp merge)."""
+    """Any split count gives the same attention (log-sum-exp merge).  The
+    split kernel here is exact fp32; the combine's V-up takes the merged
+    latent into the tensor cores as two 16-bit parts (22 significant bits),
+    so split counts, which round the merged latent differently, agree to a
+    few units of 2^-22 per term summed over r."""
     case = case_for(key)
     g = GpuCase(case)
     base, _ = g.decode(num_splits=1)
     got, _ = g.decode(num_splits=splits)
-    assert rel_err(got, base) <= 1e-5
+    assert rel_err(got, base) <= 4e-5
     assert rel_err(got, case.reference()) <= (TOL_F32 if case.w.cache == "f32" else TOL)
 
 
