@@ -57,6 +57,8 @@ namespace qsvd {
 namespace {
 
 constexpr int kThreadsTc = 256;
+constexpr int kConvWarps = 3;      // quantised latent: converting warps per stream
+constexpr int kThreadsTcQ = 256 + 64 * (kConvWarps - 1);   // warps 8.. convert too
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
 constexpr int kMaxSlots = 8;                   // per ring
 constexpr int kMaxGroupBufs = 4;               // S accumulators per channel group (quantised latent)
@@ -99,9 +101,8 @@ struct Smem {
   uint64_t* drain;       // [2] one per MMA issuer
   uint64_t* sg_full;     // [kMaxGroupBufs] quantised latent: S of one channel group complete
   uint64_t* sg_empty;    // [kMaxGroupBufs] ... read by the softmax
-  uint8_t* sraw;         // quantised latent: raw-code rings (S, Z) and two tiles of Z scales
+  uint8_t* sraw;         // quantised latent: raw-code rings (S, Z)
   uint8_t* zraw;
-  uint8_t* zscale;
   uint64_t* sraw_full;   // [kMaxRaw]
   uint64_t* zraw_full;   // [kMaxRaw]
   float* red;            // [4][NP] per-warp partial max / sum
@@ -114,9 +115,8 @@ struct Smem {
 
 // P buffers: 2 (double buffer) x PS parts (bf16: hi + lo) x pbuf_bytes.
 // Quantised latent: raw codes of one item (S: 128 rows x 64 channels; Z: 64
-// rows x 128 channels) are QB x 1024 bytes; Z scales of one tile 128 x r/128.
+// rows x 128 channels) are QB x 1024 bytes.
 __host__ __device__ constexpr int raw_bytes(int qb) { return qb * 1024; }
-__host__ __device__ inline int zscale_bytes(int r) { return 256 * (r / 128); }
 
 template <int NP, int QS, int PS, bool SG>
 __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
@@ -126,8 +126,7 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   s.pbuf = s.zring + size_t(nz) * kZSlotBytes;
   s.sraw = s.pbuf + 2 * PS * pbuf_bytes<NP>();
   s.zraw = s.sraw + size_t(nraw) * raw_bytes(qb);
-  s.zscale = s.zraw + size_t(nraw) * raw_bytes(qb);
-  uint8_t* m = s.zscale + (qb ? 2 * zscale_bytes(r) : 0);
+  uint8_t* m = s.zraw + size_t(nraw) * raw_bytes(qb);
   uint64_t* bars = reinterpret_cast<uint64_t*>(m);
   s.s_full = bars;
   s.s_empty = bars + kMaxSlots;
@@ -277,7 +276,7 @@ __device__ __forceinline__ void convert_s_box(uint32_t d, uint32_t raw, int nv, 
 // [QB x 16 bytes]): channels 128 j .. 128 j + 127 of rows 64 h .. 64 h + 63,
 // dequantised (code x group scale, one fp16 rounding of the exact product),
 // two 64-channel boxes of 64 rows, 128-byte swizzled; rows >= nv are zeros.
-// tsc: the tile's scales [128][ngroups] (shared or global memory).
+// tsc: the tile's scales [128][ngroups] in global memory.
 template <int QB>
 __device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const __half* tsc,
                                                int ngroups, int j, int h, int nv, int lane) {
@@ -302,23 +301,23 @@ __device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const _
   __syncwarp();
 }
 
-// Bulk (untiled) copy global -> shared, completion on an mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-
-// Producer of one ring for a quantised latent (warp-wide).  The raw codes of
-// each item arrive by TMA into a ring of nraw slots, issued nraw items ahead
-// (nraw <= items per tile); the warp converts them into the fp16 slot the
+// Producer of one ring for a quantised latent: nsub warps share a stream,
+// warp wsub taking the items k == wsub (mod nsub) of the stream's sequence.
+// The raw codes of each item arrive by TMA into a ring of nraw slots (nraw a
+// multiple of nsub, so a slot is always refilled by the warp that drained
+// it), issued nraw items ahead; the warp converts them into the fp16 slot the
 // MMAs read (S: exact integers, plus the query box by TMA; Z: dequantised,
-// with the tile's scales, which ride with the tile's first Z item when their
-// block is 16-byte aligned and the tile is full).
+// the token's group scale read from global memory).  Conversion is
+// latency-bound per warp (dependent integer/half2 chains, the proxy fence
+// before each hand-off), so the stream's throughput grows with nsub.
+// *last_item / *last_raw: the last item this warp produced / issued (-1 if
+// none), for the drain after an abort.  Returns false on a wait that expired
+// or an abort.
 template <int NP, int QS, int QB>
-__device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, const CUtensorMap* tm_q,
-                          const __half* scales, const int32_t* sched, int B, int r, int max_len,
-                          long long tb, long long te, int n, int nslots, int nraw, int lane,
-                          long long* issued, long long* raw_issued) {
+__device__ bool produce_q(int kind, int wsub, int nsub, const Smem& s, const CUtensorMap* tm_raw,
+                          const CUtensorMap* tm_q, const __half* scales, const int32_t* sched, int B,
+                          int r, int max_len, long long tb, long long te, int n, int nslots, int nraw,
+                          int lane, long long* last_item, long long* last_raw) {
   const int NI = r / 64, NG = r / 128;
   uint8_t* ring = kind == 0 ? s.sring : s.zring;
   const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
@@ -326,27 +325,27 @@ __device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, co
   uint64_t* empty = kind == 0 ? s.s_empty : s.z_empty;
   uint8_t* raw = kind == 0 ? s.sraw : s.zraw;
   uint64_t* rfull = kind == 0 ? s.sraw_full : s.zraw_full;
-  const uint32_t ring0 = saddr(ring), raw0 = saddr(raw), zsc0 = saddr(s.zscale);
+  const uint32_t ring0 = saddr(ring), raw0 = saddr(raw);
   constexpr uint32_t RB = uint32_t(raw_bytes(QB));
-  const uint32_t ZSB = uint32_t(zscale_bytes(r));
   const long long total = (long long)n * NI;
-  // issue side: nraw items ahead of the conversion
+  *last_item = -1;
+  *last_raw = -1;
+  // issue side: walks every item of the stream, issues this warp's
   TileIter ia;
   ia.init(sched, B, tb, te);
   int ia_i = 0, ua = 0;
   long long ki = 0;
-  auto issue_one = [&]() {
-    const int slot = int(ki % nraw);
-    const uint32_t fb = saddr(&rfull[slot]);
-    const int row = ia.b * max_len + ia.t0();
-    const size_t sc_off = size_t(row) * NG * 2;
-    const bool sc_bulk = kind == 1 && ua == 0 && ia.nvalid() == kTile && sc_off % 16 == 0;
-    if (lane == int(ki & 31)) {   // rotating issuing lane
-      mbar_expect_tx(fb, RB + (sc_bulk ? ZSB : 0u));
-      if (kind == 0) tma_load_2d(raw0 + slot * RB, tm_raw, ua * (QB * 8), row, fb);
-      else tma_load_2d(raw0 + slot * RB, tm_raw, (ua >> 1) * (QB * 16), row + 64 * (ua & 1), fb);
-      if (sc_bulk)
-        bulk_load(zsc0 + (ia_i & 1) * ZSB, reinterpret_cast<const uint8_t*>(scales) + sc_off, ZSB, fb);
+  auto issue_next = [&]() {
+    if (ki % nsub == wsub) {
+      const int slot = int(ki % nraw);
+      const uint32_t fb = saddr(&rfull[slot]);
+      const int row = ia.b * max_len + ia.t0();
+      if (lane == int((ki / nsub) & 31)) {   // rotating issuing lane
+        mbar_expect_tx(fb, RB);
+        if (kind == 0) tma_load_2d(raw0 + slot * RB, tm_raw, ua * (QB * 8), row, fb);
+        else tma_load_2d(raw0 + slot * RB, tm_raw, (ua >> 1) * (QB * 16), row + 64 * (ua & 1), fb);
+      }
+      *last_raw = ki;
     }
     ++ki;
     if (++ua == NI) {
@@ -354,28 +353,21 @@ __device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, co
       if (++ia_i < n) ia.next();
     }
   };
-  for (long long x = 0; x < total && x < nraw; ++x) issue_one();
+  for (long long x = 0; x < total && x < nraw; ++x) issue_next();
   TileIter it;
   it.init(sched, B, tb, te);
-  Ring rg(nslots);
-  long long k = 0;
+  long long k = 0;   // item index of the stream
   for (int i = 0; i < n; ++i) {
     const int nv = it.nvalid(), b = it.b;
-    const int row = b * max_len + it.t0();
-    const size_t sc_off = size_t(row) * NG * 2;
-    const bool sc_smem = kind == 1 && nv == kTile && sc_off % 16 == 0;
-    const __half* tsc = sc_smem ? reinterpret_cast<const __half*>(s.zscale + (i & 1) * ZSB)
-                                : scales + size_t(row) * NG;
-    for (int u = 0; u < NI; ++u) {
-      const int rs = int(k % nraw);
+    const __half* tsc = scales + (size_t(b) * max_len + it.t0()) * NG;   // the tile's scales [128][NG]
+    for (int u = 0; u < NI; ++u, ++k) {
+      if (k % nsub != wsub) continue;
+      const int rs = int(k % nraw), slot = int(k % nslots);
       if (!__all_sync(0xffffffffu, mbar_wait(saddr(&rfull[rs]), uint32_t(k / nraw) & 1u)) ||
-          !__all_sync(0xffffffffu, mbar_wait(saddr(&empty[rg.slot]), rg.phase ^ 1u))) {   // warp-uniform
-        *issued = k;
-        *raw_issued = ki;
-        return false;
-      }
-      const uint32_t dst = ring0 + uint32_t(rg.slot) * slot_bytes;
-      const uint32_t fb = saddr(&full[rg.slot]);
+          !__all_sync(0xffffffffu, mbar_wait(saddr(&empty[slot]), (uint32_t(k / nslots) & 1u) ^ 1u)))
+        return false;   // warp-uniform
+      const uint32_t dst = ring0 + uint32_t(slot) * slot_bytes;
+      const uint32_t fb = saddr(&full[slot]);
       if (kind == 0) {
         if (lane == 0) {   // the query box; the slot completes on this and the codes' arrival
           mbar_expect_tx(fb, uint32_t(QS * NP * 128));
@@ -386,22 +378,31 @@ __device__ bool produce_q(int kind, const Smem& s, const CUtensorMap* tm_raw, co
         convert_z_item<QB>(dst, raw0 + uint32_t(rs) * RB, tsc, NG, u >> 1, u & 1, nv, lane);
       }
       if (lane == 0) mbar_arrive(fb);
-      // the raw slot has been read: refill it nraw items ahead
-      if (ki < total) issue_one();
+      *last_item = k;
+      // the raw slot has been read: the item nraw ahead (also this warp's) refills it
+      for (int x = 0; x < nsub && ki < total; ++x) issue_next();
       __syncwarp();
-      rg.advance();
-      ++k;
     }
     it.next();
-    if (__any_sync(0xffffffffu, *s.abort_flag)) {
-      *issued = k;
-      *raw_issued = ki;
-      return false;
-    }
+    if (__any_sync(0xffffffffu, *s.abort_flag)) return false;
   }
-  *issued = k;
-  *raw_issued = ki;
   return true;
+}
+
+// After an abort: wait (bounded) for the copies this warp may have in flight
+// -- the last raw load into each of its raw slots, the query boxes of its
+// last S items -- so that none lands after the CTA has left.
+__device__ void drain_q(int kind, int wsub, int nsub, const Smem& s, int nslots, int nraw,
+                        long long last_item, long long last_raw) {
+  uint64_t* rfull = kind == 0 ? s.sraw_full : s.zraw_full;
+  for (int slot = wsub; slot < nraw; slot += nsub) {
+    if (last_raw < slot) continue;
+    const long long kk = slot + (last_raw - slot) / nraw * nraw;   // last item issued into the slot
+    mbar_wait(saddr(&rfull[slot]), uint32_t(kk / nraw) & 1u);
+  }
+  if (kind == 0)
+    for (long long kk = last_item; kk >= 0 && kk > last_item - nslots; kk -= nsub)
+      mbar_wait(saddr(&s.s_full[int(kk % nslots)]), uint32_t(kk / nslots) & 1u);
 }
 
 // Producer of one ring (warp-wide).  kind 0: S ring (latent box from HBM,
@@ -500,7 +501,7 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 // blockIdx.x / ch), each owning every ch-th chunk; all of them run the same
 // softmax on the same scores and part 0 writes m and l.
 template <int NP, bool BF16, int QS, int PS, int QB, bool SG>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(QB ? kThreadsTcQ : kThreadsTc, 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
            const __grid_constant__ CUtensorMap tm_q,
            const uint8_t* __restrict__ cache, const __half* __restrict__ scales,
@@ -566,22 +567,25 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = *s.tmem_holder;
 
-  if (warp == 0 || warp == 2) {
+  if (warp == 0 || warp == 2 || (QB && warp >= 8)) {
     // ----------------------------------------------------------- producers
-    const int kind = warp >> 1;
+    // quantised latent: S converters warps 0, 8, 10, ..., Z converters 2, 9, 11, ...
+    const int kind = (warp == 0 || (warp >= 8 && (warp & 1) == 0)) ? 0 : 1;
+    const int wsub = warp >= 8 ? (warp - 8) / 2 + 1 : 0;
     const int nslots = kind == 0 ? ns : nz;
     long long issued = 0, raw_issued = 0;
     bool ok;
-    if constexpr (QB != 0)   // quantised latent: tm_cs / tm_cz map the raw codes
-      ok = produce_q<NP, QS, QB>(kind, s, kind == 0 ? &tm_cs : &tm_cz, &tm_q, scales, sched, B, r,
-                                 max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
-    else
+    if constexpr (QB != 0) {   // tm_cs / tm_cz map the raw codes
+      ok = produce_q<NP, QS, QB>(kind, wsub, kConvWarps, s, kind == 0 ? &tm_cs : &tm_cz, &tm_q, scales,
+                                 sched, B, r, max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
+    } else {
       ok = produce<NP, QS, SG>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te,
                                n, nslots, lane, &issued, ch, cpart);
+    }
     if (!ok && lane == 0) {
       set_abort(s, status);
-      drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
-      if (QB) drain_ring(kind == 0 ? s.sraw_full : s.zraw_full, raw_issued, nraw);
+      if constexpr (QB != 0) drain_q(kind, wsub, kConvWarps, s, nslots, nraw, issued, raw_issued);
+      else drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
     }
     __syncwarp();
   } else if (warp == 1 && !SG) {
@@ -1189,14 +1193,15 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   if constexpr (QB != 0) {
     // quantised latent: the fp16 slots are filled by conversion (short
     // latency), so three of each; the raw-code rings take the rest, at most
-    // one tile of items ahead (the Z scales are double-buffered per tile)
+    // one tile of items ahead
     ns = nz = 3;
-    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>() - 2 * zscale_bytes(d.r) -
+    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>() -
                       ns * s_slot_bytes<NP, QS>() - nz * kZSlotBytes;
     nraw = avail / (2 * raw_bytes(QB));
     if (nraw > kMaxRaw) nraw = kMaxRaw;
     if (nraw > d.r / 64) nraw = d.r / 64;
-    if (nraw < 2) return cudaErrorInvalidConfiguration;
+    nraw -= nraw % kConvWarps;   // a raw slot is always refilled by the warp that drained it
+    if (nraw < kConvWarps) return cudaErrorInvalidConfiguration;
   }
   if constexpr (SG) {
     // no S items: both rings carry Z items and share the budget
@@ -1211,12 +1216,12 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   if (QB && nsg < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + size_t(ns) * a_slot_bytes<NP, QS, SG>() + size_t(nz) * kZSlotBytes +
                       2 * PS * pbuf_bytes<NP>() +
-                      (QB ? 2 * size_t(nraw) * raw_bytes(QB) + 2 * zscale_bytes(d.r) : 0) + kMiscBytes;
+                      (QB ? 2 * size_t(nraw) * raw_bytes(QB) : 0) + kMiscBytes;
   auto kern = k_split_tc<NP, BF16, QS, PS, QB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   {
-    const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(kThreadsTc), smem, s,
+    const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(QB ? kThreadsTcQ : kThreadsTc), smem, s,
                                      tcs, tcz, tq, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch);
     if (le != cudaSuccess) return le;
   }
