@@ -259,12 +259,20 @@ __device__ __forceinline__ void convert_s_box(uint32_t d, uint32_t raw, int nv, 
   constexpr int VPR = RPB / 16;           // 16-byte vectors per row
   constexpr int CPV = QB == 4 ? 4 : 2;    // 16-byte fp16 chunks per vector
   constexpr int NV = 128 * VPR / 32;      // vectors per lane: 8 (int4), 16 (int8)
+  // every raw vector's load is issued before the first store (the shared
+  // accesses are ordered asm statements: interleaved, each load would wait
+  // behind the previous vector's stores)
+  uint4 rv[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int v = lane + 32 * i, t = v / VPR, q = v % VPR;
-    const uint4 rv = t < nv ? lds128(raw + t * RPB + q * 16) : make_uint4(0, 0, 0, 0);
+    rv[i] = t < nv ? lds128(raw + t * RPB + q * 16) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int v = lane + 32 * i, t = v / VPR, q = v % VPR;
     uint4 out[CPV];
-    codes_to_half<QB>(rv, false, __half2(), out);   // zero codes give zeros
+    codes_to_half<QB>(rv[i], false, __half2(), out);   // zero codes give zeros
 #pragma unroll
     for (int c = 0; c < CPV; ++c) sts128(d + t * 128 + (((q * CPV + c) ^ (t & 7)) << 4), out[c]);
   }
@@ -284,14 +292,21 @@ __device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const _
   constexpr int VPR = RPB / 16;
   constexpr int CPV = QB == 4 ? 4 : 2;
   constexpr int NV = 64 * VPR / 32;       // vectors per lane: 8 (int4), 16 (int8)
+  // all raw vectors and scales requested before the first store (see convert_s_box)
+  uint4 rv[NV];
+  __half sc[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int v = lane + 32 * i, tt = v / VPR, q = v % VPR, t = 64 * h + tt;
     const bool in = t < nv;
-    const uint4 rv = in ? lds128(raw + tt * RPB + q * 16) : make_uint4(0, 0, 0, 0);
-    const __half sc = in ? tsc[t * ngroups + j] : __float2half(0.f);
+    rv[i] = in ? lds128(raw + tt * RPB + q * 16) : make_uint4(0, 0, 0, 0);
+    sc[i] = in ? tsc[t * ngroups + j] : __float2half(0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR;
     uint4 out[CPV];
-    codes_to_half<QB>(rv, true, __halves2half2(sc, sc), out);
+    codes_to_half<QB>(rv[i], true, __halves2half2(sc[i], sc[i]), out);
     const int ch = q * (CPV * 8);         // first channel of the vector within the 128
     const int box = ch >> 6, c0 = (ch & 63) >> 3;
 #pragma unroll
@@ -1192,16 +1207,21 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   ring_slots<NP, QS, PS>(&ns, &nz);
   if constexpr (QB != 0) {
     // quantised latent: the fp16 slots are filled by conversion (short
-    // latency), so three of each; the raw-code rings take the rest, at most
-    // one tile of items ahead
-    ns = nz = 3;
-    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>() -
-                      ns * s_slot_bytes<NP, QS>() - nz * kZSlotBytes;
-    nraw = avail / (2 * raw_bytes(QB));
-    if (nraw > kMaxRaw) nraw = kMaxRaw;
-    if (nraw > d.r / 64) nraw = d.r / 64;
-    nraw -= nraw % kConvWarps;   // a raw slot is always refilled by the warp that drained it
-    if (nraw < kConvWarps) return cudaErrorInvalidConfiguration;
+    // latency); each converting warp holds one while it converts, so the
+    // rings need more slots than converters to keep conversion off the MMAs'
+    // path.  The raw-code rings (a multiple of kConvWarps slots each) take
+    // what is left; of 6 or 3 raw slots, the choice with more fp16 slots.
+    const int base = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
+    const int pair = s_slot_bytes<NP, QS>() + kZSlotBytes;
+    int best = 0;
+    for (int cand = 2 * kConvWarps; cand >= kConvWarps; cand -= kConvWarps) {
+      if (cand > kMaxRaw || cand > d.r / 64) continue;
+      int slots = (base - 2 * cand * raw_bytes(QB)) / pair;
+      if (slots > kMaxSlots) slots = kMaxSlots;
+      if (slots > best) { best = slots; nraw = cand; }
+    }
+    ns = nz = best;
+    if (nraw < kConvWarps || best < 2) return cudaErrorInvalidConfiguration;
   }
   if constexpr (SG) {
     // no S items: both rings carry Z items and share the budget
