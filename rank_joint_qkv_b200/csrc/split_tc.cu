@@ -584,9 +584,11 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 
   if (warp == 0 || warp == 2 || (QB && warp >= 8)) {
     // ----------------------------------------------------------- producers
-    // quantised latent: S converters warps 0, 8, 10, ..., Z converters 2, 9, 11, ...
-    const int kind = (warp == 0 || (warp >= 8 && (warp & 1) == 0)) ? 0 : 1;
-    const int wsub = warp >= 8 ? (warp - 8) / 2 + 1 : 0;
+    // quantised latent: S converters warps 0, 9, 10 and Z converters 2, 8, 11
+    // (warp w issues on scheduler w % 4: each stream on three schedulers)
+    static_assert(kConvWarps == 3, "converter warp map");
+    const int kind = (warp == 0 || warp == 9 || warp == 10) ? 0 : 1;
+    const int wsub = warp < 8 ? 0 : (warp == 8 || warp == 9 ? 1 : 2);
     const int nslots = kind == 0 ? ns : nz;
     long long issued = 0, raw_issued = 0;
     bool ok;
