@@ -449,11 +449,12 @@ def oracle_sample(w, n_tokens: int, b: int):
 
 
 def time_oracle(w, n_tokens, budget_s, max_seqs=None):
+    """The oracle on sequences of n_tokens: until budget_s seconds are spent,
+    or exactly max_seqs sequences when that is given."""
     from oracle import qsvd_ref as ref
     rb = w.rope_base if w.rope else None
     done_tokens, spent, seqs = 0, 0.0, 0
-    wts = None
-    while spent < budget_s and (max_seqs is None or seqs < max_seqs):
+    while (seqs < max_seqs) if max_seqs is not None else (spent < budget_s):
         c, cnew, wuq, wuk, wuv = oracle_sample(w, n_tokens, seqs % w.B)
         t = time.perf_counter()
         ref.decode_materialized([c], [n_tokens], cnew, wuq, wuk, wuv, w.H, rope_base=rb)
@@ -486,6 +487,11 @@ def run_reference(args, rank, world):
     n = int(min(int(np.max(lens)), 8192))
     for _ in range(args.warmup):
         time_oracle(w, min(n, 512), 0.0, max_seqs=1)
+    # one sequence per step; its length bounded so that the K steps take
+    # about two minutes at most (the oracle's cost grows with the tokens)
+    t1, s1, _ = time_oracle(w, min(n, 1024), 0.0, max_seqs=1)
+    per_token = s1 / t1
+    n = int(max(128, min(n, 120.0 / (max(1, args.steps) * per_token))))
     tokens, spent, seqs = 0, 0.0, 0
     for _ in range(args.steps):
         t, s, k = time_oracle(w, n, 0.0, max_seqs=1)
