@@ -193,12 +193,14 @@ class ClockSampler:
 
 
 def measured_peaks():
+    """HBM copy GB/s, bf16 TFLOP/s burst and sustained, and whose numbers."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def kernel_source_hash(files) -> str:
@@ -379,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return None
-    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    hbm_peak, tc_burst, tc_sustained, peak_kind = measured_peaks()
     dom_mean = statistics.mean(dom_ms)
     lat_b = latent_bytes(w, lens)
     kname = ("k_rope_scores" if rope_tc
@@ -395,9 +397,12 @@ def run_ours(args, rank, world, local_rank):
         # keys rebuilt per head: K_h = C W^u_{k,h}, 2 r E flop per valid token
         flops = 2.0 * w.r * w.E * float(np.sum(lens))
         achieved = flops / (dom_mean / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak, "traffic": traffic, "kernel": kname,
-                "peak_kind": peak_kind + " bf16 burst (fp16 has the same dense rate)",
+        # the scores kernel runs back to back inside long runs of steps (the
+        # power cap sets its clock): the sustained GEMM peak is its ceiling
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_sustained, "unit": "TFLOP/s",
+                "frac": achieved / tc_sustained, "traffic": traffic, "kernel": kname,
+                "peak_kind": peak_kind + " bf16 sustained (fp16 has the same dense rate)",
+                "frac_of_burst_peak": achieved / tc_burst,
                 "flops_per_launch": flops, "launch_ms": dom_mean}
     else:
         achieved = lat_b / (dom_mean / 1e3) / 1e9

@@ -125,8 +125,6 @@ __global__ void __launch_bounds__(128)
 k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ q, float scale,
              float* __restrict__ qt32, QT16* __restrict__ qt16, int B, int H, int d_h, int r, int E,
              int32_t* status) {
-  dev::pdl_wait();   // see launch_pdl
-  dev::pdl_trigger();
   using namespace gemv_mma;
   constexpr bool BF16 = std::is_same<WT, __nv_bfloat16>::value;
   constexpr bool SCALE = !BF16;           // fp16 range needs the power-of-two scale
@@ -155,6 +153,9 @@ k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__
           "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"(h * d_h + 64 * c), "r"(j0), "r"(bar_s)
           : "memory");
   }
+  // the weight tile is in flight; what follows reads what earlier kernels wrote
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
   const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);   // ldmatrix: this lane's row of its 8x8 matrix
   const int mcol = 8 * (lane >> 4);
   const uint32_t xs_s = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
