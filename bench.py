@@ -204,10 +204,17 @@ def measured_peaks():
 
 
 def kernel_source_hash(files) -> str:
+    """Hash of the code in the kernel's source files, comments and whitespace
+    left out: a committed DRAM-traffic figure stays valid across comment
+    edits and goes stale with any change of code."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "rank_joint_qkv_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "rank_joint_qkv_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

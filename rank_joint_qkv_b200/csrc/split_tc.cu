@@ -1,4 +1,8 @@
-// Split phase on the 5th-generation tensor cores: absorbed query, 16-bit latent.
+// Split phase on the 5th-generation tensor cores, one CTA per split (a
+// persistent CTA walks its split's run of tiles): absorbed query with a
+// 16-bit or int4/int8 latent, and the rotary mode's two passes (the scores
+// kernel k_rope_scores at the end of this file, then this kernel with the
+// scores given).
 //
 // Per 128-token latent tile of one sequence (QSVD digest, Method, Step 1: keys
 // and values are never rebuilt when no rotary embedding is applied; WSVD
@@ -35,6 +39,10 @@
 //   warps 4-7  softmax over the S accumulator (one TMEM lane = one token),
 //              conditional rescale of Z, P written to shared memory, and the
 //              per-segment epilogue (partials m, l, z to global memory)
+// Quantised latent (384 threads): raw codes arrive by TMA and three warps
+// per stream convert them (S: warps 0, 9, 10; Z: warps 2, 8, 11); S is
+// accumulated per 128-channel group and scaled per token by the softmax.
+// Scores given (rotary mode): no S pass; warps 1 and 3 both issue Z MMAs.
 //
 // Precision: the absorbed query enters the MMA as hi + lo 16-bit parts and,
 // for bf16 latents, P does too (two accumulating MMAs); accumulation is fp32.
