@@ -45,6 +45,12 @@ def case(key):
             "i8": synthetic.replace(synthetic.SHRUNK[3], cache="i8", name="shrunk-int8-h2"),
             "i4h32": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=768, B=2, L=600,
                                        h2_n=256),
+            # r 256: four items per tile, three raw slots per stream (one per converter)
+            "i4r256": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0),
+            "i8r256": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0, cache="i8",
+                                        name="shrunk-int8-r256"),
+            "i4r256rag": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0, B=4, L=700,
+                                           ragged=(1, 700)),
             # cluster shapes: 6 CTAs of 256 channels (the LLaVA-7B rank), 8 of 256
             "c6": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=300),
             "c6bf": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=290, cache="bf16",
@@ -68,7 +74,7 @@ _KEYS16 = ["full", "f16", "bf16", "h32", "r768", "c6", "c6bf", "c8"]
 
 
 @pytest.mark.parametrize("key,kern", [(k, v) for k in _KEYS16 for v in BOTH] +
-                         [(k, CTA) for k in ("i4", "i8", "i4h32")])
+                         [(k, CTA) for k in ("i4", "i8", "i4h32", "i4r256", "i8r256", "i4r256rag")])
 def test_tc_matches_oracle(cuda_ok, key, kern):
     c = case(key)
     g = GpuCase(c, kernel=kern)
@@ -111,6 +117,17 @@ def test_tc_split_invariance(cuda_ok, splits, kern):
     # each split rounds P = 2^(s - m_split) to fp16 against its own reference
     # max, so split counts differ at the level of fp16 rounding (2^-11)
     assert rel_err(got, base) <= 1e-3
+    assert rel_err(got, c.reference()) <= TOL
+
+
+@pytest.mark.parametrize("key", ["i4", "i8r256"])
+@pytest.mark.parametrize("splits", [1, 3, 1000])
+def test_tc_int_split_invariance(cuda_ok, key, splits):
+    """Quantised latents at any split count (each converting warp's share of
+    items changes with the split boundaries)."""
+    c = case(key)
+    got, ws = GpuCase(c, kernel=CTA).decode(num_splits=splits)
+    assert q.status_word(ws) == 0
     assert rel_err(got, c.reference()) <= TOL
 
 
