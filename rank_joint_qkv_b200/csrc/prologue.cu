@@ -303,7 +303,7 @@ k_rope_query(const float* __restrict__ q, const int32_t* __restrict__ sched,
 // ---------------------------------------------------------------------------
 // Split-KV schedule: clamped lengths and the tile prefix over sequences.
 // sched[0..B] = tiles before sequence b (sched[B] = total), sched[B+1+b] = len.
-// grid 1, block 1024.  Also records G in the workspace header.
+// grid 1, block 32 .. 1024 (a multiple of 32).  Also records G in the workspace header.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
@@ -311,9 +311,10 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
            int32_t* __restrict__ tickets, int n_tickets) {
   dev::pdl_wait();   // see launch_pdl
   dev::pdl_trigger();
-  for (int i = threadIdx.x; i < n_tickets; i += 1024) tickets[i] = 0;
-  __shared__ int32_t part[1024];
+  for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0;
+  __shared__ int32_t wsum[32];
   __shared__ int32_t carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   if (threadIdx.x == 0) {
     carry = 0;
     hdr->status = 0;   // reset before any thread flags a clamped length
@@ -322,7 +323,7 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
     hdr->kernel = kernel;
   }
   __syncthreads();
-  for (int b0 = 0; b0 < B; b0 += 1024) {
+  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
     const int b = b0 + threadIdx.x;
     int nt = 0;
     if (b < B) {
@@ -330,18 +331,29 @@ k_schedule(const int32_t* __restrict__ lengths, int B, int max_len, int G,
       sched[B + 1 + b] = n;
       nt = dev::tiles_of(n);
     }
-    part[threadIdx.x] = nt;
-    __syncthreads();
-    // inclusive Hillis-Steele scan
-    for (int o = 1; o < 1024; o <<= 1) {
-      const int v = threadIdx.x >= o ? part[threadIdx.x - o] : 0;
-      __syncthreads();
-      part[threadIdx.x] += v;
-      __syncthreads();
+    // inclusive scan: within each warp by shuffles, then over the warp totals
+    int v = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
     }
-    if (b < B) sched[b + 1] = carry + part[threadIdx.x];
+    if (lane == 31) wsum[warp] = v;
     __syncthreads();
-    if (threadIdx.x == 1023) carry += part[1023];
+    if (warp == 0) {
+      int t = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += u;
+      }
+      if (lane < nw) wsum[lane] = t;
+    }
+    __syncthreads();
+    const int incl = v + (warp > 0 ? wsum[warp - 1] : 0);
+    if (b < B) sched[b + 1] = carry + incl;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry += incl;
     __syncthreads();
   }
   if (threadIdx.x == 0) sched[0] = 0;
@@ -410,7 +422,8 @@ cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, i
                             WsHeader* hdr, int kernel, int32_t* tickets, int n_tickets,
                             cudaStream_t s) {
   {
-    const cudaError_t le = launch_pdl(k_schedule, dim3(1), dim3(1024), 0, s,
+    const int threads = d.batch <= 1024 ? (d.batch + 31) / 32 * 32 : 1024;   // a warp for small batches
+    const cudaError_t le = launch_pdl(k_schedule, dim3(1), dim3(threads), 0, s,
                                      lengths, d.batch, d.max_len, G, sched, hdr, kernel, tickets, n_tickets);
     if (le != cudaSuccess) return le;
   }
