@@ -288,7 +288,9 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (d.rope)
       e = launch_rope_query(d, qsrc, sched, rope_tab, sl2, qt32, s);
     else
-      e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, qt16, &hdr->status, s);
+      // only the copy the split kernel reads: fp32 for CUDA cores, 16-bit hi/lo for tensor cores
+      e = launch_absorb(d, qsrc, P + L.wuk, sl2, kernel == QSVD_KERNEL_SIMT ? qt32 : nullptr,
+                        kernel == QSVD_KERNEL_SIMT ? nullptr : qt16, &hdr->status, s);
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (split_any) {

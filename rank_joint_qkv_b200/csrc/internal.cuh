@@ -169,6 +169,8 @@ cudaError_t launch_schedule(const qsvd_dims& d, const int32_t* lengths, int G, i
 cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* wuq,
                              float* qpart, int KS, float* q, int32_t* tickets, int32_t* status,
                              cudaStream_t s);
+// qt32 (fp32, for the CUDA-core split) and qt16 ([B][2][H][r] hi/lo, for the
+// tensor cores) are each written only when non-null.
 cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale_log2,
                           float* qt32, void* qt16, int32_t* status, cudaStream_t s);
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,

@@ -97,14 +97,16 @@ k_absorb(const float* __restrict__ q, const WT* __restrict__ W, float scale,
         if (j - j0 < jn && b < B) {
           const float v = acc[a][c] * scale;
           const size_t o = (size_t(b) * H + h) * r + j;
-          qt32[o] = v;
-          // 16-bit copy for the tensor cores, [B][2][H][r]: the rounded value
-          // and its rounding residual (hi + lo carries ~2x the mantissa bits;
-          // one 16-bit part alone perturbs peaked softmaxes by ~1e-2)
-          const QT16 hi = dev::from_f<QT16>(v);
-          const size_t o2 = ((size_t(b) * 2) * H + h) * r + j;
-          qt16[o2] = hi;
-          qt16[o2 + size_t(H) * r] = dev::from_f<QT16>(v - dev::to_f(hi));
+          if (qt32) qt32[o] = v;
+          if (qt16) {
+            // 16-bit copy for the tensor cores, [B][2][H][r]: the rounded value
+            // and its rounding residual (hi + lo carries ~2x the mantissa bits;
+            // one 16-bit part alone perturbs peaked softmaxes by ~1e-2)
+            const QT16 hi = dev::from_f<QT16>(v);
+            const size_t o2 = ((size_t(b) * 2) * H + h) * r + j;
+            qt16[o2] = hi;
+            qt16[o2 + size_t(H) * r] = dev::from_f<QT16>(v - dev::to_f(hi));
+          }
         }
       }
   }
@@ -259,7 +261,8 @@ k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__
         const float sc = scale * inv_scale[bb];
         const float v0 = acc[t][2 * half] * sc, v1 = acc[t][2 * half + 1] * sc;
         const size_t o = (size_t(b) * H + h) * r + j0 + jl;
-        *reinterpret_cast<float2*>(qt32 + o) = make_float2(v0, v1);
+        if (qt32) *reinterpret_cast<float2*>(qt32 + o) = make_float2(v0, v1);
+        if (!qt16) continue;
         // 16-bit copy for the tensor cores, [B][2][H][r]: the rounded value
         // and its rounding residual
         const QT16 h0 = dev::from_f<QT16>(v0), h1 = dev::from_f<QT16>(v1);
