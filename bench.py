@@ -491,6 +491,56 @@ def cpu_baseline(w, lens, budget_s=15.0):
                       f"(keys/values materialised), {spent:.1f} s"}
 
 
+def run_prefill(args):
+    """qsvd_prefill_latent on the workload's whole cache (every token of every
+    sequence, B x L rows): one GEMM x W^d with the cache's rounding or
+    quantisation fused, timed with CUDA events over K launches."""
+    import rank_joint_qkv_b200 as q
+    device = "cuda:0"
+    torch.cuda.set_device(device)
+    w = synthetic.CONFIGS[args.config]
+    max_len = w.L
+    n = w.B * max_len
+    dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
+                       group=w.group)
+    wt = torch.bfloat16 if w.weight == "bf16" else torch.float16
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    wd = (torch.randn(w.E, w.r, device=device, generator=g) / math.sqrt(w.E)).to(wt)
+    wu = torch.zeros(w.r, w.E, dtype=wt, device=device)
+    packed = q.qsvd_prepare_weights(dims, wd, wu, wu, wu)
+    x = torch.randn(n, w.E, device=device, generator=g).to(wt)
+    rowb = {"f16": 2 * w.r, "bf16": 2 * w.r, "f32": 4 * w.r, "i8": w.r, "i4": w.r // 2}[w.cache]
+    cache = torch.empty(n, rowb, dtype=torch.uint8, device=device)
+    scales = (torch.empty(n, w.r // w.group, dtype=torch.float16, device=device)
+              if w.cache in ("i4", "i8") else None)
+    dst = torch.arange(n, dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    for _ in range(args.warmup):
+        q.qsvd_prefill_latent(dims, packed, x, dst, cache, scales, None, status)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            q.qsvd_prefill_latent(dims, packed, x, dst, cache, scales, None, status)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.0 * n * w.E * w.r
+    achieved = flops / (ms / 1e3) / 1e12
+    _, burst, sustained, kind = measured_peaks()
+    return {"metric": "prefill latent rows/s (x W^d, rounded or quantised into the cache)",
+            "value": n / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": w.weight, "data": "synthetic",
+            "config": {"workload": w.name, "E": w.E, "r": w.r, "rows": n, "cache": w.cache},
+            "roofline": {"bound": "tensor", "achieved": achieved, "unit": "TFLOP/s",
+                         "peak": sustained, "frac": achieved / sustained,
+                         "frac_of_burst_peak": achieved / burst, "peak_kind": kind + " bf16 sustained",
+                         "kernel": "k_prefill", "flops_per_launch": flops},
+            "status": int(status.item()), "clocks": clk.summary()}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -536,6 +586,8 @@ def main():
     ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05", "cta", "cluster"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time qsvd_prefill_latent over the workload's whole cache instead of a decode step")
     ap.add_argument("--eager", action="store_true",
                     help="time the API calls as issued instead of a CUDA-graph replay of one step")
     args = ap.parse_args()
@@ -545,7 +597,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.prefill:
+        line = run_prefill(args)
+    elif args.impl == "reference":
         line = run_reference(args, rank, world)
     else:
         if world > 1:

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define QSVD_ABI_VERSION 1
+#define QSVD_ABI_VERSION 2
 
 typedef enum {
   QSVD_OK = 0,
@@ -175,6 +175,36 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed,
                                void* scales, float* c_out, int32_t* status,
                                void* workspace, size_t* workspace_bytes,
                                void* stream);
+
+/*
+ * qsvd_prefill_latent -- the latent rows of many tokens at once (a prompt):
+ * c_i = x_i W^d for n_rows rows of x, each rounded to the cache type or
+ * quantised exactly as qsvd_append_latent does, stored at cache row
+ * dst_rows[i] (= b * max_len + t for token t of sequence b).
+ * Source: QSVD paper notes, 关键设计 (only C = X W^d is cached); QSVD digest,
+ * Method, Step 3 (quantised latent).  One tensor-core GEMM with the rounding
+ * or quantisation fused into its epilogue.
+ *   x             device, n_rows x E, weight_dtype, row-major, 16-byte aligned.
+ *   n_rows        >= 0 (0: nothing is enqueued).
+ *   dst_rows      device, n_rows int32: destination cache row of each x row;
+ *                 rows outside [0, B * max_len) are skipped and flagged
+ *                 (QSVD_STATUS_POS_OOB).
+ *   cache, scales as in qsvd_append_latent.
+ *   c_fp32_debug  device, n_rows x r float32 (16-byte aligned), or NULL:
+ *                 receives c before rounding, the exact input of the
+ *                 quantiser.
+ *   status        device int32 word or NULL; bits QSVD_STATUS_* are OR-ed in.
+ * Requires 16-bit weights, r % 256 == 0, E % 64 == 0, group == 128 for int
+ * caches, and H2 folded into the weights (dims->h2 == 0); else UNSUPPORTED.
+ * The tensor cores sum the fp32 products in their own order, so c can differ
+ * from qsvd_append_latent's in the last bits; a given c is rounded and
+ * quantised identically.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+qsvd_status qsvd_prefill_latent(const qsvd_dims* dims, const void* packed,
+                                const void* x, int n_rows, const int32_t* dst_rows,
+                                void* cache, void* scales, float* c_fp32_debug,
+                                int32_t* status, void* stream);
 
 /*
  * qsvd_append_latent_static -- qsvd_append_latent without a workspace.

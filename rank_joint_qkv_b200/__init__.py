@@ -57,6 +57,7 @@ _sigs = {
                          ctypes.c_uint, _P],
     "qsvd_combine_splits": [_D, _P, _P, ctypes.c_int, _P, _P, _P],
     "qsvd_append_latent_static": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
+    "qsvd_prefill_latent": [_D, _P, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -153,6 +154,16 @@ def qsvd_append_latent(dims: qsvd_dims, packed, x, pos, cache, scales=None, c_ou
                                    _ptr(workspace), ctypes.byref(n), _stream(stream)),
            "qsvd_append_latent")
     return workspace
+
+
+def qsvd_prefill_latent(dims: qsvd_dims, packed, x, dst_rows, cache, scales=None,
+                        c_out=None, status=None, stream=None):
+    """Latent rows of x.shape[0] tokens at once, row i stored at cache row
+    dst_rows[i] (b * max_len + t)."""
+    _check(_lib.qsvd_prefill_latent(ctypes.byref(dims), _ptr(packed), _ptr(x), int(x.shape[0]),
+                                    _ptr(dst_rows), _ptr(cache), _ptr(scales), _ptr(c_out),
+                                    _ptr(status), _stream(stream)),
+           "qsvd_prefill_latent")
 
 
 def qsvd_append_latent_static(dims: qsvd_dims, packed, x, pos, cache, scales=None,

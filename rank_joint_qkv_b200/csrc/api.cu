@@ -216,6 +216,29 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed, const 
   return QSVD_OK;
 }
 
+qsvd_status qsvd_prefill_latent(const qsvd_dims* dims, const void* packed, const void* x, int n_rows,
+                                const int32_t* dst_rows, void* cache, void* scales, float* c_fp32_debug,
+                                int32_t* status, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (n_rows < 0) return fail(QSVD_ERR_INVALID_ARG, "n_rows must be >= 0");
+  if (!prefill_supported(d) || (cache_is_int(d) && d.group != 128))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "prefill needs 16-bit weights, r %% 256 == 0, E %% 64 == 0, group 128, H2 folded into the weights");
+  if (n_rows == 0) return QSVD_OK;
+  if (!packed || !x || !dst_rows || !cache) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (cache_is_int(d) && !scales) return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
+  if (!aligned16(x) || !aligned16(cache) || (c_fp32_debug && !aligned16(c_fp32_debug)))
+    return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const PackedLayout L = packed_layout(d);
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  cudaError_t e = launch_prefill(d, P + L.wd, x, n_rows, dst_rows, cache, scales, c_fp32_debug, status,
+                                 static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_latent");
+  return QSVD_OK;
+}
+
 static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const float* qin,
                                int qin_is_latent, const void* cache, const void* scales,
                                const int32_t* lengths, int num_splits, void* workspace,

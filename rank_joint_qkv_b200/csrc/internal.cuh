@@ -215,6 +215,14 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s);
 
+// Prefill of the latent cache (tcgen05 GEMM x W^d with the append path's
+// rounding / quantisation fused): 16-bit weights, r % 256 == 0, E % 64 == 0,
+// H2 folded into the weights (not the online mode).
+bool prefill_supported(const qsvd_dims& d);
+cudaError_t launch_prefill(const qsvd_dims& d, const void* wd, const void* x, int n_rows,
+                           const int32_t* dst_rows, void* cache, void* scales, float* c_out,
+                           int32_t* status, cudaStream_t s);
+
 // Combine phase.  16-bit weights with d_h % 64 == 0: a merge kernel writes
 // the merged latents zm, then the tensor-core GEMV applies W^u_v per head;
 // otherwise one kernel merges and applies W^u_v per (head, 128 rows of r).

@@ -161,3 +161,27 @@ def test_cluster_kernel_refused_where_it_does_not_apply(bad):
     with pytest.raises(q.QsvdError) as e:
         q.decode_workspace_bytes(d, num_splits=4)
     assert e.value.status == q.QSVD_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bad", [dict(weight="f32", cache="f32"), dict(r=384, E=512),
+                                 dict(h2=True, h2_m=2), dict(cache="i4", group=64)])
+def test_prefill_refused_where_it_does_not_apply(bad):
+    """qsvd_prefill_latent: dims it has no kernel for are UNSUPPORTED, on the
+    host, before any pointer is looked at."""
+    lib = ctypes.CDLL(q.LIB_PATH)
+    lib.qsvd_prefill_latent.argtypes = q._sigs["qsvd_prefill_latent"]
+    d = _dims(**bad)
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.qsvd_prefill_latent(ctypes.byref(d), fake, fake, 4, fake, fake, fake, None, None, None)
+    assert st == q.QSVD_ERR_UNSUPPORTED, q._lib.qsvd_last_error()
+
+
+def test_prefill_row_count_checked_on_host():
+    lib = ctypes.CDLL(q.LIB_PATH)
+    lib.qsvd_prefill_latent.argtypes = q._sigs["qsvd_prefill_latent"]
+    d = _dims()
+    st = lib.qsvd_prefill_latent(ctypes.byref(d), None, None, -1, None, None, None, None, None, None)
+    assert st == q.QSVD_ERR_INVALID_ARG
+    # no rows: nothing to do, no pointer needed
+    st = lib.qsvd_prefill_latent(ctypes.byref(d), None, None, 0, None, None, None, None, None, None)
+    assert st == q.QSVD_OK
