@@ -270,3 +270,72 @@ def attention_uncompressed(xs: Sequence[np.ndarray], lengths, x_query: np.ndarra
             e = np.exp(logits - m)
             out[b, lo:hi] = (e / e.sum()) @ vv[:, lo:hi]
     return out
+
+
+# --------------------------------------------------------------------------
+# Output projection (the layer's W_O after attention)
+# --------------------------------------------------------------------------
+
+def output_projection(o: np.ndarray, wo: np.ndarray) -> np.ndarray:
+    """y = o W_O: the attention output (B x E, heads concatenated) times the
+    layer's output projection (E x E; row h*d_h + i multiplies channel i of
+    head h)."""
+    return np.asarray(o, np.float64) @ np.asarray(wo, np.float64)
+
+
+def fold_value_output(wuv: np.ndarray, wo: np.ndarray, H: int) -> np.ndarray:
+    """Per-head merge of the value up-projection into the output projection.
+
+    WSVD digest, Method, fused kernel (§3.4): the value factor of each head
+    is fused into the output projection so that V is never rebuilt.  With a
+    shared latent the value factor of head h is W^u_{v,h} (the d_h columns of
+    W^u_v that belong to h, r x d_h) and the matching slice of W_O is its rows
+    h*d_h .. h*d_h + d_h - 1 (d_h x E).  Returns F stacked by head: rows
+    h*r .. h*r + r - 1 hold F_h = W^u_{v,h} W_{O,h} (H*r x E)."""
+    wuv = np.asarray(wuv, np.float64)
+    wo = np.asarray(wo, np.float64)
+    r, E = wuv.shape
+    d_h = E // H
+    f = np.zeros((H * r, wo.shape[1]))
+    for h in range(H):
+        cols = slice(h * d_h, (h + 1) * d_h)
+        f[h * r:(h + 1) * r] = wuv[:, cols] @ wo[cols]
+    return f
+
+
+def decode_absorbed_latents(caches: Sequence[np.ndarray], lengths, qin: np.ndarray,
+                            wuq, wuk, H: int, *, qin_is_latent: bool = True,
+                            scale: Optional[float] = None) -> np.ndarray:
+    """Per-head attention-weighted latent z_h = p_h^T C (B x H x r): the
+    absorbed decode before any value projection (zero for an empty
+    sequence)."""
+    wuq = np.asarray(wuq, np.float64)
+    wuk = np.asarray(wuk, np.float64)
+    E = wuk.shape[1]
+    r = wuk.shape[0]
+    d_h = E // H
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    B = len(lengths)
+    z = np.zeros((B, H, r))
+    for b in range(B):
+        n = int(lengths[b])
+        if n == 0:
+            continue
+        c = np.asarray(caches[b], np.float64)[:n]
+        qb = np.asarray(qin[b], np.float64)
+        q = qb @ wuq if qin_is_latent else qb
+        for h in range(H):
+            cols = slice(h * d_h, (h + 1) * d_h)
+            s = scale * (c @ (wuk[:, cols] @ q[cols]))
+            p = np.exp(s - np.max(s))
+            z[b, h] = (p / np.sum(p)) @ c
+    return z
+
+
+def decode_folded(z: np.ndarray, f: np.ndarray) -> np.ndarray:
+    """y_b = sum_h z_{b,h} F_h: the projected layer output straight from the
+    per-head latents (B x E_out)."""
+    z = np.asarray(z, np.float64)
+    B, H, r = z.shape
+    return z.reshape(B, H * r) @ np.asarray(f, np.float64)

@@ -363,3 +363,53 @@ def test_quantizer_error_bound_and_packing():
     assert np.array_equal(qr.unpack_int4(qr.pack_int4(codes)), codes)
     p = qr.pack_int4(np.array([[1, -1, -8, 7]], np.int8))
     assert p.tolist() == [[0xF1, 0x78]]
+
+
+# ---------------------------------------------------------- output projection
+
+def _wo(E, seed):
+    return np.random.default_rng(seed).standard_normal((E, E)) / math.sqrt(E)
+
+
+@pytest.mark.parametrize("rope_free_cfg", [1, 3])
+def test_fold_equals_projected_materialized(rope_free_cfg):
+    """sum_h z_h (W^u_{v,h} W_{O,h}) is the attention of the materialised
+    route (values rebuilt, heads concatenated) times W_O; an empty sequence
+    gives a zero row."""
+    w = synthetic.SHRUNK[rope_free_cfg]
+    case = oi.build_case(w)
+    lengths = case.lengths.copy()
+    lengths[-1] = 0
+    wo = _wo(w.E, 4)
+    want = ref.output_projection(
+        ref.decode_materialized(case.caches, lengths, case.cnew, case.wuq, case.wuk, case.wuv, w.H), wo)
+    z = ref.decode_absorbed_latents(case.caches, lengths, case.cnew, case.wuq, case.wuk, w.H)
+    got = ref.decode_folded(z, ref.fold_value_output(case.wuv, wo, w.H))
+    assert np.max(np.abs(got - want)) <= 1e-11 * np.max(np.abs(want))
+    assert np.all(got[-1] == 0.0)
+
+
+def test_fold_with_identity_output_projection():
+    """W_O = I: F_h is W^u_{v,h} placed in head h's columns, zero elsewhere
+    (fixes which rows of W_O and which columns of W^u_v meet)."""
+    E, H, r = 96, 3, 40
+    wuv = np.random.default_rng(2).standard_normal((r, E))
+    f = ref.fold_value_output(wuv, np.eye(E), H)
+    d_h = E // H
+    for h in range(H):
+        blk = f[h * r:(h + 1) * r]
+        assert np.array_equal(blk[:, h * d_h:(h + 1) * d_h], wuv[:, h * d_h:(h + 1) * d_h])
+        mask = np.ones(E, bool)
+        mask[h * d_h:(h + 1) * d_h] = False
+        assert np.all(blk[:, mask] == 0.0)
+
+
+def test_output_projection_permutation():
+    """A permutation W_O moves columns: y[:, perm[j]] = o[:, j]."""
+    g = np.random.default_rng(8)
+    o = g.standard_normal((3, 12))
+    perm = g.permutation(12)
+    wo = np.zeros((12, 12))
+    wo[np.arange(12), perm] = 1.0
+    y = ref.output_projection(o, wo)
+    assert np.array_equal(y[:, perm], o)
