@@ -262,8 +262,14 @@ def run_ours(args, rank, world, local_rank):
             "cluster": q.QSVD_KERNEL_TCGEN05_CLUSTER}[args.kernel]
     dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
                        out="f32", group=w.group, rope=w.rope, rope_base=w.rope_base,
-                       kernel=kern)
+                       kernel=kern, out_proj=args.out_proj)
     packed = q.qsvd_prepare_weights(dims, inp["wd"], inp["wuq"], inp["wuk"], inp["wuv"])
+    if args.out_proj != "none":
+        # synthetic output projection W_O (E x E), seeded like the other weights
+        gwo = torch.Generator(device=device).manual_seed(w.seed * 31 + 5)
+        wo = (torch.randn((w.E, w.E), generator=gwo, device=device) / math.sqrt(w.E)).to(TORCH_DT[w.weight])
+        q.qsvd_prepare_out_proj(dims, wo, packed)
+        del wo
     stream = torch.cuda.current_stream()
     lens_dev = torch.from_numpy(lens).to(device)
     pos_dev = (lens_dev - 1).to(torch.int32)
@@ -426,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
                    "batch_per_gpu": w.B, "kv_len": int(max_len),
                    "tokens_per_step_per_gpu": int(tokens_per_step), "cache": w.cache,
                    "weights": w.weight, "mode": "rope" if w.rope else "absorbed",
-                   "splits": args.splits, "kernel": args.kernel,
+                   "splits": args.splits, "kernel": args.kernel, "out_proj": args.out_proj,
                    "l2": "inputs larger than L2: %.0f MB latent read per step per GPU"
                          % (lat_b / 1e6),
                    "parallelism": f"dp{world}"},
@@ -586,6 +592,9 @@ def main():
     ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05", "cta", "cluster"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--out-proj", choices=["none", "chain", "fold"], default="none",
+                    help="apply the layer's output projection W_O in the combine (chain: V-up then "
+                         "W_O; fold: W^u_v folded into W_O per head)")
     ap.add_argument("--prefill", action="store_true",
                     help="time qsvd_prefill_latent over the workload's whole cache instead of a decode step")
     ap.add_argument("--eager", action="store_true",

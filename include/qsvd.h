@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define QSVD_ABI_VERSION 2
+#define QSVD_ABI_VERSION 3
 
 typedef enum {
   QSVD_OK = 0,
@@ -98,6 +98,20 @@ typedef enum {
 /* The workspace header records the kernel that ran: SIMT, TCGEN05_CTA or
  * TCGEN05_CLUSTER. */
 
+/* Output projection applied by the combine (qsvd_dims.out_proj).  WSVD
+ * digest, Method, fused kernel (§3.4): the value up-projection is merged
+ * into the attention layer's output projection W_O so that V is never built.
+ *   NONE   out = o (B x E, heads concatenated), o_h = z_h W^u_{v,h}.
+ *   CHAIN  out = o W_O: the V-up GEMV, then a GEMV by W_O (E x E).
+ *   FOLD   out = sum_h z_h F_h with F_h = W^u_{v,h} W_{O,h} (r x E), the
+ *          rows h d_h .. h d_h + d_h - 1 of W_O: one GEMV over the merged
+ *          latents, no V-up.  F (H r x E) is formed once by
+ *          qsvd_prepare_out_proj.
+ * CHAIN and FOLD need 16-bit weights and d_h % 64 == 0. */
+#define QSVD_OUT_PROJ_NONE 0
+#define QSVD_OUT_PROJ_CHAIN 1
+#define QSVD_OUT_PROJ_FOLD 2
+
 typedef struct {
   int E;               /* model width, E = H * d_h */
   int H;               /* heads */
@@ -115,6 +129,7 @@ typedef struct {
   int h2;              /* 1: append applies H2 to the latent before quantising */
   int h2_m;            /* order m of the small factor of H2 = H_{r/m} (x) Q_m */
   int kernel;          /* QSVD_KERNEL_* */
+  int out_proj;        /* QSVD_OUT_PROJ_* */
 } qsvd_dims;
 
 /*
@@ -232,6 +247,27 @@ qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const void* packed,
                                       void* stream);
 
 /*
+ * qsvd_prepare_out_proj -- add the output projection W_O to a packed buffer
+ * that qsvd_prepare_weights filled with the same dims (dims->out_proj CHAIN
+ * or FOLD; qsvd_prepare_weights reports the size with room for it).
+ * Source: WSVD digest, Method, fused kernel (§3.4).
+ *   wo            device, E x E row-major, weight_dtype: y = o W_O, row
+ *                 h d_h + i of W_O multiplies channel i of head h.
+ *   packed        the buffer of qsvd_prepare_weights (read: W^u_v, already
+ *                 rotated by H2 when one was folded in; written: the W_O
+ *                 section).  CHAIN copies W_O; FOLD writes
+ *                 F[h r + j][n] = sum_i W^u_v[j][h d_h + i] W_O[h d_h + i][n],
+ *                 accumulated in float32 over i in order and rounded once
+ *                 to weight_dtype.
+ *   packed_bytes  in: capacity of packed.
+ * Stream-ordered; nothing is allocated.
+ * Errors: INVALID_ARG (out_proj NONE, NULL pointers, small buffer),
+ * UNSUPPORTED (fp32 weights, d_h % 64 != 0), CUDA.
+ */
+qsvd_status qsvd_prepare_out_proj(const qsvd_dims* dims, const void* wo, void* packed,
+                                  size_t packed_bytes, void* stream);
+
+/*
  * qsvd_decode_attn -- one decode step of multi-head attention over the
  * latent cache, output B x E.
  * Source: QSVD digest, Method, Step 1 (keys/values rebuilt from C_qkv);
@@ -251,7 +287,8 @@ qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const void* packed,
  *                  sections): header (int32 status, G, tile, kernel), query
  *                  buffers, then per split-partial slot s = split + b:
  *                  m[s][H], l[s][H] (float32, log2 domain), z[s][H][r].
- *   out            device, B x E, out_dtype.
+ *   out            device, B x E, out_dtype: o, or the projected o W_O when
+ *                  dims->out_proj is CHAIN or FOLD.
  *   phases         QSVD_PHASE_* mask (0 = all).  Running the phases as
  *                  separate calls in order gives the same result; so does
  *                  running the split as its two rotary passes
@@ -271,6 +308,7 @@ qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed,
  * lengths and num_splits) and apply the value up-projection: with M = max_s m_s,
  * w_s = 2^(m_s - M):  z = sum_s w_s z_s / sum_s w_s l_s,  o_h = z_h W^u_{v,h}.
  * Source: WSVD digest, Method 3.4 (flash decoding); QSVD digest, Step 1.
+ * With dims->out_proj the output is o W_O (see QSVD_OUT_PROJ_*).
  * Equivalent to qsvd_decode_attn with phases = QSVD_PHASE_COMBINE.
  * Errors: INVALID_ARG, CUDA.
  */

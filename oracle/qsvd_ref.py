@@ -305,10 +305,12 @@ def fold_value_output(wuv: np.ndarray, wo: np.ndarray, H: int) -> np.ndarray:
 
 def decode_absorbed_latents(caches: Sequence[np.ndarray], lengths, qin: np.ndarray,
                             wuq, wuk, H: int, *, qin_is_latent: bool = True,
+                            rope_base: Optional[float] = None,
                             scale: Optional[float] = None) -> np.ndarray:
     """Per-head attention-weighted latent z_h = p_h^T C (B x H x r): the
-    absorbed decode before any value projection (zero for an empty
-    sequence)."""
+    decode before any value projection (zero for an empty sequence).  The
+    scores are C qt_h with qt_h = W^u_{k,h} q_h, or, with rope_base, the
+    rotated rebuilt keys R(t) (C W^u_{k,h})_t against the rotated query."""
     wuq = np.asarray(wuq, np.float64)
     wuk = np.asarray(wuk, np.float64)
     E = wuk.shape[1]
@@ -327,7 +329,12 @@ def decode_absorbed_latents(caches: Sequence[np.ndarray], lengths, qin: np.ndarr
         q = qb @ wuq if qin_is_latent else qb
         for h in range(H):
             cols = slice(h * d_h, (h + 1) * d_h)
-            s = scale * (c @ (wuk[:, cols] @ q[cols]))
+            if rope_base is None:
+                s = scale * (c @ (wuk[:, cols] @ q[cols]))
+            else:
+                kh = rope(c @ wuk[:, cols], np.arange(n), rope_base)
+                qh = rope(q[cols][None, :], np.array([n - 1]), rope_base)[0]
+                s = scale * (kh @ qh)
             p = np.exp(s - np.max(s))
             z[b, h] = (p / np.sum(p)) @ c
     return z

@@ -32,6 +32,9 @@ QSVD_PHASE_SPLIT_SCORES, QSVD_PHASE_SPLIT_ACCUM = 8, 16
 QSVD_STATUS_LEN_CLAMPED, QSVD_STATUS_POS_OOB, QSVD_STATUS_SCALE_SAT, QSVD_STATUS_TIMEOUT = 1, 2, 4, 8
 QSVD_KERNEL_AUTO, QSVD_KERNEL_SIMT, QSVD_KERNEL_TCGEN05 = 0, 1, 2
 QSVD_KERNEL_TCGEN05_CTA, QSVD_KERNEL_TCGEN05_CLUSTER = 3, 4
+QSVD_OUT_PROJ_NONE, QSVD_OUT_PROJ_CHAIN, QSVD_OUT_PROJ_FOLD = 0, 1, 2
+OUT_PROJ_CODE = {None: QSVD_OUT_PROJ_NONE, "none": QSVD_OUT_PROJ_NONE,
+                 "chain": QSVD_OUT_PROJ_CHAIN, "fold": QSVD_OUT_PROJ_FOLD}
 
 DTYPE_CODE = {"f32": QSVD_F32, "f16": QSVD_F16, "bf16": QSVD_BF16, "i8": QSVD_I8, "i4": QSVD_I4}
 
@@ -43,7 +46,7 @@ class qsvd_dims(ctypes.Structure):
         ("rope", ctypes.c_int), ("rope_base", ctypes.c_float),
         ("softmax_scale", ctypes.c_float), ("cache_dtype", ctypes.c_int),
         ("weight_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("h2", ctypes.c_int),
-        ("h2_m", ctypes.c_int), ("kernel", ctypes.c_int),
+        ("h2_m", ctypes.c_int), ("kernel", ctypes.c_int), ("out_proj", ctypes.c_int),
     ]
 
 
@@ -58,6 +61,7 @@ _sigs = {
     "qsvd_combine_splits": [_D, _P, _P, ctypes.c_int, _P, _P, _P],
     "qsvd_append_latent_static": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
     "qsvd_prefill_latent": [_D, _P, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P],
+    "qsvd_prepare_out_proj": [_D, _P, _P, ctypes.c_size_t, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -98,10 +102,12 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def make_dims(E, H, d_h, r, batch, max_len, *, cache="f16", weight="f16", out="f32",
               group=128, rope=False, rope_base=10000.0, softmax_scale=0.0, h2=False,
-              h2_m=0, kernel=QSVD_KERNEL_AUTO) -> qsvd_dims:
+              h2_m=0, kernel=QSVD_KERNEL_AUTO, out_proj=None) -> qsvd_dims:
+    """``out_proj``: None/"none", "chain" or "fold" (see QSVD_OUT_PROJ_*)."""
     return qsvd_dims(E, H, d_h, r, batch, max_len, group, int(bool(rope)), float(rope_base),
                      float(softmax_scale), DTYPE_CODE[cache], DTYPE_CODE[weight],
-                     DTYPE_CODE[out], int(bool(h2)), int(h2_m), int(kernel))
+                     DTYPE_CODE[out], int(bool(h2)), int(h2_m), int(kernel),
+                     OUT_PROJ_CODE[out_proj])
 
 
 def kernel_launches() -> int:
@@ -134,6 +140,14 @@ def qsvd_prepare_weights(dims: qsvd_dims, wd, wuq, wuk, wuv, h2_q=None, packed=N
                                      _ptr(wuv), _ptr(hq), _ptr(packed), ctypes.byref(n),
                                      _stream(stream)), "qsvd_prepare_weights")
     return packed
+
+
+def qsvd_prepare_out_proj(dims: qsvd_dims, wo, packed, stream=None):
+    """Add W_O (E x E device tensor, y = o W_O) to a buffer filled by
+    qsvd_prepare_weights with the same dims (dims.out_proj chain or fold)."""
+    _check(_lib.qsvd_prepare_out_proj(ctypes.byref(dims), _ptr(wo), _ptr(packed),
+                                      packed.numel() * packed.element_size(), _stream(stream)),
+           "qsvd_prepare_out_proj")
 
 
 def append_workspace_bytes(dims: qsvd_dims) -> int:

@@ -79,6 +79,8 @@ static qsvd_status validate(const qsvd_dims* d) {
   }
   if (d->kernel < QSVD_KERNEL_AUTO || d->kernel > QSVD_KERNEL_TCGEN05_CLUSTER)
     return fail(QSVD_ERR_INVALID_ARG, "unknown kernel choice %d", d->kernel);
+  if (d->out_proj < QSVD_OUT_PROJ_NONE || d->out_proj > QSVD_OUT_PROJ_FOLD)
+    return fail(QSVD_ERR_INVALID_ARG, "unknown out_proj %d", d->out_proj);
   return QSVD_OK;
 }
 
@@ -189,6 +191,27 @@ qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd, const vo
   return QSVD_OK;
 }
 
+qsvd_status qsvd_prepare_out_proj(const qsvd_dims* dims, const void* wo, void* packed,
+                                  size_t packed_bytes, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (d.out_proj == QSVD_OUT_PROJ_NONE)
+    return fail(QSVD_ERR_INVALID_ARG, "dims->out_proj is QSVD_OUT_PROJ_NONE");
+  if (!combine_uses_gemv(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "the output projection needs 16-bit weights, d_h %% 64 == 0, r %% 32 == 0");
+  if (!wo || !packed) return fail(QSVD_ERR_INVALID_ARG, "wo/packed is NULL");
+  const PackedLayout L = packed_layout(d);
+  if (packed_bytes < L.total)
+    return fail(QSVD_ERR_WORKSPACE, "packed buffer holds %zu bytes, %zu needed", packed_bytes, L.total);
+  if ((reinterpret_cast<uintptr_t>(packed) & 255u) != 0)
+    return fail(QSVD_ERR_INVALID_ARG, "packed must be 256-byte aligned");
+  cudaError_t e = launch_prepare_out_proj(d, wo, packed, L, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prepare_out_proj");
+  return QSVD_OK;
+}
+
 qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed, const void* x,
                                const int32_t* pos, void* cache, void* scales, float* c_out,
                                int32_t* status, void* workspace, size_t* workspace_bytes,
@@ -263,6 +286,10 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
                 "tensor-core rotary path needs d_h == 128, r %% 64 == 0, cache and weights both fp16 or both bf16");
   if (kernel == QSVD_KERNEL_SIMT && !d.rope && split_simt_grid_heads(d) == 0)
     return fail(QSVD_ERR_UNSUPPORTED, "rank too large for the CUDA-core split kernel");
+  if ((phases & QSVD_PHASE_COMBINE) && d.out_proj != QSVD_OUT_PROJ_NONE && !combine_uses_gemv(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "the output projection needs 16-bit weights, d_h %% 64 == 0, r %% 32 == 0 and "
+                "at most 2047 tiles per sequence");
   int G = 0;
   qsvd_status st = resolve_splits(d, num_splits, kernel, &G);
   if (st != QSVD_OK) return st;
@@ -343,8 +370,10 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (combine_uses_gemv(d)) {
       float* zm = reinterpret_cast<float*>(Wb + W.zm);
       int32_t* tickets = reinterpret_cast<int32_t*>(Wb + W.tickets) + W.NTQ;
+      const OutProj op{P + L.wo, reinterpret_cast<float*>(Wb + W.ow), reinterpret_cast<float*>(Wb + W.ypart),
+                       tickets + W.NTV};
       e = launch_combine_gemv(d, hdr, sched, pm, pl, pz, P + L.wuv, zm, opart, tickets, &hdr->status,
-                              out, s);
+                              out, op, s);
     } else {
       e = launch_combine(d, hdr, sched, pm, pl, pz, P + L.wuv, opart, W.JS, W.P, out, s);
     }

@@ -317,7 +317,7 @@ template <typename WT, typename OT>
 cudaError_t merge_vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                         const float* pm, const float* pl, const float* pz, const void* wuv,
                         float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
-                        cudaStream_t s) {
+                        const OutProj& op, cudaStream_t s) {
   const dim3 grid((d.r + kMergeCh - 1) / kMergeCh, d.H, d.batch);
   {
     const cudaError_t le = launch_pdl(k_merge, dim3(grid), dim3(128), 0, s,
@@ -327,9 +327,26 @@ cudaError_t merge_vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* 
   note_launch();
   cudaError_t e = check_launch();
   if (e != cudaSuccess) return e;
+  const WT* wo = static_cast<const WT*>(op.wo);
+  if (d.out_proj == QSVD_OUT_PROJ_FOLD) {
+    // out[b][n] = sum_{h, j} zm[b][h][j] F[h r + j][n]: the merged latents of
+    // all heads are one activation row of H r elements
+    const int K = d.H * d.r;
+    return launch_gemv<float, WT, OT>(zm, wo, op.ypart, d.batch, K, d.E, gemv_ksplit(K, d.weight_dtype),
+                                      static_cast<OT*>(out), op.ytickets, status, s);
+  }
   // o[b][h d_h + n] = zm[b][h] . W^u_v[:, h d_h + n]: activation row of
   // column group h (d_h columns) is zm + b H r + h r
   const XGroups xg{(long long)d.H * d.r, d.d_h, d.r};
+  if (d.out_proj == QSVD_OUT_PROJ_CHAIN) {
+    e = launch_gemv<float, WT, float>(zm, static_cast<const WT*>(wuv), vpart, d.batch, d.r, d.E,
+                                      gemv_ksplit(d.r, d.weight_dtype), op.ow, tickets, status, s, xg);
+    if (e != cudaSuccess) return e;
+    // y = o W_O with o kept in fp32 (the GEMV splits it into two 16-bit parts)
+    return launch_gemv<float, WT, OT>(op.ow, wo, op.ypart, d.batch, d.E, d.E,
+                                      gemv_ksplit(d.E, d.weight_dtype), static_cast<OT*>(out), op.ytickets,
+                                      status, s);
+  }
   return launch_gemv<float, WT, OT>(zm, static_cast<const WT*>(wuv), vpart, d.batch, d.r, d.E,
                                     gemv_ksplit(d.r, d.weight_dtype), static_cast<OT*>(out), tickets,
                                     status, s, xg);
@@ -348,15 +365,15 @@ bool combine_uses_gemv(const qsvd_dims& d) {
 cudaError_t launch_combine_gemv(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                                 const float* pm, const float* pl, const float* pz, const void* wuv,
                                 float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
-                                cudaStream_t s) {
+                                const OutProj& op, cudaStream_t s) {
 #define QSVD_MV(WT)                                                                                    \
   switch (d.out_dtype) {                                                                               \
     case QSVD_F32: return merge_vup_t<WT, float>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart, tickets,   \
-                                                 status, out, s);                                      \
+                                                 status, out, op, s);                                      \
     case QSVD_F16: return merge_vup_t<WT, __half>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart, tickets,  \
-                                                  status, out, s);                                     \
+                                                  status, out, op, s);                                     \
     case QSVD_BF16: return merge_vup_t<WT, __nv_bfloat16>(d, hdr, sched, pm, pl, pz, wuv, zm, vpart,   \
-                                                          tickets, status, out, s);                    \
+                                                          tickets, status, out, op, s);                    \
     default: return cudaErrorInvalidValue;                                                             \
   }
   if (d.weight_dtype == QSVD_BF16) { QSVD_MV(__nv_bfloat16) }

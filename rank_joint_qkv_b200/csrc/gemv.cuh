@@ -161,20 +161,6 @@ k_gemv_partial(const XT* __restrict__ x, const WT* __restrict__ W, float* __rest
 template <typename WT>
 inline size_t gemv_smem() { return size_t(gemv_rows<WT>()) * (256 * sizeof(WT) + 16 * 4); }
 
-// Split of K: one 64 KB tile per CTA -- 512 rows x 64 columns for 16-bit
-// weights (tensor cores), 64 rows x 256 columns for fp32 (CUDA cores).
-// Shape-only, device-independent.
-inline int gemv_ksplit(int K, qsvd_dtype wt) {
-  const int rt = wt == QSVD_F32 ? 64 : 512;
-  return (K + rt - 1) / rt;
-}
-
-// Ticket counters: one per (column block, block of 16 sequences).
-inline int gemv_tickets(int N, int B, qsvd_dtype wt) {
-  const int cw = wt == QSVD_F32 ? 256 : 64;
-  return ((N + cw - 1) / cw) * ((B + 15) / 16);
-}
-
 // ---------------------------------------------------------------------------
 // Tensor-core variant for 16-bit weights (mma.sync m16n8k16, fp32 accumulate).
 // At 16 sequences a CUDA-core GEMV does 16 FMAs per weight element and is

@@ -53,8 +53,15 @@ struct PackedLayout {
   size_t wukT;                // W^u_k transposed, E x r (rotary tensor-core path)
   size_t h2q;                 // h2_m x h2_m float32 (online H2 in append)
   size_t rope;                // max_len x (d_h/2) x {cos, sin} float32
+  size_t wo;                  // output projection: W_O E x E (chain) or F H r x E (fold)
   size_t total;
 };
+
+// Rows (K) of the output-projection GEMV: E for the chain, H r for the fold.
+inline size_t out_proj_rows(const qsvd_dims& d) {
+  return d.out_proj == QSVD_OUT_PROJ_FOLD ? size_t(d.H) * d.r
+                                          : d.out_proj == QSVD_OUT_PROJ_CHAIN ? size_t(d.E) : 0;
+}
 
 inline PackedLayout packed_layout(const qsvd_dims& d) {
   PackedLayout p{};
@@ -68,6 +75,7 @@ inline PackedLayout packed_layout(const qsvd_dims& d) {
   p.wukT = o; if (d.rope) o = align256(o + mat);
   p.h2q = o; o = align256(o + size_t(16) * 16 * 4);
   p.rope = o; if (d.rope) o = align256(o + size_t(d.max_len) * (d.d_h / 2) * 2 * 4);
+  p.wo = o;  o = align256(o + out_proj_rows(d) * d.E * wb);
   p.total = o;
   return p;
 }
@@ -81,9 +89,25 @@ struct WsHeader {
 };
 
 struct WsLayout {
-  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, zm, scores, total;
-  int G, P, KS, JS, NT, NTQ;   // NT tickets in all, the first NTQ for the query GEMV
+  size_t hdr, sched, tickets, q, qt32, qt16, qpart, pm, pl, pz, opart, zm, scores, ow, ypart, total;
+  int G, P, KS, JS, NT, NTQ, NTV;   // NT tickets in all: NTQ query GEMV, NTV V-up GEMV, then the
+                                    // output projection's
+  int KSY;                          // split-K of the output-projection GEMV
 };
+
+// GEMV (gemv.cuh) split of K: one 64 KB tile per CTA -- 512 rows x 64 columns for 16-bit
+// weights (tensor cores), 64 rows x 256 columns for fp32 (CUDA cores).
+// Shape-only, device-independent.
+inline int gemv_ksplit(int K, qsvd_dtype wt) {
+  const int rt = wt == QSVD_F32 ? 64 : 512;
+  return (K + rt - 1) / rt;
+}
+
+// Ticket counters: one per (column block, block of 16 sequences).
+inline int gemv_tickets(int N, int B, qsvd_dtype wt) {
+  const int cw = wt == QSVD_F32 ? 256 : 64;
+  return ((N + cw - 1) / cw) * ((B + 15) / 16);
+}
 
 // Split-K factor of the query projection and j-splits of the combine.
 int prologue_ksplit(const qsvd_dims& d);   // split of r in q = c_new W^u_q
@@ -99,7 +123,9 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.KS = prologue_ksplit(d);
   w.JS = combine_jsplit(d);
   w.NTQ = prologue_tickets(d);
-  w.NT = w.NTQ + gemv_tickets_vup(d);   // then the V-up GEMV's (combine)
+  w.NTV = gemv_tickets_vup(d);          // then the V-up GEMV's (combine)
+  w.KSY = d.out_proj ? gemv_ksplit(int(out_proj_rows(d)), d.weight_dtype) : 0;
+  w.NT = w.NTQ + w.NTV + (d.out_proj ? gemv_tickets(d.E, d.batch, d.weight_dtype) : 0);
   const size_t B = d.batch, E = d.E, H = d.H, r = d.r;
   size_t o = 0;
   w.hdr = o;   o = align256(o + sizeof(WsHeader));
@@ -115,6 +141,8 @@ inline WsLayout ws_layout(const qsvd_dims& d, int G) {
   w.opart = o; o = align256(o + size_t(w.JS) * B * E * 4);   // also the V-up GEMV's partials
   w.zm = o;    o = align256(o + B * H * r * 4);                 // merged latents [B][H][r]
   w.scores = o; if (d.rope) o = align256(o + B * H * size_t(d.max_len) * 4);   // rotary: [B][H][max_len]
+  w.ow = o;    if (d.out_proj == QSVD_OUT_PROJ_CHAIN) o = align256(o + B * E * 4);   // o before W_O
+  w.ypart = o; o = align256(o + size_t(w.KSY) * B * E * 4);    // output-projection partials
   w.total = o;
   return w;
 }
@@ -227,10 +255,21 @@ cudaError_t launch_prefill(const qsvd_dims& d, const void* wd, const void* x, in
 // the merged latents zm, then the tensor-core GEMV applies W^u_v per head;
 // otherwise one kernel merges and applies W^u_v per (head, 128 rows of r).
 bool combine_uses_gemv(const qsvd_dims& d);
+// Merge + V-up on the tensor-core GEMV.  With d.out_proj the output is
+// projected by W_O: CHAIN runs the V-up into `ow` (B x E fp32) and a second
+// GEMV by `wo` (E x E); FOLD skips the V-up and runs one GEMV of the merged
+// latents (B x H r) by `wo` = F (H r x E).  `ypart` holds that GEMV's KSY
+// split-K partials; `ytickets` its ticket counters.
+struct OutProj {
+  const void* wo;
+  float* ow;
+  float* ypart;
+  int32_t* ytickets;
+};
 cudaError_t launch_combine_gemv(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                                 const float* pm, const float* pl, const float* pz, const void* wuv,
                                 float* zm, float* vpart, int32_t* tickets, int32_t* status, void* out,
-                                cudaStream_t s);
+                                const OutProj& op, cudaStream_t s);
 cudaError_t launch_combine(const qsvd_dims& d, const WsHeader* hdr, const int32_t* sched,
                            const float* pm, const float* pl, const float* pz,
                            const void* wuv, float* opart, int JS, int P, void* out,
@@ -247,6 +286,10 @@ cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
 cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
                            const void* wuk, const void* wuv, const float* h2q_host,
                            void* packed, const PackedLayout& L, cudaStream_t s);
+// Output-projection section of the packed buffer: W_O copied (CHAIN) or the
+// per-head fold F = W^u_{v,h} W_{O,h} (FOLD); W^u_v read from the buffer.
+cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* packed,
+                                    const PackedLayout& L, cudaStream_t s);
 
 }  // namespace qsvd
 

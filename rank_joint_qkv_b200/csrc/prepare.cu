@@ -93,6 +93,65 @@ __global__ void k_rope_table(float* __restrict__ tab, int max_len, int half, dou
   }
 }
 
+// Per-head fold of the value up-projection into the output projection (WSVD
+// digest, Method, fused kernel §3.4): F[h r + j][n] = sum_i W^u_v[j][h d_h + i]
+// W_O[h d_h + i][n].  One 64 x 64 tile of F per CTA (grid ceil(E/64),
+// ceil(r/64), H; block 16 x 16, 4 x 4 outputs per thread); i runs in order,
+// fp32 fma, rounded once to WT.
+template <typename WT>
+__global__ void __launch_bounds__(256)
+k_fold_vo(const WT* __restrict__ wuv, const WT* __restrict__ wo, WT* __restrict__ f, int E, int r,
+          int d_h) {
+  __shared__ float as[64][33];   // [j][i]
+  __shared__ float bs[32][65];   // [i][n]
+  const int n0 = blockIdx.x * 64, j0 = blockIdx.y * 64, h = blockIdx.z;
+  const int tx = threadIdx.x, ty = threadIdx.y, t = ty * 16 + tx;
+  float acc[4][4] = {};
+  for (int i0 = 0; i0 < d_h; i0 += 32) {
+    for (int k = t; k < 64 * 32; k += 256) {
+      const int jj = k / 32, ii = k % 32;
+      const int j = j0 + jj, i = i0 + ii;
+      as[jj][ii] = (j < r && i < d_h) ? dev::to_f(wuv[size_t(j) * E + size_t(h) * d_h + i]) : 0.f;
+    }
+    for (int k = t; k < 32 * 64; k += 256) {
+      const int ii = k / 64, nn = k % 64;
+      const int i = i0 + ii, n = n0 + nn;
+      bs[ii][nn] = (i < d_h && n < E) ? dev::to_f(wo[(size_t(h) * d_h + i) * E + n]) : 0.f;
+    }
+    __syncthreads();
+    const int iend = min(32, d_h - i0);
+    for (int ii = 0; ii < iend; ++ii) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { a[u] = as[ty * 4 + u][ii]; b[u] = bs[ii][tx * 4 + u]; }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int j = j0 + ty * 4 + u;
+    if (j >= r) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int n = n0 + tx * 4 + v;
+      if (n < E) f[(size_t(h) * r + j) * E + n] = dev::from_f<WT>(acc[u][v]);
+    }
+  }
+}
+
+template <typename WT>
+cudaError_t fold_vo_t(const qsvd_dims& d, const void* wuv, const void* wo, void* f, cudaStream_t s) {
+  const dim3 grid((d.E + 63) / 64, (d.r + 63) / 64, d.H);
+  k_fold_vo<WT><<<grid, dim3(16, 16), 0, s>>>(static_cast<const WT*>(wuv), static_cast<const WT*>(wo),
+                                              static_cast<WT*>(f), d.E, d.r, d.d_h);
+  note_launch();
+  return check_launch();
+}
+
 template <typename WT>
 cudaError_t fold_t(WT* base, int nvec, size_t es, size_t vs, int r, int m, const float* q,
                    float scale, cudaStream_t s) {
@@ -161,6 +220,19 @@ cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
     case QSVD_F32: return prepare_t<float>(d, h2q_host, P, L, s);
     case QSVD_F16: return prepare_t<__half>(d, h2q_host, P, L, s);
     case QSVD_BF16: return prepare_t<__nv_bfloat16>(d, h2q_host, P, L, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* packed,
+                                    const PackedLayout& L, cudaStream_t s) {
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  if (d.out_proj == QSVD_OUT_PROJ_CHAIN)
+    return cudaMemcpyAsync(P + L.wo, wo, size_t(d.E) * d.E * dtype_bytes(d.weight_dtype),
+                           cudaMemcpyDeviceToDevice, s);
+  switch (d.weight_dtype) {
+    case QSVD_F16: return fold_vo_t<__half>(d, P + L.wuv, wo, P + L.wo, s);
+    case QSVD_BF16: return fold_vo_t<__nv_bfloat16>(d, P + L.wuv, wo, P + L.wo, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -126,7 +126,8 @@ def test_header_constants_match_binding():
     """Every QSVD_PHASE_ / QSVD_STATUS_ / QSVD_KERNEL_ value of the header
     has the same value in the Python binding."""
     src = open(HEADER).read()
-    consts = dict(re.findall(r"#define (QSVD_(?:PHASE|STATUS|KERNEL)_[A-Z0-9_]+) (\d+)u?", src))
+    consts = dict(re.findall(r"#define (QSVD_(?:PHASE|STATUS|KERNEL|OUT_PROJ)_[A-Z0-9_]+) (\d+)u?", src))
+    assert "QSVD_OUT_PROJ_FOLD" in consts
     assert any(k.startswith("QSVD_PHASE_SPLIT_") for k in consts)
     assert "QSVD_KERNEL_TCGEN05" in consts
     for name, val in consts.items():
@@ -185,3 +186,47 @@ def test_prefill_row_count_checked_on_host():
     # no rows: nothing to do, no pointer needed
     st = lib.qsvd_prefill_latent(ctypes.byref(d), None, None, 0, None, None, None, None, None, None)
     assert st == q.QSVD_OK
+
+
+def _packed_bytes(d):
+    n = ctypes.c_size_t(0)
+    st = q._lib.qsvd_prepare_weights(ctypes.byref(d), None, None, None, None, None, None,
+                                     ctypes.byref(n), None)
+    assert st == q.QSVD_OK
+    return n.value
+
+
+def test_out_proj_sections_sized_on_host():
+    """The packed buffer gains W_O (E x E) for the chain and F (H r x E) for
+    the fold; the decode workspace gains the projection's partials."""
+    base = _packed_bytes(_dims())
+    E, H, r = 512, 4, 256
+    assert _packed_bytes(_dims(out_proj="chain")) == base + E * E * 2
+    assert _packed_bytes(_dims(out_proj="fold")) == base + H * r * E * 2
+    w0 = q.decode_workspace_bytes(_dims(), num_splits=4)
+    # chain: o (B x E fp32) + ceil(E/512) partials of B x E
+    assert q.decode_workspace_bytes(_dims(out_proj="chain"), num_splits=4) >= w0 + 2 * 512 * 4 * 2
+    # fold: ceil(H r / 512) = 2 partials of B x E
+    assert q.decode_workspace_bytes(_dims(out_proj="fold"), num_splits=4) >= w0 + 2 * 2 * 512 * 4
+
+
+def test_out_proj_refused_on_host():
+    d = _dims()
+    d.out_proj = 3
+    with pytest.raises(q.QsvdError) as e:
+        q.decode_workspace_bytes(d, num_splits=4)
+    assert e.value.status == q.QSVD_ERR_INVALID_ARG
+    # fp32 weights have no tensor-core GEMV: the projection is UNSUPPORTED
+    d = _dims(weight="f32", cache="f32", out_proj="fold")
+    with pytest.raises(q.QsvdError) as e:
+        q.decode_workspace_bytes(d, num_splits=4)
+    assert e.value.status == q.QSVD_ERR_UNSUPPORTED
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the checks fail first
+    assert q._lib.qsvd_prepare_out_proj(ctypes.byref(d), fake, fake, 1 << 30, None) == \
+        q.QSVD_ERR_UNSUPPORTED
+    d = _dims()
+    assert q._lib.qsvd_prepare_out_proj(ctypes.byref(d), fake, fake, 1 << 30, None) == \
+        q.QSVD_ERR_INVALID_ARG
+    d = _dims(out_proj="chain")
+    assert q._lib.qsvd_prepare_out_proj(ctypes.byref(d), fake, fake, 256, None) == \
+        q.QSVD_ERR_WORKSPACE

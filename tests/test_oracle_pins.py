@@ -371,19 +371,22 @@ def _wo(E, seed):
     return np.random.default_rng(seed).standard_normal((E, E)) / math.sqrt(E)
 
 
-@pytest.mark.parametrize("rope_free_cfg", [1, 3])
-def test_fold_equals_projected_materialized(rope_free_cfg):
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_fold_equals_projected_materialized(cfg):
     """sum_h z_h (W^u_{v,h} W_{O,h}) is the attention of the materialised
-    route (values rebuilt, heads concatenated) times W_O; an empty sequence
-    gives a zero row."""
-    w = synthetic.SHRUNK[rope_free_cfg]
+    route (values rebuilt, heads concatenated) times W_O, with and without
+    rotary embedding; an empty sequence gives a zero row."""
+    w = synthetic.SHRUNK[cfg]
     case = oi.build_case(w)
     lengths = case.lengths.copy()
     lengths[-1] = 0
     wo = _wo(w.E, 4)
+    rb = w.rope_base if w.rope else None
     want = ref.output_projection(
-        ref.decode_materialized(case.caches, lengths, case.cnew, case.wuq, case.wuk, case.wuv, w.H), wo)
-    z = ref.decode_absorbed_latents(case.caches, lengths, case.cnew, case.wuq, case.wuk, w.H)
+        ref.decode_materialized(case.caches, lengths, case.cnew, case.wuq, case.wuk, case.wuv, w.H,
+                                rope_base=rb), wo)
+    z = ref.decode_absorbed_latents(case.caches, lengths, case.cnew, case.wuq, case.wuk, w.H,
+                                    rope_base=rb)
     got = ref.decode_folded(z, ref.fold_value_output(case.wuv, wo, w.H))
     assert np.max(np.abs(got - want)) <= 1e-11 * np.max(np.abs(want))
     assert np.all(got[-1] == 0.0)
