@@ -38,6 +38,7 @@ import synthetic  # noqa: E402
 METRIC = "decode-attn KV-tokens/s over C_qkv latent cache; achieved HBM GB/s vs peak"
 UNIT = "KV-tokens/s"
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+CALIB_SEQS, CALIB_LEN = 256, 640   # calibration set: sequences x tokens (image + text)
 ROW_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "i8": 1, "i4": 0.5}
 
 
@@ -547,6 +548,69 @@ def run_prefill(args):
             "status": int(status.item()), "clocks": clk.summary()}
 
 
+def run_beta(args):
+    """One split-exponent evaluation of the calibration objective per step
+    (factors for beta, layout with H2, three prefills, two decodes, the
+    squared output error on the host) on the workload's shapes with
+    ``CALIB_SEQS`` synthetic calibration sequences of ``CALIB_LEN`` tokens;
+    the oracle's objective timed beside it on a bounded sample of them."""
+    import rank_joint_qkv_b200 as q
+    from rank_joint_qkv_b200.calibrate import BetaObjective
+    device = "cuda:0"
+    torch.cuda.set_device(device)
+    w = synthetic.CONFIGS[args.config]
+    n_seq, L = CALIB_SEQS, CALIB_LEN
+    g = torch.Generator(device=device).manual_seed(w.seed * 131 + 7)
+    # leading singular triplets of a joint [W_Q W_K W_V]: orthonormal columns / rows
+    u = torch.linalg.qr(torch.randn(w.E, w.r, generator=g, device=device))[0]
+    vt = torch.linalg.qr(torch.randn(3 * w.E, w.r, generator=g, device=device))[0].T.contiguous()
+    sig = synthetic.spectrum(w.E)[: w.r]
+    x = torch.randn(n_seq * L, w.E, generator=g, device=device)
+    x[:, torch.from_numpy(synthetic.outlier_channels(w)).to(device)] *= w.outlier_scale
+    x = x.to(TORCH_DT[w.weight])
+    lens = np.full(n_seq, L, np.int64)
+    h2_m = w.h2_m if w.h2_n else 0
+    h2_q = synthetic.small_orthogonal(h2_m) if h2_m else None
+    obj = BetaObjective(u, sig, vt, x, lens, w.H, cache=w.cache, group=w.group, weight=w.weight,
+                        h2_q=h2_q, h2_m=h2_m)
+    betas = [0.5 + 0.4 * math.sin(1.7 * k) for k in range(args.warmup + args.steps)]
+    for b in betas[: args.warmup]:
+        obj(b)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    vals = [obj(b) for b in betas[args.warmup:]]
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 2 * 2.0 * n_seq * L * w.E * w.r     # the two full prefills dominate
+    line = {"metric": "beta-search objective evaluations/s (calibration latents quantised, decode-step outputs)",
+            "value": 1.0 / dt, "unit": "evaluations/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "dtype": w.weight, "data": "synthetic",
+            "config": {"workload": w.name, "E": w.E, "H": w.H, "r": w.r, "cache": w.cache,
+                       "h2": f"H_{w.r // h2_m} x Q_{h2_m} folded" if h2_m else None,
+                       "calibration": f"{n_seq} sequences x {L} tokens"},
+            "timing": "host wall clock per evaluation, including the two B x E outputs read back",
+            "prefill_flop_per_step": flops, "objective_sample": vals[:3],
+            "status": obj.status_word()}
+    # the oracle on a bounded sample: the same objective for a few sequences
+    from oracle import beta_ref as br
+    k = 2
+    u64, vt64 = u.double().cpu().numpy(), vt.double().cpu().numpy()
+    s_full = np.asarray(sig, np.float64)
+    xs = [x[i * L:(i + 1) * L].float().cpu().numpy().astype(np.float64) for i in range(k)]
+    h2 = None
+    if h2_m:
+        from oracle import qsvd_ref as ref
+        h2 = ref.h2_matrix(w.r // h2_m, h2_q)
+    t0 = time.perf_counter()
+    br.calibration_objective(u64, s_full, vt64, w.r, 0.5, xs, lens[:k], w.H,
+                             bits=4 if w.cache == "i4" else 8, group=w.group, weight=w.weight, h2=h2)
+    cdt = (time.perf_counter() - t0) * n_seq / k
+    line["cpu_baseline"] = {"value": 1.0 / cdt, "unit": "evaluations/s", "cores": torch.get_num_threads(),
+                            "kind": "oracle",
+                            "sample": f"{k} of {n_seq} calibration sequences, scaled by {n_seq // k}"}
+    return line
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -595,6 +659,8 @@ def main():
     ap.add_argument("--out-proj", choices=["none", "chain", "fold"], default="none",
                     help="apply the layer's output projection W_O in the combine (chain: V-up then "
                          "W_O; fold: W^u_v folded into W_O per head)")
+    ap.add_argument("--beta-search", action="store_true",
+                    help="time one evaluation of the split-exponent calibration objective per step")
     ap.add_argument("--prefill", action="store_true",
                     help="time qsvd_prefill_latent over the workload's whole cache instead of a decode step")
     ap.add_argument("--eager", action="store_true",
@@ -608,6 +674,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.prefill:
         line = run_prefill(args)
+    elif args.beta_search:
+        line = run_beta(args)
     elif args.impl == "reference":
         line = run_reference(args, rank, world)
     else:

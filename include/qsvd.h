@@ -247,6 +247,28 @@ qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const void* packed,
                                       void* stream);
 
 /*
+ * qsvd_split_factors -- the rank-r factors for one split of the singular
+ * values between the down- and the up-projection (QSVD paper notes, 关键设计:
+ * the latent is X U_r Sigma_r^beta; 核心创新: beta is fitted on calibration
+ * data): W^d = U_r diag(a), [W^u_q W^u_k W^u_v] = diag(b) V_r^T, each entry
+ * one float32 product rounded once to weight_dtype.  For a split exponent
+ * beta the caller passes a_j = sigma_j^beta, b_j = sigma_j^(1 - beta).
+ *   u      device, E x r float32 row-major: the first r left singular vectors.
+ *   vt     device, r x 3E float32 row-major: the first r right singular
+ *          vectors of [W_Q W_K W_V] (columns 0..E-1 belong to W_Q, E..2E-1
+ *          to W_K, 2E..3E-1 to W_V).
+ *   a, b   device, r float32 each.
+ *   wd     device, E x r, weight_dtype (written).
+ *   wuq, wuk, wuv  device, r x E each, weight_dtype (written); the inputs
+ *          of qsvd_prepare_weights.
+ * Stream-ordered; nothing is allocated.
+ * Errors: INVALID_ARG (NULL pointer, bad dims), CUDA.
+ */
+qsvd_status qsvd_split_factors(const qsvd_dims* dims, const float* u, const float* vt,
+                               const float* a, const float* b, void* wd, void* wuq, void* wuk,
+                               void* wuv, void* stream);
+
+/*
  * qsvd_prepare_out_proj -- add the output projection W_O to a packed buffer
  * that qsvd_prepare_weights filled with the same dims (dims->out_proj CHAIN
  * or FOLD; qsvd_prepare_weights reports the size with room for it).

@@ -62,6 +62,7 @@ _sigs = {
     "qsvd_append_latent_static": [_D, _P, _P, _P, _P, _P, _P, _P, _P],
     "qsvd_prefill_latent": [_D, _P, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P],
     "qsvd_prepare_out_proj": [_D, _P, _P, ctypes.c_size_t, _P],
+    "qsvd_split_factors": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -148,6 +149,15 @@ def qsvd_prepare_out_proj(dims: qsvd_dims, wo, packed, stream=None):
     _check(_lib.qsvd_prepare_out_proj(ctypes.byref(dims), _ptr(wo), _ptr(packed),
                                       packed.numel() * packed.element_size(), _stream(stream)),
            "qsvd_prepare_out_proj")
+
+
+def qsvd_split_factors(dims: qsvd_dims, u, vt, a, b, wd, wuq, wuk, wuv, stream=None):
+    """Fill wd (E x r) and wuq/wuk/wuv (r x E), weight-dtype device tensors,
+    with U diag(a) and diag(b) V^T (u: E x r, vt: r x 3E, a, b: r; float32
+    device tensors)."""
+    _check(_lib.qsvd_split_factors(ctypes.byref(dims), _ptr(u), _ptr(vt), _ptr(a), _ptr(b), _ptr(wd),
+                                   _ptr(wuq), _ptr(wuk), _ptr(wuv), _stream(stream)),
+           "qsvd_split_factors")
 
 
 def append_workspace_bytes(dims: qsvd_dims) -> int:

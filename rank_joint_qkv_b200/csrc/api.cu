@@ -191,6 +191,19 @@ qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd, const vo
   return QSVD_OK;
 }
 
+qsvd_status qsvd_split_factors(const qsvd_dims* dims, const float* u, const float* vt,
+                               const float* a, const float* b, void* wd, void* wuq, void* wuk,
+                               void* wuv, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  if (!u || !vt || !a || !b || !wd || !wuq || !wuk || !wuv)
+    return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  cudaError_t e = launch_split_factors(*dims, u, vt, a, b, wd, wuq, wuk, wuv,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "split_factors");
+  return QSVD_OK;
+}
+
 qsvd_status qsvd_prepare_out_proj(const qsvd_dims* dims, const void* wo, void* packed,
                                   size_t packed_bytes, void* stream) {
   qsvd_status st = validate(dims);

@@ -286,6 +286,10 @@ cudaError_t launch_append(const qsvd_dims& d, const void* x, const void* wd,
 cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
                            const void* wuk, const void* wuv, const float* h2q_host,
                            void* packed, const PackedLayout& L, cudaStream_t s);
+// Factors of one singular-value split: W^d = U diag(a), W^u = diag(b) V^T.
+cudaError_t launch_split_factors(const qsvd_dims& d, const float* u, const float* vt, const float* a,
+                                 const float* b, void* wd, void* wuq, void* wuk, void* wuv,
+                                 cudaStream_t s);
 // Output-projection section of the packed buffer: W_O copied (CHAIN) or the
 // per-head fold F = W^u_{v,h} W_{O,h} (FOLD); W^u_v read from the buffer.
 cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* packed,

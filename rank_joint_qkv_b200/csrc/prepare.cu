@@ -5,6 +5,7 @@
 // Y = (X H1^T)(H1 W^d H2^T)(H2 W^u)), stores W^u_k transposed for the rotary
 // tensor-core kernel and a float32 cos/sin table whose angles are formed in
 // float64 (positions up to 32k lose ~2^-9 rad if formed in float32).
+#include <algorithm>
 #include <cmath>
 
 #include "internal.cuh"
@@ -220,6 +221,55 @@ cudaError_t launch_prepare(const qsvd_dims& d, const void* wd, const void* wuq,
     case QSVD_F32: return prepare_t<float>(d, h2q_host, P, L, s);
     case QSVD_F16: return prepare_t<__half>(d, h2q_host, P, L, s);
     case QSVD_BF16: return prepare_t<__nv_bfloat16>(d, h2q_host, P, L, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+namespace {
+
+// wd[e][j] = u[e][j] a[j] (E x r); wu_k[j][n] = b[j] vt[j][k E + n] for
+// k = q, k, v (r x E each).  Grid-stride over the 4 r E outputs.
+template <typename WT>
+__global__ void __launch_bounds__(256)
+k_split_factors(const float* __restrict__ u, const float* __restrict__ vt, const float* __restrict__ a,
+                const float* __restrict__ b, WT* __restrict__ wd, WT* __restrict__ wuq, WT* __restrict__ wuk,
+                WT* __restrict__ wuv, int E, int r) {
+  const size_t m = size_t(E) * r;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < 4 * m;
+       i += size_t(gridDim.x) * blockDim.x) {
+    if (i < m) {
+      wd[i] = dev::from_f<WT>(u[i] * a[i % r]);
+    } else {
+      const size_t t = i - m;
+      const int k = int(t / m);              // 0: q, 1: k, 2: v
+      const size_t rem = t % m;
+      const int j = int(rem / E), n = int(rem % E);
+      WT* dst = k == 0 ? wuq : (k == 1 ? wuk : wuv);
+      dst[rem] = dev::from_f<WT>(b[j] * vt[size_t(j) * 3 * E + size_t(k) * E + n]);
+    }
+  }
+}
+
+template <typename WT>
+cudaError_t split_factors_t(const qsvd_dims& d, const float* u, const float* vt, const float* a,
+                            const float* b, void* wd, void* wuq, void* wuk, void* wuv, cudaStream_t s) {
+  const size_t n = size_t(4) * d.E * d.r;
+  const unsigned blocks = unsigned(std::min<size_t>((n + 255) / 256, 148 * 16));
+  k_split_factors<WT><<<blocks, 256, 0, s>>>(u, vt, a, b, static_cast<WT*>(wd), static_cast<WT*>(wuq),
+                                             static_cast<WT*>(wuk), static_cast<WT*>(wuv), d.E, d.r);
+  note_launch();
+  return check_launch();
+}
+
+}  // namespace
+
+cudaError_t launch_split_factors(const qsvd_dims& d, const float* u, const float* vt, const float* a,
+                                 const float* b, void* wd, void* wuq, void* wuk, void* wuv,
+                                 cudaStream_t s) {
+  switch (d.weight_dtype) {
+    case QSVD_F32: return split_factors_t<float>(d, u, vt, a, b, wd, wuq, wuk, wuv, s);
+    case QSVD_F16: return split_factors_t<__half>(d, u, vt, a, b, wd, wuq, wuk, wuv, s);
+    case QSVD_BF16: return split_factors_t<__nv_bfloat16>(d, u, vt, a, b, wd, wuq, wuk, wuv, s);
     default: return cudaErrorInvalidValue;
   }
 }

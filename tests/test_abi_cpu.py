@@ -230,3 +230,11 @@ def test_out_proj_refused_on_host():
     d = _dims(out_proj="chain")
     assert q._lib.qsvd_prepare_out_proj(ctypes.byref(d), fake, fake, 256, None) == \
         q.QSVD_ERR_WORKSPACE
+
+
+def test_split_factors_pointers_checked_on_host():
+    d = _dims()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the NULL check fails first
+    st = q._lib.qsvd_split_factors(ctypes.byref(d), fake, fake, fake, None, fake, fake, fake, fake, None)
+    assert st == q.QSVD_ERR_INVALID_ARG
+    assert b"NULL" in q._lib.qsvd_last_error()
