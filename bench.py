@@ -611,6 +611,57 @@ def run_beta(args):
     return line
 
 
+def run_per_head(args):
+    """qsvd_decode_attn_per_head on the workload's shapes with per-head key
+    and value latents of rank ``--per-head-rank``: K launches timed with
+    CUDA events; HBM figure = latent bytes per launch / launch time."""
+    import rank_joint_qkv_b200 as q
+    device = "cuda:0"
+    torch.cuda.set_device(device)
+    w = synthetic.CONFIGS[args.config]
+    r = args.per_head_rank
+    cache = w.cache if w.cache in ("f16", "bf16", "f32") else "f16"
+    wt = TORCH_DT[w.weight]
+    g = torch.Generator(device=device).manual_seed(w.seed * 17 + 3)
+    lat = torch.empty((w.B, w.H, w.L, r), dtype=TORCH_DT[cache], device=device)
+    lat_v = torch.empty_like(lat)
+    for t in (lat, lat_v):
+        for b in range(w.B):   # per sequence keeps the fp32 temporary small
+            t[b].copy_(torch.randn((w.H, w.L, r), generator=g, device=device))
+    bk = (torch.randn((w.H, r, w.d_h), generator=g, device=device) / math.sqrt(r)).to(wt)
+    bv = (torch.randn((w.H, r, w.d_h), generator=g, device=device) / math.sqrt(r)).to(wt)
+    qv = torch.randn((w.B, w.E), generator=g, device=device)
+    lens = torch.full((w.B,), w.L, dtype=torch.int32, device=device)
+    dims = q.make_dims(w.E, w.H, w.d_h, r, w.B, w.L, cache=cache, weight=w.weight)
+    out = torch.empty((w.B, w.E), dtype=torch.float32, device=device)
+    ws = torch.empty(q.per_head_workspace_bytes(dims), dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        q.qsvd_decode_attn_per_head(dims, bk, bv, qv, lat, lat_v, lens, out, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = q.kernel_launches()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            q.qsvd_decode_attn_per_head(dims, bk, bv, qv, lat, lat_v, lens, out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    lat_b = 2.0 * lat.numel() * lat.element_size()
+    hbm, _, _, kind = measured_peaks()
+    gbs = lat_b / (ms / 1e3) / 1e9
+    return {"metric": "per-head latent decode KV-tokens/s (key and value latents per head)",
+            "value": w.B * w.L / (ms / 1e3), "unit": "KV-tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": cache,
+            "data": "synthetic",
+            "config": {"workload": w.name + "-per-head", "E": w.E, "H": w.H, "d_h": w.d_h, "r_per_head": r,
+                       "batch": w.B, "kv_len": w.L, "cache": cache, "weights": w.weight},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": None, "kernel": "qsvd_decode_attn_per_head (3 kernels)",
+                         "peak_kind": kind, "bytes_per_launch": lat_b},
+            "gpu_launches": q.kernel_launches() - n0, "clocks": clk.summary()}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -659,6 +710,8 @@ def main():
     ap.add_argument("--out-proj", choices=["none", "chain", "fold"], default="none",
                     help="apply the layer's output projection W_O in the combine (chain: V-up then "
                          "W_O; fold: W^u_v folded into W_O per head)")
+    ap.add_argument("--per-head-rank", type=int, default=0,
+                    help="time the per-head latent decode (key and value latents of this rank per head)")
     ap.add_argument("--beta-search", action="store_true",
                     help="time one evaluation of the split-exponent calibration objective per step")
     ap.add_argument("--prefill", action="store_true",
@@ -676,6 +729,8 @@ def main():
         line = run_prefill(args)
     elif args.beta_search:
         line = run_beta(args)
+    elif args.per_head_rank:
+        line = run_per_head(args)
     elif args.impl == "reference":
         line = run_reference(args, rank, world)
     else:

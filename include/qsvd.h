@@ -338,6 +338,37 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
                                 void* workspace, int num_splits,
                                 const int32_t* lengths, void* out, void* stream);
 
+/*
+ * qsvd_decode_attn_per_head -- decode-step attention over per-head latents
+ * (WSVD digest, Method, per-head SVD §3.1, fused kernel §3.4).  Head h keeps
+ * its own key latent C_{Kh} = X A_{Kh} and value latent C_{Vh} = X A_{Vh}
+ * (L x r each; dims->r is the per-head rank) with W_{Kh} = A_{Kh} B_{Kh},
+ * W_{Vh} = A_{Vh} B_{Vh}.  With tau = dims->softmax_scale (<= 0: 1/sqrt(d_h)):
+ *   qt_h = tau B_{Kh} q_h,  s_t = C_{Kh,t} . qt_h,  p = softmax(s),
+ *   o_h = (p^T C_{Vh}) B_{Vh}.
+ * No rotary embedding (dims->rope must be 0).  Computed in float32 on CUDA
+ * cores, 256 tokens per split CTA, chunks merged in the log2 domain.
+ *   bk, bv     device, H x r x d_h each, weight_dtype (F32, F16 or BF16):
+ *              B_{Kh} and B_{Vh} stacked by head.
+ *   q          device, B x E float32: the query (head h in columns
+ *              h d_h .. h d_h + d_h - 1).
+ *   ck, cv     device, B x H x max_len x r each, cache_dtype (F32, F16 or
+ *              BF16): rows 0 .. len_b - 1 of every head are read.
+ *   lengths    device, B int32; clamped to [0, max_len] and flagged
+ *              (QSVD_STATUS_LEN_CLAMPED); len 0 gives a zero output row.
+ *   workspace  device scratch, 16-byte aligned, or NULL to query the size
+ *              into *workspace_bytes (in: capacity).  Its first int32 is the
+ *              status word.
+ *   out        device, B x E, out_dtype.
+ * Stream-ordered; nothing is allocated.
+ * Errors: INVALID_ARG, UNSUPPORTED (rotary mode, int caches, online H2, an
+ * output projection, max_len beyond ~50 M tokens), WORKSPACE, CUDA.
+ */
+qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, const void* bv,
+                                      const float* q, const void* ck, const void* cv,
+                                      const int32_t* lengths, void* workspace,
+                                      size_t* workspace_bytes, void* out, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* qsvd_status_string(qsvd_status s);
 

@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "internal.cuh"
+#include "wsvd.cuh"
 
 namespace qsvd {
 
@@ -405,6 +406,33 @@ qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed, const fl
   if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
   return decode_impl(*dims, packed, qin, qin_is_latent, cache, scales, lengths, num_splits,
                      workspace, workspace_bytes, out, phases, static_cast<cudaStream_t>(stream));
+}
+
+qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, const void* bv,
+                                      const float* q, const void* ck, const void* cv,
+                                      const int32_t* lengths, void* workspace, size_t* workspace_bytes,
+                                      void* out, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  if (d.rope) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no rotary mode");
+  if (cache_is_int(d)) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: F32, F16 or BF16 caches");
+  if (d.h2 || d.out_proj != QSVD_OUT_PROJ_NONE)
+    return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no online H2, no output projection");
+  const WsvdLayout W = wsvd_layout(d);
+  if ((size_t(W.S) + d.r + 4) * 4 > 227 * 1024)
+    return fail(QSVD_ERR_UNSUPPORTED, "max_len too large for the per-head merge");
+  if (!workspace) { *workspace_bytes = W.total; return QSVD_OK; }
+  if (*workspace_bytes < W.total)
+    return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, W.total);
+  if (!bk || !bv || !q || !ck || !cv || !lengths || !out)
+    return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(workspace)) return fail(QSVD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  cudaError_t e = launch_wsvd_decode(d, bk, bv, q, ck, cv, lengths, score_scale_log2(d), workspace, W, out,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attn_per_head");
+  return QSVD_OK;
 }
 
 qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed, void* workspace,

@@ -1,0 +1,143 @@
+"""Host-side checks of the per-head latent decode (qsvd_decode_attn_per_head),
+no GPU: refusals, the workspace size, and the index arithmetic of its three
+kernels replayed on the CPU for every CTA and thread of small and ragged
+launches (every access inside its buffer, every valid token of every head
+read exactly once, every chunk the merge reads written by the split).
+
+The replay restates the kernels' index formulas (split_wsvd.cu); it checks
+where they point, not what they compute.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import rank_joint_qkv_b200 as q
+
+CHUNK, T = 256, 128
+
+
+def _dims(**kw):
+    base = dict(E=512, H=4, d_h=128, r=64, batch=3, max_len=700)
+    base.update(kw)
+    opts = {k: base.pop(k) for k in list(base) if k not in ("E", "H", "d_h", "r", "batch", "max_len")}
+    return q.make_dims(base["E"], base["H"], base["d_h"], base["r"], base["batch"], base["max_len"], **opts)
+
+
+def _align(n):
+    return (n + 255) // 256 * 256
+
+
+def _layout(B, H, r, max_len):
+    S = (max_len + CHUNK - 1) // CHUNK
+    o = 0
+    hdr = o; o = _align(o + 16)
+    qt = o; o = _align(o + B * H * r * 4)
+    m = o; o = _align(o + B * H * S * 4)
+    l_ = o; o = _align(o + B * H * S * 4)
+    z = o; o = _align(o + B * H * S * r * 4)
+    return dict(S=S, hdr=hdr, qt=qt, m=m, l=l_, z=z, total=o)
+
+
+@pytest.mark.parametrize("shape", [dict(), dict(r=32, max_len=256), dict(r=96, max_len=1000),
+                                   dict(r=256, batch=1, max_len=5000)])
+def test_workspace_size_matches_layout(shape):
+    d = _dims(**shape)
+    want = _layout(d.batch, d.H, d.r, d.max_len)["total"]
+    assert q.per_head_workspace_bytes(d) == want
+
+
+@pytest.mark.parametrize("bad,status", [(dict(rope=True), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(cache="i4", r=128), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(out_proj="chain"), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(h2=True, h2_m=2), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(r=48), q.QSVD_ERR_INVALID_ARG)])
+def test_refusals_on_host(bad, status):
+    with pytest.raises(q.QsvdError) as e:
+        q.per_head_workspace_bytes(_dims(**bad))
+    assert e.value.status == status
+
+
+def test_null_pointers_and_small_workspace():
+    d = _dims()
+    n = ctypes.c_size_t(64)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the checks fail first
+    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake,
+                                          ctypes.byref(n), fake, None)
+    assert st == q.QSVD_ERR_WORKSPACE
+    n = ctypes.c_size_t(1 << 30)
+    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), None, fake, fake, fake, fake, fake, fake,
+                                          ctypes.byref(n), fake, None)
+    assert st == q.QSVD_ERR_INVALID_ARG
+
+
+def _replay(B, H, d_h, r, max_len, lengths):
+    """Replay the three launches' index arithmetic; return the read counts
+    of every latent row (b, h, t)."""
+    E = H * d_h
+    W = _layout(B, H, r, max_len)
+    S = W["S"]
+    n_cache = B * H * max_len * r
+    rows_read = np.zeros((B, H, max_len), np.int64)
+    written = np.zeros(B * H * S, bool)
+    # absorb: grid (H, B); q reads and qt writes
+    for b in range(B):
+        for h in range(H):
+            qrow = (b * H + h) * d_h
+            assert 0 <= qrow and qrow + d_h <= B * E
+            assert (b * H + h) * r + r <= B * H * r
+            assert h * r * d_h + r * d_h <= H * r * d_h          # B_K rows of head h
+    # split: grid (S, H, B)
+    ng = T // r if (r < T and T % r == 0) else 1
+    smem = r + CHUNK + 4 + ng * r
+    assert ng * r <= max(r, T)
+    for b in range(B):
+        ln = min(max(int(lengths[b]), 0), max_len)
+        for h in range(H):
+            for sp in range(S):
+                t0 = sp * CHUNK
+                if t0 >= ln:
+                    continue
+                n = min(CHUNK, ln - t0)
+                bh = b * H + h
+                kb = (bh * max_len + t0) * r
+                for t in range(n):                         # score rows (warp per row)
+                    lo, hi = kb + t * r, kb + t * r + r
+                    assert 0 <= lo and hi <= n_cache
+                    rows_read[b, h, t0 + t] += 1
+                assert n <= CHUNK                           # ss[t] inside its section
+                if ng > 1:                                  # value rows by token groups
+                    for tid in range(T):
+                        g, j = tid // r, tid % r
+                        assert g * r + j < ng * r
+                        for t in range(g, n, ng):
+                            assert kb + t * r + j < n_cache
+                slot = bh * S + sp
+                assert slot < B * H * S and (slot + 1) * r <= B * H * S * r
+                written[slot] = True
+    # combine: grid (H, B); reads the chunks s < ceil(len / CHUNK)
+    for b in range(B):
+        ln = min(max(int(lengths[b]), 0), max_len)
+        su = (ln + CHUNK - 1) // CHUNK
+        assert su <= S and S + r + 4 <= 227 * 1024 // 4
+        for h in range(H):
+            base = (b * H + h) * S
+            for s in range(su):
+                assert written[base + s]
+            assert (b * H + h) * d_h + d_h <= B * E             # output row
+    return rows_read, smem
+
+
+@pytest.mark.parametrize("B,H,d_h,r,max_len,lengths", [
+    (3, 4, 128, 64, 700, [700, 1, 300]),
+    (2, 2, 64, 32, 256, [256, 255]),
+    (2, 3, 128, 96, 513, [513, 0]),
+    (1, 2, 128, 256, 1000, [777]),
+    (2, 2, 64, 128, 300, [-5, 9999]),                      # clamped to 0 and max_len
+])
+def test_index_replay(B, H, d_h, r, max_len, lengths):
+    rows, smem = _replay(B, H, d_h, r, max_len, lengths)
+    for b in range(B):
+        ln = min(max(lengths[b], 0), max_len)
+        assert np.all(rows[b, :, :ln] == 1) and np.all(rows[b, :, ln:] == 0)
+    assert smem * 4 <= 227 * 1024
