@@ -346,3 +346,40 @@ def decode_folded(z: np.ndarray, f: np.ndarray) -> np.ndarray:
     z = np.asarray(z, np.float64)
     B, H, r = z.shape
     return z.reshape(B, H * r) @ np.asarray(f, np.float64)
+
+
+# --------------------------------------------------------------------------
+# Prefill attention (all prompt tokens at once, causal)
+# --------------------------------------------------------------------------
+
+def prefill_attention(c: np.ndarray, wuq, wuk, wuv, H: int, *, rope_base: Optional[float] = None,
+                      scale: Optional[float] = None) -> np.ndarray:
+    """Causal self-attention over one prompt whose latent rows are ``c``
+    (L x r): Q = C W^u_q, K = C W^u_k, V = C W^u_v rebuilt in full (QSVD
+    digest, Method, Step 1), token t attends to tokens 0..t; with rope_base
+    every query and key is rotated by its own position.  Output L x E
+    (heads concatenated)."""
+    c = np.asarray(c, np.float64)
+    wuq = np.asarray(wuq, np.float64)
+    wuk = np.asarray(wuk, np.float64)
+    wuv = np.asarray(wuv, np.float64)
+    L = c.shape[0]
+    E = wuk.shape[1]
+    d_h = E // H
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    q, k, v = c @ wuq, c @ wuk, c @ wuv
+    out = np.zeros((L, E))
+    pos = np.arange(L)
+    for h in range(H):
+        cols = slice(h * d_h, (h + 1) * d_h)
+        qh, kh = q[:, cols], k[:, cols]
+        if rope_base is not None:
+            qh, kh = rope(qh, pos, rope_base), rope(kh, pos, rope_base)
+        logits = scale * (qh @ kh.T)
+        logits[np.triu_indices(L, 1)] = -np.inf
+        logits -= logits.max(axis=1, keepdims=True)
+        p = np.exp(logits)
+        p /= p.sum(axis=1, keepdims=True)
+        out[:, cols] = p @ v[:, cols]
+    return out

@@ -416,3 +416,44 @@ def test_output_projection_permutation():
     wo[np.arange(12), perm] = 1.0
     y = ref.output_projection(o, wo)
     assert np.array_equal(y[:, perm], o)
+
+
+# ------------------------------------------------------------- prefill attention
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_prefill_last_rows_are_decode_steps(cfg):
+    """Row t of the causal prefill is the decode step of a sequence of t + 1
+    tokens whose current latent is row t (rotary: query at position t)."""
+    w = synthetic.SHRUNK[cfg]
+    case = oi.build_case(w)
+    c = case.caches[0]
+    n = c.shape[0]
+    rb = w.rope_base if w.rope else None
+    pre = ref.prefill_attention(c, case.wuq, case.wuk, case.wuv, w.H, rope_base=rb)
+    for t in (0, 1, n // 2, n - 1):
+        dec = ref.decode_materialized([c[:t + 1]], [t + 1], c[t:t + 1], case.wuq, case.wuk, case.wuv,
+                                      w.H, rope_base=rb)
+        assert np.max(np.abs(pre[t] - dec[0])) <= 1e-11 * np.max(np.abs(dec))
+
+
+def test_prefill_brute_force_loops():
+    """Scalar loops over tokens, heads and channels on a tiny case."""
+    g = np.random.default_rng(6)
+    L, r, H, d_h = 5, 6, 2, 4
+    E = H * d_h
+    c = g.standard_normal((L, r))
+    wuq, wuk, wuv = (g.standard_normal((r, E)) for _ in range(3))
+    got = ref.prefill_attention(c, wuq, wuk, wuv, H)
+    tau = 1.0 / math.sqrt(d_h)
+    for t in range(L):
+        for h in range(H):
+            qv = [sum(c[t][j] * wuq[j][h * d_h + i] for j in range(r)) for i in range(d_h)]
+            logits = []
+            for u in range(t + 1):
+                kv = [sum(c[u][j] * wuk[j][h * d_h + i] for j in range(r)) for i in range(d_h)]
+                logits.append(tau * sum(qv[i] * kv[i] for i in range(d_h)))
+            mx = max(logits)
+            ws = [math.exp(x - mx) for x in logits]
+            for i in range(d_h):
+                num = sum(ws[u] * sum(c[u][j] * wuv[j][h * d_h + i] for j in range(r)) for u in range(t + 1))
+                assert abs(got[t][h * d_h + i] - num / sum(ws)) <= 1e-12 * (1 + abs(num / sum(ws)))
