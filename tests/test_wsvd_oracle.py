@@ -80,3 +80,15 @@ def test_fold_pays_below_model_width():
     # a shared latent of rank 1536 read by all 32 heads: folding reads 8.7x more
     ratio = wr.out_proj_weight_elems(E, H, 1536, True) / (1536 * E + E * E)
     assert 8.6 < ratio < 8.8
+
+
+def test_per_head_traffic_ratio():
+    """Key Contributions: per head and step, a per-head latent moves L r
+    elements where a shared one moves L R, a ratio r / R.  LLaVA-7B shapes:
+    a shared latent of rank 1536 read for each of 32 heads against per-head
+    key and value latents of rank 64."""
+    L = 8192
+    assert wr.latent_bytes_per_head(L, 64, 2) / wr.latent_bytes_per_head(L, 1536, 2) == 64 / 1536
+    shared_reloaded = 32 * wr.latent_bytes_per_head(L, 1536, 2)
+    per_head_kv = 32 * 2 * wr.latent_bytes_per_head(L, 64, 2)
+    assert shared_reloaded == 805306368 and per_head_kv == 67108864
