@@ -352,8 +352,14 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  *              B_{Kh} and B_{Vh} stacked by head.
  *   q          device, B x E float32: the query (head h in columns
  *              h d_h .. h d_h + d_h - 1).
- *   ck, cv     device, B x H x max_len x r each, cache_dtype (F32, F16 or
- *              BF16): rows 0 .. len_b - 1 of every head are read.
+ *   ck, cv     device, cache_dtype (F32, F16 or BF16), in one of two
+ *              layouts (rows 0 .. len_b - 1 of every head are read):
+ *              QSVD_PER_HEAD_HEAD_MAJOR   B x H x max_len x r;
+ *              QSVD_PER_HEAD_TOKEN_MAJOR  B x max_len x H x r: row t of a
+ *              sequence holds every head's latent, so it is exactly the
+ *              cache row that qsvd_prefill_latent / qsvd_append_latent write
+ *              with W^d = [A_1 .. A_H] (E x H r) and rank H r.
+ *   layout     QSVD_PER_HEAD_*.
  *   lengths    device, B int32; clamped to [0, max_len] and flagged
  *              (QSVD_STATUS_LEN_CLAMPED); len 0 gives a zero output row.
  *   workspace  device scratch, 16-byte aligned, or NULL to query the size
@@ -361,12 +367,15 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  *              status word.
  *   out        device, B x E, out_dtype.
  * Stream-ordered; nothing is allocated.
- * Errors: INVALID_ARG, UNSUPPORTED (rotary mode, int caches, online H2, an
- * output projection, max_len beyond ~50 M tokens), WORKSPACE, CUDA.
+ * Errors: INVALID_ARG (also an unknown layout), UNSUPPORTED (rotary mode,
+ * int caches, online H2, an output projection, max_len beyond ~50 M
+ * tokens), WORKSPACE, CUDA.
  */
+#define QSVD_PER_HEAD_HEAD_MAJOR 0
+#define QSVD_PER_HEAD_TOKEN_MAJOR 1
 qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, const void* bv,
                                       const float* q, const void* ck, const void* cv,
-                                      const int32_t* lengths, void* workspace,
+                                      const int32_t* lengths, int layout, void* workspace,
                                       size_t* workspace_bytes, void* out, void* stream);
 
 /* Human-readable name of a status code (static string). */

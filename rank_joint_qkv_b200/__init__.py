@@ -33,6 +33,7 @@ QSVD_STATUS_LEN_CLAMPED, QSVD_STATUS_POS_OOB, QSVD_STATUS_SCALE_SAT, QSVD_STATUS
 QSVD_KERNEL_AUTO, QSVD_KERNEL_SIMT, QSVD_KERNEL_TCGEN05 = 0, 1, 2
 QSVD_KERNEL_TCGEN05_CTA, QSVD_KERNEL_TCGEN05_CLUSTER = 3, 4
 QSVD_OUT_PROJ_NONE, QSVD_OUT_PROJ_CHAIN, QSVD_OUT_PROJ_FOLD = 0, 1, 2
+QSVD_PER_HEAD_HEAD_MAJOR, QSVD_PER_HEAD_TOKEN_MAJOR = 0, 1
 OUT_PROJ_CODE = {None: QSVD_OUT_PROJ_NONE, "none": QSVD_OUT_PROJ_NONE,
                  "chain": QSVD_OUT_PROJ_CHAIN, "fold": QSVD_OUT_PROJ_FOLD}
 
@@ -63,7 +64,7 @@ _sigs = {
     "qsvd_prefill_latent": [_D, _P, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P],
     "qsvd_prepare_out_proj": [_D, _P, _P, ctypes.c_size_t, _P],
     "qsvd_split_factors": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P],
-    "qsvd_decode_attn_per_head": [_D, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
+    "qsvd_decode_attn_per_head": [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _SZ, _P, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -224,22 +225,23 @@ def qsvd_decode_attn(dims: qsvd_dims, packed, qin, qin_is_latent, cache, scales,
 
 def per_head_workspace_bytes(dims: qsvd_dims) -> int:
     n = ctypes.c_size_t(0)
-    _check(_lib.qsvd_decode_attn_per_head(ctypes.byref(dims), None, None, None, None, None, None, None,
+    _check(_lib.qsvd_decode_attn_per_head(ctypes.byref(dims), None, None, None, None, None, None, 0, None,
                                           ctypes.byref(n), None, None),
            "qsvd_decode_attn_per_head(size)")
     return n.value
 
 
 def qsvd_decode_attn_per_head(dims: qsvd_dims, bk, bv, q, ck, cv, lengths, out, workspace=None,
-                              stream=None):
-    """Decode over per-head key/value latents (ck, cv: B x H x max_len x r);
-    bk, bv: H x r x d_h; q: B x E float32.  Returns the workspace (its
-    first int32 is the status word)."""
+                              layout=QSVD_PER_HEAD_HEAD_MAJOR, stream=None):
+    """Decode over per-head key/value latents (ck, cv: B x H x max_len x r,
+    or B x max_len x H x r with layout QSVD_PER_HEAD_TOKEN_MAJOR); bk, bv:
+    H x r x d_h; q: B x E float32.  Returns the workspace (its first int32
+    is the status word)."""
     if workspace is None:
         workspace = _empty_bytes(per_head_workspace_bytes(dims), q.device)
     n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
     _check(_lib.qsvd_decode_attn_per_head(ctypes.byref(dims), _ptr(bk), _ptr(bv), _ptr(q), _ptr(ck),
-                                          _ptr(cv), _ptr(lengths), _ptr(workspace), ctypes.byref(n),
+                                          _ptr(cv), _ptr(lengths), int(layout), _ptr(workspace), ctypes.byref(n),
                                           _ptr(out), _stream(stream)),
            "qsvd_decode_attn_per_head")
     return workspace

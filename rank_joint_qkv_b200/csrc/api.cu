@@ -410,8 +410,8 @@ qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed, const fl
 
 qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, const void* bv,
                                       const float* q, const void* ck, const void* cv,
-                                      const int32_t* lengths, void* workspace, size_t* workspace_bytes,
-                                      void* out, void* stream) {
+                                      const int32_t* lengths, int layout, void* workspace,
+                                      size_t* workspace_bytes, void* out, void* stream) {
   qsvd_status st = validate(dims);
   if (st != QSVD_OK) return st;
   const qsvd_dims& d = *dims;
@@ -420,6 +420,8 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
   if (cache_is_int(d)) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: F32, F16 or BF16 caches");
   if (d.h2 || d.out_proj != QSVD_OUT_PROJ_NONE)
     return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no online H2, no output projection");
+  if (layout != QSVD_PER_HEAD_HEAD_MAJOR && layout != QSVD_PER_HEAD_TOKEN_MAJOR)
+    return fail(QSVD_ERR_INVALID_ARG, "unknown per-head latent layout %d", layout);
   const WsvdLayout W = wsvd_layout(d);
   if ((size_t(W.S) + d.r + 4) * 4 > 227 * 1024)
     return fail(QSVD_ERR_UNSUPPORTED, "max_len too large for the per-head merge");
@@ -430,7 +432,7 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
     return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
   if (!aligned16(workspace)) return fail(QSVD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   cudaError_t e = launch_wsvd_decode(d, bk, bv, q, ck, cv, lengths, score_scale_log2(d), workspace, W, out,
-                                     static_cast<cudaStream_t>(stream));
+                                     layout == QSVD_PER_HEAD_TOKEN_MAJOR, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_per_head");
   return QSVD_OK;
 }

@@ -75,11 +75,14 @@ k_wsvd_absorb(const WT* __restrict__ bk, const float* __restrict__ q, float* __r
 
 // One chunk of one (sequence, head).  grid (S, H, B).  Writes the chunk's
 // m = max s, l = sum 2^(s - m), z = sum 2^(s - m) C_V,t (log2-domain s).
+// Latent row (b, h, t) starts at ((b H + h) max_len + t) r (head-major) or
+// ((b max_len + t) H + h) r (token-major); consecutive tokens are r or H r
+// elements apart.
 template <typename CT>
 __global__ void __launch_bounds__(kT)
 k_wsvd_split(const CT* __restrict__ ck, const CT* __restrict__ cv, const float* __restrict__ qt,
              const int32_t* __restrict__ lengths, float* __restrict__ pm, float* __restrict__ pl,
-             float* __restrict__ pz, int H, int r, int max_len, int S) {
+             float* __restrict__ pz, int H, int r, int max_len, int S, int token_major) {
   extern __shared__ float sm[];
   float* qs = sm;                   // r
   float* ss = qs + r;               // kWsvdChunk scores, then weights
@@ -91,13 +94,15 @@ k_wsvd_split(const CT* __restrict__ ck, const CT* __restrict__ cv, const float* 
   if (t0 >= len) return;            // the same for every thread of the CTA
   const int n = min(kWsvdChunk, len - t0);
   const size_t bh = size_t(b) * H + h;
-  const CT* kb = ck + (bh * max_len + t0) * size_t(r);
-  const CT* vb = cv + (bh * max_len + t0) * size_t(r);
+  const size_t row0 = token_major ? (size_t(b) * max_len + t0) * H + h : bh * max_len + t0;
+  const size_t rs = token_major ? size_t(H) * r : size_t(r);   // elements between tokens
+  const CT* kb = ck + row0 * size_t(r);
+  const CT* vb = cv + row0 * size_t(r);
   for (int j = threadIdx.x; j < r; j += kT) qs[j] = qt[bh * r + j];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int t = warp; t < n; t += kT / 32) {
-    const CT* row = kb + size_t(t) * r;
+    const CT* row = kb + size_t(t) * rs;
     float acc = 0.f;
     for (int j = lane; j < r; j += 32) acc = fmaf(dev::to_f(row[j]), qs[j], acc);
     acc = warp_sum(acc);
@@ -120,7 +125,7 @@ k_wsvd_split(const CT* __restrict__ ck, const CT* __restrict__ cv, const float* 
   if (ng > 1) {
     const int g = threadIdx.x / r, j = threadIdx.x % r;
     float acc = 0.f;
-    for (int t = g; t < n; t += ng) acc = fmaf(ss[t], dev::to_f(vb[size_t(t) * r + j]), acc);
+    for (int t = g; t < n; t += ng) acc = fmaf(ss[t], dev::to_f(vb[size_t(t) * rs + j]), acc);
     zp[g * r + j] = acc;
     __syncthreads();
     for (int jj = threadIdx.x; jj < r; jj += kT) {
@@ -131,7 +136,7 @@ k_wsvd_split(const CT* __restrict__ ck, const CT* __restrict__ cv, const float* 
   } else {
     for (int j = threadIdx.x; j < r; j += kT) {
       float acc = 0.f;
-      for (int t = 0; t < n; ++t) acc = fmaf(ss[t], dev::to_f(vb[size_t(t) * r + j]), acc);
+      for (int t = 0; t < n; ++t) acc = fmaf(ss[t], dev::to_f(vb[size_t(t) * rs + j]), acc);
       zrow[j] = acc;
     }
   }
@@ -198,7 +203,7 @@ cudaError_t allow_smem(K kern, size_t bytes) {
 template <typename WT, typename CT, typename OT>
 cudaError_t wsvd_t(const qsvd_dims& d, const void* bk, const void* bv, const float* q, const void* ck,
                    const void* cv, const int32_t* lengths, float sl2, void* workspace,
-                   const WsvdLayout& W, void* out, cudaStream_t s) {
+                   const WsvdLayout& W, void* out, int token_major, cudaStream_t s) {
   uint8_t* wb = static_cast<uint8_t*>(workspace);
   int32_t* status = reinterpret_cast<int32_t*>(wb + W.hdr);
   float* qt = reinterpret_cast<float*>(wb + W.qt);
@@ -220,7 +225,8 @@ cudaError_t wsvd_t(const qsvd_dims& d, const void* bk, const void* bv, const flo
   note_launch();
   if ((e = check_launch()) != cudaSuccess) return e;
   ks<<<dim3(W.S, d.H, d.batch), kT, s_split, s>>>(static_cast<const CT*>(ck), static_cast<const CT*>(cv),
-                                                  qt, lengths, pm, pl, pz, d.H, d.r, d.max_len, W.S);
+                                                  qt, lengths, pm, pl, pz, d.H, d.r, d.max_len, W.S,
+                                                  token_major);
   note_launch();
   if ((e = check_launch()) != cudaSuccess) return e;
   kc<<<dim3(d.H, d.batch), kT, s_comb, s>>>(pm, pl, pz, static_cast<const WT*>(bv), lengths,
@@ -232,11 +238,11 @@ cudaError_t wsvd_t(const qsvd_dims& d, const void* bk, const void* bv, const flo
 template <typename WT, typename CT>
 cudaError_t wsvd_out(const qsvd_dims& d, const void* bk, const void* bv, const float* q, const void* ck,
                      const void* cv, const int32_t* lengths, float sl2, void* ws, const WsvdLayout& W,
-                     void* out, cudaStream_t s) {
+                     void* out, int tm, cudaStream_t s) {
   switch (d.out_dtype) {
-    case QSVD_F32: return wsvd_t<WT, CT, float>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
-    case QSVD_F16: return wsvd_t<WT, CT, __half>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
-    case QSVD_BF16: return wsvd_t<WT, CT, __nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
+    case QSVD_F32: return wsvd_t<WT, CT, float>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
+    case QSVD_F16: return wsvd_t<WT, CT, __half>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
+    case QSVD_BF16: return wsvd_t<WT, CT, __nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -244,11 +250,11 @@ cudaError_t wsvd_out(const qsvd_dims& d, const void* bk, const void* bv, const f
 template <typename WT>
 cudaError_t wsvd_cache(const qsvd_dims& d, const void* bk, const void* bv, const float* q, const void* ck,
                        const void* cv, const int32_t* lengths, float sl2, void* ws, const WsvdLayout& W,
-                       void* out, cudaStream_t s) {
+                       void* out, int tm, cudaStream_t s) {
   switch (d.cache_dtype) {
-    case QSVD_F32: return wsvd_out<WT, float>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
-    case QSVD_F16: return wsvd_out<WT, __half>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
-    case QSVD_BF16: return wsvd_out<WT, __nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, s);
+    case QSVD_F32: return wsvd_out<WT, float>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
+    case QSVD_F16: return wsvd_out<WT, __half>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
+    case QSVD_BF16: return wsvd_out<WT, __nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, ws, W, out, tm, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -257,12 +263,14 @@ cudaError_t wsvd_cache(const qsvd_dims& d, const void* bk, const void* bv, const
 
 cudaError_t launch_wsvd_decode(const qsvd_dims& d, const void* bk, const void* bv, const float* q,
                                const void* ck, const void* cv, const int32_t* lengths, float sl2,
-                               void* workspace, const WsvdLayout& W, void* out, cudaStream_t s) {
+                               void* workspace, const WsvdLayout& W, void* out, int token_major,
+                               cudaStream_t s) {
+  const int tm = token_major;
   switch (d.weight_dtype) {
-    case QSVD_F32: return wsvd_cache<float>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, s);
-    case QSVD_F16: return wsvd_cache<__half>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, s);
+    case QSVD_F32: return wsvd_cache<float>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, tm, s);
+    case QSVD_F16: return wsvd_cache<__half>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, tm, s);
     case QSVD_BF16:
-      return wsvd_cache<__nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, s);
+      return wsvd_cache<__nv_bfloat16>(d, bk, bv, q, ck, cv, lengths, sl2, workspace, W, out, tm, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -34,6 +34,7 @@ inline WsvdLayout wsvd_layout(const qsvd_dims& d) {
 // o_h = z_h B_{Vh}).
 cudaError_t launch_wsvd_decode(const qsvd_dims& d, const void* bk, const void* bv, const float* q,
                                const void* ck, const void* cv, const int32_t* lengths, float sl2,
-                               void* workspace, const WsvdLayout& W, void* out, cudaStream_t s);
+                               void* workspace, const WsvdLayout& W, void* out, int token_major,
+                               cudaStream_t s);
 
 }  // namespace qsvd

@@ -53,10 +53,13 @@ def _case(E, H, r, lengths, cache, weight):
     return dims, dev, want
 
 
-def _run(dims, dev, out_dtype=torch.float32):
+def _run(dims, dev, out_dtype=torch.float32, layout=q.QSVD_PER_HEAD_HEAD_MAJOR):
     out = torch.full((dims.batch, dims.E), float("nan"), dtype=out_dtype, device="cuda")
-    ws = q.qsvd_decode_attn_per_head(dims, dev["bk"], dev["bv"], dev["q"], dev["ck"], dev["cv"],
-                                     dev["lengths"], out)
+    ck, cv = dev["ck"], dev["cv"]
+    if layout == q.QSVD_PER_HEAD_TOKEN_MAJOR:   # B x H x L x r -> B x L x H x r
+        ck, cv = ck.transpose(1, 2).contiguous(), cv.transpose(1, 2).contiguous()
+    ws = q.qsvd_decode_attn_per_head(dims, dev["bk"], dev["bv"], dev["q"], ck, cv,
+                                     dev["lengths"], out, layout=layout)
     torch.cuda.synchronize()
     return out.float().cpu().numpy(), int(ws[:4].view(torch.int32).item())
 
@@ -73,6 +76,9 @@ def test_matches_oracle(cuda_ok, E, H, r, lengths, cache, weight):
     got, status = _run(dims, dev)
     assert status == 0
     assert rel_err(got, want) <= TOL
+    # the token-major layout reads the same rows: the same bits
+    got_tm, status = _run(dims, dev, layout=q.QSVD_PER_HEAD_TOKEN_MAJOR)
+    assert status == 0 and np.array_equal(got_tm, got)
 
 
 def test_empty_and_clamped_lengths(cuda_ok):
@@ -97,3 +103,47 @@ def test_out_dtypes_round_the_float32_result(cuda_ok):
         got, _ = _run(dims, dev, td)
         want = oi.from_device_dtype(oi.to_device_dtype(ref32, dt), dt)
         assert np.array_equal(got, want.astype(np.float32))
+
+
+def test_latents_from_prefill(cuda_ok):
+    """Per-head key and value latents written by qsvd_prefill_latent (W^d =
+    [A_1 .. A_H], rank H r, one cache row per token holding every head) and
+    read by the per-head decode in the token-major layout."""
+    E, H, r, lengths = 512, 4, 64, [300, 1, 513]
+    d_h = E // H
+    w = synthetic.replace(synthetic.SHRUNK[1], E=E, H=H, d_h=d_h, r=r, B=len(lengths), L=max(lengths))
+    wq, wk, wv = synthetic.qkv_weights(w)
+    rnd = lambda m: oi.from_device_dtype(oi.to_device_dtype(m, "f16"), "f16")
+    fk = [(rnd(a), rnd(b)) for a, b in wr.per_head_factors(wk, H, r)]
+    fv = [(rnd(a), rnd(b)) for a, b in wr.per_head_factors(wv, H, r)]
+    max_len = max(lengths) + 5
+    xs = [rnd(synthetic.sequence_activations(w, b, n)) for b, n in enumerate(lengths)]
+    ck = [rnd(wr.per_head_latents(x, fk)) for x in xs]          # H x len x r, rounded like the cache
+    cv = [rnd(wr.per_head_latents(x, fv)) for x in xs]
+    qv = np.stack([(x[-1] @ wq.astype(np.float64)).astype(np.float32) for x in xs])
+    want = wr.decode_absorbed(ck, cv, np.asarray(lengths), qv.astype(np.float64), fk, fv)
+
+    R = H * r
+    pdims = q.make_dims(E, H, d_h, R, len(lengths), max_len, cache="f16", weight="f16")
+    x_all = torch.from_numpy(np.concatenate(xs).astype(np.float16)).cuda()
+    rows = torch.from_numpy(np.concatenate([b * max_len + np.arange(n) for b, n in enumerate(lengths)])
+                            .astype(np.int32)).cuda()
+    zeros = torch.zeros((R, E), dtype=torch.float16, device="cuda")
+    caches = []
+    for fac in (fk, fv):
+        a_all = torch.from_numpy(np.concatenate([a for a, _ in fac], axis=1).astype(np.float16)).cuda()
+        packed = q.qsvd_prepare_weights(pdims, a_all, zeros, zeros, zeros)
+        cache = torch.full((len(lengths), max_len, R), PAD, dtype=torch.float16, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        q.qsvd_prefill_latent(pdims, packed, x_all, rows, cache, status=st)
+        caches.append(cache)
+    dims = q.make_dims(E, H, d_h, r, len(lengths), max_len, cache="f16", weight="f16")
+    bk = torch.from_numpy(np.stack([b for _, b in fk]).astype(np.float16)).cuda()
+    bv = torch.from_numpy(np.stack([b for _, b in fv]).astype(np.float16)).cuda()
+    out = torch.full((len(lengths), E), float("nan"), dtype=torch.float32, device="cuda")
+    ws = q.qsvd_decode_attn_per_head(dims, bk, bv, torch.from_numpy(qv).cuda(), caches[0], caches[1],
+                                     torch.tensor(lengths, dtype=torch.int32, device="cuda"), out,
+                                     layout=q.QSVD_PER_HEAD_TOKEN_MAJOR)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and int(ws[:4].view(torch.int32).item()) == 0
+    assert rel_err(out.cpu().numpy(), want) <= TOL

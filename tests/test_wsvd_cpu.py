@@ -62,16 +62,19 @@ def test_null_pointers_and_small_workspace():
     d = _dims()
     n = ctypes.c_size_t(64)
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the checks fail first
-    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake,
+    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), fake, fake, fake, fake, fake, fake, 0, fake,
                                           ctypes.byref(n), fake, None)
     assert st == q.QSVD_ERR_WORKSPACE
     n = ctypes.c_size_t(1 << 30)
-    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), None, fake, fake, fake, fake, fake, fake,
+    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), None, fake, fake, fake, fake, fake, 0, fake,
                                           ctypes.byref(n), fake, None)
     assert st == q.QSVD_ERR_INVALID_ARG
+    st = q._lib.qsvd_decode_attn_per_head(ctypes.byref(d), fake, fake, fake, fake, fake, fake, 2, None,
+                                          ctypes.byref(n), fake, None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"layout" in q._lib.qsvd_last_error()
 
 
-def _replay(B, H, d_h, r, max_len, lengths):
+def _replay(B, H, d_h, r, max_len, lengths, token_major=False):
     """Replay the three launches' index arithmetic; return the read counts
     of every latent row (b, h, t)."""
     E = H * d_h
@@ -100,10 +103,16 @@ def _replay(B, H, d_h, r, max_len, lengths):
                     continue
                 n = min(CHUNK, ln - t0)
                 bh = b * H + h
-                kb = (bh * max_len + t0) * r
+                row0 = (b * max_len + t0) * H + h if token_major else bh * max_len + t0
+                rs = H * r if token_major else r
+                kb = row0 * r
                 for t in range(n):                         # score rows (warp per row)
-                    lo, hi = kb + t * r, kb + t * r + r
+                    lo, hi = kb + t * rs, kb + t * rs + r
                     assert 0 <= lo and hi <= n_cache
+                    # the row this is in the caller's layout
+                    want = ((b * max_len + t0 + t) * H + h) * r if token_major else \
+                        ((b * H + h) * max_len + t0 + t) * r
+                    assert lo == want
                     rows_read[b, h, t0 + t] += 1
                 assert n <= CHUNK                           # ss[t] inside its section
                 if ng > 1:                                  # value rows by token groups
@@ -111,7 +120,7 @@ def _replay(B, H, d_h, r, max_len, lengths):
                         g, j = tid // r, tid % r
                         assert g * r + j < ng * r
                         for t in range(g, n, ng):
-                            assert kb + t * r + j < n_cache
+                            assert kb + t * rs + j < n_cache
                 slot = bh * S + sp
                 assert slot < B * H * S and (slot + 1) * r <= B * H * S * r
                 written[slot] = True
@@ -135,8 +144,9 @@ def _replay(B, H, d_h, r, max_len, lengths):
     (1, 2, 128, 256, 1000, [777]),
     (2, 2, 64, 128, 300, [-5, 9999]),                      # clamped to 0 and max_len
 ])
-def test_index_replay(B, H, d_h, r, max_len, lengths):
-    rows, smem = _replay(B, H, d_h, r, max_len, lengths)
+@pytest.mark.parametrize("token_major", [False, True])
+def test_index_replay(B, H, d_h, r, max_len, lengths, token_major):
+    rows, smem = _replay(B, H, d_h, r, max_len, lengths, token_major)
     for b in range(B):
         ln = min(max(lengths[b], 0), max_len)
         assert np.all(rows[b, :, :ln] == 1) and np.all(rows[b, :, ln:] == 0)
