@@ -26,6 +26,7 @@ import statistics
 import subprocess
 import sys
 import time
+from typing import Optional
 
 import numpy as np
 import torch
@@ -46,10 +47,20 @@ ROW_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "i8": 1, "i4": 0.5}
 # inputs
 # ---------------------------------------------------------------------------
 
-def bench_inputs(cfg: int, device: str, rank: int = 0):
+def workload(cfg: int, cache: Optional[str] = None):
+    """Configuration ``cfg``; ``cache`` overrides its latent type (the int4
+    workload also runs with an int8 latent: same shapes, 780 bytes a token)."""
+    w = synthetic.CONFIGS[cfg]
+    if cache and cache != w.cache:
+        w = synthetic.replace(w, cache=cache, name=w.name.replace(w.cache.replace("i", "int"),
+                                                                  cache.replace("i", "int")))
+    return w
+
+
+def bench_inputs(cfg: int, device: str, rank: int = 0, cache: Optional[str] = None):
     """Device-resident synthetic inputs of configuration ``cfg`` (the same
     recipe on every rank, seeded by rank)."""
-    w = synthetic.CONFIGS[cfg]
+    w = workload(cfg, cache)
     lens = synthetic.lengths(w)
     max_len = int(lens.max())
     cs, _ = synthetic.direct_channel_scales(w)

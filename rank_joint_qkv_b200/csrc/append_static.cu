@@ -8,6 +8,7 @@
 // file-scope device array that every GPU loading the library keeps until the
 // process exits.
 #include <cmath>
+#include <cstdio>
 #include <mutex>
 
 #include "internal.cuh"
@@ -41,6 +42,8 @@ cudaError_t scratch_on_current_device(float** out) {
   return cudaSuccess;
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 }  // namespace
 }  // namespace qsvd
 
@@ -59,12 +62,20 @@ extern "C" qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const vo
   if (st != QSVD_OK) return st;
   const int KS = append_ksplit(d);
   const size_t need = size_t(KS) * d.batch * d.r;
-  if (need > kStaticScratchFloats)
-    return set_error(QSVD_ERR_WORKSPACE,
-                     "qsvd_append_latent_static: ceil(E / 128) * batch * r exceeds the "
-                     "1048576-float static scratch; use qsvd_append_latent with a workspace");
+  if (need > kStaticScratchFloats) {
+    char msg[256];
+    snprintf(msg, sizeof(msg),
+             "qsvd_append_latent_static: ksplit * batch * r = %zu floats exceeds the %zu-float "
+             "static scratch (ksplit = ceil(E/512) for 16-bit weights, ceil(E/64) for float32); "
+             "use qsvd_append_latent with a workspace", need, kStaticScratchFloats);
+    return set_error(QSVD_ERR_WORKSPACE, msg);
+  }
   if (!packed || !x || !pos || !cache)
     return set_error(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  // The GEMV reads x with 8- and 16-byte vector loads and the finish kernel
+  // stores whole rows: the same alignment the workspace entry point demands.
+  if (!aligned16(x) || !aligned16(cache))
+    return set_error(QSVD_ERR_INVALID_ARG, "x and cache must be 16-byte aligned");
   if (cache_is_int(d) && !scales) return set_error(QSVD_ERR_INVALID_ARG, "int caches need scales");
   float* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess)

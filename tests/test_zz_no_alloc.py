@@ -86,3 +86,20 @@ def test_static_append_rejects_oversize_requests():
     st = lib.qsvd_append_latent_static(ctypes.byref(dims), p, p, p, p, None, None, None, None)
     assert st == q.QSVD_ERR_WORKSPACE
     assert b"static scratch" in q._lib.qsvd_last_error()
+
+
+def test_static_append_rejects_misaligned_pointers():
+    """x and cache are read and written with vector accesses, so, as with the
+    workspace entry point, a pointer off a 16-byte boundary is refused on the
+    host before anything is enqueued (the pointers are never dereferenced)."""
+    dims = q.make_dims(1024, 8, 128, 256, 4, 16, cache="f16", weight="f16")
+    lib = ctypes.CDLL(q.LIB_PATH)
+    lib.qsvd_append_latent_static.argtypes = q._sigs["qsvd_append_latent_static"]
+    lib.qsvd_append_latent_static.restype = ctypes.c_int
+    good = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    for x, cache in ((bad, good), (good, bad)):
+        st = lib.qsvd_append_latent_static(ctypes.byref(dims), good, x, good, cache, None, None,
+                                           None, None)
+        assert st == q.QSVD_ERR_INVALID_ARG
+        assert b"16-byte aligned" in q._lib.qsvd_last_error()
