@@ -7,8 +7,13 @@ One step = the whole hot path for one batch: append the current token of
 every sequence (c = x W^d, written as row len-1), then decode attention over
 the latent cache (query projection and absorption, split-KV flash decoding,
 cross-split merge and value up-projection).  Inputs are synthetic and seeded
-(``synthetic``); the latent cache is far larger than L2, so no flush is
-needed between steps.  Prints one JSON line (rank 0).
+(``synthetic``); the latent cache is far larger than L2.  The timed region
+is exactly K steps of a CUDA-graph replay, repeated back to back until about
+0.3 s have passed (so the clock record holds enough samples) and reported as
+the median region; a second figure times single steps after a 256 MB write
+that flushes L2.  At N = 1 the line also carries the other workloads (int4
+and int8 latents, the two rotary layers), each with its own roofline.
+Prints one JSON line (rank 0).
 
 Multi-GPU (torchrun): every rank holds its own batch of sequences (weak
 scaling, no collective on the data path); the step time is the max over
@@ -262,142 +267,263 @@ def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, ms_ma
 # our implementation
 # ---------------------------------------------------------------------------
 
+class DecodeStep:
+    """One decode step of a workload on this rank's GPU: append the current
+    token of every sequence, then the decode phases, each one API call.
+    Rotary mode on the tensor cores runs the split as its two passes so that
+    the scores pass (the dominant kernel there) is timed on its own."""
+
+    def __init__(self, q, cfg, cache_override, args, device, rank):
+        self.q = q
+        inp = bench_inputs(cfg, device, rank, cache=cache_override)
+        self.inp = inp
+        w, lens, max_len = inp["w"], inp["lens"], inp["max_len"]
+        self.w, self.lens, self.max_len, self.device = w, lens, max_len, device
+        kern = {"auto": q.QSVD_KERNEL_AUTO, "simt": q.QSVD_KERNEL_SIMT,
+                "tcgen05": q.QSVD_KERNEL_TCGEN05, "cta": q.QSVD_KERNEL_TCGEN05_CTA,
+                "cluster": q.QSVD_KERNEL_TCGEN05_CLUSTER}[args.kernel]
+        self.splits = args.splits
+        self.dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
+                                out="f32", group=w.group, rope=w.rope, rope_base=w.rope_base,
+                                kernel=kern, out_proj=args.out_proj)
+        self.packed = q.qsvd_prepare_weights(self.dims, inp["wd"], inp["wuq"], inp["wuk"], inp["wuv"])
+        if args.out_proj != "none":
+            # synthetic output projection W_O (E x E), seeded like the other weights
+            gwo = torch.Generator(device=device).manual_seed(w.seed * 31 + 5)
+            wo = (torch.randn((w.E, w.E), generator=gwo, device=device) / math.sqrt(w.E)).to(TORCH_DT[w.weight])
+            q.qsvd_prepare_out_proj(self.dims, wo, self.packed)
+            del wo
+        self.stream = torch.cuda.current_stream()
+        self.lens_dev = torch.from_numpy(lens).to(device)
+        self.pos_dev = (self.lens_dev - 1).to(torch.int32)
+        self.x_dev = inp["x_host"].to(device)
+        self.cnew = torch.empty((w.B, w.r), dtype=torch.float32, device=device)
+        self.out = torch.empty((w.B, w.E), dtype=torch.float32, device=device)
+        self.app_ws = torch.empty(q.append_workspace_bytes(self.dims), dtype=torch.uint8, device=device)
+        self.dec_ws = torch.empty(q.decode_workspace_bytes(self.dims, self.splits), dtype=torch.uint8,
+                                  device=device)
+        # which split kernel these dims run (workspace header), from one full call
+        self._append(self.stream)
+        self._decode(q.QSVD_PHASE_ALL, self.stream)
+        torch.cuda.synchronize()
+        self.kernel_used = int(self.dec_ws[12:16].view(torch.int32).item())
+        self.rope_tc = w.rope and self.kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
+        split_phases = ([("scores", q.QSVD_PHASE_SPLIT_SCORES), ("accum", q.QSVD_PHASE_SPLIT_ACCUM)]
+                        if self.rope_tc else [("split", q.QSVD_PHASE_SPLIT)])
+        self.phases = ([("append", None), ("prologue", q.QSVD_PHASE_PROLOGUE)] + split_phases +
+                       [("combine", q.QSVD_PHASE_COMBINE)])
+        self.graph = None
+
+    def _append(self, st):
+        self.q.qsvd_append_latent(self.dims, self.packed, self.x_dev, self.pos_dev, self.inp["cache"],
+                                  self.inp["scales"], self.cnew, None, self.app_ws, stream=st)
+
+    def _decode(self, ph, st):
+        self.q.qsvd_decode_attn(self.dims, self.packed, self.cnew, True, self.inp["cache"],
+                                self.inp["scales"], self.lens_dev, self.out, num_splits=self.splits,
+                                workspace=self.dec_ws, phases=ph, stream=st)
+
+    def step(self, ev=None, st=None):
+        """ev: len(phases) + 1 events bracketing the phases."""
+        st = self.stream if st is None else st
+        for k, (name, ph) in enumerate(self.phases):
+            if ev is not None:
+                ev[k].record(st)
+            if ph is None:
+                self._append(st)
+            else:
+                self._decode(ph, st)
+        if ev is not None:
+            ev[len(self.phases)].record(st)
+
+    def eager_pass(self, steps):
+        """The API calls per step with events between the phases: per-phase
+        mean times, the dominant kernel's per-launch times, kernels per step."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+              for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0 = self.q.kernel_launches()
+        torch.cuda.synchronize()
+        t0.record(self.stream)
+        for i in range(steps):
+            self.step(ev[i])
+        t1.record(self.stream)
+        torch.cuda.synchronize()
+        per_step = (self.q.kernel_launches() - n0) // steps
+        phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
+                    for k, (name, _) in enumerate(self.phases)}
+        dom = 2   # the split (absorbed) or the scores pass (rotary)
+        dom_ms = [e[dom].elapsed_time(e[dom + 1]) for e in ev]
+        return t0.elapsed_time(t1), phase_ms, dom_ms, per_step
+
+    def capture(self):
+        """One step captured as a CUDA graph: the same kernels with the same
+        arguments, without the host work between launches."""
+        gstream = torch.cuda.Stream(self.device)
+        gstream.wait_stream(self.stream)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=gstream):
+            self.step(st=gstream)
+        for _ in range(3):
+            self.graph.replay()
+        torch.cuda.synchronize()
+
+    def run(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.step()
+
+    def timed_regions(self, steps, world, min_seconds):
+        """Regions of exactly `steps` steps, each bracketed by a barrier and a
+        synchronize, repeated back to back until `min_seconds` have passed
+        (at least one): per-region milliseconds."""
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        regions, spent = [], 0.0
+        while not regions or spent < min_seconds * 1e3:
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            t0.record(self.stream)
+            for _ in range(steps):
+                self.run()
+            t1.record(self.stream)
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            regions.append(t0.elapsed_time(t1))
+            spent += regions[-1]
+            if world > 1:   # every rank runs the same number of regions
+                more = torch.tensor([1.0 if spent < min_seconds * 1e3 else 0.0], device=self.device)
+                torch.distributed.all_reduce(more, op=torch.distributed.ReduceOp.MAX)
+                if more.item() == 0.0:
+                    break
+        return regions
+
+    def flushed_steps(self, n, flush):
+        """n steps, each preceded by a write of `flush` (a buffer larger than
+        L2) and timed alone: per-step milliseconds."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(self.stream)
+            self.run()
+            b.record(self.stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def roofline(self, dom_ms):
+        """Roofline object of the dominant kernel from its per-launch times."""
+        q, w = self.q, self.w
+        hbm_peak, tc_burst, tc_sustained, peak_kind = measured_peaks()
+        dom_mean = statistics.mean(dom_ms)
+        lat_b = latent_bytes(w, self.lens)
+        kname = ("k_rope_scores" if self.rope_tc
+                 else "k_split_cl" if self.kernel_used == q.QSVD_KERNEL_TCGEN05_CLUSTER
+                 else "k_split_tc" if self.kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
+                 else "k_split_rope" if w.rope else "k_split_abs")
+        src = (["split_cluster.cu", "tc_common.cuh", "internal.cuh"] if kname == "k_split_cl"
+               else ["split_tc.cu", "tc_common.cuh", "internal.cuh"] if kname in ("k_split_tc", "k_rope_scores")
+               else ["split_simt.cu", "internal.cuh"])
+        traffic = profiled_traffic(kname, w.name, src)
+        if self.rope_tc:
+            # keys rebuilt per head: K_h = C W^u_{k,h}, 2 r E flop per valid token
+            flops = 2.0 * w.r * w.E * float(np.sum(self.lens))
+            achieved = flops / (dom_mean / 1e3) / 1e12
+            # the scores kernel runs back to back inside long runs of steps (the
+            # power cap sets its clock): the sustained GEMM peak is its ceiling
+            return {"bound": "tensor", "achieved": achieved, "peak": tc_sustained, "unit": "TFLOP/s",
+                    "frac": achieved / tc_sustained, "traffic": traffic, "kernel": kname,
+                    "peak_kind": peak_kind + " bf16 sustained (fp16 has the same dense rate)",
+                    "frac_of_burst_peak": achieved / tc_burst,
+                    "flops_per_launch": flops, "launch_ms": dom_mean,
+                    "launch_ms_median": statistics.median(dom_ms)}
+        achieved = lat_b / (dom_mean / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic,
+                "kernel": kname, "peak_kind": peak_kind,
+                "bytes_per_launch": lat_b, "launch_ms": dom_mean,
+                "launch_ms_median": statistics.median(dom_ms)}
+
+
+def other_workloads(q, args, device):
+    """The other workloads of the path, each timed in this run on its own
+    inputs: its dominant kernel's roofline and its graph-replayed step.
+    Parity cases of the test suite, reported here so that one bench line
+    carries every workload's measured fraction."""
+    out = []
+    for cfg, cache in ((3, None), (3, "i8"), (2, None), (4, None)):
+        st = DecodeStep(q, cfg, cache, args, device, 0)
+        for _ in range(3):
+            st.step()
+        _, phase_ms, dom_ms, _ = st.eager_pass(args.extra_steps)
+        st.capture()
+        regions = st.timed_regions(args.extra_steps, 1, 0.0)
+        ms = regions[0] / args.extra_steps
+        tokens = float(np.sum(st.lens))
+        out.append({"workload": st.w.name, "cache": st.w.cache,
+                    "mode": "rope" if st.w.rope else "absorbed",
+                    "tokens_per_step": int(tokens), "ms_per_step": ms,
+                    "value": tokens / (ms / 1e3), "unit": UNIT,
+                    "step_hbm_gbs": (latent_bytes(st.w, st.lens) + weight_bytes(st.w)) / (ms / 1e3) / 1e9,
+                    "phase_ms": phase_ms, "roofline": st.roofline(dom_ms),
+                    "steps": args.extra_steps})
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import rank_joint_qkv_b200 as q
 
     device = f"cuda:{local_rank}"
     torch.cuda.set_device(device)
-    inp = bench_inputs(args.config, device, rank)
-    w, lens, max_len = inp["w"], inp["lens"], inp["max_len"]
-    kern = {"auto": q.QSVD_KERNEL_AUTO, "simt": q.QSVD_KERNEL_SIMT,
-            "tcgen05": q.QSVD_KERNEL_TCGEN05, "cta": q.QSVD_KERNEL_TCGEN05_CTA,
-            "cluster": q.QSVD_KERNEL_TCGEN05_CLUSTER}[args.kernel]
-    dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
-                       out="f32", group=w.group, rope=w.rope, rope_base=w.rope_base,
-                       kernel=kern, out_proj=args.out_proj)
-    packed = q.qsvd_prepare_weights(dims, inp["wd"], inp["wuq"], inp["wuk"], inp["wuv"])
-    if args.out_proj != "none":
-        # synthetic output projection W_O (E x E), seeded like the other weights
-        gwo = torch.Generator(device=device).manual_seed(w.seed * 31 + 5)
-        wo = (torch.randn((w.E, w.E), generator=gwo, device=device) / math.sqrt(w.E)).to(TORCH_DT[w.weight])
-        q.qsvd_prepare_out_proj(dims, wo, packed)
-        del wo
-    stream = torch.cuda.current_stream()
-    lens_dev = torch.from_numpy(lens).to(device)
-    pos_dev = (lens_dev - 1).to(torch.int32)
-    x_dev = inp["x_host"].to(device)
-    cnew = torch.empty((w.B, w.r), dtype=torch.float32, device=device)
-    out = torch.empty((w.B, w.E), dtype=torch.float32, device=device)
-    app_ws = torch.empty(q.append_workspace_bytes(dims), dtype=torch.uint8, device=device)
-    dec_ws = torch.empty(q.decode_workspace_bytes(dims, args.splits), dtype=torch.uint8,
-                         device=device)
-    cache, scales = inp["cache"], inp["scales"]
-
-    def decode(ph, st):
-        q.qsvd_decode_attn(dims, packed, cnew, True, cache, scales, lens_dev, out,
-                           num_splits=args.splits, workspace=dec_ws, phases=ph, stream=st)
-
-    # which split kernel these dims run (workspace header), from one full call
-    q.qsvd_append_latent(dims, packed, x_dev, pos_dev, cache, scales, cnew, None, app_ws,
-                         stream=stream)
-    decode(q.QSVD_PHASE_ALL, stream)
-    torch.cuda.synchronize()
-    kernel_used = int(dec_ws[12:16].view(torch.int32).item())   # workspace header: kernel
-    rope_tc = w.rope and kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
-    # the phases of one step, one API call each; rotary mode on the tensor
-    # cores runs the split as its two passes so that the scores pass (the
-    # dominant kernel there) is timed on its own
-    split_phases = ([("scores", q.QSVD_PHASE_SPLIT_SCORES), ("accum", q.QSVD_PHASE_SPLIT_ACCUM)]
-                    if rope_tc else [("split", q.QSVD_PHASE_SPLIT)])
-    phases = ([("append", None), ("prologue", q.QSVD_PHASE_PROLOGUE)] + split_phases +
-              [("combine", q.QSVD_PHASE_COMBINE)])
-
-    def step(ev=None, st=None):
-        # ev: len(phases) + 1 events bracketing the phases
-        st = stream if st is None else st
-        for k, (name, ph) in enumerate(phases):
-            if ev is not None:
-                ev[k].record(st)
-            if ph is None:
-                q.qsvd_append_latent(dims, packed, x_dev, pos_dev, cache, scales, cnew, None,
-                                     app_ws, stream=st)
-            else:
-                decode(ph, st)
-        if ev is not None:
-            ev[len(phases)].record(st)
-
+    st = DecodeStep(q, args.config, args.cache, args, device, rank)
+    w, lens, max_len = st.w, st.lens, st.max_len
     for _ in range(args.warmup):
-        step()
+        st.step()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
 
-    # eager pass: the four API calls per step, with events between the phases
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)]
-          for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = q.kernel_launches()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    t0.record(stream)
-    for i in range(args.steps):
-        step(ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    launches_per_step = (q.kernel_launches() - launches0) // args.steps
-    ms_eager = max_over_ranks(t0.elapsed_time(t1), device, world)
-    phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
-                for k, (name, _) in enumerate(phases)}
-    # the dominant kernel's launches: the split (absorbed), the scores pass (rotary)
-    dom = 2
-    dom_ms = [e[dom].elapsed_time(e[dom + 1]) for e in ev]
-
-    # timed pass: one step captured as a CUDA graph (the same kernels with the
-    # same arguments, without the host work between launches), replayed
-    graph = None
+    ms_eager, phase_ms, dom_ms, launches_per_step = st.eager_pass(args.steps)
+    ms_eager = max_over_ranks(ms_eager, device, world)
     if not args.eager:
-        gstream = torch.cuda.Stream(device)
-        gstream.wait_stream(stream)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=gstream):
-            step(st=gstream)
-        for _ in range(3):
-            graph.replay()
-        torch.cuda.synchronize()
-    run = (lambda: graph.replay()) if graph is not None else (lambda: step())
+        st.capture()
+    # the timed region: exactly K steps, repeated back to back until about
+    # 0.3 s have passed so that the clock record holds enough samples; the
+    # reported time is the median region's
     with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        t0.record(stream)
-        for i in range(args.steps):
-            run()
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-    launches = launches_per_step * args.steps
-    ms = t0.elapsed_time(t1)
+        regions = st.timed_regions(args.steps, world, args.min_region_s)
+    ms = statistics.median(regions)
     ms_max = max_over_ranks(ms, device, world)
+    launches = launches_per_step * args.steps
     tokens_per_step = float(np.sum(lens))
     value = whole_job_rate(tokens_per_step, args.steps, world, ms_max)
 
+    # L2 flushed before every step (a 256 MB write), each step timed alone
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    fl = st.flushed_steps(max(10, min(args.steps, 50)), flush)
+    del flush
+    fl_ms = max_over_ranks(statistics.median(fl), device, world)
+
     # end to end through the public API with host buffers
-    x_pin = inp["x_host"].pin_memory()
+    x_pin = st.inp["x_host"].pin_memory()
     lens_pin = torch.from_numpy(lens).pin_memory()
     out_pin = torch.empty((w.B, w.E), dtype=torch.float32).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ke = max(3, args.steps)
     torch.cuda.synchronize()
-    e0.record(stream)
+    e0.record(st.stream)
     for _ in range(ke):
-        x_dev.copy_(x_pin, non_blocking=True)
-        lens_dev.copy_(lens_pin, non_blocking=True)
-        torch.sub(lens_dev, 1, out=pos_dev)
-        step()
-        out_pin.copy_(out, non_blocking=True)
-    e1.record(stream)
+        st.x_dev.copy_(x_pin, non_blocking=True)
+        st.lens_dev.copy_(lens_pin, non_blocking=True)
+        torch.sub(st.lens_dev, 1, out=st.pos_dev)
+        st.step()
+        out_pin.copy_(st.out, non_blocking=True)
+    e1.record(st.stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
     e2e_value = whole_job_rate(tokens_per_step, ke, world, e2e_ms)
@@ -406,60 +532,43 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return None
-    hbm_peak, tc_burst, tc_sustained, peak_kind = measured_peaks()
-    dom_mean = statistics.mean(dom_ms)
     lat_b = latent_bytes(w, lens)
-    kname = ("k_rope_scores" if rope_tc
-             else "k_split_cl" if kernel_used == q.QSVD_KERNEL_TCGEN05_CLUSTER
-             else "k_split_tc" if kernel_used == q.QSVD_KERNEL_TCGEN05_CTA
-             else "k_split_rope" if w.rope else "k_split_abs")
-    src = (["split_cluster.cu", "tc_common.cuh", "internal.cuh"] if kname == "k_split_cl"
-           else ["split_tc.cu", "tc_common.cuh", "internal.cuh"] if kname in ("k_split_tc", "k_rope_scores")
-           else ["split_simt.cu", "internal.cuh"])
-    workload = w.name
-    traffic = profiled_traffic(kname, workload, src)
-    if rope_tc:
-        # keys rebuilt per head: K_h = C W^u_{k,h}, 2 r E flop per valid token
-        flops = 2.0 * w.r * w.E * float(np.sum(lens))
-        achieved = flops / (dom_mean / 1e3) / 1e12
-        # the scores kernel runs back to back inside long runs of steps (the
-        # power cap sets its clock): the sustained GEMM peak is its ceiling
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_sustained, "unit": "TFLOP/s",
-                "frac": achieved / tc_sustained, "traffic": traffic, "kernel": kname,
-                "peak_kind": peak_kind + " bf16 sustained (fp16 has the same dense rate)",
-                "frac_of_burst_peak": achieved / tc_burst,
-                "flops_per_launch": flops, "launch_ms": dom_mean}
-    else:
-        achieved = lat_b / (dom_mean / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": traffic,
-                "kernel": kname, "peak_kind": peak_kind,
-                "bytes_per_launch": lat_b, "launch_ms": dom_mean}
     step_gbs = (lat_b + weight_bytes(w)) / (ms_max / args.steps / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.cache, "data": "synthetic",
-        "config": {"workload": workload, "E": w.E, "H": w.H, "d_h": w.d_h, "r": w.r,
+        "config": {"workload": w.name, "E": w.E, "H": w.H, "d_h": w.d_h, "r": w.r,
                    "batch_per_gpu": w.B, "kv_len": int(max_len),
                    "tokens_per_step_per_gpu": int(tokens_per_step), "cache": w.cache,
                    "weights": w.weight, "mode": "rope" if w.rope else "absorbed",
                    "splits": args.splits, "kernel": args.kernel, "out_proj": args.out_proj,
-                   "l2": "inputs larger than L2: %.0f MB latent read per step per GPU"
+                   "l2": "inputs larger than L2: %.0f MB latent read per step per GPU; "
+                         "l2_flushed: the same step after a 256 MB write, timed alone"
                          % (lat_b / 1e6),
                    "parallelism": f"dp{world}"},
         "steps_per_s": args.steps * 1e3 / ms_max,
         "timing": ("CUDA-graph replay of one captured step (the kernels of the four API calls)"
-                   if graph is not None else "eager API calls"),
+                   if st.graph is not None else "eager API calls"),
+        "timed_regions": {"count": len(regions), "steps_each": args.steps,
+                          "ms_median": statistics.median(regions), "ms_min": min(regions),
+                          "ms_max": max(regions)},
         "ms_per_step_eager": ms_eager / args.steps,
         "phase_ms": phase_ms,
         "step_hbm_gbs": step_gbs,
-        "roofline": roof,
+        "l2_flushed": {"ms_per_step": fl_ms, "value": whole_job_rate(tokens_per_step, 1, world, fl_ms),
+                       "steps": len(fl), "stat": "median"},
+        "roofline": st.roofline(dom_ms),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches),
+        "gpu_launches_all_regions": int(launches * len(regions)),
     }
     line["clocks"] = clk.summary()
+    del st
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extra and args.config == 1 and args.cache is None:
+        line["other_workloads"] = other_workloads(q, args, device)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, lens, budget_s=args.cpu_seconds)
     return line
@@ -559,6 +668,60 @@ def run_prefill(args):
             "status": int(status.item()), "clocks": clk.summary()}
 
 
+def run_prefill_attn(args):
+    """qsvd_prefill_attention over every prompt of the workload (B prompts of
+    L tokens: Q, K, V rebuilt from the latent rows by three GEMMs, then causal
+    attention on the tensor cores), timed with CUDA events over K calls."""
+    import rank_joint_qkv_b200 as q
+    device = "cuda:0"
+    torch.cuda.set_device(device)
+    w = synthetic.CONFIGS[args.config]
+    inp = bench_inputs(args.config, device)
+    lens = inp["lens"]
+    max_len = inp["max_len"]
+    dims = q.make_dims(w.E, w.H, w.d_h, w.r, w.B, max_len, cache=w.cache, weight=w.weight,
+                       rope=w.rope, rope_base=w.rope_base)
+    packed = q.qsvd_prepare_weights(dims, inp["wd"], inp["wuq"], inp["wuk"], inp["wuv"])
+    lens_dev = torch.from_numpy(lens).to(device)
+    out = torch.empty((w.B, max_len, w.E), dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = torch.empty(q.prefill_attention_workspace_bytes(dims), dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        q.qsvd_prefill_attention(dims, packed, inp["cache"], lens_dev, out, status, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = q.kernel_launches()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            q.qsvd_prefill_attention(dims, packed, inp["cache"], lens_dev, out, status, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    L = lens.astype(np.float64)
+    rows = float(w.B * max_len)
+    attn_flops = float(np.sum(2.0 * w.E * L * (L + 1.0)))      # causal Q K^T and P V
+    gemm_flops = 3 * 2.0 * rows * w.r * w.E                      # Q, K, V = C W^u
+    flops = attn_flops + gemm_flops
+    achieved = flops / (ms / 1e3) / 1e12
+    _, burst, sustained, kind = measured_peaks()
+    parts = 3.0   # S: 3 part products; P V: 3 part products
+    return {"metric": "prefill attention prompt tokens/s (Q, K, V rebuilt from the latent rows, causal)",
+            "value": float(np.sum(L)) / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": w.cache,
+            "data": "synthetic",
+            "config": {"workload": w.name + "-prefill-attention", "E": w.E, "H": w.H, "r": w.r,
+                       "prompts": w.B, "prompt_len": int(max_len), "rope": bool(w.rope)},
+            "roofline": {"bound": "tensor", "achieved": achieved, "unit": "TFLOP/s", "peak": sustained,
+                         "frac": achieved / sustained, "frac_of_burst_peak": achieved / burst,
+                         "peak_kind": kind + " bf16 sustained", "traffic": None,
+                         "kernel": "qsvd_prefill_attention (3 latent GEMMs, 3 part kernels, k_prefill_attn)",
+                         "flops_per_call": flops, "attention_flops": attn_flops, "gemm_flops": gemm_flops,
+                         "tensor_work_per_attention_flop": parts},
+            "gpu_launches": q.kernel_launches() - n0, "status": int(status.item()),
+            "clocks": clk.summary()}
+
+
 def run_beta(args):
     """One split-exponent evaluation of the calibration objective per step
     (factors for beta, layout with H2, three prefills, two decodes, the
@@ -643,7 +806,8 @@ def run_per_head(args):
     bv = (torch.randn((w.H, r, w.d_h), generator=g, device=device) / math.sqrt(r)).to(wt)
     qv = torch.randn((w.B, w.E), generator=g, device=device)
     lens = torch.full((w.B,), w.L, dtype=torch.int32, device=device)
-    dims = q.make_dims(w.E, w.H, w.d_h, r, w.B, w.L, cache=cache, weight=w.weight)
+    dims = q.make_dims(w.E, w.H, w.d_h, r, w.B, w.L, cache=cache, weight=w.weight, rope=w.rope,
+                       rope_base=w.rope_base)
     out = torch.empty((w.B, w.E), dtype=torch.float32, device=device)
     ws = torch.empty(q.per_head_workspace_bytes(dims), dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
@@ -666,9 +830,10 @@ def run_per_head(args):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": cache,
             "data": "synthetic",
             "config": {"workload": w.name + "-per-head", "E": w.E, "H": w.H, "d_h": w.d_h, "r_per_head": r,
+                       "mode": "rope" if w.rope else "absorbed",
                        "batch": w.B, "kv_len": w.L, "cache": cache, "weights": w.weight},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "traffic": None, "kernel": "qsvd_decode_attn_per_head (3 kernels)",
+                         "traffic": None, "kernel": "qsvd_decode_attn_per_head (all its kernels)",
                          "peak_kind": kind, "bytes_per_launch": lat_b},
             "gpu_launches": q.kernel_launches() - n0, "clocks": clk.summary()}
 
@@ -676,7 +841,7 @@ def run_per_head(args):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    w = synthetic.CONFIGS[args.config]
+    w = workload(args.config, args.cache)
     lens = synthetic.lengths(w)
     n = int(min(int(np.max(lens)), 8192))
     for _ in range(args.warmup):
@@ -710,9 +875,17 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--cache", choices=["i4", "i8"], default=None,
+                    help="latent type of a quantised workload (the int4 workload also runs with int8)")
+    ap.add_argument("--min-region-s", type=float, default=0.3,
+                    help="repeat the K-step timed region until this many seconds have passed")
+    ap.add_argument("--extra-steps", type=int, default=30,
+                    help="steps per timed region of the other workloads")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads' measurements")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05", "cta", "cluster"], default="auto")
@@ -727,6 +900,8 @@ def main():
                     help="time one evaluation of the split-exponent calibration objective per step")
     ap.add_argument("--prefill", action="store_true",
                     help="time qsvd_prefill_latent over the workload's whole cache instead of a decode step")
+    ap.add_argument("--prefill-attn", action="store_true",
+                    help="time qsvd_prefill_attention over the workload's prompts (all B x L tokens)")
     ap.add_argument("--eager", action="store_true",
                     help="time the API calls as issued instead of a CUDA-graph replay of one step")
     args = ap.parse_args()
@@ -738,6 +913,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.prefill:
         line = run_prefill(args)
+    elif args.prefill_attn:
+        line = run_prefill_attn(args)
     elif args.beta_search:
         line = run_beta(args)
     elif args.per_head_rank:

@@ -222,6 +222,63 @@ qsvd_status qsvd_prefill_latent(const qsvd_dims* dims, const void* packed,
                                 int32_t* status, void* stream);
 
 /*
+ * qsvd_beta_exponents -- the split exponents of one beta for
+ * qsvd_split_factors: a_j = float(sigma_j^beta), b_j = float(sigma_j^(1 -
+ * beta)), the powers taken in float64 (QSVD paper notes, 关键设计: the latent
+ * is X U_r Sigma_r^beta; the up-projection carries Sigma_r^(1 - beta)).
+ *   sigma  device, r float32 singular values (>= 0); 1 <= r <= 8192.
+ *   a, b   device, r float32 each (written).
+ * Stream-ordered.  Errors: INVALID_ARG, CUDA.
+ */
+qsvd_status qsvd_beta_exponents(const float* sigma, int r, double beta, float* a, float* b, void* stream);
+
+/*
+ * qsvd_sq_diff_sum -- *out = sum_i (y_i - yq_i)^2 over n float32 pairs,
+ * accumulated in float64 on the device: the calibration objective
+ * sum_d ||Y_d - Y'_d||^2 of the beta search (QSVD paper notes, 核心创新) over
+ * the decode outputs from the float32 and the quantised latent rows.
+ *   y, yq  device, n float32 each.
+ *   out    device, one float64 (overwritten; the sum of per-block partials,
+ *          added in an unspecified order).
+ * Stream-ordered.  Errors: INVALID_ARG, CUDA.
+ */
+qsvd_status qsvd_sq_diff_sum(const float* y, const float* yq, int64_t n, double* out, void* stream);
+
+/*
+ * qsvd_prefill_attention -- causal attention over the prompts whose latent
+ * rows are in the cache (the attention of a prefill step).  Source: QSVD
+ * digest, Method, Step 1 (queries, keys and values are rebuilt from the
+ * buffered latent: Q = C W^u_q, K = C W^u_k, V = C W^u_v) and Key
+ * Contributions (the prompt is read once, into the latent); rotary embedding
+ * as in the decode (WSVD digest, Method §3.4).  For prompt b of length
+ * len_b (its latent rows are cache rows b max_len + t, t < len_b) and head h:
+ *   o_t = sum_{u <= t} softmax_u(tau q_t . k_u) v_u
+ * with q_t, k_u rotated to their own positions when dims->rope is set and
+ * tau = dims->softmax_scale (<= 0: 1/sqrt(d_h)).  Q, K and V are rebuilt by
+ * the tensor-core latent GEMM in float32 and held as two 16-bit parts each
+ * (hi and rounding residual); the attention runs on tcgen05 with float32
+ * accumulation.
+ *   packed     from qsvd_prepare_weights (its W^u_q, W^u_k, W^u_v and, with
+ *              dims->rope, its rotary table).
+ *   cache      device, B x max_len x r, cache_dtype (F16 or BF16, equal to
+ *              weight_dtype), 16-byte aligned.
+ *   lengths    device, B int32 prompt lengths, clamped to [0, max_len].
+ *   workspace  device scratch, 16-byte aligned, or NULL to query its size
+ *              into *workspace_bytes (in: capacity):
+ *              B max_len E (4 + 6 x 2) bytes.
+ *   out        device, B x max_len x E, out_dtype, 16-byte aligned: rows
+ *              t < len_b are written, other rows are left as they were.
+ *   status     device int32 word; QSVD_STATUS_TIMEOUT is OR-ed in if a
+ *              pipeline wait expired.
+ * Requires d_h == 128, E % 256 == 0, r % 64 == 0; else UNSUPPORTED.
+ * Stream-ordered; nothing is allocated.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+qsvd_status qsvd_prefill_attention(const qsvd_dims* dims, const void* packed, const void* cache,
+                                   const int32_t* lengths, void* workspace, size_t* workspace_bytes,
+                                   void* out, int32_t* status, void* stream);
+
+/*
  * qsvd_append_latent_static -- qsvd_append_latent without a workspace.
  * The paper has no counterpart: this is an interface variant for callers
  * that cannot allocate device memory -- a serving engine or plugin host that
@@ -347,12 +404,16 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  *   qt_h = tau B_{Kh} q_h,  s_t = C_{Kh,t} . qt_h,  p = softmax(s),
  *   o_h = (p^T C_{Vh}) B_{Vh}.
  * No rotary embedding (dims->rope must be 0).  Computed in float32 on CUDA
- * cores, 256 tokens per split CTA, chunks merged in the log2 domain.
+ * cores, 256 tokens per split CTA, chunks merged in the log2 domain; 16-bit
+ * latents with r = 64, 128 or 256 are read as 16-byte vectors.
  *   bk, bv     device, H x r x d_h each, weight_dtype (F32, F16 or BF16):
- *              B_{Kh} and B_{Vh} stacked by head.
- *   q          device, B x E float32: the query (head h in columns
- *              h d_h .. h d_h + d_h - 1).
- *   ck, cv     device, cache_dtype (F32, F16 or BF16), in one of two
+ *              B_{Kh} and B_{Vh} stacked by head.  With dims->out_proj ==
+ *              QSVD_OUT_PROJ_FOLD (16-bit weights), bv is instead the fold
+ *              F = [B_{V1} W_{O,1}; ..; B_{VH} W_{O,H}] (H r x E, from
+ *              qsvd_prepare_per_head_fold) and out receives y = o W_O.
+ *   q          device, B x E float32, 16-byte aligned: the query (head h
+ *              in columns h d_h .. h d_h + d_h - 1).
+ *   ck, cv     device, 16-byte aligned, cache_dtype (F32, F16 or BF16), in one of two
  *              layouts (rows 0 .. len_b - 1 of every head are read):
  *              QSVD_PER_HEAD_HEAD_MAJOR   B x H x max_len x r;
  *              QSVD_PER_HEAD_TOKEN_MAJOR  B x max_len x H x r: row t of a
@@ -368,8 +429,8 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  *   out        device, B x E, out_dtype.
  * Stream-ordered; nothing is allocated.
  * Errors: INVALID_ARG (also an unknown layout), UNSUPPORTED (rotary mode,
- * int caches, online H2, an output projection, max_len beyond ~50 M
- * tokens), WORKSPACE, CUDA.
+ * int caches, online H2, the chained output projection, the fold with
+ * float32 weights, max_len beyond ~50 M tokens), WORKSPACE, CUDA.
  */
 #define QSVD_PER_HEAD_HEAD_MAJOR 0
 #define QSVD_PER_HEAD_TOKEN_MAJOR 1
@@ -377,6 +438,22 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
                                       const float* q, const void* ck, const void* cv,
                                       const int32_t* lengths, int layout, void* workspace,
                                       size_t* workspace_bytes, void* out, void* stream);
+
+/*
+ * qsvd_prepare_per_head_fold -- the per-head value factor folded into the
+ * output projection (WSVD digest, Method, fused kernel §3.4):
+ *   F[h r + j][n] = sum_i B_{Vh}[j][i] W_O[h d_h + i][n]
+ * in float32, rounded once to weight_dtype.  With it the per-head decode
+ * (dims->out_proj = QSVD_OUT_PROJ_FOLD) ends in one GEMV of the merged
+ * latents (B x H r) by F instead of B_{Vh} then W_O.
+ *   bv  device, H x r x d_h, weight_dtype (F16 or BF16).
+ *   wo  device, E x E, weight_dtype (row h d_h + i multiplies channel i of
+ *       head h).
+ *   f   device, H r x E, weight_dtype (written).
+ * Stream-ordered.  Errors: INVALID_ARG, UNSUPPORTED (float32 weights), CUDA.
+ */
+qsvd_status qsvd_prepare_per_head_fold(const qsvd_dims* dims, const void* bv, const void* wo, void* f,
+                                       void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* qsvd_status_string(qsvd_status s);
@@ -389,6 +466,20 @@ uint64_t qsvd_kernel_launches(void);
 
 /* QSVD_ABI_VERSION of the loaded library. */
 int qsvd_abi_version(void);
+
+/*
+ * qsvd_testing_set_score_wait_ns -- failure injection for tests (the pages
+ * have no counterpart).  Every wait inside a kernel gives up after 2 s and
+ * records QSVD_STATUS_TIMEOUT.  With ns != 0, the softmax warps of the
+ * tensor-core split kernel (absorbed mode) begin their first tile by waiting
+ * on a barrier that nothing releases, with a limit of ns nanoseconds: the
+ * wait expires on every call, without any fault -- the kernel flags the
+ * timeout, the other roles stop, wait (with the normal limit) for their
+ * copies and MMAs in flight, free TMEM and return.  Applies to the current
+ * device; ns = 0 turns it off.  Synchronous; for tests only.
+ * Errors: CUDA.
+ */
+qsvd_status qsvd_testing_set_score_wait_ns(unsigned long long ns);
 
 #ifdef __cplusplus
 }

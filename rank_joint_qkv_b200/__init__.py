@@ -65,6 +65,11 @@ _sigs = {
     "qsvd_prepare_out_proj": [_D, _P, _P, ctypes.c_size_t, _P],
     "qsvd_split_factors": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "qsvd_decode_attn_per_head": [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _SZ, _P, _P],
+    "qsvd_testing_set_score_wait_ns": [ctypes.c_ulonglong],
+    "qsvd_prefill_attention": [_D, _P, _P, _P, _P, _SZ, _P, _P, _P],
+    "qsvd_prepare_per_head_fold": [_D, _P, _P, _P, _P],
+    "qsvd_beta_exponents": [_P, ctypes.c_int, ctypes.c_double, _P, _P, _P],
+    "qsvd_sq_diff_sum": [_P, _P, ctypes.c_int64, _P, _P],
 }
 for _name, _args in _sigs.items():
     _f = getattr(_lib, _name)
@@ -119,6 +124,13 @@ def kernel_launches() -> int:
 
 def abi_version() -> int:
     return int(_lib.qsvd_abi_version())
+
+
+def qsvd_testing_set_score_wait_ns(ns: int) -> None:
+    """Failure-detection tests only: with ns != 0 the tensor-core split
+    kernel's softmax warps wait on a barrier nothing releases, giving up
+    after ns nanoseconds (current device); 0 turns it off."""
+    _check(_lib.qsvd_testing_set_score_wait_ns(int(ns)), "qsvd_testing_set_score_wait_ns")
 
 
 def _empty_bytes(n: int, device) -> torch.Tensor:
@@ -190,6 +202,48 @@ def qsvd_prefill_latent(dims: qsvd_dims, packed, x, dst_rows, cache, scales=None
                                     _ptr(dst_rows), _ptr(cache), _ptr(scales), _ptr(c_out),
                                     _ptr(status), _stream(stream)),
            "qsvd_prefill_latent")
+
+
+def qsvd_beta_exponents(sigma, beta: float, a, b, stream=None) -> None:
+    """a = sigma^beta, b = sigma^(1 - beta) (float64 powers), device tensors."""
+    _check(_lib.qsvd_beta_exponents(_ptr(sigma), int(sigma.numel()), float(beta), _ptr(a), _ptr(b),
+                                    _stream(stream)), "qsvd_beta_exponents")
+
+
+def qsvd_sq_diff_sum(y, yq, out, stream=None) -> None:
+    """out[0] = sum (y - yq)^2 in float64 (device tensors; out float64)."""
+    _check(_lib.qsvd_sq_diff_sum(_ptr(y), _ptr(yq), int(y.numel()), _ptr(out), _stream(stream)),
+           "qsvd_sq_diff_sum")
+
+
+def qsvd_prepare_per_head_fold(dims: qsvd_dims, bv, wo, f=None, stream=None) -> torch.Tensor:
+    """F = [B_{Vh} W_{O,h}]_h (H r x E) in the weight type; returns F."""
+    if f is None:
+        f = torch.empty((dims.H * dims.r, dims.E), dtype=wo.dtype, device=wo.device)
+    _check(_lib.qsvd_prepare_per_head_fold(ctypes.byref(dims), _ptr(bv), _ptr(wo), _ptr(f), _stream(stream)),
+           "qsvd_prepare_per_head_fold")
+    return f
+
+
+def prefill_attention_workspace_bytes(dims: qsvd_dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.qsvd_prefill_attention(ctypes.byref(dims), None, None, None, None, ctypes.byref(n),
+                                       None, None, None), "qsvd_prefill_attention(size)")
+    return n.value
+
+
+def qsvd_prefill_attention(dims: qsvd_dims, packed, cache, lengths, out, status, workspace=None,
+                           stream=None):
+    """Causal attention over the prompts' latent rows (cache rows b * max_len
+    + t, t < lengths[b]); out is B x max_len x E.  Returns the workspace."""
+    if workspace is None:
+        workspace = _empty_bytes(prefill_attention_workspace_bytes(dims), cache.device)
+    n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _check(_lib.qsvd_prefill_attention(ctypes.byref(dims), _ptr(packed), _ptr(cache), _ptr(lengths),
+                                       _ptr(workspace), ctypes.byref(n), _ptr(out), _ptr(status),
+                                       _stream(stream)),
+           "qsvd_prefill_attention")
+    return workspace
 
 
 def qsvd_append_latent_static(dims: qsvd_dims, packed, x, pos, cache, scales=None,

@@ -12,8 +12,9 @@ fold), qsvd_prefill_latent three times (the calibration latents rounded to
 float32 for Y, quantised into the cache for Y', and the float32 latent of
 each sequence's last token, the decode query), and qsvd_decode_attn twice.
 Y_d and Y'_d are the decode-step outputs of calibration sequence d (its last
-token attending to all its tokens); the host adds up the squared
-differences of the two B x E outputs.
+token attending to all its tokens); qsvd_beta_exponents forms sigma^beta and
+sigma^(1 - beta) and qsvd_sq_diff_sum adds up the squared differences of the
+two B x E outputs in float64 on the device: the host reads one number.
 
 The search: a grid over [0, 1], then a golden-section search (Kiefer, 1953)
 between the best grid point's neighbours; the best beta evaluated wins.
@@ -26,8 +27,8 @@ from typing import Dict, Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-from . import (QSVD_KERNEL_AUTO, make_dims, qsvd_decode_attn, qsvd_prefill_latent,
-               qsvd_prepare_weights, qsvd_split_factors)
+from . import (QSVD_KERNEL_AUTO, make_dims, qsvd_beta_exponents, qsvd_decode_attn, qsvd_prefill_latent,
+               qsvd_prepare_weights, qsvd_split_factors, qsvd_sq_diff_sum)
 
 _GOLDEN = (math.sqrt(5.0) - 1.0) / 2.0
 _TORCH = {"f16": torch.float16, "bf16": torch.bfloat16}
@@ -81,14 +82,16 @@ class BetaObjective:
         self.yq = torch.empty((B, E), dtype=torch.float32, device=dev)
         self.ws_f = self.ws_q = None
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.sigma = torch.from_numpy(self.s.astype(np.float32)).to(dev)
+        self.a = torch.empty(r, dtype=torch.float32, device=dev)
+        self.b = torch.empty(r, dtype=torch.float32, device=dev)
+        self.obj = torch.zeros(1, dtype=torch.float64, device=dev)
         self.evaluations = 0
 
     def outputs(self, beta: float) -> Tuple[torch.Tensor, torch.Tensor]:
         """Y (float32 latent rows) and Y' (quantised rows) on the device."""
-        dev = self.x.device
-        a = torch.from_numpy((self.s ** beta).astype(np.float32)).to(dev)
-        b = torch.from_numpy((self.s ** (1.0 - beta)).astype(np.float32)).to(dev)
-        qsvd_split_factors(self.dims_f, self.u, self.vt, a, b, self.wd, *self.wu)
+        qsvd_beta_exponents(self.sigma, beta, self.a, self.b)
+        qsvd_split_factors(self.dims_f, self.u, self.vt, self.a, self.b, self.wd, *self.wu)
         self.packed = qsvd_prepare_weights(self.dims_f, self.wd, *self.wu, h2_q=self.h2_q,
                                            packed=self.packed)
         qsvd_prefill_latent(self.dims_f, self.packed, self.x, self.rows, self.cache_f,
@@ -106,8 +109,8 @@ class BetaObjective:
 
     def __call__(self, beta: float) -> float:
         y, yq = self.outputs(beta)
-        d = y.cpu().numpy().astype(np.float64) - yq.cpu().numpy().astype(np.float64)
-        return float(np.sum(d * d))
+        qsvd_sq_diff_sum(y, yq, self.obj)   # on the device, float64
+        return float(self.obj.item())
 
     def status_word(self) -> int:
         return int(self.status.item())

@@ -168,6 +168,12 @@ uint64_t qsvd_kernel_launches(void) { return g_launches.load(std::memory_order_r
 
 int qsvd_abi_version(void) { return QSVD_ABI_VERSION; }
 
+qsvd_status qsvd_testing_set_score_wait_ns(unsigned long long ns) {
+  const cudaError_t e = set_score_wait_ns(ns);
+  if (e != cudaSuccess) return cuda_fail(e, "qsvd_testing_set_score_wait_ns");
+  return QSVD_OK;
+}
+
 qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd, const void* wuq,
                                  const void* wuk, const void* wuv, const float* h2_q,
                                  void* packed, size_t* packed_bytes, void* stream) {
@@ -202,6 +208,22 @@ qsvd_status qsvd_split_factors(const qsvd_dims* dims, const float* u, const floa
   cudaError_t e = launch_split_factors(*dims, u, vt, a, b, wd, wuq, wuk, wuv,
                                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "split_factors");
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_beta_exponents(const float* sigma, int r, double beta, float* a, float* b, void* stream) {
+  if (r < 1 || r > 8192) return fail(QSVD_ERR_INVALID_ARG, "r (%d) must be in [1, 8192]", r);
+  if (!sigma || !a || !b) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  cudaError_t e = launch_beta_split(sigma, beta, a, b, r, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "beta_exponents");
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_sq_diff_sum(const float* y, const float* yq, int64_t n, double* out, void* stream) {
+  if (n < 0) return fail(QSVD_ERR_INVALID_ARG, "n must be >= 0");
+  if (!y || !yq || !out) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  cudaError_t e = launch_sq_diff_sum(y, yq, size_t(n), out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sq_diff_sum");
   return QSVD_OK;
 }
 
@@ -273,6 +295,35 @@ qsvd_status qsvd_prefill_latent(const qsvd_dims* dims, const void* packed, const
   cudaError_t e = launch_prefill(d, P + L.wd, x, n_rows, dst_rows, cache, scales, c_fp32_debug, status,
                                  static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prefill_latent");
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_prefill_attention(const qsvd_dims* dims, const void* packed, const void* cache,
+                                   const int32_t* lengths, void* workspace, size_t* workspace_bytes,
+                                   void* out, int32_t* status, void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  if (!prefill_attention_supported(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "prefill attention needs d_h == 128, an F16 or BF16 cache of the weight type, "
+                "E %% 256 == 0 and r %% 64 == 0");
+  const PrefillAttnWs need = prefill_attention_ws(d, nullptr);
+  if (!workspace) { *workspace_bytes = need.total; return QSVD_OK; }
+  if (*workspace_bytes < need.total)
+    return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, need.total);
+  if (!packed || !cache || !lengths || !out || !status)
+    return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(workspace) || !aligned16(cache) || !aligned16(out))
+    return fail(QSVD_ERR_INVALID_ARG, "workspace, cache and out must be 16-byte aligned");
+  const PackedLayout L = packed_layout(d);
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  cudaError_t e = launch_prefill_attention(d, P + L.wuq, P + L.wuk, P + L.wuv,
+                                           reinterpret_cast<const float*>(P + L.rope), cache, lengths,
+                                           prefill_attention_ws(d, workspace), out, status,
+                                           score_scale_log2(d), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_attention");
   return QSVD_OK;
 }
 
@@ -416,10 +467,15 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
   if (st != QSVD_OK) return st;
   const qsvd_dims& d = *dims;
   if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
-  if (d.rope) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no rotary mode");
+  if (d.rope && !wsvd_rope_supported(d))
+    return fail(QSVD_ERR_UNSUPPORTED,
+                "per-head latents, rotary mode: d_h == 128, r in {64, 128, 256}, an F16 or BF16 cache "
+                "of the weight type");
   if (cache_is_int(d)) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: F32, F16 or BF16 caches");
-  if (d.h2 || d.out_proj != QSVD_OUT_PROJ_NONE)
-    return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no online H2, no output projection");
+  if (d.h2 || d.out_proj == QSVD_OUT_PROJ_CHAIN)
+    return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no online H2, no chained output projection");
+  if (d.out_proj == QSVD_OUT_PROJ_FOLD && d.weight_dtype == QSVD_F32)
+    return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: the folded output projection needs 16-bit weights");
   if (layout != QSVD_PER_HEAD_HEAD_MAJOR && layout != QSVD_PER_HEAD_TOKEN_MAJOR)
     return fail(QSVD_ERR_INVALID_ARG, "unknown per-head latent layout %d", layout);
   const WsvdLayout W = wsvd_layout(d);
@@ -430,10 +486,24 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
     return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, W.total);
   if (!bk || !bv || !q || !ck || !cv || !lengths || !out)
     return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!aligned16(workspace)) return fail(QSVD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (!aligned16(workspace) || !aligned16(ck) || !aligned16(cv) || !aligned16(q))
+    return fail(QSVD_ERR_INVALID_ARG, "workspace, q, ck and cv must be 16-byte aligned");
   cudaError_t e = launch_wsvd_decode(d, bk, bv, q, ck, cv, lengths, score_scale_log2(d), workspace, W, out,
                                      layout == QSVD_PER_HEAD_TOKEN_MAJOR, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_per_head");
+  return QSVD_OK;
+}
+
+qsvd_status qsvd_prepare_per_head_fold(const qsvd_dims* dims, const void* bv, const void* wo, void* f,
+                                       void* stream) {
+  qsvd_status st = validate(dims);
+  if (st != QSVD_OK) return st;
+  const qsvd_dims& d = *dims;
+  if (d.weight_dtype != QSVD_F16 && d.weight_dtype != QSVD_BF16)
+    return fail(QSVD_ERR_UNSUPPORTED, "the per-head fold needs 16-bit weights");
+  if (!bv || !wo || !f) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
+  cudaError_t e = launch_per_head_fold(d, bv, wo, f, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prepare_per_head_fold");
   return QSVD_OK;
 }
 

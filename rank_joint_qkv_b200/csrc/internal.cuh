@@ -254,7 +254,23 @@ cudaError_t launch_prefill(const qsvd_dims& d, const void* wd, const void* x, in
 // Combine phase.  16-bit weights with d_h % 64 == 0: a merge kernel writes
 // the merged latents zm, then the tensor-core GEMV applies W^u_v per head;
 // otherwise one kernel merges and applies W^u_v per (head, 128 rows of r).
+// Prefill attention (prefill_attn.cu): workspace sections and launcher.
+struct PrefillAttnWs {
+  float* stage;     // [B max_len][E] float32 rows of the GEMM (Q, then K, then V)
+  void* q[2];       // hi, lo parts [B max_len][E], cache type
+  void* k[2];
+  void* v[2];
+  size_t total;     // bytes
+};
+bool prefill_attention_supported(const qsvd_dims& d);
+PrefillAttnWs prefill_attention_ws(const qsvd_dims& d, void* workspace);
+cudaError_t launch_prefill_attention(const qsvd_dims& d, const void* wuq, const void* wuk, const void* wuv,
+                                     const float* rope_tab, const void* cache, const int32_t* lengths,
+                                     const PrefillAttnWs& w, void* out, int32_t* status, float sl2,
+                                     cudaStream_t s);
+
 bool combine_uses_gemv(const qsvd_dims& d);
+cudaError_t set_score_wait_ns(unsigned long long ns);   // test hook of the split kernel
 // Merge + V-up on the tensor-core GEMV.  With d.out_proj the output is
 // projected by W_O: CHAIN runs the V-up into `ow` (B x E fp32) and a second
 // GEMV by `wo` (E x E); FOLD skips the V-up and runs one GEMV of the merged
@@ -292,6 +308,9 @@ cudaError_t launch_split_factors(const qsvd_dims& d, const float* u, const float
                                  cudaStream_t s);
 // Output-projection section of the packed buffer: W_O copied (CHAIN) or the
 // per-head fold F = W^u_{v,h} W_{O,h} (FOLD); W^u_v read from the buffer.
+cudaError_t launch_beta_split(const float* sigma, double beta, float* a, float* b, int r, cudaStream_t s);
+cudaError_t launch_sq_diff_sum(const float* y, const float* yq, size_t n, double* out, cudaStream_t s);
+cudaError_t launch_per_head_fold(const qsvd_dims& d, const void* bv, const void* wo, void* f, cudaStream_t s);
 cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* packed,
                                     const PackedLayout& L, cudaStream_t s);
 

@@ -229,7 +229,7 @@ k_prefill(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
       const int m = m0 + t;
       long long row = -1;
       if (m < n_rows) {
-        const int dr = dst_rows[m];
+        const int dr = dst_rows ? dst_rows[m] : m;   // no row list: row m of the output
         if (dr >= 0 && dr < n_dst_rows) row = dr;
         else if (status) atomicOr(status, QSVD_STATUS_POS_OOB);
       }

@@ -95,14 +95,16 @@ __global__ void k_rope_table(float* __restrict__ tab, int max_len, int half, dou
 }
 
 // Per-head fold of the value up-projection into the output projection (WSVD
-// digest, Method, fused kernel §3.4): F[h r + j][n] = sum_i W^u_v[j][h d_h + i]
-// W_O[h d_h + i][n].  One 64 x 64 tile of F per CTA (grid ceil(E/64),
-// ceil(r/64), H; block 16 x 16, 4 x 4 outputs per thread); i runs in order,
-// fp32 fma, rounded once to WT.
+// digest, Method, fused kernel §3.4): F[h r + j][n] = sum_i V_h[j][i]
+// W_O[h d_h + i][n], with V_h[j][i] at v[j sj + h sh + i]: the head's d_h
+// columns of the shared W^u_v (sj = E, sh = d_h) or the per-head factor
+// B_{Vh} stacked by head (sj = d_h, sh = r d_h).  One 64 x 64 tile of F per
+// CTA (grid ceil(E/64), ceil(r/64), H; block 16 x 16, 4 x 4 outputs per
+// thread); i runs in order, fp32 fma, rounded once to WT.
 template <typename WT>
 __global__ void __launch_bounds__(256)
 k_fold_vo(const WT* __restrict__ wuv, const WT* __restrict__ wo, WT* __restrict__ f, int E, int r,
-          int d_h) {
+          int d_h, long long sj, long long sh) {
   __shared__ float as[64][33];   // [j][i]
   __shared__ float bs[32][65];   // [i][n]
   const int n0 = blockIdx.x * 64, j0 = blockIdx.y * 64, h = blockIdx.z;
@@ -112,7 +114,7 @@ k_fold_vo(const WT* __restrict__ wuv, const WT* __restrict__ wo, WT* __restrict_
     for (int k = t; k < 64 * 32; k += 256) {
       const int jj = k / 32, ii = k % 32;
       const int j = j0 + jj, i = i0 + ii;
-      as[jj][ii] = (j < r && i < d_h) ? dev::to_f(wuv[size_t(j) * E + size_t(h) * d_h + i]) : 0.f;
+      as[jj][ii] = (j < r && i < d_h) ? dev::to_f(wuv[size_t(j) * sj + size_t(h) * sh + i]) : 0.f;
     }
     for (int k = t; k < 32 * 64; k += 256) {
       const int ii = k / 64, nn = k % 64;
@@ -145,10 +147,12 @@ k_fold_vo(const WT* __restrict__ wuv, const WT* __restrict__ wo, WT* __restrict_
 }
 
 template <typename WT>
-cudaError_t fold_vo_t(const qsvd_dims& d, const void* wuv, const void* wo, void* f, cudaStream_t s) {
+cudaError_t fold_vo_t(const qsvd_dims& d, const void* wuv, const void* wo, void* f, cudaStream_t s,
+                      bool per_head = false) {
   const dim3 grid((d.E + 63) / 64, (d.r + 63) / 64, d.H);
+  const long long sj = per_head ? d.d_h : d.E, sh = per_head ? (long long)d.r * d.d_h : d.d_h;
   k_fold_vo<WT><<<grid, dim3(16, 16), 0, s>>>(static_cast<const WT*>(wuv), static_cast<const WT*>(wo),
-                                              static_cast<WT*>(f), d.E, d.r, d.d_h);
+                                              static_cast<WT*>(f), d.E, d.r, d.d_h, sj, sh);
   note_launch();
   return check_launch();
 }
@@ -250,6 +254,37 @@ k_split_factors(const float* __restrict__ u, const float* __restrict__ vt, const
   }
 }
 
+// The split exponents of one beta: a_j = float(sigma_j^beta), b_j =
+// float(sigma_j^(1 - beta)), powers in float64.  One CTA, r <= 8192.
+__global__ void __launch_bounds__(256)
+k_beta_split(const float* __restrict__ sigma, double beta, float* __restrict__ a, float* __restrict__ b, int r) {
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    const double sj = double(sigma[j]);
+    a[j] = float(pow(sj, beta));
+    b[j] = float(pow(sj, 1.0 - beta));
+  }
+}
+
+// sum over i of (y_i - yq_i)^2 in float64, added into *out (zeroed first).
+__global__ void __launch_bounds__(256)
+k_sq_diff_sum(const float* __restrict__ y, const float* __restrict__ yq, size_t n, double* __restrict__ out) {
+  __shared__ double red[8];
+  double acc = 0.0;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x) {
+    const double d = double(y[i]) - double(yq[i]);
+    acc = fma(d, d, acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) t += red[w];
+    atomicAdd(out, t);
+  }
+}
+
 template <typename WT>
 cudaError_t split_factors_t(const qsvd_dims& d, const float* u, const float* vt, const float* a,
                             const float* b, void* wd, void* wuq, void* wuk, void* wuv, cudaStream_t s) {
@@ -274,6 +309,21 @@ cudaError_t launch_split_factors(const qsvd_dims& d, const float* u, const float
   }
 }
 
+cudaError_t launch_beta_split(const float* sigma, double beta, float* a, float* b, int r, cudaStream_t s) {
+  k_beta_split<<<1, 256, 0, s>>>(sigma, beta, a, b, r);
+  note_launch();
+  return check_launch();
+}
+
+cudaError_t launch_sq_diff_sum(const float* y, const float* yq, size_t n, double* out, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(double), s);
+  if (e != cudaSuccess) return e;
+  const unsigned blocks = unsigned(std::min<size_t>((n + 255) / 256, 148 * 4));
+  k_sq_diff_sum<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(y, yq, n, out);
+  note_launch();
+  return check_launch();
+}
+
 cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* packed,
                                     const PackedLayout& L, cudaStream_t s) {
   uint8_t* P = static_cast<uint8_t*>(packed);
@@ -285,6 +335,23 @@ cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* pa
     case QSVD_BF16: return fold_vo_t<__nv_bfloat16>(d, P + L.wuv, wo, P + L.wo, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_per_head_fold(const qsvd_dims& d, const void* bv, const void* wo, void* f, cudaStream_t s) {
+  switch (d.weight_dtype) {
+    case QSVD_F16: return fold_vo_t<__half>(d, bv, wo, f, s, true);
+    case QSVD_BF16: return fold_vo_t<__nv_bfloat16>(d, bv, wo, f, s, true);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_rope_table(float* tab, int max_len, int d_h, float base, cudaStream_t s) {
+  const int half = d_h / 2;
+  const size_t n = size_t(max_len) * half;
+  const unsigned blocks = unsigned(std::min<size_t>((n + 255) / 256, 4096));
+  k_rope_table<<<blocks, 256, 0, s>>>(tab, max_len, half, std::log(double(base)), d_h);
+  note_launch();
+  return check_launch();
 }
 
 }  // namespace qsvd

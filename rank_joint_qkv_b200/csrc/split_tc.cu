@@ -73,6 +73,12 @@ constexpr int kMaxGroupBufs = 4;               // S accumulators per channel gro
 constexpr int kMaxRaw = 8;                     // raw-code slots per stream (quantised latent)
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
+// Failure injection for tests (qsvd_testing_set_score_wait_ns): when
+// non-zero, the softmax warps start their first tile by waiting on a barrier
+// that is never released, giving up after this many nanoseconds -- the
+// timeout path runs without any fault.  0: no injection.
+__device__ unsigned long long g_score_wait_ns = 0;
+
 
 // Shared-memory carve.  Both rings carry items of 1/(r/64) of a tile.
 //   S slot: one 64-channel box of the latent tile (128 tokens x 128 bytes,
@@ -113,6 +119,7 @@ struct Smem {
   uint8_t* zraw;
   uint64_t* sraw_full;   // [kMaxRaw]
   uint64_t* zraw_full;   // [kMaxRaw]
+  uint64_t* never;       // never released (failure injection)
   float* red;            // [4][NP] per-warp partial max / sum
   float* m_run;          // [NP] running reference max per head (log2 domain)
   float* l_run;          // [NP] running sum of P per head
@@ -148,6 +155,7 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   s.sg_empty = s.sg_full + kMaxGroupBufs;
   s.sraw_full = s.sg_empty + kMaxGroupBufs;
   s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + 2 kMaxRaw = 64 barriers
+  s.never = s.zraw_full + kMaxRaw;       // the 65th (the barrier area holds 80)
   static_assert(640 + 4 * NP * 4 + 32 + 3 * NP * 4 <= kMiscBytes, "misc region");
   s.red = reinterpret_cast<float*>(m + 640);
   s.tmem_holder = reinterpret_cast<uint32_t*>(m + 640 + 4 * NP * 4);
@@ -566,6 +574,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       mbar_init(saddr(&s.sraw_full[i]), 1);
       mbar_init(saddr(&s.zraw_full[i]), 1);
     }
+    mbar_init(saddr(s.never), 1);
     for (int i = 0; i < nz; ++i) {
       mbar_init(saddr(&s.z_full[i]), 1);
       mbar_init(saddr(&s.z_empty[i]), 1);
@@ -710,6 +719,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     const int q = warp & 3;
     const int t = 32 * q + lane;              // token row in the tile == TMEM lane
     const uint32_t lane_off = uint32_t(32 * q) << 16;
+    const uint64_t inject_ns = g_score_wait_ns;
     // m and l per head live in shared memory (identical for the four warps);
     // thread t < NP owns head t's entries
     TileIter it;
@@ -720,6 +730,10 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       const bool first = it.first(tb), last = it.last();
       const int nv = it.nvalid();
       int fail = 0;
+      if (inject_ns && i == 0 && group_or(!mbar_wait_ns(saddr(s.never), 0, inject_ns))) {
+        if (t == 0) set_abort(s, status);
+        break;
+      }
       float sv[NP];
       if (QB) {
         // s_t = sum_g scale_{t,g} (codes_{t,g} . qt_g), one TMEM buffer per group
@@ -1372,6 +1386,10 @@ cudaError_t launch_split_tc_scores(const qsvd_dims& d, const float* scores, cons
     return np == 16 ? QSVD_SG(16, true) : np == 32 ? QSVD_SG(32, true) : QSVD_SG(48, true);
   return np == 16 ? QSVD_SG(16, false) : np == 32 ? QSVD_SG(32, false) : QSVD_SG(48, false);
 #undef QSVD_SG
+}
+
+cudaError_t set_score_wait_ns(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_score_wait_ns, &ns, sizeof(ns));
 }
 
 bool rope_tc_supported(const qsvd_dims& d) {

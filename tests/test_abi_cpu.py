@@ -238,3 +238,19 @@ def test_split_factors_pointers_checked_on_host():
     st = q._lib.qsvd_split_factors(ctypes.byref(d), fake, fake, fake, None, fake, fake, fake, fake, None)
     assert st == q.QSVD_ERR_INVALID_ARG
     assert b"NULL" in q._lib.qsvd_last_error()
+
+
+def test_prefill_attention_host_checks():
+    """Workspace size and refusals of qsvd_prefill_attention, no GPU."""
+    d = q.make_dims(512, 4, 128, 256, 3, 305, cache="f16", weight="f16")
+    n = 3 * 305
+    al = lambda x: (x + 255) // 256 * 256
+    want = al(n * 512 * 4) + 6 * al(n * 512 * 2)
+    assert q.prefill_attention_workspace_bytes(d) == want
+    for bad in (q.make_dims(512, 8, 64, 256, 3, 305, cache="f16", weight="f16"),      # d_h 64
+                q.make_dims(512, 4, 128, 256, 3, 305, cache="i4", weight="f16"),      # int cache
+                q.make_dims(512, 4, 128, 256, 3, 305, cache="bf16", weight="f16"),    # mixed types
+                q.make_dims(640, 5, 128, 256, 3, 305, cache="f16", weight="f16")):    # E % 256
+        with pytest.raises(q.QsvdError) as e:
+            q.prefill_attention_workspace_bytes(bad)
+        assert e.value.status == q.QSVD_ERR_UNSUPPORTED

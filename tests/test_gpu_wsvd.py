@@ -50,6 +50,7 @@ def _case(E, H, r, lengths, cache, weight):
         cv=oi.as_torch(oi.to_device_dtype(cv, cache), cache).cuda(),
         q=torch.from_numpy(qv).cuda(),
         lengths=torch.tensor(lengths, dtype=torch.int32).cuda())
+    dev["host"] = ([ck[b] for b in range(len(lengths))], [cv[b] for b in range(len(lengths))], qv, fk, fv)
     return dims, dev, want
 
 
@@ -169,3 +170,53 @@ def test_latents_from_prefill(cuda_ok):
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
     assert rel_err(out.cpu().numpy(), want) <= TOL
+
+
+@pytest.mark.parametrize("weight", ["f16", "bf16"])
+def test_value_factor_folded_into_output_projection(cuda_ok, weight):
+    """B_{Vh} folded into W_O on the GPU (WSVD digest, Method, fused kernel
+    §3.4): F = [B_{Vh} W_{O,h}]_h against the oracle's fold (float32
+    accumulation over d_h terms plus one rounding to the weight type), and
+    the folded decode y = z F against the oracle's merged latents times the
+    stored F (float32 arithmetic: the per-head bar)."""
+    E, H, r, lengths = 512, 4, 64, [300, 1, 130]
+    d_h = E // H
+    dims, dev, _ = _case(E, H, r, lengths, weight, weight)
+    g = np.random.default_rng(3)
+    wo = oi.from_device_dtype(oi.to_device_dtype(g.standard_normal((E, E)) / np.sqrt(E), weight), weight)
+    wo_t = oi.as_torch(oi.to_device_dtype(wo, weight), weight).cuda()
+    f = q.qsvd_prepare_per_head_fold(dims, dev["bv"], wo_t)
+    torch.cuda.synchronize()
+    f_np = f.float().cpu().numpy().astype(np.float64)
+    ck, cv, qv, fk, fv = dev["host"]
+    f64 = wr.fold_values(fv, wo)
+    acc = np.concatenate([np.abs(b) @ np.abs(wo[h * d_h:(h + 1) * d_h]) for h, (_, b) in enumerate(fv)])
+    ulp = 2.0 ** (-11 if weight == "f16" else -8)
+    assert np.all(np.abs(f_np - f64) <= ulp * np.abs(f64) + d_h * 2.0 ** -23 * acc + 1e-30)
+    dims.out_proj = q.OUT_PROJ_CODE["fold"]
+    out = torch.full((dims.batch, E), float("nan"), dtype=torch.float32, device="cuda")
+    ws = q.qsvd_decode_attn_per_head(dims, dev["bk"], f, dev["q"], dev["ck"], dev["cv"], dev["lengths"], out)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    z = wr.decode_latents(ck, cv, np.asarray(lengths), qv.astype(np.float64), fk)
+    want = z.reshape(len(lengths), -1) @ f_np
+    assert rel_err(out.cpu().numpy(), want) <= TOL
+
+
+@pytest.mark.parametrize("r,dt,layout", [(64, "f16", q.QSVD_PER_HEAD_HEAD_MAJOR),
+                                         (128, "bf16", q.QSVD_PER_HEAD_TOKEN_MAJOR),
+                                         (64, "f16", q.QSVD_PER_HEAD_TOKEN_MAJOR)])
+def test_rotary_keys_rebuilt_on_tensor_cores(cuda_ok, r, dt, layout):
+    """Rotary mode (WSVD digest, Method §3.4: keys rebuilt from the per-head
+    latent tile and rotated before the scores): K_h = C_{Kh} B_{Kh} on
+    tcgen05, rotated at each position, the query at len - 1; against the
+    oracle's rebuilt-key decode.  Bar: 2e-3 (16-bit operands, float32
+    tensor-core accumulation)."""
+    E, H, lengths = 512, 4, [300, 1, 513]
+    dims, dev, _ = _case(E, H, r, lengths, dt, dt)
+    ck, cv, qv, fk, fv = dev["host"]
+    want = wr.decode(ck, cv, np.asarray(lengths), qv.astype(np.float64), fk, fv, rope_base=10000.0)
+    dims.rope, dims.rope_base = 1, 10000.0
+    got, status = _run(dims, dev, layout=layout)
+    assert status == 0
+    assert rel_err(got, want) <= 2e-3

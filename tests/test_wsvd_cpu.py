@@ -28,11 +28,11 @@ def _align(n):
     return (n + 255) // 256 * 256
 
 
-def _layout(B, H, r, max_len):
+def _layout(B, H, r, max_len, d_h=128):
     S = (max_len + CHUNK - 1) // CHUNK
     o = 0
     hdr = o; o = _align(o + 16)
-    qt = o; o = _align(o + B * H * r * 4)
+    qt = o; o = _align(o + B * H * max(r, d_h) * 4)
     m = o; o = _align(o + B * H * S * 4)
     l_ = o; o = _align(o + B * H * S * 4)
     z = o; o = _align(o + B * H * S * r * 4)
@@ -47,9 +47,12 @@ def test_workspace_size_matches_layout(shape):
     assert q.per_head_workspace_bytes(d) == want
 
 
-@pytest.mark.parametrize("bad,status", [(dict(rope=True), q.QSVD_ERR_UNSUPPORTED),
+@pytest.mark.parametrize("bad,status", [(dict(rope=True, r=96), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(rope=True, cache="f32"), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(rope=True, cache="bf16"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(cache="i4", r=128), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(out_proj="chain"), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(out_proj="fold", weight="f32"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(h2=True, h2_m=2), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(r=48), q.QSVD_ERR_INVALID_ARG)])
 def test_refusals_on_host(bad, status):
@@ -151,3 +154,60 @@ def test_index_replay(B, H, d_h, r, max_len, lengths, token_major):
         ln = min(max(lengths[b], 0), max_len)
         assert np.all(rows[b, :, :ln] == 1) and np.all(rows[b, :, ln:] == 0)
     assert smem * 4 <= 227 * 1024
+
+
+def _replay_vec(B, H, r, max_len, lengths, token_major):
+    """The 16-byte-vector split kernel (16-bit latents, r in {64, 128, 256}):
+    grid (S, H, B), 256 threads; thread (vj = tid % (r / 8), tg = tid // (r / 8))
+    reads vector vj of rows t = p * (256 / (r / 8)) + tg.  Returns how often
+    each element of the cache is read (keys; the value side is identical)."""
+    TPR = r // 8
+    TPP = 256 // TPR
+    NP = CHUNK // TPP
+    assert NP * TPP == CHUNK
+    S = (max_len + CHUNK - 1) // CHUNK
+    n_cache = B * H * max_len * r
+    hits = np.zeros(n_cache, np.int64)
+    for b in range(B):
+        ln = min(max(int(lengths[b]), 0), max_len)
+        for h in range(H):
+            for sp in range(S):
+                t0 = sp * CHUNK
+                if t0 >= ln:
+                    continue
+                n = min(CHUNK, ln - t0)
+                row0 = (b * max_len + t0) * H + h if token_major else (b * H + h) * max_len + t0
+                rsv = (H * r if token_major else r) // 8
+                for tid in range(256):
+                    vj, tg = tid % TPR, tid // TPR
+                    assert tg < TPP and 8 * vj + 7 < r            # zr[tg][8 vj + e]
+                    for p in range(NP):
+                        t = p * TPP + tg
+                        assert t < CHUNK                            # ss[t]
+                        if t >= n:
+                            continue
+                        v = row0 * r // 8 + vj + t * rsv            # 16-byte vector index
+                        assert (row0 * r) % 8 == 0
+                        lo = 8 * v
+                        assert 0 <= lo and lo + 8 <= n_cache
+                        hits[lo:lo + 8] += 1
+    return hits
+
+
+@pytest.mark.parametrize("B,H,r,max_len,lengths", [
+    (3, 4, 64, 700, [700, 1, 300]),
+    (2, 2, 128, 513, [513, 0]),
+    (1, 2, 256, 1000, [777]),
+    (2, 2, 64, 300, [-5, 9999]),
+])
+@pytest.mark.parametrize("token_major", [False, True])
+def test_vector_split_index_replay(B, H, r, max_len, lengths, token_major):
+    hits = _replay_vec(B, H, r, max_len, lengths, token_major)
+    want = np.zeros((B, max_len, H, r) if token_major else (B, H, max_len, r), np.int64)
+    for b in range(B):
+        ln = min(max(lengths[b], 0), max_len)
+        if token_major:
+            want[b, :ln] = 1
+        else:
+            want[b, :, :ln] = 1
+    assert np.array_equal(hits, want.reshape(-1))    # every valid element once, nothing else
