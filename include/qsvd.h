@@ -403,9 +403,14 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  * W_{Vh} = A_{Vh} B_{Vh}.  With tau = dims->softmax_scale (<= 0: 1/sqrt(d_h)):
  *   qt_h = tau B_{Kh} q_h,  s_t = C_{Kh,t} . qt_h,  p = softmax(s),
  *   o_h = (p^T C_{Vh}) B_{Vh}.
- * No rotary embedding (dims->rope must be 0).  Computed in float32 on CUDA
- * cores, 256 tokens per split CTA, chunks merged in the log2 domain; 16-bit
- * latents with r = 64, 128 or 256 are read as 16-byte vectors.
+ * Computed in float32 on CUDA cores, 256 tokens per split CTA, chunks merged
+ * in the log2 domain; 16-bit latents with r = 64, 128 or 256 are read as
+ * 16-byte vectors.  With dims->rope (rotary mode; d_h == 128, r = 64 or
+ * 128, an F16 or BF16 cache of the weight type): keys are rebuilt per
+ * 128-token tile on the tensor cores, K_h = C_{Kh} B_{Kh}, rotated to their
+ * positions and dotted with the query rotated to len_b - 1 (base
+ * dims->rope_base; the cos/sin table of every position, from float64 angles,
+ * is built in the workspace by each call).
  *   bk, bv     device, H x r x d_h each, weight_dtype (F32, F16 or BF16):
  *              B_{Kh} and B_{Vh} stacked by head.  With dims->out_proj ==
  *              QSVD_OUT_PROJ_FOLD (16-bit weights), bv is instead the fold
@@ -428,9 +433,10 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  *              status word.
  *   out        device, B x E, out_dtype.
  * Stream-ordered; nothing is allocated.
- * Errors: INVALID_ARG (also an unknown layout), UNSUPPORTED (rotary mode,
- * int caches, online H2, the chained output projection, the fold with
- * float32 weights, max_len beyond ~50 M tokens), WORKSPACE, CUDA.
+ * Errors: INVALID_ARG (also an unknown layout), UNSUPPORTED (rotary mode
+ * outside the shapes above, int caches, online H2, the chained output
+ * projection, the fold with float32 weights, max_len beyond ~50 M tokens),
+ * WORKSPACE, CUDA.
  */
 #define QSVD_PER_HEAD_HEAD_MAJOR 0
 #define QSVD_PER_HEAD_TOKEN_MAJOR 1

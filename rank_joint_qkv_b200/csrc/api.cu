@@ -469,7 +469,7 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
   if (!workspace_bytes) return fail(QSVD_ERR_INVALID_ARG, "workspace_bytes is NULL");
   if (d.rope && !wsvd_rope_supported(d))
     return fail(QSVD_ERR_UNSUPPORTED,
-                "per-head latents, rotary mode: d_h == 128, r in {64, 128, 256}, an F16 or BF16 cache "
+                "per-head latents, rotary mode: d_h == 128, r in {64, 128}, an F16 or BF16 cache "
                 "of the weight type");
   if (cache_is_int(d)) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: F32, F16 or BF16 caches");
   if (d.h2 || d.out_proj == QSVD_OUT_PROJ_CHAIN)

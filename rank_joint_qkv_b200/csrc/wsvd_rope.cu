@@ -5,13 +5,14 @@
 // scaled by tau log2(e); s_t = q'_h . R(t) K_h[t].  Values stay in latent
 // space (z_h = p^T C_{Vh}, o_h = z_h B_{Vh}) as in the absorbed mode.
 //
-// k_wsvd_rope_scores, one CTA per (128 tokens, head, sequence), 128 threads:
-// the latent tile (128 x r, K-major) and B_{Kh} (r x d_h, read in place as the
-// MN-major B operand) arrive by TMA (128-byte swizzle); one thread issues
-// r / 16 tcgen05 MMAs (M = 128 tokens, N = d_h = 128, K = 16) into TMEM; every
-// thread then takes its token's key row (TMEM lane = token), rotates the
-// pairs (i, i + 64) with the fp64-built cos/sin row of its position and dots
-// it with the rotated query.  Both MMA operands are the stored 16-bit values,
+// k_wsvd_rope_scores, one CTA per (128 tokens, sequence) walking the heads:
+// per head the latent tile (128 x r, K-major) and B_{Kh} (r x d_h, read in
+// place as the MN-major B operand) arrive by TMA (128-byte swizzle, two
+// stages); one thread issues r / 16 tcgen05 MMAs (M = 128 tokens, N = d_h =
+// 128, K = 16) into one of two TMEM buffers; every epilogue thread then takes
+// its token's key row (TMEM lane = token), rotates the pairs (i, i + 64) with
+// the fp64-built cos/sin row of its position (staged once for all heads) and
+// dots it with the rotated query.  Both MMA operands are the stored 16-bit values,
 // so every product is exact and only the float32 accumulation rounds.  The
 // scores ([B][H][max_len]) go to the chunk kernel of split_wsvd.cu, which
 // runs the softmax and the value side.
@@ -25,8 +26,6 @@
 
 namespace qsvd {
 namespace {
-
-constexpr int kWrT = 128;   // threads (tokens) per scores CTA
 
 // q'[b][h][i] = sl2 R(len_b - 1) q[b][h d + i], pairs (i, i + d/2).  grid (H, B).
 __global__ void __launch_bounds__(128)
@@ -51,102 +50,164 @@ k_wsvd_rope_query(const float* __restrict__ q, const int32_t* __restrict__ lengt
   }
 }
 
-// grid (ceil(max_len / 128), H, B), block 128.  R: per-head rank (64, 128 or
-// 256); d_h = 128.  TMA maps: latent rows (head-major: 2D {r, rows}; token-
-// major: 3D {r, H, B max_len} with a box one head high), B_K as 2D {d_h, H r}.
+// grid (ceil(max_len / 128), B), block 160.  R: per-head rank (64 or 128);
+// d_h = 128.  One CTA walks every head of its 128 positions: warp 4's
+// first thread loads (TMA: the head's latent tile and B_{Kh}, two stages)
+// and issues the MMAs into one of two TMEM buffers; warps 0-3 (TMEM lanes
+// 32 w .., one token each) rotate and score, with the positions' cos/sin rows
+// staged once in shared memory for all heads.  TMA maps: latent rows
+// (head-major: 2D {r, rows}; token-major: 3D {r, H, B max_len} with a box one
+// head high), B_K as 2D {d_h, H r}.
+constexpr int kWrTab = 130;   // floats per staged table row (pitch: 2-way bank conflicts at most)
 template <bool BF16, int R>
-__global__ void __launch_bounds__(kWrT)
+__global__ void __launch_bounds__(160, 1)
 k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
                    const float* __restrict__ qr, const float* __restrict__ tab,
                    const int32_t* __restrict__ lengths, float* __restrict__ scores,
                    int32_t* __restrict__ status, int H, int max_len, int token_major) {
   constexpr int D = 128, NB = R / 64;
-  constexpr int CBYTES = 128 * R * 2, BBYTES = R * D * 2;
+  constexpr int CBYTES = 128 * R * 2, BBYTES = R * D * 2, STAGE = CBYTES + BBYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + CBYTES + BBYTES);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2);
-  __shared__ float qs[D];
+  float* tabs = reinterpret_cast<float*>(base + 2 * STAGE);            // [128][kWrTab]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 128 * kWrTab);
+  uint64_t* full = bars;        // [2] stage loaded
+  uint64_t* empty = bars + 2;   // [2] stage's MMAs done
+  uint64_t* done = bars + 4;    // [2] TMEM buffer holds a head's keys
+  uint64_t* tfree = bars + 6;   // [2] TMEM buffer read by the epilogue
+  uint64_t* drain = bars + 8;   // the MMA thread's last commit
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int b = blockIdx.y;
   const int len = min(max(lengths[b], 0), max_len);
   const int t0 = blockIdx.x * 128;
   if (t0 >= len) return;   // uniform across the CTA, before any barrier or TMEM use
   const uint32_t s0 = saddr(base);
-  const uint32_t full = saddr(&bars[0]), done = saddr(&bars[1]);
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(saddr(&full[i]), 1);
+      mbar_init(saddr(&empty[i]), 1);
+      mbar_init(saddr(&done[i]), 1);
+      mbar_init(saddr(&tfree[i]), 1);
+    }
+    mbar_init(saddr(drain), 1);
+    *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(
+  if (warp == 4) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
                      saddr(tmem_holder))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     tc_fence_before();
+  } else {
+    // this token's cos/sin row (64 pairs), staged once for every head
+    const int p = t0 + threadIdx.x;
+    const float4* src = reinterpret_cast<const float4*>(tab + size_t(p < max_len ? p : 0) * D);
+    float* dst = tabs + threadIdx.x * kWrTab;
+#pragma unroll 8
+    for (int v = 0; v < D / 4; ++v) {
+      const float4 x = __ldg(src + v);
+      dst[4 * v] = x.x; dst[4 * v + 1] = x.y; dst[4 * v + 2] = x.z; dst[4 * v + 3] = x.w;
+    }
   }
-  for (int i = threadIdx.x; i < D; i += kWrT) qs[i] = qr[(size_t(b) * H + h) * D + i];
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(full, uint32_t(CBYTES + BBYTES));
-#pragma unroll
-    for (int kb = 0; kb < NB; ++kb) {
-      if (token_major)
-        tma_load_3d_hint(s0 + kb * 128 * 128, &tm_c, 64 * kb, h, b * max_len + t0, full, policy_evict_first());
-      else
-        tma_load_2d(s0 + kb * 128 * 128, &tm_c, 64 * kb, (b * H + h) * max_len + t0, full);
-    }
-    tma_load_2d(s0 + CBYTES, &tm_b, 0, h * R, full);
-    tma_load_2d(s0 + CBYTES + R * 128, &tm_b, 64, h * R, full);
-    ok = mbar_wait(full, 0);
-    if (ok) {
-      tc_fence_after();
+
+  if (warp == 4) {
+    if (lane == 0) {
       constexpr uint32_t id = idesc_f16(128, D, BF16, false, true);   // B MN-major
+      bool ok = true;
+      int issued = 0;
+      auto load = [&](int h) -> bool {
+        const int st = h & 1;
+        if (!mbar_wait(saddr(&empty[st]), (uint32_t(h >> 1) & 1u) ^ 1u)) return false;
+        const uint32_t dst = s0 + uint32_t(st * STAGE), fb = saddr(&full[st]);
+        mbar_expect_tx(fb, uint32_t(STAGE));
 #pragma unroll
-      for (int kk = 0; kk < R / 16; ++kk) {   // K = 16 latent channels per MMA
-        const uint64_t a = sdesc(s0 + uint32_t((kk >> 2) * 128 * 128 + (kk & 3) * 32), 16, 1024);
-        const uint64_t bd = sdesc(s0 + CBYTES + uint32_t(kk * 16 * 128), R * 128, 1024);
-        tc_mma(tmem, a, bd, id, kk > 0 ? 1u : 0u);
+        for (int kb = 0; kb < NB; ++kb) {
+          if (token_major)
+            tma_load_3d_hint(dst + kb * 128 * 128, &tm_c, 64 * kb, h, b * max_len + t0, fb, policy_evict_first());
+          else
+            tma_load_2d(dst + kb * 128 * 128, &tm_c, 64 * kb, (b * H + h) * max_len + t0, fb);
+        }
+        tma_load_2d(dst + CBYTES, &tm_b, 0, h * R, fb);
+        tma_load_2d(dst + CBYTES + R * 128, &tm_b, 64, h * R, fb);
+        ++issued;
+        return true;
+      };
+      ok = load(0);
+      for (int h = 0; h < H && ok; ++h) {
+        if (h + 1 < H && !load(h + 1)) { ok = false; break; }
+        const int st = h & 1;
+        if (!mbar_wait(saddr(&full[st]), uint32_t(h >> 1) & 1u)) { ok = false; break; }
+        if (h >= 2 && !mbar_wait(saddr(&tfree[st]), uint32_t((h - 2) >> 1) & 1u)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sb = s0 + uint32_t(st * STAGE);
+#pragma unroll
+        for (int kk = 0; kk < R / 16; ++kk) {   // K = 16 latent channels per MMA
+          const uint64_t a = sdesc(sb + uint32_t((kk >> 2) * 128 * 128 + (kk & 3) * 32), 16, 1024);
+          const uint64_t bd = sdesc(sb + CBYTES + uint32_t(kk * 16 * 128), R * 128, 1024);
+          tc_mma(tmem + uint32_t(st * D), a, bd, id, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(saddr(&done[st]));
+        tc_commit(saddr(&empty[st]));
+        if (*abort_flag) ok = false;
       }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(status, QSVD_STATUS_TIMEOUT);
+        // every copy issued has landed before the CTA may leave
+        for (int h = issued > 2 ? issued - 2 : 0; h < issued; ++h)
+          mbar_wait(saddr(&full[h & 1]), uint32_t(h >> 1) & 1u);
+      }
+      tc_commit(saddr(drain));   // every MMA issued has completed before TMEM is freed
+      mbar_wait(saddr(drain), 0);
     }
-    tc_commit(done);   // also when nothing was issued: the epilogue's wait completes
-  }
-  __syncwarp();
-  const bool got = __syncthreads_and(mbar_wait(done, 0) && ok);
-  if (!got) {
-    if (threadIdx.x == 0) atomicOr(status, QSVD_STATUS_TIMEOUT);
+    __syncwarp();
   } else {
-    tc_fence_after();
     const int t = threadIdx.x, p = t0 + t;
-    const uint32_t ta = tmem + (uint32_t(32 * warp) << 16);
-    const float* trow = tab + size_t(p < max_len ? p : 0) * D;   // (cos, sin) x 64
-    float s = 0.f;
-#pragma unroll 1
-    for (int i0 = 0; i0 < 64; i0 += 16) {
-      float klo[16], khi[16];
-      tmem_ld16(ta + uint32_t(i0), klo);
-      tmem_ld16(ta + uint32_t(64 + i0), khi);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int j = i0 + e;
-        const float2 cs = *reinterpret_cast<const float2*>(trow + 2 * j);
-        s = fmaf(qs[j], fmaf(klo[e], cs.x, -khi[e] * cs.y), s);
-        s = fmaf(qs[64 + j], fmaf(khi[e], cs.x, klo[e] * cs.y), s);
+    const uint32_t lane_off = uint32_t(32 * warp) << 16;
+    const float* trow = tabs + t * kWrTab;
+    for (int h = 0; h < H; ++h) {
+      const int st = h & 1;
+      if (group_or(!mbar_wait(saddr(&done[st]), uint32_t(h >> 1) & 1u))) {
+        if (t == 0) { *abort_flag = 1; atomicOr(status, QSVD_STATUS_TIMEOUT); }
+        break;
       }
+      tc_fence_after();
+      const float* qh = qr + (size_t(b) * H + h) * D;
+      const uint32_t ta = tmem + lane_off + uint32_t(st * D);
+      float s = 0.f;
+#pragma unroll 1
+      for (int i0 = 0; i0 < 64; i0 += 16) {
+        float klo[16], khi[16];
+        tmem_ld16(ta + uint32_t(i0), klo);
+        tmem_ld16(ta + uint32_t(64 + i0), khi);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = i0 + e;
+          const float c = trow[2 * j], sn = trow[2 * j + 1];
+          s = fmaf(__ldg(qh + j), fmaf(klo[e], c, -khi[e] * sn), s);
+          s = fmaf(__ldg(qh + 64 + j), fmaf(khi[e], c, klo[e] * sn), s);
+        }
+      }
+      tc_fence_before();
+      group_sync();
+      if (t == 0) mbar_arrive(saddr(&tfree[st]));
+      if (p < len) scores[(size_t(b) * H + h) * max_len + p] = s;
+      if (group_or(*abort_flag)) break;
     }
-    if (p < len) scores[(size_t(b) * H + h) * max_len + p] = s;
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 4) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
   }
 }
 
@@ -189,12 +250,12 @@ cudaError_t scores_t(const qsvd_dims& d, const void* bk, const void* ck, const f
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int smem = 1024 + 128 * R * 2 + R * 128 * 2 + 64;
+  const int smem = 1024 + 2 * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128;
   auto kern = k_wsvd_rope_scores<BF16, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((d.max_len + 127) / 128, d.H, d.batch), kWrT, smem, s>>>(tc, tb, qr, tab, lengths, scores, status,
-                                                                     d.H, d.max_len, token_major);
+  kern<<<dim3((d.max_len + 127) / 128, d.batch), 160, smem, s>>>(tc, tb, qr, tab, lengths, scores, status,
+                                                               d.H, d.max_len, token_major);
   note_launch();
   return check_launch();
 }
@@ -205,7 +266,6 @@ cudaError_t scores_r(const qsvd_dims& d, const void* bk, const void* ck, const f
   switch (d.r) {
     case 64: return scores_t<BF16, 64>(d, bk, ck, qr, tab, lengths, scores, status, tm, s);
     case 128: return scores_t<BF16, 128>(d, bk, ck, qr, tab, lengths, scores, status, tm, s);
-    case 256: return scores_t<BF16, 256>(d, bk, ck, qr, tab, lengths, scores, status, tm, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -214,7 +274,7 @@ cudaError_t scores_r(const qsvd_dims& d, const void* bk, const void* ck, const f
 
 bool wsvd_rope_supported(const qsvd_dims& d) {
   return d.d_h == 128 && (d.cache_dtype == QSVD_F16 || d.cache_dtype == QSVD_BF16) &&
-         d.weight_dtype == d.cache_dtype && (d.r == 64 || d.r == 128 || d.r == 256);
+         d.weight_dtype == d.cache_dtype && (d.r == 64 || d.r == 128);   // a head's key rank is <= d_h
 }
 
 cudaError_t launch_wsvd_rope_front(const qsvd_dims& d, const void* bk, const float* q, const void* ck,
