@@ -80,18 +80,23 @@ def bench_inputs(cfg: int, device: str, rank: int = 0, cache: Optional[str] = No
             rows = torch.randn((max_len, r), generator=gen, device=device) * cs_t
             cache[b].copy_(rows)
     else:
-        # random codes on the symmetric grid and positive fp16 group scales
-        g = w.group
-        if w.cache == "i8":
-            cache = torch.randint(-127, 128, (B, max_len, r), generator=gen, device=device,
-                                  dtype=torch.int8)
-        else:
-            lo = torch.randint(-7, 8, (B, max_len, r // 2), generator=gen, device=device)
-            hi = torch.randint(-7, 8, (B, max_len, r // 2), generator=gen, device=device)
-            cache = ((lo & 0xF) | ((hi & 0xF) << 4)).to(torch.uint8)
-        grp = cs_t.view(r // g, g).amax(dim=1) * 3.0 / (7 if w.cache == "i4" else 127)
-        scales = (grp[None, None, :] * (0.5 + torch.rand((B, max_len, r // g), generator=gen,
-                                                          device=device))).to(torch.float16)
+        # rows drawn as in the 16-bit case, then quantised per (token, group):
+        # fp16 scale = group amax / qmax, code = rint(value / scale) (the
+        # latent quantiser's own rule), int4 packed two codes per byte
+        g, qmax = w.group, (7 if w.cache == "i4" else 127)
+        cache = torch.empty((B, max_len, r if w.cache == "i8" else r // 2),
+                            dtype=torch.int8 if w.cache == "i8" else torch.uint8, device=device)
+        scales = torch.empty((B, max_len, r // g), dtype=torch.float16, device=device)
+        for b in range(B):
+            rows = (torch.randn((max_len, r), generator=gen, device=device) * cs_t).view(max_len, r // g, g)
+            sc = (rows.abs().amax(dim=2) / qmax).to(torch.float16)
+            codes = torch.round(rows / sc.float().clamp_min(1e-30)[..., None]).clamp_(-qmax, qmax)
+            codes = codes.to(torch.int8).view(max_len, r)
+            scales[b].copy_(sc)
+            if w.cache == "i8":
+                cache[b].copy_(codes)
+            else:
+                cache[b].copy_(((codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)).to(torch.uint8))
     wuq, wuk, wuv = (torch.from_numpy(a).to(device=device, dtype=TORCH_DT[w.weight])
                      for a in synthetic.direct_up_weights_np(w))
     wd = torch.from_numpy(synthetic.direct_down_weight_np(w)).to(device=device,

@@ -327,6 +327,13 @@ qsvd_status qsvd_prefill_attention(const qsvd_dims* dims, const void* packed, co
   return QSVD_OK;
 }
 
+// Quantised latent on the tensor cores: the int8 query parts [B][3][H][r]
+// take the first three quarters of the 16-bit parts' section ([B][2][H][r]
+// 16-bit), their per-(sequence, head) scales [B][H] the rest.
+static float* quant_query_scales(const qsvd_dims& d, void* qt16) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(qt16) + size_t(3) * d.batch * d.H * d.r);
+}
+
 static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const float* qin,
                                int qin_is_latent, const void* cache, const void* scales,
                                const int32_t* lengths, int num_splits, void* workspace,
@@ -403,9 +410,18 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     if (d.rope)
       e = launch_rope_query(d, qsrc, sched, rope_tab, sl2, qt32, s);
     else
-      // only the copy the split kernel reads: fp32 for CUDA cores, 16-bit hi/lo for tensor cores
-      e = launch_absorb(d, qsrc, P + L.wuk, sl2, kernel == QSVD_KERNEL_SIMT ? qt32 : nullptr,
-                        kernel == QSVD_KERNEL_SIMT ? nullptr : qt16, &hdr->status, s);
+      // only the copy the split kernel reads: fp32 for CUDA cores, 16-bit hi/lo
+      // for tensor cores; a quantised latent on the tensor cores takes int8
+      // parts (in the 16-bit parts' section) with their scales and offset
+      // terms (in the fp32 section, unused on that path)
+      if (kernel != QSVD_KERNEL_SIMT && cache_is_int(d)) {
+        e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, nullptr, &hdr->status, s);
+        if (e == cudaSuccess)
+          e = launch_quant_query(d, qt32, static_cast<int8_t*>(qt16), quant_query_scales(d, qt16), s);
+      } else {
+        e = launch_absorb(d, qsrc, P + L.wuk, sl2, kernel == QSVD_KERNEL_SIMT ? qt32 : nullptr,
+                          kernel == QSVD_KERNEL_SIMT ? nullptr : qt16, &hdr->status, s);
+      }
     if (e != cudaSuccess) return cuda_fail(e, "query prologue");
   }
   if (split_any) {
@@ -426,7 +442,8 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
     else if (kernel == QSVD_KERNEL_TCGEN05_CLUSTER)
       e = launch_split_cl(d, cache, qt16, sched, G, pm, pl, pz, &hdr->status, s);
     else if (kernel == QSVD_KERNEL_TCGEN05_CTA)
-      e = launch_split_tc(d, cache, scales, qt16, sched, G, pm, pl, pz, &hdr->status, s);
+      e = launch_split_tc(d, cache, scales, qt16, sched, G, pm, pl, pz, &hdr->status, s,
+                          quant_query_scales(d, qt16));
     else
       e = launch_split_simt_absorbed(d, qt32, cache, scales, sched, G, pm, pl, pz, s);
     if (e != cudaSuccess) return cuda_fail(e, "split phase");

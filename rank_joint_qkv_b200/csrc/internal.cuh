@@ -201,6 +201,9 @@ cudaError_t launch_q_partial(const qsvd_dims& d, const float* qin, const void* w
 // tensor cores) are each written only when non-null.
 cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, float scale_log2,
                           float* qt32, void* qt16, int32_t* status, cudaStream_t s);
+// Quantised latent on the tensor cores: qt32 [B][H][r] -> three int8 parts
+// qp [B][3][H][r] and one power-of-two scale qs [B][H] per (sequence, head).
+cudaError_t launch_quant_query(const qsvd_dims& d, const float* qt, int8_t* qp, float* qs, cudaStream_t s);
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,
                               const float* rope_tab, float scale_log2, float* qrot,
                               cudaStream_t s);
@@ -241,7 +244,7 @@ cudaError_t launch_split_cl(const qsvd_dims& d, const void* cache, const void* q
                             int G, float* pm, float* pl, float* pz, int32_t* status, cudaStream_t s);
 cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
-                            int32_t* status, cudaStream_t s);
+                            int32_t* status, cudaStream_t s, const float* qsh = nullptr);
 
 // Prefill of the latent cache (tcgen05 GEMM x W^d with the append path's
 // rounding / quantisation fused): 16-bit weights, r % 256 == 0, E % 64 == 0,

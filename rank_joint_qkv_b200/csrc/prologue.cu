@@ -278,6 +278,49 @@ k_absorb_mma(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
+// Quantised latents on the tensor cores: the absorbed query of each
+// (sequence, head) as three int8 parts with one power-of-two scale,
+//   qt = s (Q0 + Q1 / 128 + Q2 / 16384),  s = 2^ceil(log2(max_j |qt_j| / 127)),
+// Q0 = rint(qt / s) (|Q0| <= 127), Q1 = rint(128 (qt - s Q0) / s), Q2 likewise
+// (|Q1|, |Q2| <= 64; remainder <= s / 32768): the integer MMAs of the split
+// kernel take the parts, the softmax applies s once per head.  qp [B][3][H][r]
+// int8, qs [B][H].  grid (H, B), block 128.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+k_quant_query(const float* __restrict__ qt, int8_t* __restrict__ qp, float* __restrict__ qs, int H, int r) {
+  dev::pdl_wait();   // see launch_pdl
+  dev::pdl_trigger();
+  __shared__ float red[4];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const float* row = qt + (size_t(b) * H + h) * r;
+  float m = 0.f;
+  for (int j = threadIdx.x; j < r; j += 128) m = fmaxf(m, fabsf(row[j]));
+  m = dev::warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  // the smallest power of two >= m / 127 (1 for an all-zero query)
+  const float f = m / 127.f;
+  const float sq = f > 0.f ? __uint_as_float((__float_as_uint(f) + 0x007FFFFFu) & 0xFF800000u) : 1.f;
+  const float isq = 1.f / sq;   // exact: a power of two
+  if (threadIdx.x == 0) qs[size_t(b) * H + h] = sq;
+  int8_t* p0 = qp + ((size_t(b) * 3 + 0) * H + h) * r;
+  int8_t* p1 = qp + ((size_t(b) * 3 + 1) * H + h) * r;
+  int8_t* p2 = qp + ((size_t(b) * 3 + 2) * H + h) * r;
+  for (int j = threadIdx.x; j < r; j += 128) {
+    const float v = row[j];
+    const float q0 = rintf(v * isq);
+    const float r1 = v - sq * q0;
+    const float q1 = rintf(r1 * isq * 128.f);
+    const float r2 = r1 - sq * (1.f / 128.f) * q1;
+    const float q2 = rintf(r2 * isq * 16384.f);
+    p0[j] = int8_t(q0);
+    p1[j] = int8_t(q1);
+    p2[j] = int8_t(q2);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Rotary query: q_h <- scale * R(len_b - 1) q_h, pairs (i, i + d_h/2).
 // grid (B), block 256.
 // ---------------------------------------------------------------------------
@@ -460,6 +503,15 @@ cudaError_t launch_absorb(const qsvd_dims& d, const float* q, const void* wuk, f
                 : absorb_t<__nv_bfloat16, __half>(d, q, wuk, scale, qt32, qt16, status, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_quant_query(const qsvd_dims& d, const float* qt, int8_t* qp, float* qs, cudaStream_t s) {
+  {
+    const cudaError_t le = launch_pdl(k_quant_query, dim3(d.H, d.batch), dim3(128), 0, s, qt, qp, qs, d.H, d.r);
+    if (le != cudaSuccess) return le;
+  }
+  note_launch();
+  return check_launch();
 }
 
 cudaError_t launch_rope_query(const qsvd_dims& d, const float* q, const int32_t* sched,

@@ -65,12 +65,12 @@ namespace qsvd {
 namespace {
 
 constexpr int kThreadsTc = 256;
-constexpr int kConvWarps = 3;      // quantised latent: converting warps per stream
-constexpr int kThreadsTcQ = 256 + 64 * (kConvWarps - 1);   // warps 8.. convert too
+constexpr int kThreadsTcQ = 384;   // quantised latent: warps 8-11 convert too
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
 constexpr int kMaxSlots = 8;                   // per ring
 constexpr int kMaxGroupBufs = 4;               // S accumulators per channel group (quantised latent)
 constexpr int kMaxRaw = 8;                     // raw-code slots per stream (quantised latent)
+constexpr int kScaleBufs = 3;                  // group-scale tables of tiles in flight (quantised latent)
 constexpr float kRescaleLog2 = 8.f;             // P <= 2^8 before a rescale
 
 // Failure injection for tests (qsvd_testing_set_score_wait_ns): when
@@ -94,9 +94,16 @@ template <int NP, int QS>
 __host__ __device__ constexpr int s_slot_bytes() { return kBoxBytes + QS * NP * 128; }
 constexpr int kZBoxBytes = 64 * 128;             // 64 tokens x 64 channels x 2 bytes
 constexpr int kZSlotBytes = 2 * kZBoxBytes;
+// Quantised latent: an S item is one 128-channel group -- the codes as 8-bit
+// integers (128 tokens x 128 bytes, K-major, 128-byte swizzle) and the
+// query's three int8 parts (3 x NP rows of 128 bytes, part-major).
+template <int NP>
+__host__ __device__ constexpr int sq_slot_bytes() { return 128 * 128 + 3 * NP * 128; }
 // Scores given (SG): no S pass; ring A carries Z items too.
-template <int NP, int QS, bool SG>
-__host__ __device__ constexpr int a_slot_bytes() { return SG ? kZSlotBytes : s_slot_bytes<NP, QS>(); }
+template <int NP, int QS, bool SG, int QB = 0>
+__host__ __device__ constexpr int a_slot_bytes() {
+  return SG ? kZSlotBytes : (QB ? sq_slot_bytes<NP>() : s_slot_bytes<NP, QS>());
+}
 template <int NP>
 __host__ __device__ constexpr int pbuf_bytes() { return 2 * NP * 128; }   // one P^T part
 constexpr int kMiscBytes = 2048;
@@ -115,33 +122,41 @@ struct Smem {
   uint64_t* drain;       // [2] one per MMA issuer
   uint64_t* sg_full;     // [kMaxGroupBufs] quantised latent: S of one channel group complete
   uint64_t* sg_empty;    // [kMaxGroupBufs] ... read by the softmax
-  uint8_t* sraw;         // quantised latent: raw-code rings (S, Z)
-  uint8_t* zraw;
-  uint64_t* sraw_full;   // [kMaxRaw]
-  uint64_t* zraw_full;   // [kMaxRaw]
+  uint8_t* sraw;         // quantised latent: int4 S raw-code ring
+  uint8_t* zsc;          // quantised latent: [kScaleBufs][128 tokens][r / 128] fp16 group scales
+  uint64_t* sraw_full;   // [kMaxRaw] int4 S raw codes landed
+  uint64_t* zraw_full;   // [kMaxSlots] Z raw codes landed in their fp16 slot
   uint64_t* never;       // never released (failure injection)
+  uint64_t* zsc_full;    // [kScaleBufs] scale table of a tile written (by the S producer)
+  uint64_t* zsc_empty;   // [kScaleBufs] Z MMAs of the table's tile complete
   float* red;            // [4][NP] per-warp partial max / sum
   float* m_run;          // [NP] running reference max per head (log2 domain)
   float* l_run;          // [NP] running sum of P per head
   float* alpha;          // [NP] rescale factor of the current tile
+  float* qsig;           // [NP] quantised latent: the query parts' scale per head of the tile
   uint32_t* tmem_holder;
   volatile int* abort_flag;
 };
 
 // P buffers: 2 (double buffer) x PS parts (bf16: hi + lo) x pbuf_bytes.
-// Quantised latent: raw codes of one item (S: 128 rows x 64 channels; Z: 64
-// rows x 128 channels) are QB x 1024 bytes.
+// Quantised latent: raw codes of one Z item (64 rows x 128 channels) are
+// QB x 1024 bytes and land at the end of the item's own fp16 slot; of one S
+// item (128 rows x 128 channels) int4 only, 8 KB, in a raw ring (int8 S
+// items land by TMA in their slot as they are).  One scale table: 128 tokens
+// x r / 128 groups of fp16.
 __host__ __device__ constexpr int raw_bytes(int qb) { return qb * 1024; }
+__host__ __device__ constexpr int raw_s_bytes(int qb) { return qb == 4 ? 128 * 64 : 0; }
+__host__ __device__ constexpr int scale_buf_bytes(int r) { return 256 * (r / 128); }
 
-template <int NP, int QS, int PS, bool SG>
-__device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
+template <int NP, int QS, int PS, bool SG, int QB>
+__device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int r) {
   Smem s;
   s.sring = base;
-  s.zring = s.sring + size_t(ns) * a_slot_bytes<NP, QS, SG>();
+  s.zring = s.sring + size_t(ns) * a_slot_bytes<NP, QS, SG, QB>();
   s.pbuf = s.zring + size_t(nz) * kZSlotBytes;
   s.sraw = s.pbuf + 2 * PS * pbuf_bytes<NP>();
-  s.zraw = s.sraw + size_t(nraw) * raw_bytes(qb);
-  uint8_t* m = s.zraw + size_t(nraw) * raw_bytes(qb);
+  s.zsc = s.sraw + size_t(nraw) * raw_s_bytes(QB);
+  uint8_t* m = s.zsc + (QB ? kScaleBufs * scale_buf_bytes(r) : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(m);
   s.s_full = bars;
   s.s_empty = bars + kMaxSlots;
@@ -154,15 +169,18 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int qb, int r) {
   s.sg_full = s.drain + 2;
   s.sg_empty = s.sg_full + kMaxGroupBufs;
   s.sraw_full = s.sg_empty + kMaxGroupBufs;
-  s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + 2 kMaxRaw = 64 barriers
-  s.never = s.zraw_full + kMaxRaw;       // the 65th (the barrier area holds 80)
-  static_assert(640 + 4 * NP * 4 + 32 + 3 * NP * 4 <= kMiscBytes, "misc region");
+  s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + kMaxRaw + kMaxSlots = 64
+  s.never = s.zraw_full + kMaxSlots;     // the 65th
+  s.zsc_full = s.never + 1;
+  s.zsc_empty = s.zsc_full + kScaleBufs;  // 69 barriers (the barrier area holds 80)
+  static_assert(640 + 4 * NP * 4 + 32 + (QB ? 4 : 3) * NP * 4 <= kMiscBytes, "misc region");
   s.red = reinterpret_cast<float*>(m + 640);
   s.tmem_holder = reinterpret_cast<uint32_t*>(m + 640 + 4 * NP * 4);
   s.abort_flag = reinterpret_cast<volatile int*>(m + 640 + 4 * NP * 4 + 16);
   s.m_run = reinterpret_cast<float*>(m + 640 + 4 * NP * 4 + 32);
   s.l_run = s.m_run + NP;
   s.alpha = s.l_run + NP;
+  s.qsig = s.alpha + NP;
   return s;
 }
 
@@ -265,59 +283,35 @@ __device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
                : "memory");
 }
 
-// S item of a quantised tile from its raw codes in shared memory
-// ([128 rows][QB x 8 bytes]): channel box u as fp16 integers, unscaled (the
-// group scales are applied to S per token), in the 128-byte-swizzled K-major
-// layout; rows >= nv are zeros.  Warp-wide.
-template <int QB>
-__device__ __forceinline__ void convert_s_box(uint32_t d, uint32_t raw, int nv, int lane) {
-  constexpr int RPB = QB * 8;             // raw bytes per row: 32 (int4), 64 (int8)
-  constexpr int VPR = RPB / 16;           // 16-byte vectors per row
-  constexpr int CPV = QB == 4 ? 4 : 2;    // 16-byte fp16 chunks per vector
-  constexpr int NV = 128 * VPR / 32;      // vectors per lane: 8 (int4), 16 (int8)
-  // every raw vector's load is issued before the first store (the shared
-  // accesses are ordered asm statements: interleaved, each load would wait
-  // behind the previous vector's stores)
-  uint4 rv[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int v = lane + 32 * i, t = v / VPR, q = v % VPR;
-    rv[i] = t < nv ? lds128(raw + t * RPB + q * 16) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int v = lane + 32 * i, t = v / VPR, q = v % VPR;
-    uint4 out[CPV];
-    codes_to_half<QB>(rv[i], false, __half2(), out);   // zero codes give zeros
-#pragma unroll
-    for (int c = 0; c < CPV; ++c) sts128(d + t * 128 + (((q * CPV + c) ^ (t & 7)) << 4), out[c]);
-  }
-  fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
-  __syncwarp();
+__device__ __forceinline__ __half lds16h(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return __ushort_as_half(v);
 }
 
-// Z item of a quantised tile from its raw codes in shared memory ([64 rows]
-// [QB x 16 bytes]): channels 128 j .. 128 j + 127 of rows 64 h .. 64 h + 63,
-// dequantised (code x group scale, one fp16 rounding of the exact product),
-// two 64-channel boxes of 64 rows, 128-byte swizzled; rows >= nv are zeros.
-// tsc: the tile's scales [128][ngroups] in global memory.
+// Z item of a quantised tile, expanded in place: its raw codes ([64 rows]
+// [QB x 16 bytes], at the end of the fp16 slot) become channels 128 j ..
+// 128 j + 127 of rows 64 h .. 64 h + 63, dequantised (code x group scale,
+// one fp16 rounding of the exact product), two 64-channel boxes of 64 rows,
+// 128-byte swizzled.  sct: the tile's scale table [128][ngroups] (zeros for
+// rows past the length, which therefore come out as zeros).  Warp-wide: the
+// whole item is read into registers before the first store overwrites it.
 template <int QB>
-__device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const __half* tsc,
-                                               int ngroups, int j, int h, int nv, int lane) {
+__device__ __forceinline__ void convert_z_inplace(uint32_t d, uint32_t sct, int ngroups, int j, int h, int lane) {
   constexpr int RPB = QB * 16;            // raw bytes per row: 64 (int4), 128 (int8)
   constexpr int VPR = RPB / 16;
   constexpr int CPV = QB == 4 ? 4 : 2;
   constexpr int NV = 64 * VPR / 32;       // vectors per lane: 8 (int4), 16 (int8)
-  // all raw vectors and scales requested before the first store (see convert_s_box)
+  const uint32_t raw = d + uint32_t(kZSlotBytes - 64 * RPB);
   uint4 rv[NV];
   __half sc[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
-    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR, t = 64 * h + tt;
-    const bool in = t < nv;
-    rv[i] = in ? lds128(raw + tt * RPB + q * 16) : make_uint4(0, 0, 0, 0);
-    sc[i] = in ? tsc[t * ngroups + j] : __float2half(0.f);
+    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR;
+    rv[i] = lds128(raw + tt * RPB + q * 16);
+    sc[i] = lds16h(sct + uint32_t(((64 * h + tt) * ngroups + j) * 2));
   }
+  asm volatile("bar.warp.sync 0xffffffff;" ::: "memory");   // all loads before any store
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int v = lane + 32 * i, tt = v / VPR, q = v % VPR;
@@ -328,91 +322,238 @@ __device__ __forceinline__ void convert_z_item(uint32_t d, uint32_t raw, const _
 #pragma unroll
     for (int c = 0; c < CPV; ++c) sts128(d + box * kZBoxBytes + tt * 128 + (((c0 + c) ^ (tt & 7)) << 4), out[c]);
   }
-  fence_proxy_async();
+  fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
   __syncwarp();
 }
 
-// Producer of one ring for a quantised latent: nsub warps share a stream,
-// warp wsub taking the items k == wsub (mod nsub) of the stream's sequence.
-// The raw codes of each item arrive by TMA into a ring of nraw slots (nraw a
-// multiple of nsub, so a slot is always refilled by the warp that drained
-// it), issued nraw items ahead; the warp converts them into the fp16 slot the
-// MMAs read (S: exact integers, plus the query box by TMA; Z: dequantised,
-// the token's group scale read from global memory).  Conversion is
-// latency-bound per warp (dependent integer/half2 chains, the proxy fence
-// before each hand-off), so the stream's throughput grows with nsub.
-// *last_item / *last_raw: the last item this warp produced / issued (-1 if
-// none), for the drain after an abort.  Returns false on a wait that expired
-// or an abort.
-template <int NP, int QS, int QB>
-__device__ bool produce_q(int kind, int wsub, int nsub, const Smem& s, const CUtensorMap* tm_raw,
-                          const CUtensorMap* tm_q, const __half* scales, const int32_t* sched, int B,
-                          int r, int max_len, long long tb, long long te, int n, int nslots, int nraw,
-                          int lane, long long* last_item, long long* last_raw) {
-  const int NI = r / 64, NG = r / 128;
-  uint8_t* ring = kind == 0 ? s.sring : s.zring;
-  const uint32_t slot_bytes = kind == 0 ? uint32_t(s_slot_bytes<NP, QS>()) : uint32_t(kZSlotBytes);
-  uint64_t* full = kind == 0 ? s.s_full : s.z_full;
-  uint64_t* empty = kind == 0 ? s.s_empty : s.z_empty;
-  uint8_t* raw = kind == 0 ? s.sraw : s.zraw;
-  uint64_t* rfull = kind == 0 ? s.sraw_full : s.zraw_full;
-  const uint32_t ring0 = saddr(ring), raw0 = saddr(raw);
+// Scale table of one tile (quantised latent), written by the S producer when
+// it starts the tile: the tile's group scales [128][r / 128] (rows past the
+// length as zeros, which the Z items then dequantise to zeros), read by the
+// softmax (S) and the converting warps (Z).  A table is reused once the Z
+// MMAs of its tile are complete.  Warp-wide; false if the wait expired.
+__device__ bool write_scale_table(const Smem& s, const __half* scales, int row, int nv, int r, Ring& sb, int lane) {
+  const int NG = r / 128;
+  if (!__all_sync(0xffffffffu, mbar_wait(saddr(&s.zsc_empty[sb.slot]), sb.phase ^ 1u))) return false;
+  const __half* tsc = scales + size_t(row) * NG;
+  __half* tab = reinterpret_cast<__half*>(s.zsc + sb.slot * scale_buf_bytes(r));
+  for (int e = lane; e < 128 * NG; e += 32) tab[e] = e < nv * NG ? tsc[e] : __float2half(0.f);
+  mbar_arrive(saddr(&s.zsc_full[sb.slot]));   // every lane (count 32), releasing its own stores
+  sb.advance();
+  return true;
+}
+
+// Z stream of a quantised latent, issuing warp: per item, a free fp16 slot,
+// then the item's raw codes by TMA into the slot's end, where a converting
+// warp expands them in place.  *issued: items issued.
+template <int QB>
+__device__ bool produce_zq(const Smem& s, const CUtensorMap* tm_raw, const int32_t* sched, int B, int r,
+                           int max_len, long long tb, long long te, int n, int nz, int lane, long long* issued) {
+  const int NI = r / 64;
   constexpr uint32_t RB = uint32_t(raw_bytes(QB));
-  const long long total = (long long)n * NI;
+  const uint32_t ring0 = saddr(s.zring);
+  TileIter it;
+  it.init(sched, B, tb, te);
+  Ring rg(nz);
+  long long k = 0;
+  for (int i = 0; i < n; ++i) {
+    const int row = it.b * max_len + it.t0();
+    for (int u = 0; u < NI; ++u) {
+      if (!__all_sync(0xffffffffu, mbar_wait(saddr(&s.z_empty[rg.slot]), rg.phase ^ 1u))) { *issued = k; return false; }
+      const uint32_t fb = saddr(&s.zraw_full[rg.slot]);
+      if (lane == int(k & 31)) {   // rotating issuing lane
+        mbar_expect_tx(fb, RB);
+        tma_load_2d(ring0 + uint32_t(rg.slot) * kZSlotBytes + (kZSlotBytes - RB), tm_raw, (u >> 1) * (QB * 16),
+                    row + 64 * (u & 1), fb);
+      }
+      __syncwarp();
+      rg.advance();
+      ++k;
+    }
+    it.next();
+    if (__any_sync(0xffffffffu, *s.abort_flag)) { *issued = k; return false; }
+  }
+  *issued = k;
+  return true;
+}
+
+// Z stream of a quantised latent, converting warps: warp wsub of nsub takes
+// the items k == wsub (mod nsub), waits for the tile's scale table (once per
+// tile) and the item's raw codes, expands the item in place and hands the
+// slot to the Z MMAs.  Issues no copies (nothing to drain after an abort).
+template <int QB>
+__device__ bool convert_zq(int wsub, int nsub, const Smem& s, int r, int n, int nz, int lane) {
+  const int NI = r / 64, NG = r / 128;
+  const uint32_t ring0 = saddr(s.zring), sct0 = saddr(s.zsc);
+  Ring rg(nz), sb(kScaleBufs);
+  int k_sub = 0;
+  for (int i = 0; i < n; ++i) {
+    bool have = false;
+    for (int u = 0; u < NI; ++u) {
+      if (k_sub == wsub) {
+        if (!have && !__all_sync(0xffffffffu, mbar_wait(saddr(&s.zsc_full[sb.slot]), sb.phase))) return false;
+        have = true;
+        if (!__all_sync(0xffffffffu, mbar_wait(saddr(&s.zraw_full[rg.slot]), rg.phase))) return false;
+        convert_z_inplace<QB>(ring0 + uint32_t(rg.slot) * kZSlotBytes, sct0 + uint32_t(sb.slot * scale_buf_bytes(r)),
+                              NG, u >> 1, u & 1, lane);
+        if (lane == 0) mbar_arrive(saddr(&s.z_full[rg.slot]));
+      }
+      if (++k_sub == nsub) k_sub = 0;
+      rg.advance();
+    }
+    sb.advance();
+    if (__any_sync(0xffffffffu, *s.abort_flag)) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------- quantised latent, S stream
+// The scores pass of a quantised latent runs on the integer tensor cores:
+// per 128-channel group g, S_g = C_g Qp_g^T with C_g the codes (int8 as
+// stored; int4 unpacked to sign-extended bytes) and Qp_g the absorbed
+// query's three int8 parts (rows k NP + h), int32 exact; the softmax warps
+// then form s = sigma_h sum_g scale_{t,g} (S_0 + S_1 / 128 + S_2 / 16384)
+// with sigma_h the query parts' scale of the head (see k_quant_query).
+
+// Eight int4 codes (one word) -> eight signed bytes in channel order.
+__device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t& a, uint32_t& b) {
+  uint32_t lo = w & 0x0F0F0F0Fu;                 // channels 0, 2, 4, 6 (two's-complement nibbles)
+  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;          // channels 1, 3, 5, 7
+  lo |= (lo & 0x08080808u) * 0x1Eu;              // sign-extend each nibble to its byte (0x08 * 0x1E = 0xF0)
+  hi |= (hi & 0x08080808u) * 0x1Eu;
+  a = __byte_perm(lo, hi, 0x5140);               // channels 0 1 2 3
+  b = __byte_perm(lo, hi, 0x7362);               // channels 4 5 6 7
+}
+
+// One S item of int4 codes (raw [128 rows][64 bytes]) -> the A operand: 128
+// rows of 128 signed bytes, K-major, 128-byte swizzled.  Warp-wide;
+// every raw vector of a half is requested before the first store.
+__device__ __forceinline__ void unpack_s_group(uint32_t d, uint32_t raw, int lane) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint4 rv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rv[i] = lds128(raw + uint32_t(lane + 32 * (8 * half + i)) * 16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int v = lane + 32 * (8 * half + i), t = v >> 2, c0 = 2 * (v & 3);   // row, first 16-byte chunk
+      uint32_t o[8];
+      unpack_int4x8(rv[i].x, o[0], o[1]);
+      unpack_int4x8(rv[i].y, o[2], o[3]);
+      unpack_int4x8(rv[i].z, o[4], o[5]);
+      unpack_int4x8(rv[i].w, o[6], o[7]);
+      sts128(d + t * 128 + ((c0 ^ (t & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+      sts128(d + t * 128 + (((c0 + 1) ^ (t & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+    }
+  }
+  fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
+  __syncwarp();
+}
+
+// S stream, int8 codes: one warp; per item the codes (TMA, 128-byte swizzle,
+// straight from the cache) and the query parts (TMA) into one slot.  Rows of
+// a ragged last tile past the length are read as stored (finite integers;
+// the softmax masks them).  *issued: items issued.
+template <int NP>
+__device__ bool produce_qs8(const Smem& s, const CUtensorMap* tm_a, const CUtensorMap* tm_q, const __half* scales,
+                            const int32_t* sched, int B, int r, int max_len, long long tb, long long te, int n,
+                            int nslots, int lane, long long* issued) {
+  const int NG = r / 128;
+  constexpr uint32_t SQ = uint32_t(sq_slot_bytes<NP>());
+  const uint32_t ring0 = saddr(s.sring);
+  TileIter it;
+  it.init(sched, B, tb, te);
+  Ring rg(nslots), sb(kScaleBufs);
+  long long k = 0;
+  for (int i = 0; i < n; ++i) {
+    const int row = it.b * max_len + it.t0(), b = it.b;
+    if (!write_scale_table(s, scales, row, it.nvalid(), r, sb, lane)) { *issued = k; return false; }
+    for (int u = 0; u < NG; ++u) {
+      if (!__all_sync(0xffffffffu, mbar_wait(saddr(&s.s_empty[rg.slot]), rg.phase ^ 1u))) { *issued = k; return false; }
+      const uint32_t dst = ring0 + uint32_t(rg.slot) * SQ, fb = saddr(&s.s_full[rg.slot]);
+      const int ln = int(k & 15) * 2;   // rotating issuing lanes (see produce)
+      if (lane == 0) mbar_expect_tx(fb, SQ);
+      __syncwarp();
+      if (lane == ln) tma_load_2d(dst, tm_a, 128 * u, row, fb);
+      if (lane == ln + 1) tma_load_3d(dst + 128 * 128, tm_q, 128 * u, 0, 3 * b, fb);
+      __syncwarp();
+      rg.advance();
+      ++k;
+    }
+    it.next();
+    if (__any_sync(0xffffffffu, *s.abort_flag)) { *issued = k; return false; }
+  }
+  *issued = k;
+  return true;
+}
+
+// S stream, int4 codes: nsub warps share the items (item k to warp k % nsub);
+// raw codes by TMA into a ring of nraw slots (a multiple of nsub, so a slot is
+// always refilled by the warp that drained it) issued nraw items ahead,
+// unpacked into the slot; the query parts by TMA.  The slot completes on the
+// query's bytes and the warp's arrive.
+template <int NP>
+__device__ bool produce_qs4(int wsub, int nsub, const Smem& s, const CUtensorMap* tm_raw, const CUtensorMap* tm_q,
+                            const __half* scales, const int32_t* sched, int B, int r, int max_len, long long tb,
+                            long long te, int n, int nslots, int nraw, int lane, long long* last_item,
+                            long long* last_raw) {
+  const int NG = r / 128;
+  constexpr uint32_t SQ = uint32_t(sq_slot_bytes<NP>());
+  constexpr uint32_t RB = uint32_t(raw_s_bytes(4));
+  const uint32_t ring0 = saddr(s.sring), raw0 = saddr(s.sraw);
+  const int total = n * NG;
   *last_item = -1;
   *last_raw = -1;
-  // issue side: walks every item of the stream, issues this warp's
   TileIter ia;
   ia.init(sched, B, tb, te);
-  int ia_i = 0, ua = 0;
-  long long ki = 0;
+  int ia_i = 0, ua = 0, ki = 0, ki_sub = 0, own = 0;
+  Ring ri(nraw);
   auto issue_next = [&]() {
-    if (ki % nsub == wsub) {
-      const int slot = int(ki % nraw);
-      const uint32_t fb = saddr(&rfull[slot]);
+    if (ki_sub == wsub) {
+      const uint32_t fb = saddr(&s.sraw_full[ri.slot]);
       const int row = ia.b * max_len + ia.t0();
-      if (lane == int((ki / nsub) & 31)) {   // rotating issuing lane
+      if (lane == (own & 31)) {   // rotating issuing lane
         mbar_expect_tx(fb, RB);
-        if (kind == 0) tma_load_2d(raw0 + slot * RB, tm_raw, ua * (QB * 8), row, fb);
-        else tma_load_2d(raw0 + slot * RB, tm_raw, (ua >> 1) * (QB * 16), row + 64 * (ua & 1), fb);
+        tma_load_2d(raw0 + ri.slot * RB, tm_raw, ua * 64, row, fb);
       }
+      ++own;
       *last_raw = ki;
     }
     ++ki;
-    if (++ua == NI) {
+    if (++ki_sub == nsub) ki_sub = 0;
+    ri.advance();
+    if (++ua == NG) {
       ua = 0;
       if (++ia_i < n) ia.next();
     }
   };
-  for (long long x = 0; x < total && x < nraw; ++x) issue_next();
+  for (int x = 0; x < total && x < nraw; ++x) issue_next();
   TileIter it;
   it.init(sched, B, tb, te);
-  long long k = 0;   // item index of the stream
+  int k = 0, k_sub = 0;
+  Ring rr(nraw), rs(nslots), sb(kScaleBufs);
   for (int i = 0; i < n; ++i) {
-    const int nv = it.nvalid(), b = it.b;
-    const __half* tsc = scales + (size_t(b) * max_len + it.t0()) * NG;   // the tile's scales [128][NG]
-    for (int u = 0; u < NI; ++u, ++k) {
-      if (k % nsub != wsub) continue;
-      const int rs = int(k % nraw), slot = int(k % nslots);
-      if (!__all_sync(0xffffffffu, mbar_wait(saddr(&rfull[rs]), uint32_t(k / nraw) & 1u)) ||
-          !__all_sync(0xffffffffu, mbar_wait(saddr(&empty[slot]), (uint32_t(k / nslots) & 1u) ^ 1u)))
-        return false;   // warp-uniform
-      const uint32_t dst = ring0 + uint32_t(slot) * slot_bytes;
-      const uint32_t fb = saddr(&full[slot]);
-      if (kind == 0) {
-        if (lane == 0) {   // the query box; the slot completes on this and the codes' arrival
-          mbar_expect_tx(fb, uint32_t(QS * NP * 128));
-          tma_load_4d(dst + kBoxBytes, tm_q, 0, 0, QS * b, u, fb);
+    const int b = it.b;
+    if (wsub == 0 && !write_scale_table(s, scales, b * max_len + it.t0(), it.nvalid(), r, sb, lane)) return false;
+    for (int u = 0; u < NG; ++u) {
+      if (k_sub == wsub) {
+        if (!__all_sync(0xffffffffu, mbar_wait(saddr(&s.sraw_full[rr.slot]), rr.phase)) ||
+            !__all_sync(0xffffffffu, mbar_wait(saddr(&s.s_empty[rs.slot]), rs.phase ^ 1u)))
+          return false;   // warp-uniform
+        const uint32_t dst = ring0 + uint32_t(rs.slot) * SQ, fb = saddr(&s.s_full[rs.slot]);
+        if (lane == 0) {
+          mbar_expect_tx(fb, uint32_t(3 * NP * 128));
+          tma_load_3d(dst + 128 * 128, tm_q, 128 * u, 0, 3 * b, fb);
         }
-        convert_s_box<QB>(dst, raw0 + uint32_t(rs) * RB, nv, lane);
-      } else {
-        convert_z_item<QB>(dst, raw0 + uint32_t(rs) * RB, tsc, NG, u >> 1, u & 1, nv, lane);
+        unpack_s_group(dst, raw0 + uint32_t(rr.slot) * RB, lane);
+        if (lane == 0) mbar_arrive(fb);
+        *last_item = k;
+        for (int x = 0; x < nsub && ki < total; ++x) issue_next();
+        __syncwarp();
       }
-      if (lane == 0) mbar_arrive(fb);
-      *last_item = k;
-      // the raw slot has been read: the item nraw ahead (also this warp's) refills it
-      for (int x = 0; x < nsub && ki < total; ++x) issue_next();
-      __syncwarp();
+      ++k;
+      if (++k_sub == nsub) k_sub = 0;
+      rr.advance();
+      rs.advance();
     }
     it.next();
     if (__any_sync(0xffffffffu, *s.abort_flag)) return false;
@@ -420,20 +561,19 @@ __device__ bool produce_q(int kind, int wsub, int nsub, const Smem& s, const CUt
   return true;
 }
 
-// After an abort: wait (bounded) for the copies this warp may have in flight
-// -- the last raw load into each of its raw slots, the query boxes of its
-// last S items -- so that none lands after the CTA has left.
-__device__ void drain_q(int kind, int wsub, int nsub, const Smem& s, int nslots, int nraw,
-                        long long last_item, long long last_raw) {
-  uint64_t* rfull = kind == 0 ? s.sraw_full : s.zraw_full;
+// After an abort (int4 S unpacking warps): wait (bounded) for the copies
+// this warp may have in flight -- the last raw load into each of its raw
+// slots, the query boxes of its last S items -- so that none lands after the
+// CTA has left.
+__device__ void drain_q(int wsub, int nsub, const Smem& s, int nslots, int nraw, long long last_item,
+                        long long last_raw) {
   for (int slot = wsub; slot < nraw; slot += nsub) {
     if (last_raw < slot) continue;
     const long long kk = slot + (last_raw - slot) / nraw * nraw;   // last item issued into the slot
-    mbar_wait(saddr(&rfull[slot]), uint32_t(kk / nraw) & 1u);
+    mbar_wait(saddr(&s.sraw_full[slot]), uint32_t(kk / nraw) & 1u);
   }
-  if (kind == 0)
-    for (long long kk = last_item; kk >= 0 && kk > last_item - nslots; kk -= nsub)
-      mbar_wait(saddr(&s.s_full[int(kk % nslots)]), uint32_t(kk / nslots) & 1u);
+  for (long long kk = last_item; kk >= 0 && kk > last_item - nslots; kk -= nsub)
+    mbar_wait(saddr(&s.s_full[int(kk % nslots)]), uint32_t(kk / nslots) & 1u);
 }
 
 // Producer of one ring (warp-wide).  kind 0: S ring (latent box from HBM,
@@ -539,15 +679,17 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
            const float* __restrict__ scores, const int32_t* __restrict__ sched,
            float* __restrict__ pm, float* __restrict__ pl, float* __restrict__ pz,
            int32_t* __restrict__ status, int B, int H, int r, int max_len, int G, int ns, int nz,
-           int nsg, int nraw, int ch) {
+           int nsg, int nraw, int ch, const float* __restrict__ qsh) {
   dev::pdl_wait();   // see launch_pdl
   dev::pdl_trigger();
   static_assert(!(SG && QB), "scores given: 16-bit latent only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const Smem s = carve<NP, QS, PS, SG>(base, ns, nz, nraw, QB, r);
-  constexpr int SW = QS * NP;                 // S accumulator columns per buffer
+  const Smem s = carve<NP, QS, PS, SG, QB>(base, ns, nz, nraw, r);
+  // S accumulator columns per buffer: hi and lo query parts (16-bit), or the
+  // three int8 query parts' int32 sums of one group (quantised)
+  constexpr int SW = QB ? 3 * NP : QS * NP;
   const int ZC0 = SG ? 0 : (QB ? nsg : 2) * SW;   // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = r / 64;                      // ring items per tile
@@ -563,18 +705,20 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
-      mbar_init(saddr(&s.s_full[i]), QB ? 2 : 1);   // quantised: query TMA + converted codes
+      mbar_init(saddr(&s.s_full[i]), QB == 4 ? 2 : 1);   // int4: query TMA + unpacked codes
       mbar_init(saddr(&s.s_empty[i]), 1);
     }
     for (int i = 0; i < kMaxGroupBufs; ++i) {
       mbar_init(saddr(&s.sg_full[i]), 1);
       mbar_init(saddr(&s.sg_empty[i]), 1);
     }
-    for (int i = 0; i < kMaxRaw; ++i) {
-      mbar_init(saddr(&s.sraw_full[i]), 1);
-      mbar_init(saddr(&s.zraw_full[i]), 1);
-    }
+    for (int i = 0; i < kMaxRaw; ++i) mbar_init(saddr(&s.sraw_full[i]), 1);
+    for (int i = 0; i < kMaxSlots; ++i) mbar_init(saddr(&s.zraw_full[i]), 1);
     mbar_init(saddr(s.never), 1);
+    for (int i = 0; i < kScaleBufs; ++i) {
+      mbar_init(saddr(&s.zsc_full[i]), 32);   // the issuing warp's lanes
+      mbar_init(saddr(&s.zsc_empty[i]), 1);
+    }
     for (int i = 0; i < nz; ++i) {
       mbar_init(saddr(&s.z_full[i]), 1);
       mbar_init(saddr(&s.z_empty[i]), 1);
@@ -601,34 +745,91 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
 
   if (warp == 0 || warp == 2 || (QB && warp >= 8)) {
     // ----------------------------------------------------------- producers
-    // quantised latent: S converters warps 0, 9, 10 and Z converters 2, 8, 11
-    // (warp w issues on scheduler w % 4: each stream on three schedulers)
-    static_assert(kConvWarps == 3, "converter warp map");
-    const int kind = (warp == 0 || warp == 9 || warp == 10) ? 0 : 1;
-    const int wsub = warp < 8 ? 0 : (warp == 8 || warp == 9 ? 1 : 2);
-    const int nslots = kind == 0 ? ns : nz;
+    bool ok = true;
     long long issued = 0, raw_issued = 0;
-    bool ok;
-    if constexpr (QB != 0) {   // tm_cs / tm_cz map the raw codes
-      ok = produce_q<NP, QS, QB>(kind, wsub, kConvWarps, s, kind == 0 ? &tm_cs : &tm_cz, &tm_q, scales,
-                                 sched, B, r, max_len, tb, te, n, nslots, nraw, lane, &issued, &raw_issued);
+    if constexpr (QB != 0) {
+      // quantised latent.  S: warp 0 loads int8 codes by TMA; int4 raw codes
+      // are unpacked by warps 0 and 9.  Z: warp 2 issues the raw codes and
+      // the tiles' scale tables, warps 8-11 (int4: 8, 10, 11) expand them
+      // (warp w issues on scheduler w % 4)
+      const bool zconv = warp >= 8 && !(QB == 4 && warp == 9);
+      if (warp == 2) {
+        ok = produce_zq<QB>(s, &tm_cz, sched, B, r, max_len, tb, te, n, nz, lane, &issued);
+        if (!ok && lane == 0) {
+          set_abort(s, status);
+          drain_ring(s.zraw_full, issued, nz);
+        }
+      } else if (zconv) {
+        const int wsub = QB == 8 ? warp - 8 : (warp == 8 ? 0 : warp - 9);
+        ok = convert_zq<QB>(wsub, QB == 8 ? 4 : 3, s, r, n, nz, lane);
+        if (!ok && lane == 0) set_abort(s, status);
+      } else if (QB == 4) {   // warps 0 and 9
+        const int wsub = warp == 0 ? 0 : 1;
+        ok = produce_qs4<NP>(wsub, 2, s, &tm_cs, &tm_q, scales, sched, B, r, max_len, tb, te, n, ns, nraw, lane,
+                             &issued, &raw_issued);
+        if (!ok && lane == 0) {
+          set_abort(s, status);
+          drain_q(wsub, 2, s, ns, nraw, issued, raw_issued);
+        }
+      } else {   // int8, warp 0: no conversion
+        ok = produce_qs8<NP>(s, &tm_cs, &tm_q, scales, sched, B, r, max_len, tb, te, n, ns, lane, &issued);
+        if (!ok && lane == 0) {
+          set_abort(s, status);
+          drain_ring(s.s_full, issued, ns);
+        }
+      }
     } else {
+      const int kind = warp == 0 ? 0 : 1;
+      const int nslots = kind == 0 ? ns : nz;
       ok = produce<NP, QS, SG>(kind, s, &tm_cs, &tm_cz, &tm_q, cache, sched, B, r, max_len, tb, te,
                                n, nslots, lane, &issued, ch, cpart);
+      if (!ok && lane == 0) {
+        set_abort(s, status);
+        drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
+      }
     }
-    if (!ok && lane == 0) {
-      set_abort(s, status);
-      if constexpr (QB != 0) drain_q(kind, wsub, kConvWarps, s, nslots, nraw, issued, raw_issued);
-      else drain_ring(kind == 0 ? s.s_full : s.z_full, issued, nslots);
-    }
+    (void)raw_issued;
     __syncwarp();
   } else if (warp == 1 && !SG) {
     // ----------------------------------------------------------- S MMAs
-    if (lane == 0) {
+    if (QB && lane == 0) {
+      // quantised latent: one S item per 128-channel group, integer MMAs
+      // (M 128 tokens, N 3 NP query-part rows, K 32 bytes) accumulated onto
+      // a ring of nsg int32 group buffers that the softmax reads and refills
+      // with the bias 0x4B400000 (the bits of 1.5 x 2^23): a finished buffer
+      // holds the float 1.5 x 2^23 + S exactly (|S| < 2^22)
+      constexpr uint32_t id_q = idesc_i8(128, SW, true);   // signed codes x signed query parts
+      const uint64_t da0 = sdesc(saddr(s.sring), 16, 1024);   // K-major, 128B swizzle
+      constexpr int SQ = sq_slot_bytes<NP>();
+      Ring rg(ns);
+      Ring gr(nsg);
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        for (int u = 0; u < NC; ++u) {
+          // the buffer is released (first: initialised) biased by the softmax
+          if (!mbar_wait(saddr(&s.sg_empty[gr.slot]), gr.phase)) { ok = false; break; }
+          if (!mbar_wait(saddr(&s.s_full[rg.slot]), rg.phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t sa = da0 + uint64_t((rg.slot * SQ) >> 4);
+          const uint32_t d = tmem + uint32_t(gr.slot * SW);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // K = 32 channels (bytes) per MMA
+            tc_mma_i8(d, sa + uint64_t((kk * 32) >> 4), sa + uint64_t((128 * 128 + kk * 32) >> 4), id_q, 1u);
+          tc_commit(saddr(&s.s_empty[rg.slot]));
+          rg.advance();
+          tc_commit(saddr(&s.sg_full[gr.slot]));
+          gr.advance();
+        }
+        if (*s.abort_flag) ok = false;
+      }
+      if (!ok) set_abort(s, status);
+      tc_commit(saddr(&s.drain[0]));
+      mbar_wait(saddr(&s.drain[0]), 0);
+    } else if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(128, SW, BF16, false, false);
       const uint64_t da0 = sdesc(saddr(s.sring), 16, 1024);   // K-major, 128B swizzle
       Ring rg(ns);
-      Ring gr(QB ? nsg : 1);   // quantised latent: per-group S buffers
+      Ring gr(1);
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
         // the accumulator buffer of tile i was last read by the softmax of tile i - 2
@@ -680,6 +881,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       TileIter it;
       it.init(sched, B, tb, te);
       Ring rg(ra ? ns : nz);
+      int sbi = 0;   // quantised latent: scale table of the tile
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
         const bool first = it.first(tb);
@@ -706,6 +908,10 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         }
         if (!ok) break;
         tc_commit(saddr(&s.z_done[i & 1]));
+        if (QB) {   // the tile's scale table is free once its Z MMAs are complete
+          tc_commit(saddr(&s.zsc_empty[sbi]));
+          if (++sbi == kScaleBufs) sbi = 0;
+        }
         it.next();
         if (*s.abort_flag) ok = false;
       }
@@ -725,6 +931,20 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     TileIter it;
     it.init(sched, B, tb, te);
     Ring sgr(QB ? nsg : 1);   // quantised latent: the per-group S buffers
+    Ring scb(kScaleBufs);     // ... and the tiles' scale tables
+    float bias[16];           // 0x4B400000: 1.5 x 2^23
+#pragma unroll
+    for (int e = 0; e < 16; ++e) bias[e] = 12582912.f;
+    if (QB) {   // the group buffers start biased (each thread its own TMEM lane)
+      for (int gb = 0; gb < nsg; ++gb)
+#pragma unroll
+        for (int c = 0; c < 3 * NP / 16; ++c) tmem_st16(tmem + lane_off + uint32_t(gb * SW + 16 * c), bias);
+      tmem_wait_st();
+      tc_fence_before();
+      group_sync();
+      if (t == 0)
+        for (int gb = 0; gb < nsg; ++gb) mbar_arrive(saddr(&s.sg_empty[gb]));
+    }
     for (int i = 0; i < n; ++i) {
       const int pb = i & 1;
       const bool first = it.first(tb), last = it.last();
@@ -736,31 +956,52 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       }
       float sv[NP];
       if (QB) {
-        // s_t = sum_g scale_{t,g} (codes_{t,g} . qt_g), one TMEM buffer per group
+        // s_t = sigma_h sum_g scale_{t,g} (S0 + S1 / 128 + S2 / 16384), S_k
+        // the exact int32 sums of one group buffer (columns k NP + h) and
+        // sigma_h the query parts' scale of this (sequence, head), staged in
+        // shared memory here and read after the group loop's barriers
+        if (t < NP) s.qsig[t] = t < H ? __ldg(qsh + size_t(it.b) * H + t) : 0.f;
 #pragma unroll
         for (int h = 0; h < NP; ++h) sv[h] = 0.f;
-        const __half* tsc = scales + (size_t(it.b) * max_len + it.t0() + t) * NC;
+        fail = group_or(!mbar_wait(saddr(&s.zsc_full[scb.slot]), scb.phase));   // the tile's scale table
+        if (fail) { if (t == 0) set_abort(s, status); break; }
+        const uint32_t tsc = saddr(s.zsc) + uint32_t(scb.slot * scale_buf_bytes(r) + t * NC * 2);
+        scb.advance();
         for (int grp = 0; grp < NC; ++grp) {
-          const float sg = t < nv ? __half2float(tsc[grp]) : 0.f;
+          const float sg = __half2float(lds16h(tsc + uint32_t(grp * 2)));   // 0 past the length
           fail = group_or(!mbar_wait(saddr(&s.sg_full[sgr.slot]), sgr.phase));   // uniform
           if (fail) break;
           tc_fence_after();
           const uint32_t tg = tmem + lane_off + uint32_t(sgr.slot * SW);
 #pragma unroll
           for (int c = 0; c < NP / 16; ++c) {
-            float hi[16], lo[16];
-            tmem_ld16(tg + uint32_t(16 * c), hi);
-            tmem_ld16(tg + uint32_t(NP + 16 * c), lo);
+            float a0[16], a1[16], a2[16];
+            tmem_ld16(tg + uint32_t(16 * c), a0);
+            tmem_ld16(tg + uint32_t(NP + 16 * c), a1);
+            tmem_ld16(tg + uint32_t(2 * NP + 16 * c), a2);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) sv[16 * c + e] = fmaf(sg, hi[e] + lo[e], sv[16 * c + e]);
+            for (int e = 0; e < 16; ++e) {
+              const int h = 16 * c + e;
+              // a_k = 1.5 x 2^23 + S_k as floats (exact); subtracting the
+              // three biases (1.5 x 2^23 (1 + 2^-7 + 2^-14)) from a_0 is exact
+              // and leaves S0 + S1 / 128 + S2 / 16384 after the two fmas
+              const float g0 = a0[e] - 12681984.f;
+              sv[h] = fmaf(sg, fmaf(a2[e], 1.f / 16384.f, fmaf(a1[e], 1.f / 128.f, g0)), sv[h]);
+            }
           }
+          // refill the buffer with the bias for its next group
+#pragma unroll
+          for (int c = 0; c < 3 * NP / 16; ++c) tmem_st16(tg + uint32_t(16 * c), bias);
+          tmem_wait_st();
           tc_fence_before();
           group_sync();
           if (t == 0) mbar_arrive(saddr(&s.sg_empty[sgr.slot]));
           sgr.advance();
         }
         if (fail) { if (t == 0) set_abort(s, status); break; }
+#pragma unroll
+        for (int h = 0; h < NP; ++h) sv[h] *= s.qsig[h];
       } else if (SG) {
         // head h's scores of this tile: 128 consecutive floats per warp-row
         const float* sc = scores + size_t(it.b) * H * max_len + it.t0() + t;
@@ -1162,7 +1403,7 @@ void ring_slots(int* ns, int* nz) {
 template <int NP, bool BF16, int QB, bool SG = false>
 cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                      const float* scores, const int32_t* sched, int G, float* pm, float* pl,
-                     float* pz, int32_t* status, cudaStream_t s, int ch = 1) {
+                     float* pz, int32_t* status, cudaStream_t s, int ch = 1, const float* qsh = nullptr) {
   TensorMapEncode enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   constexpr int QS = 2;              // absorbed query as hi + lo 16-bit parts
@@ -1174,17 +1415,19 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   memset(&tcz, 0, sizeof(tcz));
   memset(&tq, 0, sizeof(tq));
   if (QB) {
-    // quantised latent: raw code rows [B * max_len][r QB / 8] bytes; S item
-    // box {QB x 8 bytes, 128 rows} (64 channels), Z item box {QB x 16 bytes,
-    // 64 rows} (128 channels); no swizzle (the warps convert them)
+    // quantised latent: code rows [B * max_len][r QB / 8] bytes.  S items are
+    // 128-channel groups of 128 rows: int8 codes straight into the MMA's
+    // layout (box {128 bytes, 128 rows}, 128-byte swizzle), int4 raw (box
+    // {64 bytes, 128 rows}, unswizzled: the warps unpack them).  Z items: box
+    // {QB x 16 bytes, 64 rows} (128 channels), unswizzled (converted).
     const cuuint64_t rb = cuuint64_t(d.r) * QB / 8;
     const cuuint64_t dims[2] = {rb, rows};
     const cuuint64_t strides[1] = {rb};
     const cuuint32_t es[2] = {1, 1};
-    const cuuint32_t bs[2] = {cuuint32_t(QB * 8), 128}, bz[2] = {cuuint32_t(QB * 16), 64};
+    const cuuint32_t bs[2] = {cuuint32_t(QB * 16), 128}, bz[2] = {cuuint32_t(QB * 16), 64};
     if (enc(&tcs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides, bs, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+            CU_TENSOR_MAP_INTERLEAVE_NONE, QB == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
         enc(&tcz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(cache), dims, strides, bz, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -1213,7 +1456,19 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  if (!SG) {
+  if (QB) {
+    // int8 query parts [B][3][H][r]: {128 channels, head, sequence x part};
+    // one box {128, NP, 3} lands as smem [part][head][128 bytes] (rows
+    // k NP + h), 128-byte swizzle.  Heads H..NP-1 arrive as zeros.
+    const cuuint64_t dims[3] = {cuuint64_t(d.r), cuuint64_t(d.H), cuuint64_t(d.batch) * 3};
+    const cuuint64_t strides[2] = {cuuint64_t(d.r), cuuint64_t(d.H) * d.r};
+    const cuuint32_t box[3] = {128, cuuint32_t(NP), 3};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(qt16), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else if (!SG) {
     // query parts: qt16 holds [B][QS][H][r] (hi, then the rounding residual),
     // seen as {64 channels, head, sequence * part, 64-channel box}; one box
     // {64, NP, QS, 1} lands as smem [part][head][64].  Heads H..NP-1 are
@@ -1230,22 +1485,20 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   int ns = 0, nz = 0, nraw = 0;
   ring_slots<NP, QS, PS>(&ns, &nz);
   if constexpr (QB != 0) {
-    // quantised latent: the fp16 slots are filled by conversion (short
-    // latency); each converting warp holds one while it converts, so the
-    // rings need more slots than converters to keep conversion off the MMAs'
-    // path.  The raw-code rings (a multiple of kConvWarps slots each) take
-    // what is left; of 6 or 3 raw slots, the choice with more fp16 slots.
-    const int base = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>();
-    const int pair = s_slot_bytes<NP, QS>() + kZSlotBytes;
-    int best = 0;
-    for (int cand = 2 * kConvWarps; cand >= kConvWarps; cand -= kConvWarps) {
-      if (cand > kMaxRaw || cand > d.r / 64) continue;
-      int slots = (base - 2 * cand * raw_bytes(QB)) / pair;
-      if (slots > kMaxSlots) slots = kMaxSlots;
-      if (slots > best) { best = slots; nraw = cand; }
+    // quantised latent: three S slots (codes + query parts, by TMA; int4:
+    // unpacked from a raw ring of 4 slots, a multiple of its two warps); the
+    // fp16 Z slots take the rest -- each converting warp holds one while it
+    // expands it, the MMAs read the ones before
+    nraw = QB == 4 ? 4 : 0;
+    const int avail = kSmemLimit - 1024 - kMiscBytes - 2 * PS * pbuf_bytes<NP>() -
+                      kScaleBufs * scale_buf_bytes(d.r) - nraw * raw_s_bytes(QB);
+    for (ns = 3; ns >= 2; --ns) {   // two S slots only where three leave fewer than 5 Z slots
+      nz = (avail - ns * sq_slot_bytes<NP>()) / kZSlotBytes;
+      if (nz >= 5) break;
     }
-    ns = nz = best;
-    if (nraw < kConvWarps || best < 2) return cudaErrorInvalidConfiguration;
+    if (ns < 2) ns = 2;
+    if (nz > kMaxSlots) nz = kMaxSlots;
+    if (nz < 4) return cudaErrorInvalidConfiguration;
   }
   if constexpr (SG) {
     // no S items: both rings carry Z items and share the budget
@@ -1254,19 +1507,20 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
     if (ns > kMaxSlots) ns = nz = kMaxSlots;
   }
   if (ns < 2 || nz < 2) return cudaErrorInvalidConfiguration;
-  // quantised latent: per-group S buffers in the TMEM left beside Z
-  int nsg = (512 - (d.r / 128) * NP) / (QS * NP);
+  // quantised latent: per-group int32 S buffers (3 NP columns) in the TMEM
+  // left beside Z
+  int nsg = (512 - (d.r / 128) * NP) / (3 * NP);
   if (nsg > kMaxGroupBufs) nsg = kMaxGroupBufs;
-  if (QB && nsg < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = 1024 + size_t(ns) * a_slot_bytes<NP, QS, SG>() + size_t(nz) * kZSlotBytes +
+  if (QB && nsg < 1) return cudaErrorInvalidConfiguration;
+  const size_t smem = 1024 + size_t(ns) * a_slot_bytes<NP, QS, SG, QB>() + size_t(nz) * kZSlotBytes +
                       2 * PS * pbuf_bytes<NP>() +
-                      (QB ? 2 * size_t(nraw) * raw_bytes(QB) : 0) + kMiscBytes;
+                      (QB ? size_t(nraw) * raw_s_bytes(QB) + kScaleBufs * scale_buf_bytes(d.r) : 0) + kMiscBytes;
   auto kern = k_split_tc<NP, BF16, QS, PS, QB, SG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   {
     const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(QB ? kThreadsTcQ : kThreadsTc), smem, s,
-                                     tcs, tcz, tq, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch);
+                                     tcs, tcz, tq, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch, qsh);
     if (le != cudaSuccess) return le;
   }
   note_launch();
@@ -1329,13 +1583,16 @@ bool split_tc_supported(const qsvd_dims& d) {
   if (d.r % 128) return false;
   const int np = split_tc_heads_padded(d);
   if (np == 0) return false;
-  if ((2 * 2 + d.r / 128) * np > 512) return false;   // two S buffers (or group buffers) of 2 np + Z
+  if (!q && (2 * 2 + d.r / 128) * np > 512) return false;   // two S buffers of 2 np + Z
+  if (q && (3 + d.r / 128) * np > 512) return false;        // one int32 group buffer of 3 np + Z
+  // quantised: the int8 query parts come from the tensor-core absorb kernel
+  if (q && ((d.weight_dtype != QSVD_F16 && d.weight_dtype != QSVD_BF16) || d.d_h % 64 || d.d_h > 256)) return false;
   return true;
 }
 
 cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
-                            int32_t* status, cudaStream_t s) {
+                            int32_t* status, cudaStream_t s, const float* qsh) {
   const int np = split_tc_heads_padded(d);
   const float* ns = nullptr;
   switch (d.cache_dtype) {
@@ -1343,11 +1600,11 @@ cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* s
       return np == 16 ? launch_t<16, true, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
                       : launch_t<32, true, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
     case QSVD_I4:
-      return np == 16 ? launch_t<16, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s, 1, qsh)
+                      : launch_t<32, false, 4>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s, 1, qsh);
     case QSVD_I8:
-      return np == 16 ? launch_t<16, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
-                      : launch_t<32, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
+      return np == 16 ? launch_t<16, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s, 1, qsh)
+                      : launch_t<32, false, 8>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s, 1, qsh);
     default:
       return np == 16 ? launch_t<16, false, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s)
                       : launch_t<32, false, 0>(d, cache, scales, qt16, ns, sched, G, pm, pl, pz, status, s);
