@@ -294,33 +294,40 @@ __device__ __forceinline__ __half lds16h(uint32_t a) {
 // 128 j + 127 of rows 64 h .. 64 h + 63, dequantised (code x group scale,
 // one fp16 rounding of the exact product), two 64-channel boxes of 64 rows,
 // 128-byte swizzled.  sct: the tile's scale table [128][ngroups] (zeros for
-// rows past the length, which therefore come out as zeros).  Warp-wide: the
-// whole item is read into registers before the first store overwrites it.
+// rows past the length, which therefore come out as zeros).  Warp-wide, in
+// two phases of 32 rows: a phase reads its raw rows into registers before
+// its first store, and its stores overwrite only raw rows of this phase or
+// the one before (int8: output row x of the second box is raw row x; int4:
+// the second box's rows 32-63 are the raw rows).
 template <int QB>
 __device__ __forceinline__ void convert_z_inplace(uint32_t d, uint32_t sct, int ngroups, int j, int h, int lane) {
   constexpr int RPB = QB * 16;            // raw bytes per row: 64 (int4), 128 (int8)
   constexpr int VPR = RPB / 16;
   constexpr int CPV = QB == 4 ? 4 : 2;
-  constexpr int NV = 64 * VPR / 32;       // vectors per lane: 8 (int4), 16 (int8)
+  constexpr int NV = 32 * VPR / 32;       // vectors per lane per phase: 4 (int4), 8 (int8)
   const uint32_t raw = d + uint32_t(kZSlotBytes - 64 * RPB);
-  uint4 rv[NV];
-  __half sc[NV];
+#pragma unroll 1
+  for (int ph = 0; ph < 2; ++ph) {
+    uint4 rv[NV];
+    __half sc[NV];
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR;
-    rv[i] = lds128(raw + tt * RPB + q * 16);
-    sc[i] = lds16h(sct + uint32_t(((64 * h + tt) * ngroups + j) * 2));
-  }
-  asm volatile("bar.warp.sync 0xffffffff;" ::: "memory");   // all loads before any store
+    for (int i = 0; i < NV; ++i) {
+      const int v = lane + 32 * i, tt = 32 * ph + v / VPR, q = v % VPR;
+      rv[i] = lds128(raw + tt * RPB + q * 16);
+      sc[i] = lds16h(sct + uint32_t(((64 * h + tt) * ngroups + j) * 2));
+    }
+    asm volatile("bar.warp.sync 0xffffffff;" ::: "memory");   // the phase's loads before its stores
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int v = lane + 32 * i, tt = v / VPR, q = v % VPR;
-    uint4 out[CPV];
-    codes_to_half<QB>(rv[i], true, __halves2half2(sc[i], sc[i]), out);
-    const int ch = q * (CPV * 8);         // first channel of the vector within the 128
-    const int box = ch >> 6, c0 = (ch & 63) >> 3;
+    for (int i = 0; i < NV; ++i) {
+      const int v = lane + 32 * i, tt = 32 * ph + v / VPR, q = v % VPR;
+      uint4 out[CPV];
+      codes_to_half<QB>(rv[i], true, __halves2half2(sc[i], sc[i]), out);
+      const int ch = q * (CPV * 8);         // first channel of the vector within the 128
+      const int box = ch >> 6, c0 = (ch & 63) >> 3;
 #pragma unroll
-    for (int c = 0; c < CPV; ++c) sts128(d + box * kZBoxBytes + tt * 128 + (((c0 + c) ^ (tt & 7)) << 4), out[c]);
+      for (int c = 0; c < CPV; ++c) sts128(d + box * kZBoxBytes + tt * 128 + (((c0 + c) ^ (tt & 7)) << 4), out[c]);
+    }
+    asm volatile("bar.warp.sync 0xffffffff;" ::: "memory");   // the phase's stores before the next's loads
   }
   fence_proxy_async();   // generic-proxy stores -> visible to the tensor core
   __syncwarp();
@@ -710,7 +717,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     }
     for (int i = 0; i < kMaxGroupBufs; ++i) {
       mbar_init(saddr(&s.sg_full[i]), 1);
-      mbar_init(saddr(&s.sg_empty[i]), 1);
+      mbar_init(saddr(&s.sg_empty[i]), 4);   // one arrive per softmax warp
     }
     for (int i = 0; i < kMaxRaw; ++i) mbar_init(saddr(&s.sraw_full[i]), 1);
     for (int i = 0; i < kMaxSlots; ++i) mbar_init(saddr(&s.zraw_full[i]), 1);
@@ -932,17 +939,15 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     it.init(sched, B, tb, te);
     Ring sgr(QB ? nsg : 1);   // quantised latent: the per-group S buffers
     Ring scb(kScaleBufs);     // ... and the tiles' scale tables
-    float bias[16];           // 0x4B400000: 1.5 x 2^23
-#pragma unroll
-    for (int e = 0; e < 16; ++e) bias[e] = 12582912.f;
-    if (QB) {   // the group buffers start biased (each thread its own TMEM lane)
+    constexpr uint32_t kBias = 0x4B400000u;   // the bits of 1.5 x 2^23
+    if (QB) {   // the group buffers start biased (each warp its own 32 TMEM lanes)
       for (int gb = 0; gb < nsg; ++gb)
 #pragma unroll
-        for (int c = 0; c < 3 * NP / 16; ++c) tmem_st16(tmem + lane_off + uint32_t(gb * SW + 16 * c), bias);
+        for (int c = 0; c < 3 * NP / 16; ++c) tmem_fill16(tmem + lane_off + uint32_t(gb * SW + 16 * c), kBias);
       tmem_wait_st();
       tc_fence_before();
-      group_sync();
-      if (t == 0)
+      __syncwarp();
+      if (lane == 0)
         for (int gb = 0; gb < nsg; ++gb) mbar_arrive(saddr(&s.sg_empty[gb]));
     }
     for (int i = 0; i < n; ++i) {
@@ -959,17 +964,19 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
         // s_t = sigma_h sum_g scale_{t,g} (S0 + S1 / 128 + S2 / 16384), S_k
         // the exact int32 sums of one group buffer (columns k NP + h) and
         // sigma_h the query parts' scale of this (sequence, head), staged in
-        // shared memory here and read after the group loop's barriers
+        // shared memory here and read after the barrier that ends the group loop
         if (t < NP) s.qsig[t] = t < H ? __ldg(qsh + size_t(it.b) * H + t) : 0.f;
 #pragma unroll
         for (int h = 0; h < NP; ++h) sv[h] = 0.f;
-        fail = group_or(!mbar_wait(saddr(&s.zsc_full[scb.slot]), scb.phase));   // the tile's scale table
-        if (fail) { if (t == 0) set_abort(s, status); break; }
+        // the groups run without CTA-level barriers: each warp waits for a
+        // buffer itself and releases it with its own arrive; a failed wait
+        // stops that warp's loop and the four agree after it
+        fail = !__all_sync(0xffffffffu, mbar_wait(saddr(&s.zsc_full[scb.slot]), scb.phase));   // scale table
         const uint32_t tsc = saddr(s.zsc) + uint32_t(scb.slot * scale_buf_bytes(r) + t * NC * 2);
         scb.advance();
-        for (int grp = 0; grp < NC; ++grp) {
+        for (int grp = 0; grp < NC && !fail; ++grp) {
           const float sg = __half2float(lds16h(tsc + uint32_t(grp * 2)));   // 0 past the length
-          fail = group_or(!mbar_wait(saddr(&s.sg_full[sgr.slot]), sgr.phase));   // uniform
+          fail = !__all_sync(0xffffffffu, mbar_wait(saddr(&s.sg_full[sgr.slot]), sgr.phase));   // warp-uniform
           if (fail) break;
           tc_fence_after();
           const uint32_t tg = tmem + lane_off + uint32_t(sgr.slot * SW);
@@ -992,14 +999,14 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           }
           // refill the buffer with the bias for its next group
 #pragma unroll
-          for (int c = 0; c < 3 * NP / 16; ++c) tmem_st16(tg + uint32_t(16 * c), bias);
+          for (int c = 0; c < 3 * NP / 16; ++c) tmem_fill16(tg + uint32_t(16 * c), kBias);
           tmem_wait_st();
           tc_fence_before();
-          group_sync();
-          if (t == 0) mbar_arrive(saddr(&s.sg_empty[sgr.slot]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(saddr(&s.sg_empty[sgr.slot]));
           sgr.advance();
         }
-        if (fail) { if (t == 0) set_abort(s, status); break; }
+        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }   // also orders the qsig stores
 #pragma unroll
         for (int h = 0; h < NP; ++h) sv[h] *= s.qsig[h];
       } else if (SG) {
