@@ -39,9 +39,13 @@
 //   warps 4-7  softmax over the S accumulator (one TMEM lane = one token),
 //              conditional rescale of Z, P written to shared memory, and the
 //              per-segment epilogue (partials m, l, z to global memory)
-// Quantised latent (384 threads): raw codes arrive by TMA and three warps
-// per stream convert them (S: warps 0, 9, 10; Z: warps 2, 8, 11); S is
-// accumulated per 128-channel group and scaled per token by the softmax.
+// Quantised latent (384 threads; 512 with 32 padded heads): S runs on the
+// integer tensor cores per 128-channel group (int8 codes straight from the
+// cache by TMA on warp 0; int4 codes unpacked to bytes by warps 0 and 9) and
+// is scaled per token by the softmax; for Z, warp 2 loads each item's raw
+// codes into the end of its fp16 slot and warps 8-11 (int4: 8, 10, 11)
+// dequantise them in place.  With 32 padded heads a second group of softmax
+// warps (12-15) takes heads 16-31.
 // Scores given (rotary mode): no S pass; warps 1 and 3 both issue Z MMAs.
 //
 // Precision: the absorbed query enters the MMA as hi + lo 16-bit parts and,
@@ -66,6 +70,15 @@ namespace {
 
 constexpr int kThreadsTc = 256;
 constexpr int kThreadsTcQ = 384;   // quantised latent: warps 8-11 convert too
+// Softmax groups of four warps: two (the second on warps 12-15, heads split
+// in halves) for a quantised latent with 32 padded heads, whose per-group
+// score reads dominate the softmax; one otherwise.
+template <int NP, int QB>
+__host__ __device__ constexpr int softmax_groups() { return (QB && NP == 32) ? 2 : 1; }
+template <int NP, int QB>
+__host__ __device__ constexpr int split_threads() {
+  return QB ? kThreadsTcQ + 128 * (softmax_groups<NP, QB>() - 1) : kThreadsTc;
+}
 constexpr int kBoxBytes = 128 * 128;            // 128 tokens x 64 channels x 2 bytes
 constexpr int kMaxSlots = 8;                   // per ring
 constexpr int kMaxGroupBufs = 4;               // S accumulators per channel group (quantised latent)
@@ -679,7 +692,7 @@ __device__ void drain_ring(uint64_t* full, long long k, int nslots) {
 // blockIdx.x / ch), each owning every ch-th chunk; all of them run the same
 // softmax on the same scores and part 0 writes m and l.
 template <int NP, bool BF16, int QS, int PS, int QB, bool SG>
-__global__ void __launch_bounds__(QB ? kThreadsTcQ : kThreadsTc, 1)
+__global__ void __launch_bounds__(split_threads<NP, QB>(), 1)
 k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cz,
            const __grid_constant__ CUtensorMap tm_q,
            const uint8_t* __restrict__ cache, const __half* __restrict__ scales,
@@ -697,6 +710,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
   // S accumulator columns per buffer: hi and lo query parts (16-bit), or the
   // three int8 query parts' int32 sums of one group (quantised)
   constexpr int SW = QB ? 3 * NP : QS * NP;
+  constexpr int WG = softmax_groups<NP, QB>(), HW = NP / WG;   // softmax groups, heads per group
   const int ZC0 = SG ? 0 : (QB ? nsg : 2) * SW;   // first Z column
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = r / 64;                      // ring items per tile
@@ -717,7 +731,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     }
     for (int i = 0; i < kMaxGroupBufs; ++i) {
       mbar_init(saddr(&s.sg_full[i]), 1);
-      mbar_init(saddr(&s.sg_empty[i]), 4);   // one arrive per softmax warp
+      mbar_init(saddr(&s.sg_empty[i]), 4 * WG);   // one arrive per softmax warp
     }
     for (int i = 0; i < kMaxRaw; ++i) mbar_init(saddr(&s.sraw_full[i]), 1);
     for (int i = 0; i < kMaxSlots; ++i) mbar_init(saddr(&s.zraw_full[i]), 1);
@@ -732,7 +746,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(saddr(&s.acc_full[i]), 1);
-      mbar_init(saddr(&s.p_full[i]), 1);
+      mbar_init(saddr(&s.p_full[i]), WG);   // one arrive per softmax group
       mbar_init(saddr(&s.z_done[i]), SG ? 2 : 1);   // SG: one commit per Z issuer
       mbar_init(saddr(&s.drain[i]), 1);
     }
@@ -750,7 +764,7 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = *s.tmem_holder;
 
-  if (warp == 0 || warp == 2 || (QB && warp >= 8)) {
+  if (warp == 0 || warp == 2 || (QB && warp >= 8 && warp < 12)) {
     // ----------------------------------------------------------- producers
     bool ok = true;
     long long issued = 0, raw_issued = 0;
@@ -929,12 +943,17 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     __syncwarp();
   } else {
     // ------------------------------------------------ softmax and epilogue
+    // WG groups of four warps (warps 4-7, and 12-15 when WG = 2) each own
+    // HW = NP / WG heads, hb .. hb + HW - 1: their score columns, running max
+    // and sum, P rows, Z columns and partials; a group synchronises on its
+    // own named barrier (1 + wg)
     const int q = warp & 3;
     const int t = 32 * q + lane;              // token row in the tile == TMEM lane
+    const int wg = warp >= 12 ? 1 : 0, hb = wg * HW, bid = 1 + wg;
     const uint32_t lane_off = uint32_t(32 * q) << 16;
     const uint64_t inject_ns = g_score_wait_ns;
-    // m and l per head live in shared memory (identical for the four warps);
-    // thread t < NP owns head t's entries
+    // m and l per head live in shared memory (identical for the group's four
+    // warps); thread t < HW owns head hb + t's entries
     TileIter it;
     it.init(sched, B, tb, te);
     Ring sgr(QB ? nsg : 1);   // quantised latent: the per-group S buffers
@@ -943,7 +962,8 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
     if (QB) {   // the group buffers start biased (each warp its own 32 TMEM lanes)
       for (int gb = 0; gb < nsg; ++gb)
 #pragma unroll
-        for (int c = 0; c < 3 * NP / 16; ++c) tmem_fill16(tmem + lane_off + uint32_t(gb * SW + 16 * c), kBias);
+        for (int c = 0; c < 3 * HW / 16; ++c)
+          tmem_fill16(tmem + lane_off + uint32_t(gb * SW + (c / (HW / 16)) * NP + hb + 16 * (c % (HW / 16))), kBias);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -955,19 +975,19 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       const bool first = it.first(tb), last = it.last();
       const int nv = it.nvalid();
       int fail = 0;
-      if (inject_ns && i == 0 && group_or(!mbar_wait_ns(saddr(s.never), 0, inject_ns))) {
+      if (inject_ns && i == 0 && group_or(!mbar_wait_ns(saddr(s.never), 0, inject_ns), bid)) {
         if (t == 0) set_abort(s, status);
         break;
       }
-      float sv[NP];
+      float sv[HW];
       if (QB) {
         // s_t = sigma_h sum_g scale_{t,g} (S0 + S1 / 128 + S2 / 16384), S_k
         // the exact int32 sums of one group buffer (columns k NP + h) and
         // sigma_h the query parts' scale of this (sequence, head), staged in
         // shared memory here and read after the barrier that ends the group loop
-        if (t < NP) s.qsig[t] = t < H ? __ldg(qsh + size_t(it.b) * H + t) : 0.f;
+        if (t < HW) s.qsig[hb + t] = hb + t < H ? __ldg(qsh + size_t(it.b) * H + hb + t) : 0.f;
 #pragma unroll
-        for (int h = 0; h < NP; ++h) sv[h] = 0.f;
+        for (int h = 0; h < HW; ++h) sv[h] = 0.f;
         // the groups run without CTA-level barriers: each warp waits for a
         // buffer itself and releases it with its own arrive; a failed wait
         // stops that warp's loop and the four agree after it
@@ -981,11 +1001,11 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           tc_fence_after();
           const uint32_t tg = tmem + lane_off + uint32_t(sgr.slot * SW);
 #pragma unroll
-          for (int c = 0; c < NP / 16; ++c) {
+          for (int c = 0; c < HW / 16; ++c) {
             float a0[16], a1[16], a2[16];
-            tmem_ld16(tg + uint32_t(16 * c), a0);
-            tmem_ld16(tg + uint32_t(NP + 16 * c), a1);
-            tmem_ld16(tg + uint32_t(2 * NP + 16 * c), a2);
+            tmem_ld16(tg + uint32_t(hb + 16 * c), a0);
+            tmem_ld16(tg + uint32_t(NP + hb + 16 * c), a1);
+            tmem_ld16(tg + uint32_t(2 * NP + hb + 16 * c), a2);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -999,79 +1019,81 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
           }
           // refill the buffer with the bias for its next group
 #pragma unroll
-          for (int c = 0; c < 3 * NP / 16; ++c) tmem_fill16(tg + uint32_t(16 * c), kBias);
+          for (int c = 0; c < 3 * HW / 16; ++c)
+            tmem_fill16(tg + uint32_t((c / (HW / 16)) * NP + hb + 16 * (c % (HW / 16))), kBias);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(saddr(&s.sg_empty[sgr.slot]));
           sgr.advance();
         }
-        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }   // also orders the qsig stores
+        if (group_or(fail, bid)) { if (t == 0) set_abort(s, status); break; }   // also orders the qsig stores
 #pragma unroll
-        for (int h = 0; h < NP; ++h) sv[h] *= s.qsig[h];
+        for (int h = 0; h < HW; ++h) sv[h] *= s.qsig[hb + h];
       } else if (SG) {
         // head h's scores of this tile: 128 consecutive floats per warp-row
         const float* sc = scores + size_t(it.b) * H * max_len + it.t0() + t;
         const bool ok = t < nv;
 #pragma unroll
-        for (int h = 0; h < NP; ++h) sv[h] = (ok && h < H) ? __ldg(sc + size_t(h) * max_len) : -INFINITY;
+        for (int h = 0; h < HW; ++h) sv[h] = (ok && hb + h < H) ? __ldg(sc + size_t(hb + h) * max_len) : -INFINITY;
       } else {
         fail = !mbar_wait(saddr(&s.acc_full[pb]), uint32_t(i >> 1) & 1u);
-        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+        if (group_or(fail, bid)) { if (t == 0) set_abort(s, status); break; }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < NP / 16; ++c) tmem_ld16(tmem + lane_off + uint32_t(pb * SW + 16 * c), sv + 16 * c);
+        for (int c = 0; c < HW / 16; ++c) tmem_ld16(tmem + lane_off + uint32_t(pb * SW + hb + 16 * c), sv + 16 * c);
         if (QS == 2) {   // S = C (q_hi + q_lo)
-          float lo[NP];
+          float lo[HW];
 #pragma unroll
-          for (int c = 0; c < NP / 16; ++c)
-            tmem_ld16(tmem + lane_off + uint32_t(pb * SW + NP + 16 * c), lo + 16 * c);
+          for (int c = 0; c < HW / 16; ++c)
+            tmem_ld16(tmem + lane_off + uint32_t(pb * SW + NP + hb + 16 * c), lo + 16 * c);
           tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < NP; ++h) sv[h] += lo[h];
+          for (int h = 0; h < HW; ++h) sv[h] += lo[h];
         }
         tmem_wait_ld();
       }
       const bool valid = t < nv;
       int need = first;   // a segment starts: m and l are set below
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < HW; ++h) {
         if (!valid) sv[h] = -INFINITY;
-        need |= sv[h] > s.m_run[h] + kRescaleLog2;
+        need |= sv[h] > s.m_run[hb + h] + kRescaleLog2;
       }
-      if (group_or(need)) {
+      if (group_or(need, bid)) {
         // exact tile max per head over the 128 rows
         {
-          float tmp[NP];
+          float tmp[HW];
 #pragma unroll
-          for (int h = 0; h < NP; ++h) tmp[h] = sv[h];
-          reduce_heads<NP>(tmp, s.red + q * NP, lane, dev::OpMax());
+          for (int h = 0; h < HW; ++h) tmp[h] = sv[h];
+          reduce_heads<HW>(tmp, s.red + q * NP + hb, lane, dev::OpMax());
         }
-        group_sync();
-        if (t < NP) {
-          const float mt = fmaxf(fmaxf(s.red[t], s.red[NP + t]), fmaxf(s.red[2 * NP + t], s.red[3 * NP + t]));
-          const float mo = first ? -INFINITY : s.m_run[t];
+        group_sync(bid);
+        if (t < HW) {
+          const int h = hb + t;
+          const float mt = fmaxf(fmaxf(s.red[h], s.red[NP + h]), fmaxf(s.red[2 * NP + h], s.red[3 * NP + h]));
+          const float mo = first ? -INFINITY : s.m_run[h];
           const float mn = fmaxf(mo, mt);
           const float a = exp2f(mo - mn);
-          s.alpha[t] = a;
-          s.m_run[t] = mn;
-          s.l_run[t] = first ? 0.f : s.l_run[t] * a;
+          s.alpha[h] = a;
+          s.m_run[h] = mn;
+          s.l_run[h] = first ? 0.f : s.l_run[h] * a;
         }
-        group_sync();
+        group_sync(bid);
         if (!first) {
           // Z of the previous tile must be complete before it is rescaled
           fail = !mbar_wait(saddr(&s.z_done[(i - 1) & 1]), uint32_t((i - 1) >> 1) & 1u);
-          if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+          if (group_or(fail, bid)) { if (t == 0) set_abort(s, status); break; }
           tc_fence_after();
           for (int c = 0; c < NCL; ++c) {
 #pragma unroll
-            for (int h16 = 0; h16 < NP / 16; ++h16) {
+            for (int h16 = 0; h16 < HW / 16; ++h16) {
               float z[16];
-              const uint32_t ta = tmem + lane_off + uint32_t(ZC0 + c * NP + 16 * h16);
+              const uint32_t ta = tmem + lane_off + uint32_t(ZC0 + c * NP + hb + 16 * h16);
               tmem_ld16(ta, z);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 16; ++e) z[e] *= s.alpha[16 * h16 + e];
+              for (int e = 0; e < 16; ++e) z[e] *= s.alpha[hb + 16 * h16 + e];
               tmem_st16(ta, z);
             }
           }
@@ -1081,24 +1103,24 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       // P = 2^(s - m) as the B operand of the Z MMA: P^T, K-major, 128B swizzle
       if (i >= 2) {
         fail = !mbar_wait(saddr(&s.z_done[pb]), uint32_t((i - 2) >> 1) & 1u);
-        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+        if (group_or(fail, bid)) { if (t == 0) set_abort(s, status); break; }
       }
       uint8_t* pbase = s.pbuf + pb * PS * pbuf_bytes<NP>() + (t >> 6) * NP * 128;
       const int chunk = (t & 63) >> 3, within = (t & 7) * 2;
-      float mr[NP];   // m into registers first: the P stores below would order each reload
+      float mr[HW];   // m into registers first: the P stores below would order each reload
 #pragma unroll
-      for (int h4 = 0; h4 < NP / 4; ++h4) {
-        const float4 v = reinterpret_cast<const float4*>(s.m_run)[h4];
+      for (int h4 = 0; h4 < HW / 4; ++h4) {
+        const float4 v = reinterpret_cast<const float4*>(s.m_run + hb)[h4];
         mr[4 * h4] = v.x;
         mr[4 * h4 + 1] = v.y;
         mr[4 * h4 + 2] = v.z;
         mr[4 * h4 + 3] = v.w;
       }
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < HW; ++h) {
         const float p = valid ? exp2f(sv[h] - mr[h]) : 0.f;
         sv[h] = p;
-        uint8_t* dst = pbase + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
+        uint8_t* dst = pbase + (hb + h) * 128 + ((chunk ^ ((hb + h) & 7)) << 4) + within;
         if (PS == 2) {
           const __nv_bfloat16 hi = __float2bfloat16_rn(p);
           *reinterpret_cast<__nv_bfloat16*>(dst) = hi;
@@ -1110,26 +1132,30 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
       }
       fence_proxy_async();
       tc_fence_before();
-      group_sync();
-      if (t == 0) mbar_arrive(saddr(&s.p_full[pb]));
+      group_sync(bid);
+      if (t == 0) mbar_arrive(saddr(&s.p_full[pb]));   // one arrive per group
       // l += this tile's P summed over its 128 tokens (after the hand-off)
-      reduce_heads<NP>(sv, s.red + q * NP, lane, dev::OpAdd());
-      group_sync();
-      if (t < NP) s.l_run[t] += (s.red[t] + s.red[NP + t]) + (s.red[2 * NP + t] + s.red[3 * NP + t]);
+      reduce_heads<HW>(sv, s.red + q * NP + hb, lane, dev::OpAdd());
+      group_sync(bid);
+      if (t < HW) {
+        const int h = hb + t;
+        s.l_run[h] += (s.red[h] + s.red[NP + h]) + (s.red[2 * NP + h] + s.red[3 * NP + h]);
+      }
       if (last) {
         fail = !mbar_wait(saddr(&s.z_done[pb]), uint32_t(i >> 1) & 1u);
-        if (group_or(fail)) { if (t == 0) set_abort(s, status); break; }
+        if (group_or(fail, bid)) { if (t == 0) set_abort(s, status); break; }
         tc_fence_after();
         const size_t slot = size_t(g) + it.b;
         // z^T chunk c: TMEM lane = channel 128 c + t, column = head, taken
         // EW head columns at a time (registers); the load of chunk c + 1 is
         // in flight while chunk c is stored
-        constexpr int EW = NP % 32 == 0 ? 32 : 16;
+        constexpr int EW = HW % 32 == 0 ? 32 : 16;
         float* zrow = pz + slot * size_t(H) * r + t;
 #pragma unroll 1
-        for (int hg = 0; hg < NP / EW; ++hg) {
+        for (int hg = 0; hg < HW / EW; ++hg) {
           float zc[EW], zn[EW];
-          const uint32_t tcol = tmem + lane_off + uint32_t(ZC0 + hg * EW);
+          const int h0 = hb + hg * EW;   // first head of the group of columns
+          const uint32_t tcol = tmem + lane_off + uint32_t(ZC0 + h0);
 #pragma unroll
           for (int e16 = 0; e16 < EW / 16; ++e16) tmem_ld16(tcol + uint32_t(16 * e16), zc + 16 * e16);
           tmem_wait_ld();
@@ -1140,10 +1166,10 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
                 tmem_ld16(tcol + uint32_t((c + 1) * NP + 16 * e16), zn + 16 * e16);
             }
             // row pointer stepped by r: no per-store index arithmetic
-            float* zp = zrow + size_t(hg * EW) * r + 128 * (SG ? c * ch + cpart : c);
+            float* zp = zrow + size_t(h0) * r + 128 * (SG ? c * ch + cpart : c);
 #pragma unroll
             for (int e = 0; e < EW; ++e) {
-              if (hg * EW + e < H) *zp = zc[e];
+              if (h0 + e < H) *zp = zc[e];
               zp += r;
             }
             tmem_wait_ld();
@@ -1151,13 +1177,13 @@ k_split_tc(const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CU
             for (int e = 0; e < EW; ++e) zc[e] = zn[e];
           }
         }
-        if (cpart == 0 && t < H && t < NP) {   // the thread that owns head t's m and l
-          pl[slot * H + t] = s.l_run[t];
-          pm[slot * H + t] = s.m_run[t];
+        if (cpart == 0 && t < HW && hb + t < H) {   // the thread that owns head hb + t's m and l
+          pl[slot * H + hb + t] = s.l_run[hb + t];
+          pm[slot * H + hb + t] = s.m_run[hb + t];
         }
       }
       it.next();
-      if (group_or(*s.abort_flag)) break;
+      if (group_or(*s.abort_flag, bid)) break;
     }
   }
   tc_fence_before();
@@ -1526,7 +1552,7 @@ cudaError_t launch_t(const qsvd_dims& d, const void* cache, const void* scales, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   {
-    const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(QB ? kThreadsTcQ : kThreadsTc), smem, s,
+    const cudaError_t le = launch_pdl(kern, dim3(G * ch), dim3(split_threads<NP, QB>()), smem, s,
                                      tcs, tcz, tq, static_cast<const uint8_t*>(cache), static_cast<const __half*>(scales), scores, sched, pm, pl, pz, status, d.batch, d.H, d.r, d.max_len, G, ns, nz, nsg, nraw, ch, qsh);
     if (le != cudaSuccess) return le;
   }

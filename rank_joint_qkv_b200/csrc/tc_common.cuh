@@ -212,6 +212,20 @@ __device__ __forceinline__ int group_or(int pred) {
   return r;
 }
 __device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The same on named barrier `id` (a second group of 128 threads uses id 2).
+__device__ __forceinline__ int group_or(int pred, int id) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return r;
+}
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
