@@ -179,8 +179,14 @@ k_append_chunk(const float* __restrict__ cpart, int KS, const int32_t* __restric
 template <typename WT>
 cudaError_t gemv_t(const qsvd_dims& d, const void* x, const void* wd, float* cpart, int KS,
                    int32_t* status, cudaStream_t s) {
+  // W^u_q and W^u_k follow W^d in the packed weights: the decode's query
+  // GEMV and absorption read them next, so they are requested into L2 here
+  const PackedLayout L = packed_layout(d);
+  const uint8_t* wq = static_cast<const uint8_t*>(wd) + (L.wuq - L.wd);
+  const size_t pf_bytes = L.wuk + size_t(d.E) * d.r * sizeof(WT) - L.wuq;
   return launch_gemv<WT, WT>(static_cast<const WT*>(x), static_cast<const WT*>(wd), cpart, d.batch,
-                             d.E, d.r, KS, static_cast<float*>(nullptr), nullptr, status, s);
+                             d.E, d.r, KS, static_cast<float*>(nullptr), nullptr, status, s, XGroups{0, 0, 0},
+                             wq, pf_bytes);
 }
 
 int append_chunk(const qsvd_dims& d) {

@@ -31,7 +31,10 @@ constexpr int kMergeMaxSplits = 2048;   // weights kept in shared memory per (b,
 __global__ void __launch_bounds__(128)
 k_merge(const WsHeader* __restrict__ hdr, const int32_t* __restrict__ sched,
         const float* __restrict__ pm, const float* __restrict__ pl, const float* __restrict__ pz,
-        float* __restrict__ zm, int B, int H, int r) {
+        float* __restrict__ zm, int B, int H, int r, const uint8_t* __restrict__ pf,
+        unsigned long long pf_bytes) {
+  // the following GEMV's weights towards L2 (constant; a hint)
+  if (pf_bytes && threadIdx.x == 32) dev::l2_prefetch_share(pf, pf_bytes);
   dev::pdl_wait();   // see launch_pdl
   dev::pdl_trigger();
   __shared__ float wt[kMergeMaxSplits];
@@ -320,8 +323,13 @@ cudaError_t merge_vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* 
                         const OutProj& op, cudaStream_t s) {
   const dim3 grid((d.r + kMergeCh - 1) / kMergeCh, d.H, d.batch);
   {
-    const cudaError_t le = launch_pdl(k_merge, dim3(grid), dim3(128), 0, s,
-                                     hdr, sched, pm, pl, pz, zm, d.batch, d.H, d.r);
+    // the GEMV after the merge reads F (fold) or W^u_v
+    const size_t wb = sizeof(WT);
+    const void* pf = d.out_proj == QSVD_OUT_PROJ_FOLD ? op.wo : wuv;
+    const size_t pf_bytes = d.out_proj == QSVD_OUT_PROJ_FOLD ? size_t(d.H) * d.r * d.E * wb : size_t(d.r) * d.E * wb;
+    const cudaError_t le = launch_pdl(k_merge, dim3(grid), dim3(128), 0, s, hdr, sched, pm, pl, pz, zm,
+                                     d.batch, d.H, d.r, static_cast<const uint8_t*>(pf),
+                                     (unsigned long long)pf_bytes);
     if (le != cudaSuccess) return le;
   }
   note_launch();

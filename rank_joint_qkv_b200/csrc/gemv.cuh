@@ -239,7 +239,8 @@ template <typename XT, typename WT, typename OT = float>
 __global__ void __launch_bounds__(128)
 k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x, XGroups xg,
            float* __restrict__ part, int B, int K, int N, int KS, OT* __restrict__ out,
-           int32_t* __restrict__ ticket, int32_t* status) {
+           int32_t* __restrict__ ticket, int32_t* status, const uint8_t* __restrict__ pf,
+           unsigned long long pf_bytes) {
   using namespace gemv_mma;
   constexpr bool BF16 = std::is_same<WT, __nv_bfloat16>::value;
   constexpr bool SPLIT = !std::is_same<XT, WT>::value;   // activation wider than the weights
@@ -276,6 +277,8 @@ k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x, X
           : "memory");
   }
 
+  // the next kernel's weights towards L2 (constant: no need to wait for anything)
+  if (pf_bytes && tid == 32) dev::l2_prefetch_share(pf, pf_bytes);
   // the weight tile is in flight; everything below reads what earlier kernels wrote
   dev::pdl_wait();   // see launch_pdl
   dev::pdl_trigger();
@@ -441,11 +444,13 @@ k_gemv_mma(const __grid_constant__ CUtensorMap tm_w, const XT* __restrict__ x, X
 
 // Launch the GEMV: tensor cores for 16-bit weights, CUDA cores for fp32.
 // Per-group activation rows (xg) and a non-float output need the tensor-core
-// variant (16-bit weights).
+// variant (16-bit weights).  pf / pf_bytes: constant bytes the next kernel
+// reads (its weights), requested into L2 while this one runs (tensor-core
+// variant; a hint only).
 template <typename XT, typename WT, typename OT = float>
 cudaError_t launch_gemv(const XT* x, const WT* W, float* part, int B, int K, int N, int KS,
                         OT* out, int32_t* ticket, int32_t* status, cudaStream_t s,
-                        XGroups xg = XGroups{0, 0, 0}) {
+                        XGroups xg = XGroups{0, 0, 0}, const void* pf = nullptr, size_t pf_bytes = 0) {
   if (xg.cols == 0) xg = XGroups{K, N, 0};
   cudaError_t e;
   if constexpr (sizeof(WT) == 2) {
@@ -471,8 +476,9 @@ cudaError_t launch_gemv(const XT* x, const WT* W, float* part, int B, int K, int
       e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     {
-      const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(128), smem, s,
-                                       tm, x, xg, part, B, K, N, KS, out, ticket, status);
+      const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(128), smem, s, tm, x, xg, part, B, K, N, KS,
+                                       out, ticket, status, static_cast<const uint8_t*>(pf),
+                                       (unsigned long long)pf_bytes);
       if (le != cudaSuccess) return le;
     }
   } else {

@@ -323,6 +323,23 @@ cudaError_t launch_prepare_out_proj(const qsvd_dims& d, const void* wo, void* pa
 
 namespace qsvd {
 namespace dev {
+// This CTA's share of [p, p + bytes) requested into L2 by bulk prefetches
+// (16-byte granules, 64 KB per request): a hint for the kernel that reads
+// those bytes next, with no effect on any result.  p 16-byte aligned.
+__device__ __forceinline__ void l2_prefetch_share(const uint8_t* p, unsigned long long bytes) {
+  const unsigned long long ncta = (unsigned long long)gridDim.x * gridDim.y * gridDim.z;
+  const unsigned long long cta =
+      blockIdx.x + (unsigned long long)gridDim.x * (blockIdx.y + (unsigned long long)gridDim.y * blockIdx.z);
+  const unsigned long long end = bytes & ~15ull;
+  const unsigned long long share = ((end + ncta - 1) / ncta + 15) & ~15ull;
+  unsigned long long lo = cta * share;
+  const unsigned long long hi = lo + share < end ? lo + share : end;
+  for (; lo < hi; lo += 65536) {
+    const unsigned n = unsigned(hi - lo < 65536 ? hi - lo : 65536);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + lo), "r"(n) : "memory");
+  }
+}
+
 
 // See launch_pdl.  A no-op when the kernel was launched without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
