@@ -239,15 +239,18 @@ __device__ __forceinline__ void ragged_rows(uint8_t* d, const uint8_t* src, size
 // fma); byte permutes restore channel order.
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-__device__ __forceinline__ void int4x8_to_half(uint32_t w, __half2 s2, bool scaled, uint32_t& o0,
-                                               uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+__device__ __forceinline__ void int4x8_to_half(uint32_t w, __half2 s2, uint32_t& o0, uint32_t& o1,
+                                               uint32_t& o2, uint32_t& o3) {
   const uint32_t x = w ^ 0x88888888u;   // offset binary: code + 8 in 0..15
   const __half2 b1032 = u2h(0x64086408u), s16 = u2h(0x2C002C00u), b72 = u2h(0xD480D480u);   // 1032, 1/16, -72
   __half2 ha = __hsub2(u2h((x & 0x000F000Fu) | 0x64006400u), b1032);          // c0, c4
   __half2 hb = __hfma2(u2h((x & 0x00F000F0u) | 0x64006400u), s16, b72);       // c1, c5
   __half2 hc = __hsub2(u2h(((x >> 8) & 0x000F000Fu) | 0x64006400u), b1032);   // c2, c6
   __half2 hd = __hfma2(u2h(((x >> 8) & 0x00F000F0u) | 0x64006400u), s16, b72); // c3, c7
-  if (scaled) { ha = __hmul2(ha, s2); hb = __hmul2(hb, s2); hc = __hmul2(hc, s2); hd = __hmul2(hd, s2); }
+  ha = __hmul2(ha, s2);   // times the group scale: one rounding of the exact product
+  hb = __hmul2(hb, s2);
+  hc = __hmul2(hc, s2);
+  hd = __hmul2(hd, s2);
   const uint32_t ua = h2u(ha), ub = h2u(hb), uc = h2u(hc), ud = h2u(hd);
   o0 = __byte_perm(ua, ub, 0x5410);
   o1 = __byte_perm(uc, ud, 0x5410);
@@ -256,31 +259,31 @@ __device__ __forceinline__ void int4x8_to_half(uint32_t w, __half2 s2, bool scal
 }
 // Four int8 codes (one 32-bit word) -> two half2 words: each byte (offset
 // binary) placed under an 0x64 high byte, minus 1024 + 128.
-__device__ __forceinline__ void int8x4_to_half(uint32_t w, __half2 s2, bool scaled, uint32_t& o0,
-                                               uint32_t& o1) {
+__device__ __forceinline__ void int8x4_to_half(uint32_t w, __half2 s2, uint32_t& o0, uint32_t& o1) {
   const uint32_t x = w ^ 0x80808080u;
   const __half2 bias = u2h(0x64806480u);   // 1152
   __half2 lo = __hsub2(u2h(__byte_perm(x, 0x64646464u, 0x5140)), bias);
   __half2 hi = __hsub2(u2h(__byte_perm(x, 0x64646464u, 0x5342)), bias);
-  if (scaled) { lo = __hmul2(lo, s2); hi = __hmul2(hi, s2); }
+  lo = __hmul2(lo, s2);
+  hi = __hmul2(hi, s2);
   o0 = h2u(lo);
   o1 = h2u(hi);
 }
 // One 16-byte vector of codes -> QB == 4: 32 channels (four 16-byte fp16
-// chunks), QB == 8: 16 channels (two chunks); optionally times a scale
+// chunks), QB == 8: 16 channels (two chunks), each times the group scale s2
 // (one fp16 rounding of the exact product).
 template <int QB>
-__device__ __forceinline__ void codes_to_half(const uint4& v, bool scaled, __half2 s2, uint4 (&out)[QB == 4 ? 4 : 2]) {
+__device__ __forceinline__ void codes_to_half(const uint4& v, __half2 s2, uint4 (&out)[QB == 4 ? 4 : 2]) {
   if (QB == 4) {
-    int4x8_to_half(v.x, s2, scaled, out[0].x, out[0].y, out[0].z, out[0].w);
-    int4x8_to_half(v.y, s2, scaled, out[1].x, out[1].y, out[1].z, out[1].w);
-    int4x8_to_half(v.z, s2, scaled, out[2].x, out[2].y, out[2].z, out[2].w);
-    int4x8_to_half(v.w, s2, scaled, out[3].x, out[3].y, out[3].z, out[3].w);
+    int4x8_to_half(v.x, s2, out[0].x, out[0].y, out[0].z, out[0].w);
+    int4x8_to_half(v.y, s2, out[1].x, out[1].y, out[1].z, out[1].w);
+    int4x8_to_half(v.z, s2, out[2].x, out[2].y, out[2].z, out[2].w);
+    int4x8_to_half(v.w, s2, out[3].x, out[3].y, out[3].z, out[3].w);
   } else {
-    int8x4_to_half(v.x, s2, scaled, out[0].x, out[0].y);
-    int8x4_to_half(v.y, s2, scaled, out[0].z, out[0].w);
-    int8x4_to_half(v.z, s2, scaled, out[1].x, out[1].y);
-    int8x4_to_half(v.w, s2, scaled, out[1].z, out[1].w);
+    int8x4_to_half(v.x, s2, out[0].x, out[0].y);
+    int8x4_to_half(v.y, s2, out[0].z, out[0].w);
+    int8x4_to_half(v.z, s2, out[1].x, out[1].y);
+    int8x4_to_half(v.w, s2, out[1].z, out[1].w);
   }
 }
 
@@ -334,7 +337,7 @@ __device__ __forceinline__ void convert_z_inplace(uint32_t d, uint32_t sct, int 
     for (int i = 0; i < NV; ++i) {
       const int v = lane + 32 * i, tt = 32 * ph + v / VPR, q = v % VPR;
       uint4 out[CPV];
-      codes_to_half<QB>(rv[i], true, __halves2half2(sc[i], sc[i]), out);
+      codes_to_half<QB>(rv[i], __halves2half2(sc[i], sc[i]), out);
       const int ch = q * (CPV * 8);         // first channel of the vector within the 128
       const int box = ch >> 6, c0 = (ch & 63) >> 3;
 #pragma unroll
