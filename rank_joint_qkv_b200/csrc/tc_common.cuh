@@ -226,6 +226,21 @@ __device__ __forceinline__ int group_or(int pred, int id) {
   return r;
 }
 __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+// OR-reduction of a predicate / plain barrier over n threads (a multiple of
+// 32) on named barrier `id`.
+__device__ __forceinline__ int bar_or(int pred, int id, int n) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(id), "r"(n)
+      : "memory");
+  return r;
+}
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.

@@ -50,34 +50,47 @@ k_wsvd_rope_query(const float* __restrict__ q, const int32_t* __restrict__ lengt
   }
 }
 
-// grid (ceil(max_len / 128), B), block 160.  R: per-head rank (64 or 128);
-// d_h = 128.  One CTA walks every head of its 128 positions: warp 4's
-// first thread loads (TMA: the head's latent tile and B_{Kh}, two stages)
-// and issues the MMAs into one of two TMEM buffers; warps 0-3 (TMEM lanes
-// 32 w .., one token each) rotate and score, with the positions' cos/sin rows
-// staged once in shared memory for all heads.  TMA maps: latent rows
+// grid (ceil(max_len / 128), B), block kWrThreads.  R: per-head rank (64 or
+// 128); d_h = 128.  One CTA walks every head of its 128 positions: warp 4 kWrG's
+// first thread loads (TMA: the head's latent tile and B_{Kh}, a ring of
+// wr_stages<R>() stages, so that several heads' tiles are in flight) and
+// issues the MMAs into one of two TMEM buffers; kWrG groups of four warps
+// (TMEM lanes 32 (w % 4) .., one token each) rotate and score, group g over
+// its share of the 64 rotation pairs, their partial dots summed through
+// shared memory; the positions' cos/sin rows are staged once in shared
+// memory for all heads.  TMA maps: latent rows
 // (head-major: 2D {r, rows}; token-major: 3D {r, H, B max_len} with a box one
 // head high), B_K as 2D {d_h, H r}.
 constexpr int kWrTab = 130;   // floats per staged table row (pitch: 2-way bank conflicts at most)
+// Load stages: as many as fit beside the staged table (32 KB stages at r 64,
+// 64 KB at r 128); a stage's loads wait in flight for about one load latency.
+template <int R>
+__host__ __device__ constexpr int wr_stages() { return R == 64 ? 4 : 2; }
+// Scoring groups of four warps (one token per thread), each over 64 / kWrG
+// of the rotation pairs; warp 4 kWrG issues the loads and MMAs.
+constexpr int kWrG = 4;
+constexpr int kWrThreads = 128 * kWrG + 32;
 template <bool BF16, int R>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kWrThreads, 1)
 k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
                    const float* __restrict__ qr, const float* __restrict__ tab,
                    const int32_t* __restrict__ lengths, float* __restrict__ scores,
                    int32_t* __restrict__ status, int H, int max_len, int token_major) {
-  constexpr int D = 128, NB = R / 64;
+  constexpr int D = 128, NB = R / 64, NST = wr_stages<R>();
   constexpr int CBYTES = 128 * R * 2, BBYTES = R * D * 2, STAGE = CBYTES + BBYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* tabs = reinterpret_cast<float*>(base + 2 * STAGE);            // [128][kWrTab]
+  float* tabs = reinterpret_cast<float*>(base + NST * STAGE);          // [128][kWrTab]
   uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 128 * kWrTab);
-  uint64_t* full = bars;        // [2] stage loaded
-  uint64_t* empty = bars + 2;   // [2] stage's MMAs done
-  uint64_t* done = bars + 4;    // [2] TMEM buffer holds a head's keys
-  uint64_t* tfree = bars + 6;   // [2] TMEM buffer read by the epilogue
-  uint64_t* drain = bars + 8;   // the MMA thread's last commit
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* full = bars;                // [NST] stage loaded
+  uint64_t* empty = bars + NST;         // [NST] stage's MMAs done
+  uint64_t* done = bars + 2 * NST;      // [2] TMEM buffer holds a head's keys
+  uint64_t* tfree = done + 2;           // [2] TMEM buffer read by the epilogue
+  uint64_t* drain = tfree + 2;          // the MMA thread's last commit
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ float ps[kWrG - 1][2][128];   // the other groups' partial dots, by TMEM buffer
+  constexpr int MW = 4 * kWrG;             // the loading / MMA warp
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
@@ -86,9 +99,11 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
   if (t0 >= len) return;   // uniform across the CTA, before any barrier or TMEM use
   const uint32_t s0 = saddr(base);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(saddr(&full[i]), 1);
       mbar_init(saddr(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(saddr(&done[i]), 1);
       mbar_init(saddr(&tfree[i]), 1);
     }
@@ -96,13 +111,13 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == MW) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
                      saddr(tmem_holder))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     tc_fence_before();
-  } else {
+  } else if (warp < 4) {
     // this token's cos/sin row (64 pairs), staged once for every head
     const int p = t0 + threadIdx.x;
     const float4* src = reinterpret_cast<const float4*>(tab + size_t(p < max_len ? p : 0) * D);
@@ -117,14 +132,14 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == MW) {
     if (lane == 0) {
       constexpr uint32_t id = idesc_f16(128, D, BF16, false, true);   // B MN-major
       bool ok = true;
       int issued = 0;
       auto load = [&](int h) -> bool {
-        const int st = h & 1;
-        if (!mbar_wait(saddr(&empty[st]), (uint32_t(h >> 1) & 1u) ^ 1u)) return false;
+        const int st = h % NST;
+        if (!mbar_wait(saddr(&empty[st]), (uint32_t(h / NST) & 1u) ^ 1u)) return false;
         const uint32_t dst = s0 + uint32_t(st * STAGE), fb = saddr(&full[st]);
         mbar_expect_tx(fb, uint32_t(STAGE));
 #pragma unroll
@@ -139,21 +154,21 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         ++issued;
         return true;
       };
-      ok = load(0);
+      for (int x = 0; x < NST - 1 && x < H && ok; ++x) ok = load(x);   // NST - 1 heads ahead
       for (int h = 0; h < H && ok; ++h) {
-        if (h + 1 < H && !load(h + 1)) { ok = false; break; }
-        const int st = h & 1;
-        if (!mbar_wait(saddr(&full[st]), uint32_t(h >> 1) & 1u)) { ok = false; break; }
-        if (h >= 2 && !mbar_wait(saddr(&tfree[st]), uint32_t((h - 2) >> 1) & 1u)) { ok = false; break; }
+        if (h + NST - 1 < H && !load(h + NST - 1)) { ok = false; break; }
+        const int st = h % NST, tb = h & 1;   // load stage, TMEM buffer
+        if (!mbar_wait(saddr(&full[st]), uint32_t(h / NST) & 1u)) { ok = false; break; }
+        if (h >= 2 && !mbar_wait(saddr(&tfree[tb]), uint32_t((h - 2) >> 1) & 1u)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sb = s0 + uint32_t(st * STAGE);
 #pragma unroll
         for (int kk = 0; kk < R / 16; ++kk) {   // K = 16 latent channels per MMA
           const uint64_t a = sdesc(sb + uint32_t((kk >> 2) * 128 * 128 + (kk & 3) * 32), 16, 1024);
           const uint64_t bd = sdesc(sb + CBYTES + uint32_t(kk * 16 * 128), R * 128, 1024);
-          tc_mma(tmem + uint32_t(st * D), a, bd, id, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + uint32_t(tb * D), a, bd, id, kk > 0 ? 1u : 0u);
         }
-        tc_commit(saddr(&done[st]));
+        tc_commit(saddr(&done[tb]));
         tc_commit(saddr(&empty[st]));
         if (*abort_flag) ok = false;
       }
@@ -161,21 +176,23 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         *abort_flag = 1;
         atomicOr(status, QSVD_STATUS_TIMEOUT);
         // every copy issued has landed before the CTA may leave
-        for (int h = issued > 2 ? issued - 2 : 0; h < issued; ++h)
-          mbar_wait(saddr(&full[h & 1]), uint32_t(h >> 1) & 1u);
+        for (int h = issued > NST ? issued - NST : 0; h < issued; ++h)
+          mbar_wait(saddr(&full[h % NST]), uint32_t(h / NST) & 1u);
       }
       tc_commit(saddr(drain));   // every MMA issued has completed before TMEM is freed
       mbar_wait(saddr(drain), 0);
     }
     __syncwarp();
   } else {
-    const int t = threadIdx.x, p = t0 + t;
-    const uint32_t lane_off = uint32_t(32 * warp) << 16;
+    const int g = warp >> 2, t = threadIdx.x & 127, p = t0 + t;   // pair half, token
+    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const float* trow = tabs + t * kWrTab;
     for (int h = 0; h < H; ++h) {
       const int st = h & 1;
-      if (group_or(!mbar_wait(saddr(&done[st]), uint32_t(h >> 1) & 1u))) {
-        if (t == 0) { *abort_flag = 1; atomicOr(status, QSVD_STATUS_TIMEOUT); }
+      // every group takes the same decision (one barrier over all their
+      // threads), which also covers an abort flagged during the last head
+      if (bar_or(*abort_flag || !mbar_wait(saddr(&done[st]), uint32_t(h >> 1) & 1u), 1 + kWrG, 128 * kWrG)) {
+        if (threadIdx.x == 0) { *abort_flag = 1; atomicOr(status, QSVD_STATUS_TIMEOUT); }
         break;
       }
       tc_fence_after();
@@ -183,7 +200,7 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
       const uint32_t ta = tmem + lane_off + uint32_t(st * D);
       float s = 0.f;
 #pragma unroll 1
-      for (int i0 = 0; i0 < 64; i0 += 16) {
+      for (int i0 = (64 / kWrG) * g; i0 < (64 / kWrG) * (g + 1); i0 += 16) {
         float klo[16], khi[16];
         tmem_ld16(ta + uint32_t(i0), klo);
         tmem_ld16(ta + uint32_t(64 + i0), khi);
@@ -197,15 +214,19 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         }
       }
       tc_fence_before();
-      group_sync();
-      if (t == 0) mbar_arrive(saddr(&tfree[st]));
-      if (p < len) scores[(size_t(b) * H + h) * max_len + p] = s;
-      if (group_or(*abort_flag)) break;
+      if (g > 0) ps[g - 1][st][t] = s;
+      bar_sync(1 + kWrG, 128 * kWrG);   // every group's TMEM reads and partial dots are done
+      if (threadIdx.x == 0) mbar_arrive(saddr(&tfree[st]));
+      if (g == 0 && p < len) {
+#pragma unroll
+        for (int o = 0; o < kWrG - 1; ++o) s += ps[o][st][t];
+        scores[(size_t(b) * H + h) * max_len + p] = s;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == MW) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
   }
@@ -250,11 +271,11 @@ cudaError_t scores_t(const qsvd_dims& d, const void* bk, const void* ck, const f
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int smem = 1024 + 2 * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128;
+  const int smem = 1024 + wr_stages<R>() * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128;
   auto kern = k_wsvd_rope_scores<BF16, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((d.max_len + 127) / 128, d.batch), 160, smem, s>>>(tc, tb, qr, tab, lengths, scores, status,
+  kern<<<dim3((d.max_len + 127) / 128, d.batch), kWrThreads, smem, s>>>(tc, tb, qr, tab, lengths, scores, status,
                                                                d.H, d.max_len, token_major);
   note_launch();
   return check_launch();
