@@ -909,7 +909,14 @@ def main():
                     help="time qsvd_prefill_attention over the workload's prompts (all B x L tokens)")
     ap.add_argument("--eager", action="store_true",
                     help="time the API calls as issued instead of a CUDA-graph replay of one step")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="prefill-attention and per-head modes only: this many sequences instead of "
+                         "the workload's own B (a smaller case, e.g. for a profiler capture)")
     args = ap.parse_args()
+    if args.batch:
+        if not (args.prefill_attn or args.per_head_rank):
+            ap.error("--batch applies to --prefill-attn and --per-head-rank only")
+        synthetic.CONFIGS[args.config] = synthetic.replace(synthetic.CONFIGS[args.config], B=args.batch)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
 

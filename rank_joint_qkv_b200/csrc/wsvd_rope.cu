@@ -89,6 +89,7 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
   uint64_t* tfree = done + 2;           // [2] TMEM buffer read by the epilogue
   uint64_t* drain = tfree + 2;          // the MMA thread's last commit
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  float* qsm = tabs + 128 * kWrTab + 32;   // [H][128] the rotated queries (after 128 bytes of barriers)
   __shared__ float ps[kWrG - 1][2][128];   // the other groups' partial dots, by TMEM buffer
   constexpr int MW = 4 * kWrG;             // the loading / MMA warp
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -117,16 +118,21 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     tc_fence_before();
-  } else if (warp < 4) {
-    // this token's cos/sin row (64 pairs), staged once for every head
-    const int p = t0 + threadIdx.x;
-    const float4* src = reinterpret_cast<const float4*>(tab + size_t(p < max_len ? p : 0) * D);
-    float* dst = tabs + threadIdx.x * kWrTab;
+  } else {
+    if (warp < 4) {
+      // this token's cos/sin row (64 pairs), staged once for every head
+      const int p = t0 + threadIdx.x;
+      const float4* src = reinterpret_cast<const float4*>(tab + size_t(p < max_len ? p : 0) * D);
+      float* dst = tabs + threadIdx.x * kWrTab;
 #pragma unroll 8
-    for (int v = 0; v < D / 4; ++v) {
-      const float4 x = __ldg(src + v);
-      dst[4 * v] = x.x; dst[4 * v + 1] = x.y; dst[4 * v + 2] = x.z; dst[4 * v + 3] = x.w;
+      for (int v = 0; v < D / 4; ++v) {
+        const float4 x = __ldg(src + v);
+        dst[4 * v] = x.x; dst[4 * v + 1] = x.y; dst[4 * v + 2] = x.z; dst[4 * v + 3] = x.w;
+      }
     }
+    // every head's rotated query of this sequence, read by all scoring threads
+    const float* qb = qr + size_t(b) * H * D;
+    for (int i = threadIdx.x; i < H * D; i += 128 * kWrG) qsm[i] = __ldg(qb + i);
   }
   __syncthreads();
   tc_fence_after();
@@ -196,7 +202,7 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         break;
       }
       tc_fence_after();
-      const float* qh = qr + (size_t(b) * H + h) * D;
+      const float* qh = qsm + h * D;
       const uint32_t ta = tmem + lane_off + uint32_t(st * D);
       float s = 0.f;
 #pragma unroll 1
@@ -209,8 +215,8 @@ k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         for (int e = 0; e < 16; ++e) {
           const int j = i0 + e;
           const float c = trow[2 * j], sn = trow[2 * j + 1];
-          s = fmaf(__ldg(qh + j), fmaf(klo[e], c, -khi[e] * sn), s);
-          s = fmaf(__ldg(qh + 64 + j), fmaf(khi[e], c, klo[e] * sn), s);
+          s = fmaf(qh[j], fmaf(klo[e], c, -khi[e] * sn), s);
+          s = fmaf(qh[64 + j], fmaf(khi[e], c, klo[e] * sn), s);
         }
       }
       tc_fence_before();
@@ -271,7 +277,7 @@ cudaError_t scores_t(const qsvd_dims& d, const void* bk, const void* ck, const f
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int smem = 1024 + wr_stages<R>() * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128;
+  const int smem = 1024 + wr_stages<R>() * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128 + d.H * 128 * 4;
   auto kern = k_wsvd_rope_scores<BF16, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -295,7 +301,8 @@ cudaError_t scores_r(const qsvd_dims& d, const void* bk, const void* ck, const f
 
 bool wsvd_rope_supported(const qsvd_dims& d) {
   return d.d_h == 128 && (d.cache_dtype == QSVD_F16 || d.cache_dtype == QSVD_BF16) &&
-         d.weight_dtype == d.cache_dtype && (d.r == 64 || d.r == 128);   // a head's key rank is <= d_h
+         d.weight_dtype == d.cache_dtype && (d.r == 64 || d.r == 128) &&   // a head's key rank is <= d_h
+         d.H <= 64;   // every head's rotated query is staged in shared memory
 }
 
 cudaError_t launch_wsvd_rope_front(const qsvd_dims& d, const void* bk, const float* q, const void* ck,

@@ -50,6 +50,7 @@ def test_workspace_size_matches_layout(shape):
 @pytest.mark.parametrize("bad,status", [(dict(rope=True, r=96), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(rope=True, cache="f32"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(rope=True, cache="bf16"), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(rope=True, E=72 * 128, H=72), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(cache="i4", r=128), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(out_proj="chain"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(out_proj="fold", weight="f32"), q.QSVD_ERR_UNSUPPORTED),
