@@ -411,9 +411,9 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
       e = launch_rope_query(d, qsrc, sched, rope_tab, sl2, qt32, s);
     else
       // only the copy the split kernel reads: fp32 for CUDA cores, 16-bit hi/lo
-      // for tensor cores; a quantised latent on the tensor cores takes int8
-      // parts (in the 16-bit parts' section) with their scales and offset
-      // terms (in the fp32 section, unused on that path)
+      // for tensor cores; a quantised latent on the tensor cores takes the
+      // absorbed query as three int8 parts and one scale per (sequence, head),
+      // both written into the 16-bit parts' section from the fp32 copy
       if (kernel != QSVD_KERNEL_SIMT && cache_is_int(d)) {
         e = launch_absorb(d, qsrc, P + L.wuk, sl2, qt32, nullptr, &hdr->status, s);
         if (e == cudaSuccess)

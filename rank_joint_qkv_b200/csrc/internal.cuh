@@ -242,6 +242,9 @@ bool split_cl_supported(const qsvd_dims& d);
 int split_cl_clusters(const qsvd_dims& d);
 cudaError_t launch_split_cl(const qsvd_dims& d, const void* cache, const void* qt16, const int32_t* sched,
                             int G, float* pm, float* pl, float* pz, int32_t* status, cudaStream_t s);
+// Absorbed mode, one CTA per split (tcgen05).  qt16: the query as 16-bit
+// hi/lo parts, or for an int8/int4 latent its int8 parts (launch_quant_query)
+// with qsh their per-(sequence, head) scales.
 cudaError_t launch_split_tc(const qsvd_dims& d, const void* cache, const void* scales, const void* qt16,
                             const int32_t* sched, int G, float* pm, float* pl, float* pz,
                             int32_t* status, cudaStream_t s, const float* qsh = nullptr);
