@@ -1417,10 +1417,11 @@ k_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ 
 
 constexpr int kSmemLimit = 232448;   // opt-in dynamic shared memory per block on sm_100
 
-// Slots per ring.  About 96 KB in flight per ring measured best on the
-// LLaVA-7B-shaped layer (fp16 latent, r = 1536, 32 heads): 4 S slots and 6 Z
-// slots took 115.7 us, 5 + 5 118.8 us, 4 + 7 118.8 us, 3 + 7 117.8 us --
-// beyond that, more bytes in flight only lengthen every load's latency.
+// Slots per ring.  The S ring holds about 96 KB, the Z ring the rest of the
+// shared memory.  On the LLaVA-7B-shaped layer (fp16 latent, r = 1536, 32
+// heads) 4 S + 7 Z slots took 102.7 us, 4 + 6 104.5, 3 + 8 105.0, 3 + 7
+// 105.7, 5 + 5 111.1, 5 + 4 125.5, 6 + 4 128.8: the Z stream (re-reads from
+// L2) is the more sensitive of the two.
 constexpr int kRingTargetBytes = 96 * 1024;
 template <int NP, int QS, int PS>
 void ring_slots(int* ns, int* nz) {
@@ -1428,8 +1429,7 @@ void ring_slots(int* ns, int* nz) {
   const int sb = s_slot_bytes<NP, QS>();
   int s = kRingTargetBytes / sb;
   if (s > kMaxSlots) s = kMaxSlots;
-  int zbytes = avail - s * sb;
-  if (zbytes > kRingTargetBytes) zbytes = kRingTargetBytes;
+  const int zbytes = avail - s * sb;
   int z = zbytes / kZSlotBytes;
   if (z > kMaxSlots) z = kMaxSlots;
   *ns = s;
