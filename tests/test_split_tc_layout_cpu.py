@@ -112,7 +112,7 @@ def test_quantised_shared_memory_budget(np_, r):
         raw_s = 128 * 64 if qb == 4 else 0
         tables = 3 * 256 * (r // 128)
         avail = k_smem - 1024 - misc - 2 * pbuf - tables - nraw * raw_s
-        for ns in (3, 2):
+        for ns in ((2,) if qb == 4 else (3, 2)):
             nz = (avail - ns * sq) // Z_SLOT
             if nz >= 5:
                 break
