@@ -45,12 +45,17 @@ def case(key):
             "i8": synthetic.replace(synthetic.SHRUNK[3], cache="i8", name="shrunk-int8-h2"),
             "i4h32": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=768, B=2, L=600,
                                        h2_n=256),
-            # r 256: four items per tile, three raw slots per stream (one per converter)
+            # r 256: two channel groups, four Z items per tile
             "i4r256": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0),
             "i8r256": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0, cache="i8",
                                         name="shrunk-int8-r256"),
             "i4r256rag": synthetic.replace(synthetic.SHRUNK[3], r=256, h2_n=0, h2_m=0, B=4, L=700,
                                            ragged=(1, 700)),
+            # r 1536 at 32 heads: twelve Z chunks leave TMEM for one S group buffer
+            "i8r1536": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=1536, B=2, L=300,
+                                         h2_n=0, h2_m=0, cache="i8", name="shrunk-int8-r1536"),
+            "i4r1536": synthetic.replace(synthetic.SHRUNK[3], E=4096, H=32, r=1536, B=2, L=300,
+                                         h2_n=0, h2_m=0, name="shrunk-int4-r1536"),
             # cluster shapes: 6 CTAs of 256 channels (the LLaVA-7B rank), 8 of 256
             "c6": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=300),
             "c6bf": synthetic.replace(base, E=4096, H=32, r=1536, B=2, L=290, cache="bf16",
@@ -74,7 +79,8 @@ _KEYS16 = ["full", "f16", "bf16", "h32", "r768", "c6", "c6bf", "c8"]
 
 
 @pytest.mark.parametrize("key,kern", [(k, v) for k in _KEYS16 for v in BOTH] +
-                         [(k, CTA) for k in ("i4", "i8", "i4h32", "i4r256", "i8r256", "i4r256rag")])
+                         [(k, CTA) for k in ("i4", "i8", "i4h32", "i4r256", "i8r256", "i4r256rag",
+                                             "i8r1536", "i4r1536")])
 def test_tc_matches_oracle(cuda_ok, key, kern):
     c = case(key)
     g = GpuCase(c, kernel=kern)
