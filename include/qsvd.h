@@ -406,7 +406,7 @@ qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
  * Computed in float32 on CUDA cores, 256 tokens per split CTA, chunks merged
  * in the log2 domain; 16-bit latents with r = 64, 128 or 256 are read as
  * 16-byte vectors.  With dims->rope (rotary mode; d_h == 128, r = 64 or
- * 128, H <= 64, an F16 or BF16 cache of the weight type): keys are rebuilt per
+ * 128, H <= 59, an F16 or BF16 cache of the weight type): keys are rebuilt per
  * 128-token tile on the tensor cores, K_h = C_{Kh} B_{Kh}, rotated to their
  * positions and dotted with the query rotated to len_b - 1 (base
  * dims->rope_base; the cos/sin table of every position, from float64 angles,

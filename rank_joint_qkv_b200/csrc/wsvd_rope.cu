@@ -70,6 +70,16 @@ __host__ __device__ constexpr int wr_stages() { return R == 64 ? 4 : 2; }
 // of the rotation pairs; warp 4 kWrG issues the loads and MMAs.
 constexpr int kWrG = 4;
 constexpr int kWrThreads = 128 * kWrG + 32;
+// Shared memory of one CTA: the dynamic part (1024 bytes of alignment slack,
+// the load stages, the cos/sin rows, 128 bytes of barriers, every head's
+// rotated query) plus the static partial dots; the sum must not exceed the
+// per-block opt-in limit.
+constexpr int kWrStaticBytes = (kWrG - 1) * 2 * 128 * 4;
+inline int wr_dynamic_smem(int r, int H) {
+  const int stages = r == 64 ? wr_stages<64>() : wr_stages<128>();
+  return 1024 + stages * (128 * r * 2 + r * 128 * 2) + 128 * kWrTab * 4 + 128 + H * 128 * 4;
+}
+constexpr int kWrSmemLimit = 232448;   // opt-in shared memory per block on sm_100
 template <bool BF16, int R>
 __global__ void __launch_bounds__(kWrThreads, 1)
 k_wsvd_rope_scores(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
@@ -277,7 +287,7 @@ cudaError_t scores_t(const qsvd_dims& d, const void* bk, const void* ck, const f
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int smem = 1024 + wr_stages<R>() * (128 * R * 2 + R * 128 * 2) + 128 * kWrTab * 4 + 128 + d.H * 128 * 4;
+  const int smem = wr_dynamic_smem(R, d.H);
   auto kern = k_wsvd_rope_scores<BF16, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -302,7 +312,8 @@ cudaError_t scores_r(const qsvd_dims& d, const void* bk, const void* ck, const f
 bool wsvd_rope_supported(const qsvd_dims& d) {
   return d.d_h == 128 && (d.cache_dtype == QSVD_F16 || d.cache_dtype == QSVD_BF16) &&
          d.weight_dtype == d.cache_dtype && (d.r == 64 || d.r == 128) &&   // a head's key rank is <= d_h
-         d.H <= 64;   // every head's rotated query is staged in shared memory
+         // every head's rotated query is staged in shared memory: H <= 59
+         wr_dynamic_smem(d.r, d.H) + kWrStaticBytes <= kWrSmemLimit;
 }
 
 cudaError_t launch_wsvd_rope_front(const qsvd_dims& d, const void* bk, const float* q, const void* ck,

@@ -50,7 +50,7 @@ def test_workspace_size_matches_layout(shape):
 @pytest.mark.parametrize("bad,status", [(dict(rope=True, r=96), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(rope=True, cache="f32"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(rope=True, cache="bf16"), q.QSVD_ERR_UNSUPPORTED),
-                                        (dict(rope=True, E=72 * 128, H=72), q.QSVD_ERR_UNSUPPORTED),
+                                        (dict(rope=True, E=60 * 128, H=60), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(cache="i4", r=128), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(out_proj="chain"), q.QSVD_ERR_UNSUPPORTED),
                                         (dict(out_proj="fold", weight="f32"), q.QSVD_ERR_UNSUPPORTED),
@@ -212,3 +212,30 @@ def test_vector_split_index_replay(B, H, r, max_len, lengths, token_major):
         else:
             want[b, :, :ln] = 1
     assert np.array_equal(hits, want.reshape(-1))    # every valid element once, nothing else
+
+
+@pytest.mark.parametrize("r", [64, 128])
+@pytest.mark.parametrize("H", [1, 32, 40, 59])
+def test_rotary_scores_shared_memory_map(r, H):
+    """k_wsvd_rope_scores' shared memory (wsvd_rope.cu), restated: the load
+    stages, the staged cos/sin rows (128 x 130 floats), 128 bytes of
+    barriers (full / empty per stage, done / tfree per TMEM buffer, drain,
+    the TMEM address, the abort flag) and every head's rotated query
+    (H x 128 floats): disjoint and aligned inside the launch's dynamic size
+    (whose base is aligned up by at most 1023 bytes), and with the static
+    partial dots (3 x 2 x 128 floats) within the 227 KB per block."""
+    nst = 4 if r == 64 else 2
+    stage = 128 * r * 2 + r * 128 * 2
+    tab = nst * stage                       # offsets from the 1024-aligned base
+    bars = tab + 128 * 130 * 4
+    nbar = 2 * nst + 5
+    holder = bars + 8 * nbar
+    abort = holder + 4
+    qsm = bars + 128
+    assert stage % 1024 == 0 and tab % 1024 == 0          # swizzled TMA boxes
+    assert bars % 8 == 0 and abort + 4 <= qsm             # barriers inside their 128 bytes
+    assert qsm % 16 == 0
+    end = qsm + H * 128 * 4
+    dynamic = 1024 + nst * stage + 128 * 130 * 4 + 128 + H * 128 * 4   # the launch's size
+    assert end + 1023 <= dynamic
+    assert dynamic + 3 * 2 * 128 * 4 <= 232448
