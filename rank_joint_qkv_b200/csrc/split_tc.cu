@@ -185,7 +185,7 @@ __device__ Smem carve(uint8_t* base, int ns, int nz, int nraw, int r) {
   s.zraw_full = s.sraw_full + kMaxRaw;   // 4 kMaxSlots + 8 + 2 kMaxGroupBufs + kMaxRaw + kMaxSlots = 64
   s.never = s.zraw_full + kMaxSlots;     // the 65th
   s.zsc_full = s.never + 1;
-  s.zsc_empty = s.zsc_full + kScaleBufs;  // 69 barriers (the barrier area holds 80)
+  s.zsc_empty = s.zsc_full + kScaleBufs;  // 65 + 2 kScaleBufs = 71 barriers (the barrier area holds 80)
   static_assert(640 + 4 * NP * 4 + 32 + (QB ? 4 : 3) * NP * 4 <= kMiscBytes, "misc region");
   s.red = reinterpret_cast<float*>(m + 640);
   s.tmem_holder = reinterpret_cast<uint32_t*>(m + 640 + 4 * NP * 4);

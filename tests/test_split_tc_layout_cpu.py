@@ -120,3 +120,46 @@ def test_quantised_shared_memory_budget(np_, r):
         assert nz >= 4
         smem = 1024 + ns * sq + nz * Z_SLOT + 2 * pbuf + nraw * raw_s + tables + misc
         assert smem <= k_smem
+
+
+@pytest.mark.parametrize("np_,ps,qb,r", [(32, 1, 0, 1536), (16, 1, 0, 512), (32, 2, 0, 1536), (16, 2, 0, 384),
+                                          (32, 1, 8, 768), (32, 1, 4, 768), (16, 1, 8, 384),
+                                          (32, 1, 8, 1536), (32, 1, 4, 1664), (16, 1, 4, 3712)])
+def test_split_kernel_shared_memory_carve(np_, ps, qb, r):
+    """carve() and the launch's size (split_tc.cu), restated for the 16-bit
+    (qb 0) and quantised paths: slot rings and P buffers on 1024-byte
+    boundaries (128-byte-swizzled TMA boxes and MMA operands), the barrier
+    area (80 barriers, 71 used) and the misc region after them, the whole
+    within the launched size and 227 KB."""
+    k_smem, misc, max_slots, z_slot = 232448, 2048, 8, 16384
+    pbuf = 2 * np_ * 128
+    if qb == 0:
+        a_slot = 128 * 128 + 2 * np_ * 128               # latent box + hi/lo query box
+        avail = k_smem - 1024 - misc - 2 * ps * pbuf
+        ns = min(96 * 1024 // a_slot, max_slots)
+        nz = min((avail - ns * a_slot) // z_slot, max_slots)
+        nraw, raw_s, tables = 0, 0, 0
+    else:
+        a_slot = 128 * 128 + 3 * np_ * 128               # codes + int8 query parts
+        nraw, raw_s = (4, 128 * 64) if qb == 4 else (0, 0)
+        tables = 3 * 256 * (r // 128)
+        avail = k_smem - 1024 - misc - 2 * ps * pbuf - tables - nraw * raw_s
+        for ns in ((2,) if qb == 4 else (3, 2)):
+            nz = (avail - ns * a_slot) // z_slot
+            if nz >= 5:
+                break
+        nz = min(nz, max_slots)
+    zring = ns * a_slot
+    pb = zring + nz * z_slot
+    sraw = pb + 2 * ps * pbuf
+    zsc = sraw + nraw * raw_s
+    m = zsc + tables
+    assert a_slot % 1024 == 0 and zring % 1024 == 0 and pb % 1024 == 0
+    assert sraw % 1024 == 0 and zsc % 16 == 0 and m % 8 == 0
+    nbar = 4 * max_slots + 8 + 2 * 4 + 8 + max_slots + 1 + 2 * 3
+    assert nbar == 71 and nbar * 8 <= 640
+    misc_used = 640 + 4 * np_ * 4 + 32 + (4 if qb else 3) * np_ * 4
+    assert misc_used <= misc
+    size = 1024 + ns * a_slot + nz * z_slot + 2 * ps * pbuf + nraw * raw_s + tables + misc
+    assert m + misc_used + 1023 <= size <= k_smem
+    assert ns >= 2 and nz >= 4
