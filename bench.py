@@ -254,6 +254,24 @@ def profiled_traffic(kernel_name: str, workload: str, src_files):
     return float(e["dram_bytes_per_launch"])
 
 
+def agreed_regions(run_region, min_ms: float, world: int, device):
+    """run_region() (-> ms) back to back until min_ms have passed (at least
+    once).  With several ranks the decision is taken together after every
+    region (a MAX all-reduce of "wants more"), so every rank runs the same
+    number of regions and the barriers inside them stay paired."""
+    regions, spent = [], 0.0
+    while True:
+        regions.append(float(run_region()))
+        spent += regions[-1]
+        more = spent < min_ms
+        if world > 1:
+            t = torch.tensor([1.0 if more else 0.0], device=device)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            more = t.item() > 0.0
+        if not more:
+            return regions
+
+
 def max_over_ranks(x: float, device, world: int) -> float:
     """Max of a per-rank scalar over the process group (no-op for one rank)."""
     if world <= 1:
@@ -382,10 +400,10 @@ class DecodeStep:
     def timed_regions(self, steps, world, min_seconds):
         """Regions of exactly `steps` steps, each bracketed by a barrier and a
         synchronize, repeated back to back until `min_seconds` have passed
-        (at least one): per-region milliseconds."""
+        (at least one; every rank runs the same number): per-region ms."""
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        regions, spent = [], 0.0
-        while not regions or spent < min_seconds * 1e3:
+
+        def region():
             torch.cuda.synchronize()
             if world > 1:
                 torch.distributed.barrier()
@@ -396,14 +414,9 @@ class DecodeStep:
             torch.cuda.synchronize()
             if world > 1:
                 torch.distributed.barrier()
-            regions.append(t0.elapsed_time(t1))
-            spent += regions[-1]
-            if world > 1:   # every rank runs the same number of regions
-                more = torch.tensor([1.0 if spent < min_seconds * 1e3 else 0.0], device=self.device)
-                torch.distributed.all_reduce(more, op=torch.distributed.ReduceOp.MAX)
-                if more.item() == 0.0:
-                    break
-        return regions
+            return t0.elapsed_time(t1)
+
+        return agreed_regions(region, min_seconds * 1e3, world, self.device)
 
     def flushed_steps(self, n, flush):
         """n steps, each preceded by a write of `flush` (a buffer larger than
