@@ -33,7 +33,10 @@
  *     Violations only visible on the device (a length or position out of
  *     range) are clamped and recorded as bits in a device status word; no
  *     kernel traps.
- *   - Pointers must be 16-byte aligned.
+ *   - Device pointers must be 16-byte aligned, except fp16 group scales
+ *     (2-byte) and the float32 c_out of an append (4-byte).  The calls
+ *     check the pointers they vectorise or hand to TMA and return
+ *     QSVD_ERR_INVALID_ARG for a misaligned one.
  */
 #ifndef QSVD_H
 #define QSVD_H
@@ -173,9 +176,11 @@ qsvd_status qsvd_prepare_weights(const qsvd_dims* dims, const void* wd,
  *             F32/F16/BF16: r elements;  I8: r int8 codes;
  *             I4: r/2 bytes, element 2j in the low nibble, 2j+1 in the high
  *             nibble (two's complement).
- *   scales  device, B x max_len x (r/group) float16 (I8/I4 only; else NULL).
- *   c_out   device, B x r float32, or NULL: receives c = x W^d (after H2
- *           when dims->h2 == 1), i.e. the exact input of the quantiser.
+ *   scales  device, B x max_len x (r/group) float16, 2-byte aligned (I8/I4
+ *           only; else NULL).
+ *   c_out   device, B x r float32 (4-byte aligned), or NULL: receives
+ *           c = x W^d (after H2 when dims->h2 == 1), i.e. the exact input
+ *           of the quantiser.
  *   status  device int32 word or NULL; bits QSVD_STATUS_* are OR-ed in.
  *   workspace        device scratch (split-K partials of x W^d), or NULL to
  *                    query the size into *workspace_bytes (in: capacity).

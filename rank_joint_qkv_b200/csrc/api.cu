@@ -45,6 +45,10 @@ static qsvd_status cuda_fail(cudaError_t e, const char* where) {
 static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// fp16 group scales are read and written two bytes at a time, fp32 outputs
+// four (the decode's fp32 output 16: it is stored as float4)
+static bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Host-checkable constraints shared by all calls.
 static qsvd_status validate(const qsvd_dims* d) {
@@ -265,6 +269,8 @@ qsvd_status qsvd_append_latent(const qsvd_dims* dims, const void* packed, const 
   if (cache_is_int(d) && !scales) return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
   if (!aligned16(x) || !aligned16(cache) || !aligned16(workspace))
     return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((scales && !aligned2(scales)) || (c_out && !aligned4(c_out)))
+    return fail(QSVD_ERR_INVALID_ARG, "scales must be 2-byte and c_out 4-byte aligned");
   const PackedLayout L = packed_layout(d);
   const uint8_t* P = static_cast<const uint8_t*>(packed);
   const float h2_scale = d.h2 ? float(1.0 / std::sqrt(double(d.r / d.h2_m))) : 1.f;
@@ -288,6 +294,7 @@ qsvd_status qsvd_prefill_latent(const qsvd_dims* dims, const void* packed, const
   if (n_rows == 0) return QSVD_OK;
   if (!packed || !x || !dst_rows || !cache) return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
   if (cache_is_int(d) && !scales) return fail(QSVD_ERR_INVALID_ARG, "int caches need scales");
+  if (scales && !aligned2(scales)) return fail(QSVD_ERR_INVALID_ARG, "scales must be 2-byte aligned");
   if (!aligned16(x) || !aligned16(cache) || (c_fp32_debug && !aligned16(c_fp32_debug)))
     return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   const PackedLayout L = packed_layout(d);
@@ -377,6 +384,8 @@ static qsvd_status decode_impl(const qsvd_dims& d, const void* packed, const flo
   if ((phases & QSVD_PHASE_COMBINE) && !out) return fail(QSVD_ERR_INVALID_ARG, "out is NULL");
   if (!aligned16(workspace) || (cache && !aligned16(cache)) || (qin && !aligned16(qin)))
     return fail(QSVD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((out && !aligned16(out)) || (scales && !aligned2(scales)))
+    return fail(QSVD_ERR_INVALID_ARG, "out must be 16-byte and scales 2-byte aligned");
 
   const PackedLayout L = packed_layout(d);
   const uint8_t* P = static_cast<const uint8_t*>(packed);
@@ -503,8 +512,8 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
     return fail(QSVD_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", *workspace_bytes, W.total);
   if (!bk || !bv || !q || !ck || !cv || !lengths || !out)
     return fail(QSVD_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!aligned16(workspace) || !aligned16(ck) || !aligned16(cv) || !aligned16(q))
-    return fail(QSVD_ERR_INVALID_ARG, "workspace, q, ck and cv must be 16-byte aligned");
+  if (!aligned16(workspace) || !aligned16(ck) || !aligned16(cv) || !aligned16(q) || !aligned16(out))
+    return fail(QSVD_ERR_INVALID_ARG, "workspace, q, ck, cv and out must be 16-byte aligned");
   cudaError_t e = launch_wsvd_decode(d, bk, bv, q, ck, cv, lengths, score_scale_log2(d), workspace, W, out,
                                      layout == QSVD_PER_HEAD_TOKEN_MAJOR, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_per_head");

@@ -76,6 +76,8 @@ extern "C" qsvd_status qsvd_append_latent_static(const qsvd_dims* dims, const vo
   // stores whole rows: the same alignment the workspace entry point demands.
   if (!aligned16(x) || !aligned16(cache))
     return set_error(QSVD_ERR_INVALID_ARG, "x and cache must be 16-byte aligned");
+  if ((scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) || (c_out && (reinterpret_cast<uintptr_t>(c_out) & 3u)))
+    return set_error(QSVD_ERR_INVALID_ARG, "scales must be 2-byte and c_out 4-byte aligned");
   if (cache_is_int(d) && !scales) return set_error(QSVD_ERR_INVALID_ARG, "int caches need scales");
   float* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess)

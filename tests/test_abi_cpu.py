@@ -254,3 +254,32 @@ def test_prefill_attention_host_checks():
         with pytest.raises(q.QsvdError) as e:
             q.prefill_attention_workspace_bytes(bad)
         assert e.value.status == q.QSVD_ERR_UNSUPPORTED
+
+
+def test_misaligned_outputs_and_scales_are_refused():
+    """The decode's fp32 output is stored as float4 and the fp16 group scales
+    two bytes at a time: pointers off those boundaries are refused on the
+    host, before anything is enqueued (the pointers are never dereferenced)."""
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in ("qsvd_decode_attn", "qsvd_append_latent", "qsvd_decode_attn_per_head",
+                 "qsvd_prefill_latent"):
+        getattr(lib, name).argtypes = q._sigs[name]
+    fake = ctypes.c_void_p(1 << 20)
+    odd, off8 = ctypes.c_void_p((1 << 20) + 1), ctypes.c_void_p((1 << 20) + 8)
+    n = ctypes.c_size_t(1 << 40)
+    st = lib.qsvd_decode_attn(ctypes.byref(_dims()), fake, fake, 1, fake, None, fake, 4, fake,
+                              ctypes.byref(n), off8, 0, None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"out must be 16-byte" in q._lib.qsvd_last_error()
+    st = lib.qsvd_decode_attn(ctypes.byref(_dims(cache="i8")), fake, fake, 1, fake, odd, fake, 4, fake,
+                              ctypes.byref(n), fake, 0, None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"scales 2-byte" in q._lib.qsvd_last_error()
+    st = lib.qsvd_append_latent(ctypes.byref(_dims(cache="i8")), fake, fake, fake, fake, odd, fake, None,
+                                fake, ctypes.byref(n), None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"scales must be 2-byte" in q._lib.qsvd_last_error()
+    d = _dims(cache="i8", weight="f16")
+    st = lib.qsvd_prefill_latent(ctypes.byref(d), fake, fake, 4, fake, fake, odd, None, None, None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"scales must be 2-byte" in q._lib.qsvd_last_error()
+    dh = q.make_dims(512, 4, 128, 64, 3, 700, cache="f16", weight="f16")
+    st = lib.qsvd_decode_attn_per_head(ctypes.byref(dh), fake, fake, fake, fake, fake, fake, 0, fake,
+                                       ctypes.byref(n), off8, None)
+    assert st == q.QSVD_ERR_INVALID_ARG and b"out must be 16-byte" in q._lib.qsvd_last_error()

@@ -103,3 +103,8 @@ def test_static_append_rejects_misaligned_pointers():
                                            None, None)
         assert st == q.QSVD_ERR_INVALID_ARG
         assert b"16-byte aligned" in q._lib.qsvd_last_error()
+    odd = ctypes.c_void_p((1 << 20) + 1)   # fp16 scales are stored two bytes at a time
+    d8 = q.make_dims(1024, 8, 128, 256, 4, 16, cache="i8", weight="f16")
+    st = lib.qsvd_append_latent_static(ctypes.byref(d8), good, good, good, good, odd, None, None, None)
+    assert st == q.QSVD_ERR_INVALID_ARG
+    assert b"scales must be 2-byte" in q._lib.qsvd_last_error()
