@@ -364,8 +364,9 @@ qsvd_status qsvd_prepare_out_proj(const qsvd_dims* dims, const void* wo, void* p
  *                  len == 0 gives a zero output row.  Values outside
  *                  [0, max_len] are clamped and flagged.
  *   num_splits     number of split CTAs G of the split phase (0: one wave on
- *                  this device).  Tiles of 128 tokens are dealt to the G
- *                  splits in equal contiguous runs over all sequences.
+ *                  this device), capped at B x ceil(max_len / 128) and at
+ *                  2048.  Tiles of 128 tokens are dealt to the G splits in
+ *                  equal contiguous runs over all sequences.
  *   workspace      device scratch, or NULL to query the size into
  *                  *workspace_bytes (in: capacity).  Layout (256-byte aligned
  *                  sections): header (int32 status, G, tile, kernel), query

@@ -138,8 +138,8 @@ static qsvd_status resolve_splits(const qsvd_dims& d, int num_splits, int kernel
     }
   }
   if (g > max_tiles) g = max_tiles;
+  if (g > kMaxSplits) g = kMaxSplits;
   if (g < 1) g = 1;
-  if (g > (1 << 20)) return fail(QSVD_ERR_INVALID_ARG, "num_splits too large");
   *G = int(g);
   return QSVD_OK;
 }

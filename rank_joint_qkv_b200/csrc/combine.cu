@@ -25,7 +25,7 @@ namespace {
 // tensor-core GEMV with head h's output columns reading row zm[b][h].
 
 constexpr int kMergeCh = 512;   // channels per merge CTA (128 threads x 4)
-constexpr int kMergeMaxSplits = 2048;   // weights kept in shared memory per (b, h)
+constexpr int kMergeMaxSplits = kMaxSplits;   // weights kept in shared memory per (b, h): c1 - c0 < G
 
 // grid (ceil(r / 512), H, B), block 128.
 __global__ void __launch_bounds__(128)
@@ -363,8 +363,8 @@ cudaError_t merge_vup_t(const qsvd_dims& d, const WsHeader* hdr, const int32_t* 
 }  // namespace
 
 bool combine_uses_gemv(const qsvd_dims& d) {
-  // a sequence of max_len tokens meets at most tiles + 1 splits: all their
-  // merge weights must fit the merge kernel's shared memory
+  // the merge's weights fit for any G (G <= kMaxSplits, capped by the host);
+  // the tile bound is the range of sequence lengths this path supports
   const long long tiles = (d.max_len + kTile - 1) / kTile;
   return (d.weight_dtype == QSVD_F16 || d.weight_dtype == QSVD_BF16) && d.d_h % 64 == 0 &&
          d.r % 32 == 0 && tiles + 1 <= kMergeMaxSplits;

@@ -18,6 +18,11 @@
 namespace qsvd {
 
 constexpr int kTile = QSVD_TILE_TOKENS;   // tokens per split-KV tile
+// Split CTAs per call at most.  A sequence's tiles fall into a contiguous run
+// of splits c0..c1; when G exceeds the tiles actually present, empty splits
+// lie between them, so the run can span up to G indices.  The merge keeps
+// one weight per index of the run in shared memory: the host caps G here.
+constexpr int kMaxSplits = 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- layouts

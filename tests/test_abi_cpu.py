@@ -101,6 +101,43 @@ def test_workspace_query_on_host():
     assert q.append_workspace_bytes(d) > 0
 
 
+def _split_begin(c, G, T):
+    return (c * T) // G
+
+
+def _split_of_tile(t, G, T):
+    return ((t + 1) * G - 1) // T
+
+
+def test_split_count_is_capped_where_a_sequence_could_span_more_merge_weights():
+    """Tiles of all sequences are dealt to G splits in equal contiguous runs
+    (internal.cuh split_begin / split_of_tile, restated).  When G exceeds
+    the tiles present at run time, empty splits lie between a sequence's
+    tiles, and its run of split indices c0..c1 (one merge weight each, held
+    in shared memory) grows towards G, far past its tile count.  The host
+    caps G at 2048, the merge's capacity."""
+    lens = [2047] + [1] * 15                      # tiles per sequence
+    T, G = sum(lens), 16 * 2047                   # G = B x tiles(max_len)
+    t0 = 0
+    for k in lens:
+        c0, c1 = _split_of_tile(t0, G, T), _split_of_tile(t0 + k - 1, G, T)
+        assert _split_begin(c0, G, T) <= t0 < _split_begin(c0 + 1, G, T)
+        assert c1 - c0 + 1 <= G
+        if k == 2047:
+            assert c1 - c0 + 1 > 2048             # what an uncapped G would meet
+        t0 += k
+    for G in (1, 7, 148, 2048):                   # the run never exceeds G
+        t0 = 0
+        for k in lens:
+            c0, c1 = _split_of_tile(t0, G, T), _split_of_tile(t0 + k - 1, G, T)
+            assert 1 <= c1 - c0 + 1 <= min(G, k + 1)
+            t0 += k
+    d = _dims(max_len=2047 * 128)
+    d.batch = 16
+    assert q.decode_workspace_bytes(d, num_splits=4096) == q.decode_workspace_bytes(d, num_splits=2048)
+    assert q.decode_workspace_bytes(d, num_splits=2047) < q.decode_workspace_bytes(d, num_splits=2048)
+
+
 def test_too_small_workspace_and_null_pointers():
     lib = ctypes.CDLL(q.LIB_PATH)
     lib.qsvd_decode_attn.argtypes = q._sigs["qsvd_decode_attn"]
