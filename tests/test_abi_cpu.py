@@ -320,3 +320,52 @@ def test_misaligned_outputs_and_scales_are_refused():
     st = lib.qsvd_decode_attn_per_head(ctypes.byref(dh), fake, fake, fake, fake, fake, fake, 0, fake,
                                        ctypes.byref(n), off8, None)
     assert st == q.QSVD_ERR_INVALID_ARG and b"out must be 16-byte" in q._lib.qsvd_last_error()
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) of every call in the header."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][A-Za-z0-9_ \*]*?)\b(qsvd_[a-z_]+)\s*\(([^)]*)\)\s*;", src):
+        params = [" ".join(p.split()) for p in m.group(3).split(",")]
+        params = [] if params == ["void"] else [p.rsplit(" ", 1)[0] if not p.endswith("*") else p
+                                                for p in params]
+        out[m.group(2)] = (" ".join(m.group(1).split()), params)
+    return out
+
+
+def _ctype_of(param):
+    """The ctypes type a parameter of this C type must be declared with."""
+    t = param.replace("const ", "").strip()
+    if t.startswith("qsvd_dims"):
+        return ctypes.POINTER(q.qsvd_dims)
+    if t.startswith("size_t") and "*" in t:
+        return ctypes.POINTER(ctypes.c_size_t)
+    if "*" in t:
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "unsigned": ctypes.c_uint, "size_t": ctypes.c_size_t,
+            "double": ctypes.c_double, "int64_t": ctypes.c_int64,
+            "unsigned long long": ctypes.c_ulonglong, "qsvd_status": ctypes.c_int}[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every call's ctypes argtypes have the header's parameter count and
+    types (a pointer as c_void_p, size_t* and qsvd_dims* as typed
+    pointers), so no argument is dropped, narrowed or widened on the way."""
+    protos = _prototypes()
+    assert set(q._sigs) | {"qsvd_status_string", "qsvd_last_error", "qsvd_kernel_launches",
+                           "qsvd_abi_version"} == set(protos)
+    for name, args in q._sigs.items():
+        ret, params = protos[name]
+        assert ret == "qsvd_status", name
+        assert len(args) == len(params), f"{name}: {len(args)} argtypes, header has {len(params)}"
+        for i, (a, p) in enumerate(zip(args, params)):
+            want = _ctype_of(p)
+            assert a is want or (hasattr(a, "_type_") and hasattr(want, "_type_") and a._type_ is want._type_
+                                 and a.__name__ == want.__name__), f"{name} argument {i}: {p!r}"
+    # pointer-sized and 64-bit results keep their width
+    assert q._lib.qsvd_last_error.restype is ctypes.c_char_p
+    assert q._lib.qsvd_status_string.restype is ctypes.c_char_p
+    assert q._lib.qsvd_kernel_launches.restype is ctypes.c_uint64
