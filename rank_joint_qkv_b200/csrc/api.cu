@@ -53,7 +53,7 @@ static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3
 // Host-checkable constraints shared by all calls.
 static qsvd_status validate(const qsvd_dims* d) {
   if (!d) return fail(QSVD_ERR_INVALID_ARG, "dims is NULL");
-  if (d->H <= 0 || d->d_h <= 0 || d->E != d->H * d->d_h)
+  if (d->H <= 0 || d->d_h <= 0 || (long long)d->E != (long long)d->H * d->d_h)
     return fail(QSVD_ERR_INVALID_ARG, "E (%d) must equal H (%d) * d_h (%d)", d->E, d->H, d->d_h);
   if (d->E % 64) return fail(QSVD_ERR_INVALID_ARG, "E (%d) must be a multiple of 64", d->E);
   if (d->d_h % 8 || d->d_h > 256)
@@ -62,6 +62,10 @@ static qsvd_status validate(const qsvd_dims* d) {
     return fail(QSVD_ERR_INVALID_ARG, "r (%d) must be a multiple of 32 in [32, 8192]", d->r);
   if (d->batch < 1) return fail(QSVD_ERR_INVALID_ARG, "batch must be >= 1");
   if (d->max_len < 1) return fail(QSVD_ERR_INVALID_ARG, "max_len must be >= 1");
+  // cache rows b * max_len + t are tensor-map coordinates and int indices
+  if ((long long)d->batch * d->max_len > 0x7FFFFFFFLL)
+    return fail(QSVD_ERR_INVALID_ARG, "batch x max_len (%lld) must be below 2^31",
+                (long long)d->batch * d->max_len);
   if (d->cache_dtype < QSVD_F32 || d->cache_dtype > QSVD_I4)
     return fail(QSVD_ERR_INVALID_ARG, "unknown cache dtype %d", int(d->cache_dtype));
   if (d->weight_dtype < QSVD_F32 || d->weight_dtype > QSVD_BF16)
@@ -497,6 +501,8 @@ qsvd_status qsvd_decode_attn_per_head(const qsvd_dims* dims, const void* bk, con
     return fail(QSVD_ERR_UNSUPPORTED,
                 "per-head latents, rotary mode: d_h == 128, r in {64, 128}, an F16 or BF16 cache "
                 "of the weight type");
+  if (d.rope && (long long)d.batch * d.H * d.max_len > 0x7FFFFFFFLL)   // head-major rows: 32-bit coordinates
+    return fail(QSVD_ERR_UNSUPPORTED, "per-head latents, rotary mode: batch x H x max_len must be below 2^31");
   if (cache_is_int(d)) return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: F32, F16 or BF16 caches");
   if (d.h2 || d.out_proj == QSVD_OUT_PROJ_CHAIN)
     return fail(QSVD_ERR_UNSUPPORTED, "per-head latents: no online H2, no chained output projection");

@@ -239,3 +239,15 @@ def test_rotary_scores_shared_memory_map(r, H):
     dynamic = 1024 + nst * stage + 128 * 130 * 4 + 128 + H * 128 * 4   # the launch's size
     assert end + 1023 <= dynamic
     assert dynamic + 3 * 2 * 128 * 4 <= 232448
+
+
+def test_rotary_rows_beyond_32_bit_coordinates_are_refused():
+    """Head-major rows (b H + h) max_len + t are tensor-map coordinates of
+    the rotary scores kernel: B x H x max_len must stay below 2^31."""
+    ok = _dims(rope=True, E=32 * 128, H=32, batch=(1 << 11) - 1, max_len=1 << 15)
+    assert q.per_head_workspace_bytes(ok) > 0
+    bad = _dims(rope=True, E=32 * 128, H=32, batch=1 << 11, max_len=1 << 15)
+    with pytest.raises(q.QsvdError) as e:
+        q.per_head_workspace_bytes(bad)
+    assert e.value.status == q.QSVD_ERR_UNSUPPORTED
+    assert b"2^31" in q._lib.qsvd_last_error()
