@@ -120,7 +120,7 @@ typedef struct {
   int H;               /* heads */
   int d_h;             /* head dim (multiple of 8, at most 256) */
   int r;               /* retained rank (latent width; multiple of 32, 32..8192) */
-  int batch;           /* B sequences per call */
+  int batch;           /* B sequences per call (at most 65535) */
   int max_len;         /* cache rows per sequence (capacity); batch x max_len < 2^31 */
   int group;           /* channels per quantisation group (I8/I4 caches) */
   int rope;            /* 0: no rotary embedding, query absorbed; 1: rotary */

@@ -60,7 +60,8 @@ static qsvd_status validate(const qsvd_dims* d) {
     return fail(QSVD_ERR_INVALID_ARG, "d_h (%d) must be a multiple of 8, at most 256", d->d_h);
   if (d->r < 32 || d->r % 32 || d->r > 8192)
     return fail(QSVD_ERR_INVALID_ARG, "r (%d) must be a multiple of 32 in [32, 8192]", d->r);
-  if (d->batch < 1) return fail(QSVD_ERR_INVALID_ARG, "batch must be >= 1");
+  // several kernels put the sequences on a grid's y or z axis
+  if (d->batch < 1 || d->batch > 65535) return fail(QSVD_ERR_INVALID_ARG, "batch must be in [1, 65535]");
   if (d->max_len < 1) return fail(QSVD_ERR_INVALID_ARG, "max_len must be >= 1");
   // cache rows b * max_len + t are tensor-map coordinates and int indices
   if ((long long)d->batch * d->max_len > 0x7FFFFFFFLL)

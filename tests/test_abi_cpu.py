@@ -74,7 +74,8 @@ def _dims(**kw):
     dict(cache="i4", group=100), dict(cache="i8", group=96), dict(d_h=130, E=520),
     dict(h2=True, h2_m=3),                   # r/h2_m = 256/3 not an integer
     dict(H=(1 << 24) + 1, d_h=256, E=256),   # H d_h wraps to E in 32-bit arithmetic
-    dict(batch=1 << 16, max_len=1 << 15),    # 2^31 cache rows: beyond 32-bit coordinates
+    dict(batch=1 << 15, max_len=1 << 16),    # 2^31 cache rows: beyond 32-bit coordinates
+    dict(batch=65536, max_len=16),           # sequences beyond a grid's y / z extent
 ])
 def test_invalid_dims_rejected_on_host(bad):
     d = _dims(**bad)
