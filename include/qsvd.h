@@ -395,6 +395,11 @@ qsvd_status qsvd_decode_attn(const qsvd_dims* dims, const void* packed,
  * Source: WSVD digest, Method 3.4 (flash decoding); QSVD digest, Step 1.
  * With dims->out_proj the output is o W_O (see QSVD_OUT_PROJ_*).
  * Equivalent to qsvd_decode_attn with phases = QSVD_PHASE_COMBINE.
+ * The workspace's size is not passed: it must be the one the decode call
+ * used, and num_splits must be that call's (the merge takes the split
+ * count recorded in the workspace and the partials' offsets from
+ * num_splits; with another value it reads other offsets, possibly past
+ * the workspace).
  * Errors: INVALID_ARG, CUDA.
  */
 qsvd_status qsvd_combine_splits(const qsvd_dims* dims, const void* packed,
